@@ -1,0 +1,137 @@
+"""Seeded synthetic inputs for the gated delta rule.
+
+This module holds the workload table and the random draws only -- none of the
+rule's arithmetic.  Both the CUDA path's tests/benchmark and the CPU oracle are
+fed from here, so both see the same bits.
+
+Draw recipe (one ``torch.Generator`` per workload, CPU, float32): q, k, v, the
+beta logit, the gate logit, then S0, each ~N(0,1) unless stated.  q and k are
+L2-normalised per token and head in float32, then rounded to the workload's
+dtype; v is rounded to the dtype; beta = sigmoid(logit); log_alpha is one of
+    -softplus(x),  -0.1 * softplus(x)  (slow decay),  Uniform[-5, 0];
+S0 is zero or N(0, std 0.02) in float32.  The gates stay float32.
+
+The shapes and laws mirror the layers the pages train (1.3B-parameter Gated
+DeltaNet models: "Gated DeltaNet: Harmonizing Gating and the Delta Rule for
+Superior Linear RNNs", section "Experiments: Performance at Scale"); no dataset
+is involved, the inputs are synthetic stand-ins.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    T: int
+    Dk: int
+    Dv: int
+    chunk: int
+    dtype: str          # "f32" or "bf16": type of q, k, v and o
+    gate_law: str       # "softplus", "slow_softplus" or "uniform5"
+    s0_law: str         # "zero" or "normal002"
+    seed: int
+    steps: int = 0      # decode workloads: number of successive single-token steps
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+# The chunkwise-forward shapes, the headline shape and the decode shape.
+WORKLOADS = {
+    w.name: w for w in [
+        Workload("tiny_f32", 1, 2, 64, 16, 16, 16, "f32", "softplus", "zero", 1001),
+        Workload("bf16_T2k", 4, 16, 2048, 128, 128, 64, "bf16", "slow_softplus", "zero", 1002),
+        Workload("long_T32k", 1, 16, 32768, 128, 128, 64, "bf16", "uniform5", "normal002", 1003),
+        Workload("wide_dk256_dv512", 8, 6, 4096, 256, 512, 64, "bf16", "softplus", "zero", 1004),
+        Workload("decode_b256", 256, 16, 1, 128, 128, 0, "bf16", "softplus", "normal002", 1005,
+                 steps=1000),
+        Workload("headline_T4k", 4, 16, 4096, 128, 128, 64, "bf16", "slow_softplus", "zero", 1006),
+    ]
+}
+
+HEADLINE = "headline_T4k"
+
+
+def workload(name: str, **overrides) -> Workload:
+    w = WORKLOADS[name]
+    return replace(w, **overrides) if overrides else w
+
+
+def _gates(gen, shape, law):
+    beta = torch.sigmoid(torch.randn(shape, generator=gen))
+    x = torch.randn(shape, generator=gen)
+    if law == "softplus":
+        la = -torch.nn.functional.softplus(x)
+    elif law == "slow_softplus":
+        la = -0.1 * torch.nn.functional.softplus(x)
+    elif law == "uniform5":
+        la = -5.0 * torch.rand(shape, generator=gen)
+    else:
+        raise ValueError(law)
+    return la.contiguous(), beta.contiguous()
+
+
+def _unit_rows(x):
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+
+
+def chunk_inputs(w: Workload, seed: int | None = None, device="cpu"):
+    """Inputs of one chunkwise forward call, as CPU (or ``device``) tensors.
+
+    q,k [B,T,H,Dk] dtype; v [B,T,H,Dv] dtype; log_alpha, beta [B,T,H] f32;
+    S0 [B,H,Dv,Dk] f32 or None.
+    """
+    gen = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    q = _unit_rows(torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    k = _unit_rows(torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    v = torch.randn((B, T, H, Dv), generator=gen).to(w.torch_dtype)
+    la, beta = _gates(gen, (B, T, H), w.gate_law)
+    S0 = None
+    if w.s0_law == "normal002":
+        S0 = 0.02 * torch.randn((B, H, Dv, Dk), generator=gen)
+    out = dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0)
+    if device != "cpu":
+        out = {n: (t.to(device) if t is not None else None) for n, t in out.items()}
+    return out
+
+
+def decode_state(w: Workload, device="cpu"):
+    """Initial decode state S0 [B,H,Dv,Dk] f32."""
+    gen = torch.Generator().manual_seed(w.seed)
+    S0 = torch.zeros((w.B, w.H, w.Dv, w.Dk))
+    if w.s0_law == "normal002":
+        S0 = 0.02 * torch.randn((w.B, w.H, w.Dv, w.Dk), generator=gen)
+    return S0.to(device)
+
+
+def decode_step_inputs(w: Workload, step: int, device="cpu"):
+    """Token ``step`` of a decode run: q,k [B,H,Dk], v [B,H,Dv] dtype; gates [B,H] f32."""
+    gen = torch.Generator().manual_seed(w.seed * 1_000_003 + step + 1)
+    B, H, Dk, Dv = w.B, w.H, w.Dk, w.Dv
+    q = _unit_rows(torch.randn((B, H, Dk), generator=gen)).to(w.torch_dtype)
+    k = _unit_rows(torch.randn((B, H, Dk), generator=gen)).to(w.torch_dtype)
+    v = torch.randn((B, H, Dv), generator=gen).to(w.torch_dtype)
+    la, beta = _gates(gen, (B, H), w.gate_law)
+    out = dict(q=q, k=k, v=v, log_alpha=la, beta=beta)
+    if device != "cpu":
+        out = {n: t.to(device) for n, t in out.items()}
+    return out
+
+
+def sample_units(w: Workload, n: int, seed: int = 7):
+    """A fixed, seeded sample of (b*H + h) head indices, always including the first
+    and the last head."""
+    total = w.B * w.H
+    if n >= total:
+        return list(range(total))
+    gen = torch.Generator().manual_seed(seed)
+    mid = torch.randperm(total - 2, generator=gen)[: max(n - 2, 0)] + 1
+    return sorted({0, total - 1, *[int(x) for x in mid]})

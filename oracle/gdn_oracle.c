@@ -1,0 +1,222 @@
+/*
+ * gdn_oracle.c -- the ORACLE for the gated delta rule: a plain, slow, float64,
+ * token-by-token CPU recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  It exists to check the CUDA path, never to stand in
+ * for it.  Only the test suite, the smoke check and the benchmark's CPU-baseline
+ * leg may load it.  It shares no code, header, table or helper with the CUDA
+ * library; nothing here is blocked, chunked, fused or reordered.
+ *
+ * What it computes (per batch item b and head h, independently):
+ *
+ *   S_t = S_{t-1} ( alpha_t ( I - beta_t k_t k_t^T ) ) + beta_t v_t k_t^T      (1)
+ *   o_t = S_t q_t                                                             (2)
+ *
+ * (1) is the gated delta rule as stated in "Gated Delta Networks: Improving
+ * Mamba2 with Delta Rule" (atlas.scime.ai summary, section "Approach") and again,
+ * in damaged LaTeX where "k_t^{o}p" stands for k_t^T, in "Gated DeltaNet:
+ * Harmonizing Gating and the Delta Rule for Superior Linear RNNs" (wispaper.ai
+ * blog, section "Methodology: The Gated Delta Rule").  The orientation of the
+ * state follows from the write term beta v k^T: S has Dv rows and Dk columns.
+ *
+ * (2) is not written on the pages; the reading adopted is the usual linear
+ * attention read-out with the state AFTER the token's own update.
+ *
+ * Input conventions (readings where the pages are silent): the gate is passed
+ * as log(alpha) (<= 0) and alpha = exp(log alpha) is taken here; beta is passed
+ * as is.  All arithmetic is double precision.
+ *
+ * Row i of the product S_{t-1} (alpha (I - beta k k^T)) is written out as
+ *   alpha * S[i][j] - alpha * beta * (sum_m S[i][m] k[m]) * k[j]
+ * which is the same matrix product with the sum over m collected once per row.
+ *
+ * Layouts (all row-major, C order):
+ *   forward:  q,k [B,T,H,Dk]   v [B,T,H,Dv]   log_alpha,beta [B,T,H]
+ *             S0,S_T [B,H,Dv,Dk]   o [B,T,H,Dv]
+ *   decode:   q,k [steps,B,H,Dk]  v [steps,B,H,Dv]  log_alpha,beta [steps,B,H]
+ *             S [B,H,Dv,Dk] (updated in place)   o [steps,B,H,Dv]
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* One token of (1) and (2) on one head: S (Dv x Dk) is updated in place and
+ * o (Dv) receives S_t q_t. */
+static void gdn_token(double *S, const double *q, const double *k,
+                      const double *v, double log_alpha, double beta,
+                      double *o, long Dk, long Dv)
+{
+    const double alpha = exp(log_alpha);
+    for (long i = 0; i < Dv; ++i) {
+        double *row = S + i * Dk;
+        double sk = 0.0; /* (S_{t-1} k_t)_i */
+        for (long m = 0; m < Dk; ++m)
+            sk += row[m] * k[m];
+        for (long j = 0; j < Dk; ++j)
+            row[j] = alpha * row[j] - alpha * beta * sk * k[j] + beta * v[i] * k[j];
+        double oi = 0.0; /* (S_t q_t)_i */
+        for (long j = 0; j < Dk; ++j)
+            oi += row[j] * q[j];
+        o[i] = oi;
+    }
+}
+
+/* Where token t of unit u lives: element offset = base + t * stride. */
+typedef struct {
+    const double *q, *k, *v, *la, *beta;
+    double *o, *S;
+    long T, Dk, Dv;
+    long tstride_qk, tstride_v, tstride_g; /* element stride between tokens */
+    const int *units;
+    int n_units;
+    int n_threads;
+    int thread_id;
+    int mode; /* 0 forward, 1 decode */
+    long B, H;
+} job_t;
+
+static void run_unit(const job_t *j, long u)
+{
+    const long b = u / j->H, h = u % j->H;
+    long qk0, v0, g0;
+    if (j->mode == 0) { /* [B,T,H,*] */
+        qk0 = (b * j->T * j->H + h) * j->Dk;
+        v0 = (b * j->T * j->H + h) * j->Dv;
+        g0 = b * j->T * j->H + h;
+    } else { /* [steps,B,H,*] */
+        qk0 = (b * j->H + h) * j->Dk;
+        v0 = (b * j->H + h) * j->Dv;
+        g0 = b * j->H + h;
+    }
+    double *S = j->S + u * j->Dv * j->Dk;
+    for (long t = 0; t < j->T; ++t) {
+        gdn_token(S, j->q + qk0 + t * j->tstride_qk, j->k + qk0 + t * j->tstride_qk,
+                  j->v + v0 + t * j->tstride_v, j->la[g0 + t * j->tstride_g],
+                  j->beta[g0 + t * j->tstride_g], j->o + v0 + t * j->tstride_v,
+                  j->Dk, j->Dv);
+    }
+}
+
+static void *worker(void *arg)
+{
+    const job_t *j = (const job_t *)arg;
+    const long n = j->units ? j->n_units : j->B * j->H;
+    for (long i = j->thread_id; i < n; i += j->n_threads)
+        run_unit(j, j->units ? (long)j->units[i] : i);
+    return NULL;
+}
+
+static int run_job(job_t *proto, int nthreads)
+{
+    const long n = proto->units ? proto->n_units : proto->B * proto->H;
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > n)
+        nthreads = (int)(n > 0 ? n : 1);
+    job_t *jobs = (job_t *)malloc(sizeof(job_t) * (size_t)nthreads);
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!jobs || !tid) {
+        free(jobs);
+        free(tid);
+        return -2;
+    }
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = *proto;
+        jobs[i].n_threads = nthreads;
+        jobs[i].thread_id = i;
+    }
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&tid[i], NULL, worker, &jobs[i]) != 0)
+            break;
+        started = i;
+    }
+    /* thread 0 runs on the caller; if a pthread failed to start, the caller
+     * picks up its share afterwards */
+    worker(&jobs[0]);
+    for (int i = 1; i <= started; ++i)
+        pthread_join(tid[i], NULL);
+    for (int i = started + 1; i < nthreads; ++i)
+        worker(&jobs[i]);
+    free(jobs);
+    free(tid);
+    return 0;
+}
+
+static int check_units(const int *units, int n_units, long n_all)
+{
+    if (!units)
+        return 0;
+    if (n_units < 0)
+        return -1;
+    for (int i = 0; i < n_units; ++i)
+        if (units[i] < 0 || units[i] >= n_all)
+            return -1;
+    return 0;
+}
+
+/*
+ * Full-sequence recurrence.  S_T receives the final state of every processed
+ * unit (it is also the working state); S0 may be NULL for a zero initial state.
+ * units/n_units: NULL runs every (b,h) unit (u = b*H + h); otherwise only the
+ * listed units are computed and only their slices of o and S_T are written.
+ * Returns 0, or -1 on a bad argument, -2 on allocation failure.
+ */
+int gdn_oracle_forward(const double *q, const double *k, const double *v,
+                       const double *log_alpha, const double *beta,
+                       const double *S0, double *o, double *S_T,
+                       long B, long T, long H, long Dk, long Dv,
+                       const int *units, int n_units, int nthreads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !o || !S_T)
+        return -1;
+    if (B <= 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0)
+        return -1;
+    if (check_units(units, n_units, B * H))
+        return -1;
+    const long n = units ? n_units : B * H;
+    for (long i = 0; i < n; ++i) {
+        const long u = units ? units[i] : i;
+        double *dst = S_T + u * Dv * Dk;
+        if (S0)
+            memcpy(dst, S0 + u * Dv * Dk, sizeof(double) * (size_t)(Dv * Dk));
+        else
+            memset(dst, 0, sizeof(double) * (size_t)(Dv * Dk));
+    }
+    job_t j;
+    memset(&j, 0, sizeof(j));
+    j.q = q; j.k = k; j.v = v; j.la = log_alpha; j.beta = beta;
+    j.o = o; j.S = S_T;
+    j.T = T; j.Dk = Dk; j.Dv = Dv; j.B = B; j.H = H;
+    j.tstride_qk = H * Dk; j.tstride_v = H * Dv; j.tstride_g = H;
+    j.units = units; j.n_units = n_units; j.mode = 0;
+    return run_job(&j, nthreads);
+}
+
+/*
+ * `steps` successive single-token updates of the state S (in place), one token
+ * per (b,h) per step -- the recurrent (decoding) form of the same rule.
+ */
+int gdn_oracle_decode(const double *q, const double *k, const double *v,
+                      const double *log_alpha, const double *beta,
+                      double *S, double *o,
+                      long steps, long B, long H, long Dk, long Dv,
+                      const int *units, int n_units, int nthreads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !o || !S)
+        return -1;
+    if (B <= 0 || steps < 0 || H <= 0 || Dk <= 0 || Dv <= 0)
+        return -1;
+    if (check_units(units, n_units, B * H))
+        return -1;
+    job_t j;
+    memset(&j, 0, sizeof(j));
+    j.q = q; j.k = k; j.v = v; j.la = log_alpha; j.beta = beta;
+    j.o = o; j.S = S;
+    j.T = steps; j.Dk = Dk; j.Dv = Dv; j.B = B; j.H = H;
+    j.tstride_qk = B * H * Dk; j.tstride_v = B * H * Dv; j.tstride_g = B * H;
+    j.units = units; j.n_units = n_units; j.mode = 1;
+    return run_job(&j, nthreads);
+}
