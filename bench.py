@@ -1,0 +1,384 @@
+"""Benchmark of the gated delta rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one chunkwise forward (``gdn_chunk_fwd``) over the headline workload
+(B=4, H=16, T=4096, Dk=Dv=128, chunk 64, bf16 q/k/v/o, float32 gates and state),
+inputs resident in HBM.  The value is tokens/s over all ranks (weak scaling:
+every rank runs its own copy of the workload, no collective on the data path).
+The same run also times the recurrent decode step (batch 256, H 16, d 128,
+float32 state in HBM updated in place) and reports its HBM bandwidth.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU oracle
+(the only other implementation of the rule) on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_130_b200 import inputs as I  # noqa: E402
+
+METRIC = "GDN chunk fwd tokens/s (bf16,H=16,d=128,T=4K); % TC peak; decode HBM GB/s"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def chunk_flops(w) -> float:
+    """Dense contraction FLOPs of the chunkwise algorithm, 2(3 C Dk + 2 C Dv + 3 Dk Dv)
+    per token per head (the gated Gram matrix, the WY factors, the state update and
+    the output)."""
+    C = w.chunk
+    return 2.0 * (3 * C * w.Dk + 2 * C * w.Dv + 3 * w.Dk * w.Dv) * w.B * w.T * w.H
+
+
+def chunk_bytes(w, has_s0: bool) -> float:
+    """Compulsory HBM bytes of one chunkwise forward: q, k, v read and o written
+    once in the element type, both gates read once (float32), S0 read if given,
+    S_T written (float32)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    tok = w.B * w.T * w.H
+    state = w.B * w.H * w.Dv * w.Dk * 4
+    return tok * (esz * (2 * w.Dk + 2 * w.Dv) + 8) + state * (2 if has_s0 else 1)
+
+
+def decode_bytes(w) -> float:
+    """Compulsory HBM bytes of one decode step: the float32 state read and written,
+    q, k, v read and o written in the element type, the two gates read."""
+    esz = 2 if w.dtype == "bf16" else 4
+    heads = w.B * w.H
+    return heads * (8 * w.Dv * w.Dk + esz * (2 * w.Dk + 2 * w.Dv) + 8)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def time_loop(fn, steps, stream, world):
+    """Device time of exactly `steps` calls, bracketed by barrier + synchronize."""
+    _barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    return start.elapsed_time(end)  # ms
+
+
+def cpu_baseline(w, inp, budget_s=15.0):
+    """The float64 oracle on a bounded sample of whole heads, all host cores."""
+    from oracle import oracle as O
+    ncores = O.default_threads()
+    one = I.sample_units(w, 1)
+    t0 = time.perf_counter()
+    O.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"], units=one,
+              nthreads=1)
+    t_head = time.perf_counter() - t0
+    n = max(1, min(w.B * w.H, int(budget_s / max(t_head, 1e-6))))
+    units = I.sample_units(w, n)
+    t0 = time.perf_counter()
+    O.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"], units=units,
+              nthreads=ncores)
+    wall = time.perf_counter() - t0
+    tokens = len(units) * w.T / w.H  # token-heads processed, expressed in tokens
+    return {"value": tokens / wall, "unit": UNIT, "cores": min(ncores, len(units)), "kind": "oracle",
+            "sample": f"{len(units)} of {w.B * w.H} (b,h) heads, all {w.T} tokens each "
+                      f"({wall:.2f} s wall); tokens/s = heads*T/H / wall"}
+
+
+def run_reference(args):
+    """--impl reference: the float64 oracle, timed on the host cores, rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    w = I.workload(I.HEADLINE)
+    inp = I.chunk_inputs(w)
+    ncores = O.default_threads()
+    # each step: the first n_tok tokens of a sample of heads, sized so that the
+    # whole run takes about two minutes
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    units = I.sample_units(w, min(w.B * w.H, ncores))
+    probe_tok = min(w.T, 256)
+    sl = lambda x: x[:, :probe_tok].contiguous()
+    t0 = time.perf_counter()
+    O.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_alpha"]), sl(inp["beta"]),
+              None, units=units, nthreads=ncores)
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    n_tok = int(max(1, min(w.T, probe_tok * per_step / t_probe)))
+    sl = lambda x: x[:, :n_tok].contiguous()
+    args_ = [sl(inp[n]) for n in ("q", "k", "v", "log_alpha", "beta")]
+    for _ in range(args.warmup):
+        O.forward(*args_, None, units=units, nthreads=ncores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.forward(*args_, None, units=units, nthreads=ncores)
+    wall = time.perf_counter() - t0
+    tokens = args.steps * len(units) * n_tok / w.H
+    value = tokens / wall
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} Dk={w.Dk} Dv={w.Dv} "
+                               f"chunk={w.chunk} {w.dtype}", "global_batch": w.B, "seq_len": w.T,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(ncores, len(units)),
+                         "kind": "oracle",
+                         "sample": f"per step: first {n_tok} tokens of {len(units)} of "
+                                   f"{w.B * w.H} heads; tokens/s = heads*tokens/H / wall"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    world, rank, local = _dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from gated_delta_rule_130_b200 import binding as G
+
+    pk, pk_kind = peaks()
+    w = I.workload(I.HEADLINE)
+    inp_cpu = I.chunk_inputs(w, seed=w.seed + rank)
+    inp = {n: (t.to(device) if t is not None else None) for n, t in inp_cpu.items()}
+    path = G.chunk_fwd_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
+    launches_per_step = {"tcgen05": 1, "simt": 2}[path]
+    o = torch.empty((w.B, w.T, w.H, w.Dv), dtype=w.torch_dtype, device=device)
+    S_T = torch.empty((w.B, w.H, w.Dv, w.Dk), dtype=torch.float32, device=device)
+    ws_bytes = G.chunk_fwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        G.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                    chunk=w.chunk, out=o, S_T=S_T, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    steps = args.steps
+    if steps is None:  # about three seconds of timed work
+        t_one = time_loop(step, 10, stream, 1) / 10
+        steps = int(min(50000, max(100, 3000.0 / max(t_one, 1e-3))))
+        steps = int(_max_over_ranks(steps, world, device))
+    with ClockSampler(local) as clk:
+        ms = time_loop(step, steps, stream, world)
+    clocks = clk.summary()
+    ms_max = _max_over_ranks(ms, world, device)
+    ms_step = ms_max / steps
+    tokens = w.B * w.T
+    value = world * tokens / (ms_step * 1e-3)
+
+    # roofline of the dominant kernel (the whole call: one fused kernel on the
+    # tcgen05 path; the two CUDA-core kernels together on the SIMT path)
+    F = chunk_flops(w)
+    Bytes = chunk_bytes(w, inp["S0"] is not None)
+    t_s = (ms / steps) * 1e-3
+    gbs = Bytes / t_s / 1e9
+    tflops = F / t_s / 1e12
+    hbm_peak = pk["hbm_gbs"]
+    tc_peak = pk["bf16_tflops"]
+    roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": gbs / hbm_peak, "traffic": None,
+                "kernel": f"gdn_chunk_fwd ({path}, {launches_per_step} launch/step)",
+                "algorithmic_bytes": Bytes, "peak_source": f"{pk_kind} hbm_gbs",
+                "tc": {"achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                       "frac": tflops / tc_peak, "flops": F,
+                       "peak_source": f"{pk_kind} bf16_tflops (burst)"}}
+
+    # decode step: batch 256, H 16, d 128, 1000 steps, state resident in HBM
+    wd = I.workload("decode_b256")
+    S = I.decode_state(wd, device=device)
+    dec_in = [{n: t.to(device) for n, t in I.decode_step_inputs(wd, t).items()} for t in range(8)]
+    od = torch.empty((wd.B, wd.H, wd.Dv), dtype=wd.torch_dtype, device=device)
+    it = [0]
+
+    def dstep():
+        x = dec_in[it[0] % len(dec_in)]
+        it[0] += 1
+        G.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=od)
+
+    for _ in range(20):
+        dstep()
+    dms = time_loop(dstep, wd.steps, stream, world)
+    dms_max = _max_over_ranks(dms, world, device)
+    d_us = 1e3 * dms / wd.steps
+    d_gbs = decode_bytes(wd) / (d_us * 1e-6) / 1e9
+    decode = {"workload": f"decode_b256: batch={wd.B} H={wd.H} Dk={wd.Dk} Dv={wd.Dv} bf16 "
+                          f"q/k/v/o, f32 state in place, {wd.steps} steps",
+              "us_per_step": 1e3 * dms_max / wd.steps, "achieved": d_gbs, "unit": "GB/s",
+              "peak": hbm_peak, "frac": d_gbs / hbm_peak, "bytes_per_step": decode_bytes(wd),
+              "gpu_launches": wd.steps}
+
+    # end to end through the public API with host buffers: pinned host inputs
+    # copied in, the call, o and S_T copied back, every step
+    host = {n: (t.pin_memory() if t is not None else None) for n, t in inp_cpu.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    s_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    dev_bufs = {n: (torch.empty_like(t, device=device) if t is not None else None)
+                for n, t in host.items()}
+
+    def e2e_step():
+        for n, t in host.items():
+            if t is not None:
+                dev_bufs[n].copy_(t, non_blocking=True)
+        G.chunk_fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["log_alpha"],
+                    dev_bufs["beta"], dev_bufs["S0"], chunk=w.chunk, out=o, S_T=S_T, workspace=ws)
+        o_h.copy_(o, non_blocking=True)
+        s_h.copy_(S_T, non_blocking=True)
+
+    e2e_steps = max(3, min(steps, 30))
+    for _ in range(3):
+        e2e_step()
+    ems = _max_over_ranks(time_loop(e2e_step, e2e_steps, stream, world), world, device)
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+    e2e = {"value": world * tokens / (ems / e2e_steps * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp_cpu)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} Dk={w.Dk} Dv={w.Dv} "
+                                   f"chunk={w.chunk} bf16 q/k/v/o, f32 gates and state, S0=0",
+                       "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (q,k,v,o = %.0f MB per rank)" %
+                             (4 * o.numel() * o.element_size() / 1e6),
+                       "path": path},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 10
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -8,8 +8,8 @@ first such use raises if ``libgdn.so`` is missing -- there is no fallback.
 """
 
 _BINDING_NAMES = {
-    "chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "library_path", "GdnError",
-    "chunk_fwd_host",
+    "chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "chunk_fwd_path", "library_path",
+    "GdnError",
 }
 
 

@@ -1,0 +1,165 @@
+"""Thin ctypes binding of libgdn.so (C ABI in include/gdn.h).
+
+Argument marshalling only: shape/dtype checks, device pointers, the current
+torch stream, and workspace allocation through torch.  Every step of the
+computation runs in the library's CUDA kernels.  Importing this module loads the
+library and raises if it is missing -- there is no other implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+PATH_NONE, PATH_SIMT, PATH_TCGEN05 = 0, 1, 2
+PATH_NAMES = {PATH_NONE: "none", PATH_SIMT: "simt", PATH_TCGEN05: "tcgen05"}
+
+
+class GdnError(RuntimeError):
+    pass
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"libgdn.so not found at {_LIB_PATH}: build it with "
+            "`python -m gated_delta_rule_130_b200.build` (there is no fallback path)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, fp, I, Z = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, I, vp, Z, vp]
+    lib.gdn_chunk_fwd.restype = I
+    lib.gdn_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_fwd_workspace_size.restype = Z
+    lib.gdn_chunk_fwd_path.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_fwd_path.restype = I
+    lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, vp]
+    lib.gdn_decode_step.restype = I
+    lib.gdn_status_string.argtypes = [I]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    raise GdnError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise GdnError(f"{what}: {LIB.gdn_status_string(status).decode()} (status {status})")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise GdnError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise GdnError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise GdnError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise GdnError(f"{name} is on {t.device}, expected {device}")
+    return t.data_ptr()
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> int:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(LIB.gdn_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+
+
+def chunk_fwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    p = int(LIB.gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, code))
+    if p < 0:
+        raise GdnError("invalid or unsupported sizes")
+    return PATH_NAMES[p]
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=None,
+              return_state: bool = True, workspace=None):
+    """Chunkwise forward: returns (o [B,T,H,Dv], S_T [B,H,Dv,Dk] float32 or None).
+
+    q, k [B,T,H,Dk] and v [B,T,H,Dv] in float32 or bfloat16 (same type);
+    log_alpha, beta [B,T,H] float32; S0 [B,H,Dv,Dk] float32 or None (zeros).
+    ``S_T`` may be passed (and may be ``S0`` itself for in-place continuation).
+    """
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise GdnError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[3]
+    dev = q.device
+    code = _dtype_code(q)
+    args = [_dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev)]
+    if log_alpha.shape != (B, T, H) or beta.shape != (B, T, H):
+        raise GdnError("log_alpha and beta must be [B,T,H]")
+    args += [_dev(log_alpha, "log_alpha", torch.float32, dev),
+             _dev(beta, "beta", torch.float32, dev)]
+    if S0 is not None:
+        if S0.shape != (B, H, Dv, Dk):
+            raise GdnError("S0 must be [B,H,Dv,Dk]")
+        args.append(_dev(S0, "S0", torch.float32, dev))
+    else:
+        args.append(None)
+    o = out if out is not None else torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
+    if o.shape != (B, T, H, Dv):
+        raise GdnError("out must be [B,T,H,Dv]")
+    args.append(_dev(o, "out", q.dtype, dev))
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        if S_T.shape != (B, H, Dv, Dk):
+            raise GdnError("S_T must be [B,H,Dv,Dk]")
+        args.append(_dev(S_T, "S_T", torch.float32, dev))
+    else:
+        args.append(None)
+    need = int(LIB.gdn_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    st = LIB.gdn_chunk_fwd(*args, B, T, H, Dk, Dv, chunk, code, ws_ptr, ws_bytes, _stream_ptr(dev))
+    _check(st, "gdn_chunk_fwd")
+    return o, S_T
+
+
+def decode_step(q, k, v, log_alpha, beta, S, out=None):
+    """One recurrent step for every (b,h); S [B,H,Dv,Dk] float32 is updated in place.
+
+    q, k [B,H,Dk], v [B,H,Dv] float32 or bfloat16; log_alpha, beta [B,H] float32.
+    Returns o [B,H,Dv] in q's dtype.
+    """
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise GdnError("q, k must be [B,H,Dk] and v [B,H,Dv]")
+    B, H, Dk = q.shape
+    Dv = v.shape[2]
+    dev = q.device
+    code = _dtype_code(q)
+    if log_alpha.shape != (B, H) or beta.shape != (B, H) or S.shape != (B, H, Dv, Dk):
+        raise GdnError("log_alpha, beta must be [B,H] and S [B,H,Dv,Dk]")
+    o = out if out is not None else torch.empty((B, H, Dv), dtype=q.dtype, device=dev)
+    st = LIB.gdn_decode_step(
+        _dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
+        _dev(log_alpha, "log_alpha", torch.float32, dev), _dev(beta, "beta", torch.float32, dev),
+        _dev(S, "S", torch.float32, dev), _dev(o, "out", q.dtype, dev), B, H, Dk, Dv, code,
+        _stream_ptr(dev))
+    _check(st, "gdn_decode_step")
+    return o

@@ -1,0 +1,125 @@
+// C-ABI entry points of libgdn.so (declared in include/gdn.h): argument checks
+// on the host, then dispatch to the kernels.  Nothing is launched when a check
+// fails, and the library allocates nothing.
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+#include "kernels.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte ranges [a, a+na) and [b, b+nb) intersect.
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+constexpr int kMaxDk = 256, kMaxDv = 512, kMaxGrid = 65535;
+
+// 0 = fine, otherwise the status to return.
+gdn_status_t check_sizes(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
+    if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (Dk > kMaxDk || Dv > kMaxDv) return GDN_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+    if (B > kMaxGrid || H > kMaxGrid) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+bool empty_problem(int B, int T, int H) { return B == 0 || H == 0 || T == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status_t status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported size or type";
+        case GDN_ERR_CUDA: return "CUDA launch failed";
+    }
+    return "unknown status";
+}
+
+int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
+    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK) return -1;
+    if (empty_problem(B, T, H)) return GDN_PATH_NONE;
+    if (gdn::tc_supported(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16)) return GDN_PATH_TCGEN05;
+    return GDN_PATH_SIMT;
+}
+
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
+                                    gdn_dtype_t dtype) {
+    if (gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype) != GDN_PATH_SIMT) return 0;
+    return gdn::simt_workspace_bytes(B, T, H, chunk);
+}
+
+gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *S0, void *o, float *S_T, int B, int T,
+                           int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    const gdn_status_t sz = check_sizes(B, T, H, Dk, Dv, chunk, dtype);
+    if (sz != GDN_OK) return sz;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4;
+    const size_t n_tok = (size_t)B * T * H;
+    const size_t state_bytes = (size_t)B * H * Dv * Dk * sizeof(float);
+    if (B == 0 || H == 0) return GDN_OK;
+    if (T == 0) {  // no tokens: the final state is the initial one
+        if (!S_T) return GDN_OK;
+        if (!aligned16(S_T) || (S0 && !aligned16(S0))) return GDN_ERR_INVALID_ARG;
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, state_bytes,
+                                                          cudaMemcpyDeviceToDevice, st))
+                           : cudaMemsetAsync(S_T, 0, state_bytes, st);
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+    if (!q || !k || !v || !log_alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, o, S_T, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t o_bytes = n_tok * Dv * esz;
+    if (overlaps(o, o_bytes, q, n_tok * Dk * esz) || overlaps(o, o_bytes, k, n_tok * Dk * esz) ||
+        overlaps(o, o_bytes, v, n_tok * Dv * esz))
+        return GDN_ERR_INVALID_ARG;
+    if (S_T && S0 && S_T != S0 && overlaps(S_T, state_bytes, S0, state_bytes))
+        return GDN_ERR_INVALID_ARG;
+
+    const bool bf16 = dtype == GDN_BF16;
+    cudaError_t e;
+    if (gdn::tc_supported(B, T, H, Dk, Dv, chunk, bf16)) {
+        e = gdn::launch_chunk_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, st);
+    } else {
+        const size_t need = gdn::simt_workspace_bytes(B, T, H, chunk);
+        if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+        e = gdn::launch_chunk_simt(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk,
+                                   bf16, workspace, st);
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, float *S, void *o, int B, int H, int Dk, int Dv,
+                             gdn_dtype_t dtype, void *stream) {
+    if (B < 0 || H < 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (Dk > kMaxDk || Dv > kMaxDv) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4;
+    const size_t heads = (size_t)B * H;
+    if (overlaps(o, heads * Dv * esz, S, heads * Dv * Dk * sizeof(float)))
+        return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_decode(q, k, v, log_alpha, beta, S, o, B, H, Dk, Dv,
+                                             dtype == GDN_BF16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // extern "C"

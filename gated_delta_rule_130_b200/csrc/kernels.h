@@ -1,0 +1,29 @@
+// Internal launchers of the library's kernels (host side).  Each enqueues its
+// kernels on `st` and returns the launch status; argument checking is done by
+// the C-ABI layer before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdn {
+
+// Recurrent step over every (b,h): decode.cu.
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, float *S, void *o, int B, int H, int Dk, int Dv,
+                          bool bf16, cudaStream_t st);
+
+// CUDA-core chunkwise forward (any supported size, f32 or bf16): chunk_simt.cu.
+size_t simt_workspace_bytes(int B, int T, int H, int chunk);
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *S0, void *o, float *S_T, int B,
+                              int T, int H, int Dk, int Dv, int chunk, bool bf16, void *workspace,
+                              cudaStream_t st);
+
+// Fused tcgen05 chunkwise forward: chunk_tc.cu.
+bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *S0, void *o, float *S_T, int B, int T,
+                            int H, int Dk, int Dv, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,130 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdn.so.
+ *
+ * The operation is the gated delta rule of Gated DeltaNet,
+ *
+ *     S_t = S_{t-1} ( alpha_t ( I - beta_t k_t k_t^T ) ) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,
+ *
+ * as stated in "Gated Delta Networks: Improving Mamba2 with Delta Rule"
+ * (atlas.scime.ai summary, section "Approach"), computed either chunk by chunk
+ * with the gated WY/UT representation that page names ("extended WY/UT
+ * chunkwise algorithm"; "Gated DeltaNet: Harmonizing Gating and the Delta Rule
+ * for Superior Linear RNNs", section "Hardware-Efficient Training"), or one
+ * token at a time for decoding.  The read-out o_t = S_t q_t uses the state after
+ * the token's own update (the pages do not write the read-out down).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates nothing, keeps no state between calls, and only enqueues work on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream).  Calls
+ *    return as soon as the work is enqueued.
+ *  - Layouts are dense row-major (C order), no strides:
+ *        q, k      [B, T, H, Dk]     (decode: [B, H, Dk])
+ *        v, o      [B, T, H, Dv]     (decode: [B, H, Dv])
+ *        log_alpha [B, T, H] float   (decode: [B, H])   log of the gate, <= 0
+ *        beta      [B, T, H] float   (decode: [B, H])   write strength
+ *        S0, S_T, S [B, H, Dv, Dk] float  -- row i of a head's state is value
+ *                                   channel i, contiguous over the key channels.
+ *  - q, k, v and o share one element type (`dtype`); the gates and the state
+ *    are always float32.  Arithmetic is float32 (tensor-core products take
+ *    bf16 operands with float32 accumulation on the bf16 path).
+ *  - Every pointer must be 16-byte aligned.
+ *  - Errors are reported before anything is launched: GDN_ERR_INVALID_ARG for a
+ *    NULL required pointer, a negative size, a misaligned pointer or a short
+ *    workspace; GDN_ERR_UNSUPPORTED for sizes outside the limits below;
+ *    GDN_ERR_CUDA if a launch fails (the CUDA error is left for the caller to
+ *    read with cudaGetLastError / cudaPeekAtLastError).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,
+    GDN_ERR_UNSUPPORTED = 2,
+    GDN_ERR_CUDA = 3
+} gdn_status_t;
+
+typedef enum {
+    GDN_F32 = 0,   /* q, k, v, o are float32 */
+    GDN_BF16 = 1   /* q, k, v, o are bfloat16 */
+} gdn_dtype_t;
+
+/* Which kernels a chunkwise forward call with these sizes runs. */
+typedef enum {
+    GDN_PATH_NONE = 0,     /* empty problem: nothing (or only a state copy) runs */
+    GDN_PATH_SIMT = 1,     /* two CUDA-core kernels: chunk preparation, then the
+                              sequential state/output pass; needs a workspace */
+    GDN_PATH_TCGEN05 = 2   /* one fused tcgen05 tensor-core kernel, no workspace */
+} gdn_path_t;
+
+/* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0
+ * (a zero size is an empty problem and is not an error). */
+
+/*
+ * Chunkwise forward over a whole sequence (training / prefill form).
+ *
+ * Each sequence is cut into chunks of `chunk` tokens (the last one may be
+ * shorter).  Inside a chunk, with g_r the running sum of log_alpha from the
+ * chunk start and Gamma_ri = exp(g_r - g_i) for i <= r:
+ *   A    = strictly-lower( diag(beta) (Gamma o K K^T) )        gated Gram matrix
+ *   T    = (I + A)^-1                                          UT transform
+ *   U    = T diag(beta) ( V - diag(exp g) K S^T )              corrected values
+ *   O    = diag(exp g) Q S^T + (Q K^T o Gamma o causal) U     chunk output
+ *   S   <- exp(g_n) S + U^T diag(exp(g_n - g)) K               next chunk's state
+ * which reproduces the token recurrence exactly up to rounding.
+ *
+ *   q, k, v, log_alpha, beta : inputs, layouts above (required).
+ *   S0  : initial state per head, or NULL for zeros.  May equal S_T.
+ *   o   : output [B,T,H,Dv] in `dtype` (required; must not overlap an input).
+ *   S_T : final state per head, or NULL if not wanted.
+ *   workspace / workspace_bytes : device scratch of at least
+ *         gdn_chunk_fwd_workspace_size(...) bytes (NULL/0 when that is 0).
+ */
+gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *S0, void *o, float *S_T,
+                           int B, int T, int H, int Dk, int Dv, int chunk,
+                           gdn_dtype_t dtype, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace gdn_chunk_fwd needs for these sizes (0 for the
+ * fused tensor-core path and for empty problems). */
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv,
+                                    int chunk, gdn_dtype_t dtype);
+
+/* The path gdn_chunk_fwd takes for these sizes (a gdn_path_t), or -1 if the
+ * sizes are invalid or unsupported. */
+int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk,
+                       gdn_dtype_t dtype);
+
+/*
+ * One recurrent (decoding) step for every (b, h): the state is read, updated
+ * and written back in place, constant memory per head ("Gated DeltaNet-2:
+ * Decoupling Erase and Write in Linear Attention", abstract: decoding with
+ * constant memory; the rule itself from the "Approach" section cited above):
+ *   u = beta (v - alpha S k);   S <- alpha S + u k^T;   o = S q.
+ *
+ *   q, k [B,H,Dk]; v [B,H,Dv]; log_alpha, beta [B,H]; S [B,H,Dv,Dk] float32
+ *   (in place); o [B,H,Dv] in `dtype`.  All required.
+ */
+gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             float *S, void *o, int B, int H, int Dk, int Dv,
+                             gdn_dtype_t dtype, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdn_status_string(gdn_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

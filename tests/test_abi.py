@@ -1,0 +1,109 @@
+"""The C-ABI library loads without a GPU, exports every function include/gdn.h
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_130_b200 import binding
+    return binding.LIB
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ["gdn_chunk_fwd", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd_path",
+              "gdn_decode_step", "gdn_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from gated_delta_rule_130_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gdn_[a-z0-9_]+)", out))
+    for n in _declared_functions():
+        assert n in exported, f"{n} declared in gdn.h but not exported"
+        assert hasattr(lib, n)
+
+
+def test_status_strings(lib):
+    assert lib.gdn_status_string(0) == b"ok"
+    assert lib.gdn_status_string(1) == b"invalid argument"
+    assert lib.gdn_status_string(2) == b"unsupported size or type"
+    assert lib.gdn_status_string(3) == b"CUDA launch failed"
+
+
+def test_path_selection_and_workspace(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    assert b.chunk_fwd_path(1, 64, 2, 16, 16, 16, torch.float32) == "simt"
+    assert b.chunk_fwd_path(0, 64, 2, 16, 16, 16, torch.float32) == "none"
+    assert b.chunk_fwd_path(1, 0, 2, 16, 16, 16, torch.float32) == "none"
+    with pytest.raises(b.GdnError):
+        b.chunk_fwd_path(1, 64, 2, 16, 16, 48, torch.float32)
+    # the CUDA-core path stores T, P' (C x C each) and g (C) per chunk
+    C, NT = 16, 4
+    assert b.chunk_fwd_workspace_size(1, 64, 2, 16, 16, C, torch.float32) == \
+        2 * NT * (2 * C * C + C) * 4
+    assert b.chunk_fwd_workspace_size(1, 0, 2, 16, 16, C, torch.float32) == 0
+
+
+def _chunk(lib, **kw):
+    a = dict(q=16, k=16, v=16, la=16, beta=16, S0=None, o=4096, S_T=None, B=1, T=8, H=1, Dk=16,
+             Dv=16, chunk=16, dtype=0, ws=16, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return lib.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["o"],
+                             a["S_T"], a["B"], a["T"], a["H"], a["Dk"], a["Dv"], a["chunk"],
+                             a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(la=None), 1),
+    (dict(B=-1), 1), (dict(T=-3), 1), (dict(Dk=0), 1), (dict(Dv=-1), 1), (dict(dtype=7), 1),
+    (dict(chunk=48), 2), (dict(chunk=128), 2), (dict(Dk=272), 2), (dict(Dv=528), 2),
+    (dict(q=24), 1), (dict(S_T=4100), 1),                 # misaligned pointers
+    (dict(ws=None), 1), (dict(ws_bytes=64), 1),           # short workspace
+    (dict(o=16), 1),                                      # output overlaps an input
+    (dict(B=0), 0), (dict(H=0), 0),                       # empty: nothing to do
+])
+def test_chunk_fwd_rejects_before_launch(lib, kw, status):
+    # every case returns from the host-side checks; no pointer is dereferenced
+    assert _chunk(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(S=None), 1), (dict(B=-1), 1), (dict(Dk=0), 1), (dict(Dk=300), 2),
+    (dict(dtype=5), 1), (dict(o=8), 1), (dict(o=16, S=16), 1), (dict(B=0), 0),
+])
+def test_decode_step_rejects_before_launch(lib, kw, status):
+    a = dict(q=16, k=16, v=16, la=16, beta=16, S=1 << 20, o=16, B=2, H=2, Dk=16, Dv=16, dtype=1)
+    a.update(kw)
+    assert lib.gdn_decode_step(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S"], a["o"], a["B"],
+                               a["H"], a["Dk"], a["Dv"], a["dtype"], None) == status
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """Import of the binding from a copy of the package without libgdn.so raises."""
+    import shutil
+    pkg = os.path.join(ROOT, "gated_delta_rule_130_b200")
+    dst = tmp_path / "gated_delta_rule_130_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "try:\n    import gated_delta_rule_130_b200.binding\nexcept ImportError as e:\n"
+            "    print('RAISED', e)\n") % str(tmp_path)
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, timeout=120)
+    assert "RAISED" in out.stdout and "libgdn.so not found" in out.stdout
