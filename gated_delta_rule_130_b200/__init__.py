@@ -9,7 +9,7 @@ first such use raises if ``libgdn.so`` is missing -- there is no fallback.
 
 _BINDING_NAMES = {
     "chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "chunk_fwd_path", "library_path",
-    "GdnError",
+    "GdnError", "check_device_status",
 }
 
 

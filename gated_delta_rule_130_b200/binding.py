@@ -43,6 +43,8 @@ def _load():
     lib.gdn_chunk_fwd_path.restype = I
     lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, vp]
     lib.gdn_decode_step.restype = I
+    lib.gdn_check_device_status.argtypes = []
+    lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     return lib
@@ -78,6 +80,11 @@ def _dev(t: torch.Tensor, name: str, dtype=None, device=None):
 
 def _stream_ptr(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def check_device_status():
+    """Synchronise and raise if a fused tensor-core kernel timed out since the last check."""
+    _check(int(LIB.gdn_check_device_status()), "gdn_check_device_status")
 
 
 def chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> int:

@@ -102,6 +102,13 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status_t gdn_check_device_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned int flag = 0;
+    if (gdn::read_and_clear_device_error(&flag) != cudaSuccess) return GDN_ERR_CUDA;
+    return flag ? GDN_ERR_CUDA : GDN_OK;
+}
+
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                              const float *beta, float *S, void *o, int B, int H, int Dk, int Dv,
                              gdn_dtype_t dtype, void *stream) {

@@ -26,4 +26,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
                             int H, int Dk, int Dv, cudaStream_t st);
 
+// Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
+// times out (synchronous).
+cudaError_t read_and_clear_device_error(unsigned int *flag);
+
 }  // namespace gdn

@@ -120,6 +120,15 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v,
                              float *S, void *o, int B, int H, int Dk, int Dv,
                              gdn_dtype_t dtype, void *stream);
 
+/*
+ * Synchronise the current device and report whether a fused tensor-core
+ * kernel gave up since the last check: its pipeline waits are bounded (about
+ * two seconds each); a CTA that times out stops, records a flag and leaves its
+ * outputs incomplete.  Returns GDN_ERR_CUDA if the flag was set (and clears
+ * it) or if synchronising failed, GDN_OK otherwise.
+ */
+gdn_status_t gdn_check_device_status(void);
+
 /* Static, human-readable name of a status code. */
 const char *gdn_status_string(gdn_status_t status);
 
