@@ -56,6 +56,42 @@ namespace gdn {
 // Set by a fused-kernel CTA that gave up waiting (read with gdn_check_device_status).
 __device__ unsigned int g_tc_error = 0;
 
+// Optional per-role timeline of CTA (0,0,0) for performance work: build with
+// -DGDN_TRACE and read with gdn_trace_read().  Compiled out otherwise.
+#ifdef GDN_TRACE
+__device__ unsigned long long g_trace[64 * 32];
+__device__ unsigned long long g_tracew[16 * 32 * 20];
+#define GDN_TRACE_AT(c, ev)                                                            \
+    do {                                                                               \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (c) < 64)        \
+            g_trace[(c) * 32 + (ev)] = clock64();                                      \
+    } while (0)
+// warp-collective variants (every lane calls them; lane 0 records, then the
+// warp reconverges so that no later barrier sees a diverged warp)
+#define GDN_TRACE_W(c, ev)                                                             \
+    do {                                                                               \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (c) < 16 &&      \
+            (threadIdx.x & 31) == 0)                                                   \
+            g_tracew[((c) * 32 + (ev)) * 20 + (threadIdx.x >> 5)] = clock64();         \
+        __syncwarp();                                                                  \
+    } while (0)
+#define GDN_TRACE_WARP(c, ev, w)                                                       \
+    do {                                                                               \
+        if ((threadIdx.x >> 5) == (w) && (threadIdx.x & 31) == 0) GDN_TRACE_AT(c, ev); \
+        __syncwarp();                                                                  \
+    } while (0)
+#else
+#define GDN_TRACE_W(c, ev) \
+    do {                   \
+    } while (0)
+#define GDN_TRACE_WARP(c, ev, w) \
+    do {                         \
+    } while (0)
+#define GDN_TRACE_AT(c, ev) \
+    do {                    \
+    } while (0)
+#endif
+
 namespace tc {
 
 using namespace sm100;
@@ -69,7 +105,18 @@ constexpr int BLK = 8192;      // one 64 x 64 bf16 tile (64 rows of 128 bytes)
 constexpr int GRP = 3 * BLK;   // K | Q | W of one key block
 constexpr int STAGE = KB * GRP + BLK;
 constexpr int OFF_K = 0, OFF_Q = BLK, OFF_W = 2 * BLK, OFF_V = KB * GRP;
-constexpr int LDA = 65;        // padded float32 row stride of the solve buffers
+constexpr int LDA = 72;        // padded float32 row stride of A and T (16-B rows)
+constexpr int LDN = 20;        // padded row stride of the 16 x 16 N blocks
+
+// Per-stage gate vectors (float offsets), written by the TMA warp:
+constexpr int GV_G2 = 0;       // g_r log2(e), g_r = sum of log alpha over rows <= r
+constexpr int GV_BETA = 64;    // beta_r
+constexpr int GV_GAM = 128;    // gamma_r = exp(g_r)
+constexpr int GV_DCY = 192;    // exp(g_last - g_r)
+constexpr int GV_U = 256;      // exp(g_r - g_{16 R(r)})            (R(r) = r / 16)
+constexpr int GV_W = 320;      // [R][i]: exp(g_{16R} - g_i) for i < 16R, else 0
+constexpr int GV_GL = 576;     // gamma_last = exp(g_last)
+constexpr int GV_STRIDE = 640;
 
 // shared-memory map (bytes from the 1024-aligned base)
 constexpr int SM_STAGE = 0;
@@ -80,42 +127,47 @@ constexpr int SM_PT = SM_UP + BLK;             // P tiles for even / odd chunks
 constexpr int SM_TT = SM_PT + 2 * BLK;         // [T'; T''] 128 rows (K-major A)
 constexpr int SM_AF = SM_TT + 2 * BLK;         // A, float32 64 x LDA
 constexpr int SM_TF = SM_AF + 64 * LDA * 4;    // T, float32 64 x LDA
-constexpr int SM_XS = SM_TF + 64 * LDA * 4;    // solve scratch, 3 x 16 x 16 float32
-constexpr int SM_GATE = SM_XS + 3 * 256 * 4;   // 2 x {gamma[64], decay[64], gamma_last}
-constexpr int GATE_STRIDE = 256;               // floats per parity
-constexpr int SM_PG = SM_GATE + 2 * GATE_STRIDE * 4;  // prep-private: g2[64], beta[64], carry
-constexpr int SM_BAR = SM_PG + 160 * 4;
-constexpr int NBAR = 24;
+constexpr int SM_NF = SM_TF + 64 * LDA * 4;    // N_IJ = T_II A_IJ, six 16 x LDN float32 blocks
+constexpr int SM_GV = SM_NF + 6 * 16 * LDN * 4; // gate vectors, NSTAGE x GV_STRIDE floats
+constexpr int SM_BAR = SM_GV + NSTAGE * GV_STRIDE * 4;
+constexpr int NBAR = 20;
 constexpr int SM_MISC = SM_BAR + NBAR * 8;     // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr int SMEM_BYTES = SM_TOTAL + 1024;    // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(SM_BAR % 8 == 0, "mbarrier alignment");
 
 // TMEM columns
 constexpr uint32_t TM_ST = 0, TM_X = 64, TM_Y = 128, TM_G = 192, TM_WU = 256;
 constexpr uint32_t TM_U = TM_WU + DK;
 constexpr uint32_t TM_COLS = 512;
 
-// barrier indices
+// barrier indices (arrivals)
 enum {
-    B_IN_FULL = 0,      // [2] TMA -> consumers
-    B_IN_EMPTY = 2,     // [2] chain MMA (after the state update) -> TMA
-    B_G_FULL = 4,       // prep MMA -> prep
-    B_G_EMPTY = 5,      // prep -> prep MMA (128)
-    B_TT_FULL = 6,      // prep -> prep MMA (128)
-    B_WU_FULL = 7,      // prep MMA -> prep, state
-    B_WU_EMPTY = 8,     // prep (64) + state (64) -> prep MMA
-    B_PREP_FULL = 9,    // [2] prep -> chain MMA, state (128)
-    B_PT_EMPTY = 11,    // [2] chain MMA -> prep
-    B_GATE_EMPTY = 13,  // [2] state -> prep (128)
-    B_X_FULL = 15,      // chain MMA -> state
-    B_U_READY = 16,     // state (64) -> chain MMA
-    B_Y_FULL = 17,      // chain MMA -> state
-    B_ST_FULL = 18,     // chain MMA -> state
-    B_S_READY = 19,     // state (128) -> chain MMA
+    B_IN_FULL = 0,      // [2] TMA warp: gate vectors + tx bytes (1)
+    B_IN_EMPTY = 2,     // [2] chain MMA commit after the last use of the stage (1)
+    B_G_FULL = 4,       // prep MMA commit (1)
+    B_G_EMPTY = 5,      // prep warps (8)
+    B_TT_FULL = 6,      // prep warps (8)
+    B_WU_FULL = 7,      // prep MMA commit (1)
+    B_WU_EMPTY = 8,     // prep warps on lanes 0-63 + state warps on lanes 64-127 (8)
+    B_PREP_FULL = 9,    // [2] prep warps (8)
+    B_PT_EMPTY = 11,    // [2] chain MMA commit (1)
+    B_X_FULL = 13,      // chain MMA commit (1)
+    B_U_READY = 14,     // state warps (8)
+    B_Y_FULL = 15,      // chain MMA commit (1)
+    B_ST_FULL = 16,     // chain MMA commit (1)
+    B_S_READY = 17,     // state warps (8)
 };
 
-constexpr int NTHREADS = 352;
+// warp roles
+constexpr int NPREP = 8;                  // warps 0-7: chunk preparation
+constexpr int NSTATEW = 8;                // warps 8-15: sequential state / output
+constexpr int W_TMA = NPREP + NSTATEW;    // 16: TMA loads and gate vectors
+constexpr int W_CHAIN = W_TMA + 1;        // 17: sequential MMAs, TMEM owner
+constexpr int W_PMMA = W_TMA + 2;         // 18: chunk-local MMAs
+constexpr int NTHREADS = 32 * (W_PMMA + 1);
+constexpr int PREP_THREADS = 32 * NPREP;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -124,6 +176,7 @@ __device__ __forceinline__ uint64_t now_ns() {
     return t;
 }
 
+// 2^x (hardware approximation, relative error about 2^-22)
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -139,10 +192,31 @@ struct Ctx {
 // Bounded wait; false (and the CTA-wide abort flag set) on timeout or abort.
 __device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
     uint64_t *b = cx.bar + idx;
+#ifdef GDN_WAIT_TEST_SLEEP_NS
+    {
+        if (mbar_test_wait(b, parity)) return true;
+        const uint64_t t0 = now_ns();
+        for (uint32_t it = 1;; ++it) {
+            __nanosleep(GDN_WAIT_TEST_SLEEP_NS);
+            if (mbar_test_wait(b, parity)) return true;
+            if ((it & 63u) == 0) {
+                if (*cx.abort) return false;
+                if (now_ns() - t0 > kTimeoutNs) {
+                    *cx.abort = 1u;
+                    atomicOr(&g_tc_error, 1u);
+                    return false;
+                }
+            }
+        }
+    }
+#endif
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = now_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(b, parity)) return true;
+#ifdef GDN_WAIT_BACKOFF_NS
+        if (it > 32) __nanosleep(GDN_WAIT_BACKOFF_NS);
+#endif
         if ((it & 255u) == 0) {
             if (*cx.abort) return false;
             if (now_ns() - t0 > kTimeoutNs) {
@@ -154,11 +228,20 @@ __device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
     }
 }
 
-// The same wait made by every lane of a warp, with a warp-uniform result (so a
-// timeout never splits a warp in front of a warp-collective tcgen05 access).
+// A wait on behalf of a whole warp: lane 0 polls (so waiting warps do not
+// compete with working warps for the shared-memory pipe) and the result is
+// broadcast, warp-uniform, so a timeout never splits a warp in front of a
+// warp-collective tcgen05 access.
 __device__ __forceinline__ bool warp_wait(const Ctx &cx, int idx, uint32_t parity) {
-    const bool ok = wait_bar(cx, idx, parity);
-    return __all_sync(0xffffffffu, ok);
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(cx, idx, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// One arrival on behalf of a whole warp, after every lane's prior writes.
+__device__ __forceinline__ void warp_arrive(const Ctx &cx, int idx) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(cx.bar + idx);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -166,78 +249,149 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Store 64 floats as one 128-byte bf16 row `row` of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row_bf16(uint8_t *tile, int row, const float *v) {
+// Columns [16 piece, 16 piece + 16) of bf16 row `row` of a 128B-swizzled tile.
+__device__ __forceinline__ void store16_bf16(uint8_t *tile, int row, int piece, const float (&v)[16]) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int k = 0; k < 2; ++k) {
         uint4 q;
-        q.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
-        q.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
-        q.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
-        q.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, c * 16)) = q;
+        q.x = pack_bf16(v[8 * k + 0], v[8 * k + 1]);
+        q.y = pack_bf16(v[8 * k + 2], v[8 * k + 3]);
+        q.z = pack_bf16(v[8 * k + 4], v[8 * k + 5]);
+        q.w = pack_bf16(v[8 * k + 6], v[8 * k + 7]);
+        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, (2 * piece + k) * 16)) = q;
     }
 }
 
-// 64 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-    float *p = v;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tmem_ld16(taddr + 16 * j, *reinterpret_cast<float(*)[16]>(p + 16 * j));
+__device__ __forceinline__ void tmem_ld16w(uint32_t taddr, float (&v)[16]) {
+    tmem_ld16(taddr, v);
     tmem_wait_ld();
 }
 
-// T = (I + A)^-1 for the 64 x 64 strictly lower A in AF (float32, stride LDA),
-// written to TF (lower triangle and diagonal; the strict upper part is not
-// written).  Blocked by 16: the four diagonal blocks by forward substitution,
-// then T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ by block diagonals.  Called by the
-// 128 prep threads together (t = 0..127); uses named barrier 1.
-__device__ __forceinline__ void ut_solve(const float *AF, float *TF, float *XS, int t) {
-    if (t < 64) {
-        const int I = t >> 4, j = t & 15, o = 16 * I;
-        float x[16];
+// The UT transform T = (I + A)^-1 of the 64 x 64 strictly lower A (AF, float32,
+// stride LDA), blocked by 16 with D_I = I + A_II:
+//   T_II = D_I^-1                                   (ut_diag, forward substitution)
+//   N_IJ = T_II A_IJ,  I > J                        (ut_offdiag phase 1, all six blocks)
+//   T_IJ = -sum_{J <= K < I} N_IK T_KJ              (phases 2-4, by block diagonal)
+// TF receives the lower triangle and the diagonal; its strict upper part is not
+// written (and never read).
+
+// Column j of T_II for block I = p / 16 (p < 64).
+__device__ __forceinline__ void ut_diag(const float *__restrict__ AF, float *__restrict__ TF, int p) {
+    const int I = p >> 4, j = p & 15, o = 16 * I;
+    float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+    for (int r = 0; r < 16; ++r) {
+        float a[16];
 #pragma unroll
-            for (int i = 0; i < r; ++i) acc += AF[(o + r) * LDA + o + i] * x[i];
-            x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -acc);
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4 *>(AF + (o + r) * LDA + o + 4 * q);
+            a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
         }
+        float acc0 = 0.f, acc1 = 0.f;  // two partial sums: shorter dependency chains
 #pragma unroll
-        for (int r = 0; r < 16; ++r) TF[(o + r) * LDA + o + j] = x[r];
+        for (int i = 0; i < r; ++i) {
+            if (i & 1) acc1 = fmaf(a[i], x[i], acc1);
+            else acc0 = fmaf(a[i], x[i], acc0);
+        }
+        x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -(acc0 + acc1));
     }
-    named_barrier(1, 128);
-    const int c = t & 15, rr = t >> 4;  // column c, rows rr and rr + 8 of each block
-    for (int d = 1; d <= 3; ++d) {
-        const int nb = 4 - d;
-        for (int b = 0; b < nb; ++b) {
-            const int I = d + b, J = b;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = rr + 8 * h;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K) {
+    for (int r = 0; r < 16; ++r) TF[(o + r) * LDA + o + j] = x[r];
+}
+
+// acc (16 x 16 as two 16 x 8 mma tiles) += Ablk (16 x 16, stride lda) * Bblk
+// (16 x 16, stride ldb), TF32 tensor-core products with float32 accumulation;
+// one warp.
+__device__ __forceinline__ void mma16(float (&acc)[2][4], const float *__restrict__ A, int lda,
+                                      const float *__restrict__ B, int ldb, int g, int t) {
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc += AF[(16 * I + r) * LDA + 16 * K + m] * TF[(16 * K + m) * LDA + 16 * J + c];
-                }
-                XS[b * 256 + r * 16 + c] = acc;
-            }
+    for (int ks = 0; ks < 2; ++ks) {
+        const int k0 = 8 * ks;
+        const uint32_t a[4] = {to_tf32(A[g * lda + k0 + t]), to_tf32(A[(g + 8) * lda + k0 + t]),
+                               to_tf32(A[g * lda + k0 + t + 4]), to_tf32(A[(g + 8) * lda + k0 + t + 4])};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t bb[2] = {to_tf32(B[(k0 + t) * ldb + 8 * nt + g]),
+                                    to_tf32(B[(k0 + t + 4) * ldb + 8 * nt + g])};
+            mma_tf32_16x8x8(acc[nt], a, bb);
         }
-        named_barrier(1, 128);
-        for (int b = 0; b < nb; ++b) {
-            const int I = d + b, J = b;
+    }
+}
+
+__device__ __forceinline__ void store16x16(const float (&acc)[2][4], float *__restrict__ D, int ld,
+                                           float sign, int g, int t) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = rr + 8 * h;
-                float acc = 0.f;
+    for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2 *>(D + g * ld + 8 * nt + 2 * t) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
+        *reinterpret_cast<float2 *>(D + (g + 8) * ld + 8 * nt + 2 * t) = make_float2(sign * acc[nt][2], sign * acc[nt][3]);
+    }
+}
+
+// Off-diagonal blocks; all PREP_THREADS threads, one warp per 16 x 16 block
+// product.  NF block order: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
+__device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *__restrict__ TF,
+                                           float *__restrict__ NF, int p) {
+    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    const auto nf = [&](int blk) { return NF + blk * 16 * LDN; };
+    const auto tf = [&](int I, int J) { return TF + 16 * I * LDA + 16 * J; };
+    if (w < 6) {  // N_IJ = T_II A_IJ
+        const int I = (w == 0) ? 1 : (w < 3 ? 2 : 3);
+        const int J = (w == 0) ? 0 : (w < 3 ? w - 1 : w - 3);
+        float acc[2][4] = {};
+        mma16(acc, tf(I, I), LDA, AF + 16 * I * LDA + 16 * J, LDA, g, t);
+        store16x16(acc, nf(w), LDN, 1.f, g, t);
+    }
+    named_barrier(1, PREP_THREADS);
+    if (w < 3) {  // T_{J+1,J} = -N_{J+1,J} T_JJ
+        const int J = w;
+        float acc[2][4] = {};
+        mma16(acc, nf(J == 0 ? 0 : (J == 1 ? 2 : 5)), LDN, tf(J, J), LDA, g, t);
+        store16x16(acc, tf(J + 1, J), LDA, -1.f, g, t);
+    }
+    named_barrier(1, PREP_THREADS);
+    if (w < 2) {  // T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})
+        const int J = w;
+        float acc[2][4] = {};
+        mma16(acc, nf(J == 0 ? 1 : 4), LDN, tf(J, J), LDA, g, t);
+        mma16(acc, nf(J == 0 ? 2 : 5), LDN, tf(J + 1, J), LDA, g, t);
+        store16x16(acc, tf(J + 2, J), LDA, -1.f, g, t);
+    }
+    named_barrier(1, PREP_THREADS);
+    if (w == 0) {  // T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)
+        float acc[2][4] = {};
+        mma16(acc, nf(3), LDN, tf(0, 0), LDA, g, t);
+        mma16(acc, nf(4), LDN, tf(1, 0), LDA, g, t);
+        mma16(acc, nf(5), LDN, tf(2, 0), LDA, g, t);
+        store16x16(acc, tf(3, 0), LDA, -1.f, g, t);
+    }
+    named_barrier(1, PREP_THREADS);
+}
+
+// Gated Gram row, one 16-column piece at a time (columns i = 16 B + j): out[i] =
+// scale * Gamma(r, i) * gram[i] for i < r (kStrict) or i <= r, zero above, with
+// Gamma(r, i) = exp(g_r - g_i).  Off the row's diagonal 16-block R the decay
+// factors as u_r * w_R[i] (u_r = exp(g_r - g_{16R}), w_R[i] = exp(g_{16R} - g_i),
+// both <= 1, so nothing overflows); inside it, exp2 of the log2-domain
+// difference.
+template <bool kStrict>
+__device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float scale, float su,
+                                            const float *g2s, const float *w_all) {
+    const int R = r >> 4;
+    if (B < R) {
+        const float *w = w_all + R * 64 + 16 * B;
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc += TF[(16 * I + r) * LDA + 16 * I + m] * XS[b * 256 + m * 16 + c];
-                TF[(16 * I + r) * LDA + 16 * J + c] = -acc;
-            }
+        for (int j = 0; j < 16; ++j) v[j] *= su * w[j];
+    } else if (B == R) {
+        const float gr = g2s[r];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int i = 16 * B + j;
+            const bool keep = kStrict ? (i < r) : (i <= r);
+            v[j] = keep ? scale * ex2(gr - g2s[i]) * v[j] : 0.f;
         }
-        named_barrier(1, 128);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
     }
 }
 
@@ -253,14 +407,16 @@ struct Params {
 __global__ void __launch_bounds__(NTHREADS, 1)
 gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base, derived by pointer arithmetic so that the compiler
+    // keeps every access below in the shared address space
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
     cx.base = base;
     cx.bar = reinterpret_cast<uint64_t *>(base + SM_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + SM_MISC);
     cx.abort = reinterpret_cast<volatile uint32_t *>(base + SM_MISC + 4);
+    float *gv_all = reinterpret_cast<float *>(base + SM_GV);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -268,17 +424,22 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int T = p.T, H = p.H, NT = p.NT;
 
     if (tid == 0) {
-        const int counts[NBAR] = {1, 1, 1, 1, 1, 128, 128, 1, 128, 128, 128, 1, 1, 128, 128,
-                                  1, 64, 1, 1, 128, 1, 1, 1, 1};
+        int counts[NBAR];
+        for (int i = 0; i < NBAR; ++i) counts[i] = 1;
+        // one arrival per arriving warp
+        counts[B_G_EMPTY] = counts[B_TT_FULL] = NPREP;
+        counts[B_PREP_FULL] = counts[B_PREP_FULL + 1] = NPREP;
+        counts[B_WU_EMPTY] = NPREP / 2 + NSTATEW / 2;
+        counts[B_U_READY] = counts[B_S_READY] = NSTATEW;
         for (int i = 0; i < NBAR; ++i) mbar_init(cx.bar + i, counts[i]);
         *cx.abort = 0u;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == W_CHAIN) {
         tmem_alloc(tmem_slot, TM_COLS);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == W_TMA && lane == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
@@ -288,25 +449,76 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------- TMA
-        if (lane == 0) {
-            int armed = 0;
-            for (int c = 0; c < NT; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !wait_bar(cx, B_IN_EMPTY + s, ((c - 2) >> 1) & 1)) break;
+    if (warp == W_TMA) {
+        // ------------------------------------- TMA loads + per-chunk gate vectors
+        constexpr float LOG2E = 1.4426950408889634f;
+        int armed = 0;
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            if (c >= 2 && !warp_wait(cx, B_IN_EMPTY + s, ((c - 2) >> 1) & 1)) break;
+            // rows lane (lo) and lane + 32 (hi); zero past the end of the sequence
+            const int t0 = c * C;
+            float la[2], be[2];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = lane + 32 * hh;
+                const bool in = t0 + r < T;
+                const size_t gi = ((size_t)b * T + t0 + r) * H + h;
+                la[hh] = in ? p.log_alpha[gi] : 0.f;
+                be[hh] = in ? p.beta[gi] : 0.f;
+            }
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y0 = __shfl_up_sync(0xffffffffu, la[0], off);
+                const float y1 = __shfl_up_sync(0xffffffffu, la[1], off);
+                if (lane >= off) {
+                    la[0] += y0;
+                    la[1] += y1;
+                }
+            }
+            la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+            const float g0 = la[0] * LOG2E, g1 = la[1] * LOG2E;  // rows lane, lane + 32
+            const float glast = __shfl_sync(0xffffffffu, g1, 31);
+            const float gb0 = __shfl_sync(0xffffffffu, g0, lane & 16);   // g at the row's 16-block start
+            const float gb1 = __shfl_sync(0xffffffffu, g1, lane & 16);
+            const float g16 = __shfl_sync(0xffffffffu, g0, 16);
+            const float g32 = __shfl_sync(0xffffffffu, g1, 0);
+            const float g48 = __shfl_sync(0xffffffffu, g1, 16);
+            float *gv = gv_all + s * GV_STRIDE;
+            gv[GV_G2 + lane] = g0;
+            gv[GV_G2 + 32 + lane] = g1;
+            gv[GV_BETA + lane] = be[0];
+            gv[GV_BETA + 32 + lane] = be[1];
+            gv[GV_GAM + lane] = ex2(g0);
+            gv[GV_GAM + 32 + lane] = ex2(g1);
+            gv[GV_DCY + lane] = ex2(glast - g0);
+            gv[GV_DCY + 32 + lane] = ex2(glast - g1);
+            gv[GV_U + lane] = ex2(g0 - gb0);
+            gv[GV_U + 32 + lane] = ex2(g1 - gb1);
+            gv[GV_W + 0 * 64 + lane] = 0.f;
+            gv[GV_W + 0 * 64 + 32 + lane] = 0.f;
+            gv[GV_W + 1 * 64 + lane] = lane < 16 ? ex2(g16 - g0) : 0.f;
+            gv[GV_W + 1 * 64 + 32 + lane] = 0.f;
+            gv[GV_W + 2 * 64 + lane] = ex2(g32 - g0);
+            gv[GV_W + 2 * 64 + 32 + lane] = 0.f;
+            gv[GV_W + 3 * 64 + lane] = ex2(g48 - g0);
+            gv[GV_W + 3 * 64 + 32 + lane] = lane < 16 ? ex2(g48 - g1) : 0.f;
+            if (lane == 0) gv[GV_GL] = ex2(glast);
+            __syncwarp();
+            if (lane == 0) {
                 uint8_t *st = base + SM_STAGE + s * STAGE;
                 mbar_arrive_expect_tx(cx.bar + B_IN_FULL + s, (2 * KB + 1) * BLK);
-                const int t0 = c * C;
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_4d(st + kb * GRP + OFF_K, &tm_k, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
                     tma_load_4d(st + kb * GRP + OFF_Q, &tm_q, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
                 }
                 tma_load_4d(st + OFF_V, &tm_v, cx.bar + B_IN_FULL + s, v0, h, t0, b);
-                armed = c + 1;
             }
-            // never leave with copies in flight: wait for the last two stages
+            armed = c + 1;
+        }
+        // never leave with copies in flight: wait for the last two stages
+        if (lane == 0) {
             for (int c = armed - 2 < 0 ? 0 : armed - 2; c < armed; ++c) {
                 uint64_t *fb = cx.bar + B_IN_FULL + (c & 1);
                 const uint64_t t0 = now_ns();
@@ -314,7 +526,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
         }
-    } else if (warp == 10) {
+    } else if (warp == W_PMMA) {
         // ------------------------------------------- MMA: chunk-local products
         if (lane == 0) {
             const uint32_t idesc_g = idesc_bf16(128, 64, false, false);
@@ -323,7 +535,9 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int s = c & 1;
                 const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
                 if (!wait_bar(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
+                GDN_TRACE_AT(c, 10);
                 if (c >= 1 && !wait_bar(cx, B_G_EMPTY, (c - 1) & 1)) break;
+                GDN_TRACE_AT(c, 11);
                 tc_fence_after();
                 // G = [K;Q] K^T : A rows 0-63 = K, 64-127 = Q (K-major); B = K (K-major)
 #pragma unroll
@@ -333,6 +547,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                              desc_sw128(st + OFF_K + koff, 16, 1024), idesc_g, kk > 0);
                 }
                 mma_commit(cx.bar + B_G_FULL);
+                GDN_TRACE_AT(c, 8);
                 if (!wait_bar(cx, B_TT_FULL, c & 1)) break;
                 if (c >= 1 && !wait_bar(cx, B_WU_EMPTY, (c - 1) & 1)) break;
                 tc_fence_after();
@@ -343,9 +558,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     mma_bf16(tmem + TM_WU, desc_sw128(tt + kk * 32, 16, 1024),
                              desc_sw128(st + OFF_K + kk * 2048, GRP, 1024), idesc_wu, kk > 0);
                 mma_commit(cx.bar + B_WU_FULL);
+                GDN_TRACE_AT(c, 9);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == W_CHAIN) {
         // ---------------------------------------------- MMA: sequential chain
         if (lane == 0) {
             const uint32_t idesc_x = idesc_bf16(128, DVT, false, true);
@@ -368,233 +584,306 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                              desc_sw128(sb + kk * 2048, 16, 1024), idesc_x, kk > 0);
                 }
                 mma_commit(cx.bar + B_X_FULL);
+                GDN_TRACE_AT(c, 12);
                 if (!wait_bar(cx, B_U_READY, c & 1)) break;
+                GDN_TRACE_AT(c, 13);
                 tc_fence_after();
-                // Y = [P; *] U'  (rows 64-127 of the A tile are not used)
-                const uint32_t pt = smem_u32(base + SM_PT + s * BLK);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    mma_bf16(tmem + TM_Y, desc_sw128(pt + kk * 32, 16, 1024),
-                             desc_sw128(un + kk * 2048, 16, 1024), idesc_y, kk > 0);
-                mma_commit(cx.bar + B_Y_FULL);
-                mma_commit(cx.bar + B_PT_EMPTY + s);
-                // S^T += K^T (decay U') : A = K^T (MN-major, key blocks GRP apart)
+                // S^T += K^T (decay U') : A = K^T (MN-major, key blocks GRP apart).
+                // Issued first: the next chunk waits on it.
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + TM_ST, desc_sw128(st + OFF_K + kk * 2048, GRP, 1024),
                              desc_sw128(up + kk * 2048, 16, 1024), idesc_s, 1u);
                 mma_commit(cx.bar + B_ST_FULL);
+                // Y += [P; *] U'  (Y holds diag(gamma) Q S^T; rows 64-127 of A unused)
+                const uint32_t pt = smem_u32(base + SM_PT + s * BLK);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + TM_Y, desc_sw128(pt + kk * 32, 16, 1024),
+                             desc_sw128(un + kk * 2048, 16, 1024), idesc_y, 1u);
+                mma_commit(cx.bar + B_Y_FULL);
+                mma_commit(cx.bar + B_PT_EMPTY + s);
                 mma_commit(cx.bar + B_IN_EMPTY + s);
             }
         }
-    } else if (warp < 4) {
+    } else if (warp < NPREP) {
         // ------------------------------------------------------------- PREP
-        const int t = tid;  // TMEM lane t
+        // 8 warps; warp w reads TMEM lanes 32 (w % 4) .. + 31 and, with its twin
+        // w ^ 4, splits those lanes' columns in half (hf = w / 4).  Lanes 0-63
+        // carry the rows of K K^T (-> A), lanes 64-127 the rows of Q K^T (-> P).
+        const int pt = tid;                         // 0..255
+        const int q = warp & 3, hf = warp >> 2;
+        const int lrow = 32 * q + lane;             // TMEM lane of this thread
+        const bool is_a = q < 2;
         float *AF = reinterpret_cast<float *>(base + SM_AF);
         float *TF = reinterpret_cast<float *>(base + SM_TF);
-        float *XS = reinterpret_cast<float *>(base + SM_XS);
-        float *g2 = reinterpret_cast<float *>(base + SM_PG);        // g * log2(e)
-        float *bt = g2 + 64;                                          // beta
-        float *carry = bt + 64;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        constexpr float LOG2E = 1.4426950408889634f;
+        float *NF = reinterpret_cast<float *>(base + SM_NF);
+        const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+        // After the WY product: W rows (TMEM lanes 0-63) of chunk cc to its stage's
+        // W slots (twin warps take one key block each), then release the WU
+        // accumulator and publish the chunk.
+        const auto finish_chunk = [&](int cc) -> bool {
+            const int sc = cc & 1;
+            bool fine = warp_wait(cx, B_WU_FULL, cc & 1);
+            GDN_TRACE_WARP(cc, 5, 0);
+            tc_fence_after();
+            if (is_a) {
+                const int kb = hf;
+                float w0[16], w1[16], w2[16], w3[16];
+                tmem_ld16(lane_addr + TM_WU + 64 * kb, w0);
+                tmem_ld16(lane_addr + TM_WU + 64 * kb + 16, w1);
+                tmem_ld16(lane_addr + TM_WU + 64 * kb + 32, w2);
+                tmem_ld16(lane_addr + TM_WU + 64 * kb + 48, w3);
+                tmem_wait_ld();
+                uint8_t *wt = base + SM_STAGE + sc * STAGE + kb * GRP + OFF_W;
+                store16_bf16(wt, lrow, 0, w0);
+                store16_bf16(wt, lrow, 1, w1);
+                store16_bf16(wt, lrow, 2, w2);
+                store16_bf16(wt, lrow, 3, w3);
+                fence_async_smem();
+                tc_fence_before();
+                warp_arrive(cx, B_WU_EMPTY);
+            }
+            warp_arrive(cx, B_PREP_FULL + sc);
+            GDN_TRACE_WARP(cc, 6, 0);
+            return fine;
+        };
+        bool ok = true;  // false once a wait has failed; the CTA is then aborting
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
-            const int t0 = c * C;
-            uint8_t *st = base + SM_STAGE + s * STAGE;
-            float *gate = reinterpret_cast<float *>(base + SM_GATE) + s * GATE_STRIDE;
-            bool ok = true;  // false once a wait has failed; the CTA is then aborting
-            if (c >= 2) ok &= warp_wait(cx, B_GATE_EMPTY + s, ((c - 2) >> 1) & 1);
-            // gates: running sum of log alpha within the chunk (rows 0..63)
-            if (t < 64) {
-                const bool in = t0 + t < T;
-                const size_t gi = ((size_t)b * T + t0 + t) * H + h;
-                float la = in ? p.log_alpha[gi] : 0.f;
-                const float be = in ? p.beta[gi] : 0.f;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, la, off);
-                    if (lane >= off) la += y;
-                }
-                if (t == 31) carry[0] = la;
-                bt[t] = be;
-                g2[t] = la;  // within-warp prefix; rows 32..63 get the carry below
-            }
-            named_barrier(1, 128);
-            if (t < 64) {
-                const float g = g2[t] + (t >= 32 ? carry[0] : 0.f);
-                named_barrier(2, 64);
-                g2[t] = g * LOG2E;
-                named_barrier(2, 64);
-                const float glast = g2[63];
-                gate[t] = ex2(g2[t]);                  // gamma_r
-                gate[64 + t] = ex2(glast - g2[t]);     // exp(g_last - g_r)
-                if (t == 0) gate[128] = ex2(glast);    // gamma_last
-            }
-            named_barrier(1, 128);
-            // Gram matrix -> A (rows of K K^T, lanes 0-63) and P (rows of Q K^T, lanes 64-127)
+            const float *gv = gv_all + s * GV_STRIDE;
+            ok &= warp_wait(cx, B_IN_FULL + s, (c >> 1) & 1);
+            GDN_TRACE_WARP(c, 0, 0);
             ok &= warp_wait(cx, B_G_FULL, c & 1);
+            GDN_TRACE_WARP(c, 1, 0);
             tc_fence_after();
             {
-                float gv[64];
-                tmem_ld64(lane_addr + TM_G, gv);
+                const int r = lrow & 63;
+                if (!is_a && c >= 2) ok &= warp_wait(cx, B_PT_EMPTY + s, ((c - 2) >> 1) & 1);
+                const float scale = is_a ? gv[GV_BETA + r] : 1.f;
+                const float su = scale * gv[GV_U + r];
+                float v0[16], v1[16];
+                tmem_ld16(lane_addr + TM_G + 32 * hf, v0);
+                tmem_ld16(lane_addr + TM_G + 32 * hf + 16, v1);
+                tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(cx.bar + B_G_EMPTY);
-                if (t < 64) {
-                    const int r = t;
-                    const float gr = g2[r], br = bt[r];
+                warp_arrive(cx, B_G_EMPTY);
+                if (is_a) {
+                    gated_piece<true>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
+                    gated_piece<true>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        AF[r * LDA + i] = (i < r) ? br * ex2(gr - g2[i]) * gv[i] : 0.f;
+                    for (int k = 0; k < 4; ++k) {
+                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hf + 4 * k) =
+                            make_float4(v0[4 * k], v0[4 * k + 1], v0[4 * k + 2], v0[4 * k + 3]);
+                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hf + 16 + 4 * k) =
+                            make_float4(v1[4 * k], v1[4 * k + 1], v1[4 * k + 2], v1[4 * k + 3]);
+                    }
+                    // A complete (the four A warps) -> diagonal blocks of T
+                    named_barrier(3, PREP_THREADS / 2);
+                    if (pt < 64) ut_diag(AF, TF, pt);
                 } else {
-                    const int r = t - 64;
-                    if (c >= 2) ok &= warp_wait(cx, B_PT_EMPTY + s, ((c - 2) >> 1) & 1);
-                    const float gr = g2[r];
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) gv[i] = (i <= r) ? ex2(gr - g2[i]) * gv[i] : 0.f;
-                    store_row_bf16(base + SM_PT + s * BLK, r, gv);
+                    gated_piece<false>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
+                    gated_piece<false>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
+                    store16_bf16(base + SM_PT + s * BLK, r, 2 * hf, v0);
+                    store16_bf16(base + SM_PT + s * BLK, r, 2 * hf + 1, v1);
                     fence_async_smem();
                 }
             }
-            named_barrier(1, 128);
-            ut_solve(AF, TF, XS, t);
-            // [T'; T''] : row t, T'(r,i) = T(r,i) beta_i gamma_i, T''(r,i) = T(r,i) beta_i
+            named_barrier(1, PREP_THREADS);
+            GDN_TRACE_WARP(c, 2, 0);
+            ut_offdiag(AF, TF, NF, pt);
+            GDN_TRACE_WARP(c, 3, 0);
+            // [T'; T''] : row rt, T'(r,i) = T(r,i) beta_i gamma_i, T''(r,i) = T(r,i) beta_i
             {
-                const int r = t & 63;
-                float row[64];
+                const int rt = pt & 127, r = rt & 63;
+                const bool wgam = rt < 64;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float sc = bt[i] * ((t < 64) ? gate[i] : 1.f);
-                    row[i] = (i <= r) ? TF[r * LDA + i] * sc : 0.f;
-                }
-                store_row_bf16(base + SM_TT, t, row);
-                fence_async_smem();
-                mbar_arrive(cx.bar + B_TT_FULL);
-            }
-            // W rows (lanes 0-63) to the stage's W slots
-            ok &= warp_wait(cx, B_WU_FULL, c & 1);
-            tc_fence_after();
-            if (t < 64) {
+                for (int k = 0; k < 2; ++k) {
+                    const int B = 2 * (pt >> 7) + k;
+                    float v[16];
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    float w[64];
-                    tmem_ld64(lane_addr + TM_WU + 64 * kb, w);
-                    store_row_bf16(st + kb * GRP + OFF_W, t, w);
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int i = 16 * B + 4 * qq;
+                        const float4 tv = *reinterpret_cast<const float4 *>(TF + r * LDA + i);
+                        const float4 bv = *reinterpret_cast<const float4 *>(gv + GV_BETA + i);
+                        float4 gv4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                        if (wgam) gv4 = *reinterpret_cast<const float4 *>(gv + GV_GAM + i);
+                        v[4 * qq + 0] = (i + 0 <= r) ? tv.x * bv.x * gv4.x : 0.f;
+                        v[4 * qq + 1] = (i + 1 <= r) ? tv.y * bv.y * gv4.y : 0.f;
+                        v[4 * qq + 2] = (i + 2 <= r) ? tv.z * bv.z * gv4.z : 0.f;
+                        v[4 * qq + 3] = (i + 3 <= r) ? tv.w * bv.w * gv4.w : 0.f;
+                    }
+                    store16_bf16(base + SM_TT, rt, B, v);
                 }
                 fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(cx.bar + B_WU_EMPTY);
+                warp_arrive(cx, B_TT_FULL);
             }
-            mbar_arrive(cx.bar + B_PREP_FULL + s);
+            GDN_TRACE_WARP(c, 4, 0);
+            ok &= finish_chunk(c);
             // leave together: every prep thread sees the same decision
-            if (named_barrier_or(1, 128, !ok || *cx.abort)) break;
+            if (named_barrier_or(1, PREP_THREADS, !ok || *cx.abort)) break;
         }
     } else {
         // ------------------------------------------------------------ STATE
-        const int t = tid - 128;  // TMEM lane t: key channel t of S^T; chunk row for X/Y
-        const int q = warp & 3;
+        // 8 warps; warp w reads TMEM lanes 32 (w % 4) .. + 31 (a key channel of
+        // S^T, or a chunk row of X / Y) and handles half of that lane's 64
+        // columns (hf), its twin the other half.
+        const int q = warp & 3, hf = (warp - NPREP) >> 2;
+        const int lrow = 32 * q + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
-        uint8_t *sb = base + SM_SB;
+        uint8_t *sbuf = base + SM_SB;
         const size_t head = (size_t)b * H + h;
-        // initial state: S^T row t = S0[v0 .. v0+63][t]
+        // initial state: S^T row lrow = S0[v0 .. v0+63][lrow]; TMEM copy pre-scaled by gamma_last
         {
-            float sv[64];
+            const bool have = warp_wait(cx, B_IN_FULL + 0, 0);
+            const float gl = gv_all[GV_GL];
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + j) * DK + t] : 0.f;
-            store_row_bf16(sb, t, sv);
-            fence_async_smem();
-            if (warp_wait(cx, B_PREP_FULL + 0, 0)) {
-                const float gl = reinterpret_cast<const float *>(base + SM_GATE)[128];
+            for (int k = 0; k < 2; ++k) {
+                const int B = 2 * hf + k;
+                float sv[16];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) sv[j] *= gl;
+                for (int j = 0; j < 16; ++j)
+                    sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + 16 * B + j) * DK + lrow] : 0.f;
+                store16_bf16(sbuf, lrow, B, sv);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tmem_st16(lane_addr + TM_ST + 16 * j, *reinterpret_cast<float(*)[16]>(sv + 16 * j));
-                tmem_wait_st();
+                for (int j = 0; j < 16; ++j) sv[j] *= gl;
+                if (have) tmem_st16(lane_addr + TM_ST + 16 * B, sv);
             }
+            fence_async_smem();
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(cx.bar + B_S_READY);
+            warp_arrive(cx, B_S_READY);
         }
         for (int c = 0; c < NT; ++c) {
             if (__any_sync(0xffffffffu, *cx.abort != 0u)) break;
             const int s = c & 1;
             const int t0 = c * C;
-            const float *gate = reinterpret_cast<const float *>(base + SM_GATE) + s * GATE_STRIDE;
-            float oq[64];
+            const float *gv = gv_all + s * GV_STRIDE;
             if (!warp_wait(cx, B_X_FULL, c & 1)) break;
+            GDN_TRACE_WARP(c, 16, NPREP);
             tc_fence_after();
-            if (t >= 64) {
-                // U' = U - W S^T for chunk row r
-                const int r = t - 64;
-                float x[64], u[64];
-                tmem_ld64(lane_addr + TM_X, x);
-                tmem_ld64(lane_addr + TM_U, u);
+            if (q >= 2) {
+                // U' = U - W S^T for chunk row r -> U' and diag(exp(g_last - g)) U' (bf16)
+                const int r = lrow - 64;
+                const float dc = gv[GV_DCY + r];
+                float x0[16], x1[16], u0[16], u1[16];
+                tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
+                tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
+                tmem_ld16(lane_addr + TM_U + 32 * hf, u0);
+                tmem_ld16(lane_addr + TM_U + 32 * hf + 16, u1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; ++j) u[j] -= x[j];
-                store_row_bf16(base + SM_UN, r, u);
-                const float dc = gate[64 + r];
+                for (int j = 0; j < 16; ++j) {
+                    u0[j] -= x0[j];
+                    u1[j] -= x1[j];
+                }
+                store16_bf16(base + SM_UN, r, 2 * hf, u0);
+                store16_bf16(base + SM_UN, r, 2 * hf + 1, u1);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) u[j] *= dc;
-                store_row_bf16(base + SM_UP, r, u);
+                for (int j = 0; j < 16; ++j) {
+                    u0[j] *= dc;
+                    u1[j] *= dc;
+                }
+                store16_bf16(base + SM_UP, r, 2 * hf, u0);
+                store16_bf16(base + SM_UP, r, 2 * hf + 1, u1);
                 fence_async_smem();
                 tc_fence_before();
-                mbar_arrive(cx.bar + B_U_READY);
-                mbar_arrive(cx.bar + B_WU_EMPTY);
+                warp_arrive(cx, B_U_READY);
+                warp_arrive(cx, B_WU_EMPTY);
+                GDN_TRACE_WARP(c, 18, NPREP + 2);
             } else {
-                // inter-chunk part of the output for chunk row t: gamma_t (Q S^T)_t
-                tmem_ld64(lane_addr + TM_X, oq);
-                const float gr = gate[t];
+                // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y; the
+                // intra-chunk MMA accumulates onto it
+                const float gr = gv[GV_GAM + lrow];
+                float x0[16], x1[16];
+                tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
+                tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; ++j) oq[j] *= gr;
-                if (!warp_wait(cx, B_Y_FULL, c & 1)) break;
-                tc_fence_after();
-                float y[64];
-                tmem_ld64(lane_addr + TM_Y, y);
-                if (t0 + t < T) {
-                    __nv_bfloat16 *dst = p.o + (((size_t)b * T + t0 + t) * H + h) * p.Dv + v0;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint4 qv;
-                        qv.x = pack_bf16(oq[8 * cc + 0] + y[8 * cc + 0], oq[8 * cc + 1] + y[8 * cc + 1]);
-                        qv.y = pack_bf16(oq[8 * cc + 2] + y[8 * cc + 2], oq[8 * cc + 3] + y[8 * cc + 3]);
-                        qv.z = pack_bf16(oq[8 * cc + 4] + y[8 * cc + 4], oq[8 * cc + 5] + y[8 * cc + 5]);
-                        qv.w = pack_bf16(oq[8 * cc + 6] + y[8 * cc + 6], oq[8 * cc + 7] + y[8 * cc + 7]);
-                        reinterpret_cast<uint4 *>(dst)[cc] = qv;
-                    }
+                for (int j = 0; j < 16; ++j) {
+                    x0[j] *= gr;
+                    x1[j] *= gr;
                 }
+                tmem_st16(lane_addr + TM_Y + 32 * hf, x0);
+                tmem_st16(lane_addr + TM_Y + 32 * hf + 16, x1);
+                tmem_wait_st();
+                tc_fence_before();
+                warp_arrive(cx, B_U_READY);
             }
-            // state hand-off: S^T (already gamma-scaled + update) -> bf16 copy, pre-scale
+            // state hand-off: S^T (gamma-scaled + update) -> bf16 copy; TMEM pre-scaled
             if (!warp_wait(cx, B_ST_FULL, c & 1)) break;
+            GDN_TRACE_WARP(c, 20, NPREP);
             tc_fence_after();
             {
-                float sv[64];
-                tmem_ld64(lane_addr + TM_ST, sv);
-                if (c + 1 < NT) {
-                    store_row_bf16(sb, t, sv);
+                const bool last = c + 1 >= NT;
+                bool have = false;
+                float gl = 1.f;
+                if (!last) {
+                    have = warp_wait(cx, B_IN_FULL + (s ^ 1), ((c + 1) >> 1) & 1);
+                    gl = gv_all[(s ^ 1) * GV_STRIDE + GV_GL];
+                }
+                float s0[16], s1[16];
+                tmem_ld16(lane_addr + TM_ST + 32 * hf, s0);
+                tmem_ld16(lane_addr + TM_ST + 32 * hf + 16, s1);
+                tmem_wait_ld();
+                if (!last) {
+                    store16_bf16(sbuf, lrow, 2 * hf, s0);
+                    store16_bf16(sbuf, lrow, 2 * hf + 1, s1);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        s0[j] *= gl;
+                        s1[j] *= gl;
+                    }
+                    if (have) {
+                        tmem_st16(lane_addr + TM_ST + 32 * hf, s0);
+                        tmem_st16(lane_addr + TM_ST + 32 * hf + 16, s1);
+                    }
                     fence_async_smem();
-                    if (!warp_wait(cx, B_PREP_FULL + (s ^ 1), ((c + 1) >> 1) & 1)) break;
-                    const float gl = reinterpret_cast<const float *>(base + SM_GATE)[(s ^ 1) * GATE_STRIDE + 128];
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) sv[j] *= gl;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tmem_st16(lane_addr + TM_ST + 16 * j, *reinterpret_cast<float(*)[16]>(sv + 16 * j));
                     tmem_wait_st();
                 } else if (p.S_T) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) p.S_T[(head * p.Dv + v0 + j) * DK + t] = sv[j];
+                    for (int j = 0; j < 16; ++j) {
+                        p.S_T[(head * p.Dv + v0 + 32 * hf + j) * DK + lrow] = s0[j];
+                        p.S_T[(head * p.Dv + v0 + 32 * hf + 16 + j) * DK + lrow] = s1[j];
+                    }
                 }
                 tc_fence_before();
-                mbar_arrive(cx.bar + B_S_READY);
-                mbar_arrive(cx.bar + B_GATE_EMPTY + s);
+                warp_arrive(cx, B_S_READY);
+                GDN_TRACE_WARP(c, 21, NPREP);
+                if (!last && !have) break;
+            }
+            // chunk output rows (lanes 0-63)
+            if (q < 2) {
+                if (!warp_wait(cx, B_Y_FULL, c & 1)) break;
+                GDN_TRACE_WARP(c, 19, NPREP);
+                tc_fence_after();
+                float y0[16], y1[16];
+                tmem_ld16(lane_addr + TM_Y + 32 * hf, y0);
+                tmem_ld16(lane_addr + TM_Y + 32 * hf + 16, y1);
+                tmem_wait_ld();
+                if (t0 + lrow < T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        p.o + (((size_t)b * T + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        dst[k] = make_uint4(pack_bf16(y0[8 * k + 0], y0[8 * k + 1]),
+                                            pack_bf16(y0[8 * k + 2], y0[8 * k + 3]),
+                                            pack_bf16(y0[8 * k + 4], y0[8 * k + 5]),
+                                            pack_bf16(y0[8 * k + 6], y0[8 * k + 7]));
+                        dst[2 + k] = make_uint4(pack_bf16(y1[8 * k + 0], y1[8 * k + 1]),
+                                                pack_bf16(y1[8 * k + 2], y1[8 * k + 3]),
+                                                pack_bf16(y1[8 * k + 4], y1[8 * k + 5]),
+                                                pack_bf16(y1[8 * k + 6], y1[8 * k + 7]));
+                    }
+                }
+                tc_fence_before();
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == W_CHAIN) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
@@ -662,6 +951,15 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
         mq, mk, mv, p);
     return cudaPeekAtLastError();
 }
+
+#ifdef GDN_TRACE
+extern "C" int gdn_trace_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_trace, sizeof(g_trace));
+}
+extern "C" int gdn_tracew_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_tracew, sizeof(g_tracew));
+}
+#endif
 
 cudaError_t read_and_clear_device_error(unsigned int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_error, sizeof(unsigned int));
