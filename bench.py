@@ -44,6 +44,27 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def measured_traffic(path: str):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    or None if the kernel sources changed since the capture."""
+    import hashlib
+    f = os.path.join(ROOT, "profiles", "traffic_gdn_chunk_tc_kernel.txt")
+    if path != "tcgen05" or not os.path.exists(f):
+        return None
+    value, ok = None, True
+    for line in open(f):
+        line = line.strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            value = float(line.split(":", 1)[1])
+        elif line.startswith("sha256 "):
+            rel, digest = line[len("sha256 "):].split(":", 1)
+            src = os.path.join(ROOT, rel.strip())
+            if not os.path.exists(src) or \
+                    hashlib.sha256(open(src, "rb").read()).hexdigest() != digest.strip():
+                ok = False
+    return value if ok else None
+
+
 def chunk_flops(w) -> float:
     """Dense contraction FLOPs of the chunkwise algorithm, 2(3 C Dk + 2 C Dv + 3 Dk Dv)
     per token per head (the gated Gram matrix, the WY factors, the state update and
@@ -139,6 +160,14 @@ def _max_over_ranks(x: float, world: int, device) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(ms_local: float, steps: int, tokens_per_rank: int, world: int, device):
+    """Whole-job tokens/s and ms/step from this rank's device time: every rank
+    processes its own batch, the job takes as long as the slowest rank."""
+    ms_max = _max_over_ranks(ms_local, world, device)
+    ms_step = ms_max / steps
+    return world * tokens_per_rank / (ms_step * 1e-3), ms_step
 
 
 def _barrier(world):
@@ -268,10 +297,8 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         ms = time_loop(step, steps, stream, world)
     clocks = clk.summary()
-    ms_max = _max_over_ranks(ms, world, device)
-    ms_step = ms_max / steps
     tokens = w.B * w.T
-    value = world * tokens / (ms_step * 1e-3)
+    value, ms_step = weak_scaling_value(ms, steps, tokens, world, device)
 
     # roofline of the dominant kernel (the whole call: one fused kernel on the
     # tcgen05 path; the two CUDA-core kernels together on the SIMT path)
@@ -283,7 +310,7 @@ def run_ours(args):
     hbm_peak = pk["hbm_gbs"]
     tc_peak = pk["bf16_tflops"]
     roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": gbs / hbm_peak, "traffic": None,
+                "frac": gbs / hbm_peak, "traffic": measured_traffic(path),
                 "kernel": f"gdn_chunk_fwd ({path}, {launches_per_step} launch/step)",
                 "algorithmic_bytes": Bytes, "peak_source": f"{pk_kind} hbm_gbs",
                 "tc": {"achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
