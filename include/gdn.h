@@ -106,6 +106,28 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk,
                        gdn_dtype_t dtype);
 
 /*
+ * gdn_chunk_fwd without a caller workspace, for callers that cannot allocate
+ * device memory (engines that plan all buffers at start-up and forbid
+ * allocation later, paths where cudaMalloc's implicit synchronisation is not
+ * acceptable, hosts that hand the library no memory).  The pages have no
+ * counterpart: this is a property of the library, not of the method.
+ *
+ * Same arguments and results as gdn_chunk_fwd, minus the workspace.  The
+ * CUDA-core path's scratch is a fixed 8 MiB array inside the library (held on
+ * every GPU that loads it until exit); sizes whose workspace
+ * (gdn_chunk_fwd_workspace_size) exceeds 8 MiB return GDN_ERR_UNSUPPORTED with
+ * nothing launched.  The first call on a device looks up the array's address
+ * (with that device current) and must come before any stream capture.  All
+ * calls share the array: calls whose work overlaps on the GPU race and must be
+ * serialised by the caller.  Allocates nothing.
+ */
+gdn_status_t gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int Dk, int Dv, int chunk,
+                                   gdn_dtype_t dtype, void *stream);
+
+/*
  * One recurrent (decoding) step for every (b, h): the state is read, updated
  * and written back in place, constant memory per head ("Gated DeltaNet-2:
  * Decoupling Erase and Write in Linear Attention", abstract: decoding with
