@@ -165,8 +165,9 @@ constexpr int NPREP = 8;                  // warps 0-7: chunk preparation
 constexpr int NSTATEW = 8;                // warps 8-15: sequential state / output
 constexpr int W_TMA = NPREP + NSTATEW;    // 16: TMA loads and gate vectors
 constexpr int W_CHAIN = W_TMA + 1;        // 17: sequential MMAs, TMEM owner
-constexpr int W_PMMA = W_TMA + 2;         // 18: chunk-local MMAs
-constexpr int NTHREADS = 32 * (W_PMMA + 1);
+constexpr int W_PMMA = W_TMA + 2;         // 18: WY product of each chunk
+constexpr int W_GMMA = W_TMA + 3;         // 19: Gram product of each chunk
+constexpr int NTHREADS = 32 * (W_GMMA + 1);
 constexpr int PREP_THREADS = 32 * NPREP;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
@@ -330,7 +331,7 @@ __device__ __forceinline__ void store16x16(const float (&acc)[2][4], float *__re
 // Off-diagonal blocks; all PREP_THREADS threads, one warp per 16 x 16 block
 // product.  NF block order: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
 __device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *__restrict__ TF,
-                                           float *__restrict__ NF, int p) {
+                                           float *__restrict__ NF, int p, int tc_trace_chunk = 0) {
     const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
     const auto nf = [&](int blk) { return NF + blk * 16 * LDN; };
     const auto tf = [&](int I, int J) { return TF + 16 * I * LDA + 16 * J; };
@@ -342,6 +343,7 @@ __device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *
         store16x16(acc, nf(w), LDN, 1.f, g, t);
     }
     named_barrier(1, PREP_THREADS);
+    GDN_TRACE_WARP(tc_trace_chunk, 26, 0);
     if (w < 3) {  // T_{J+1,J} = -N_{J+1,J} T_JJ
         const int J = w;
         float acc[2][4] = {};
@@ -349,6 +351,7 @@ __device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *
         store16x16(acc, tf(J + 1, J), LDA, -1.f, g, t);
     }
     named_barrier(1, PREP_THREADS);
+    GDN_TRACE_WARP(tc_trace_chunk, 27, 0);
     if (w < 2) {  // T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})
         const int J = w;
         float acc[2][4] = {};
@@ -357,6 +360,7 @@ __device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *
         store16x16(acc, tf(J + 2, J), LDA, -1.f, g, t);
     }
     named_barrier(1, PREP_THREADS);
+    GDN_TRACE_WARP(tc_trace_chunk, 28, 0);
     if (w == 0) {  // T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)
         float acc[2][4] = {};
         mma16(acc, nf(3), LDN, tf(0, 0), LDA, g, t);
@@ -365,6 +369,7 @@ __device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *
         store16x16(acc, tf(3, 0), LDA, -1.f, g, t);
     }
     named_barrier(1, PREP_THREADS);
+    GDN_TRACE_WARP(tc_trace_chunk, 29, 0);
 }
 
 // Gated Gram row, one 16-column piece at a time (columns i = 16 B + j): out[i] =
@@ -428,8 +433,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int i = 0; i < NBAR; ++i) counts[i] = 1;
         // one arrival per arriving warp
         counts[B_G_EMPTY] = counts[B_TT_FULL] = NPREP;
-        counts[B_PREP_FULL] = counts[B_PREP_FULL + 1] = NPREP;
-        counts[B_WU_EMPTY] = NPREP / 2 + NSTATEW / 2;
+        counts[B_WU_EMPTY] = NSTATEW;
+        counts[B_PREP_FULL] = counts[B_PREP_FULL + 1] = NPREP / 2 + NSTATEW / 2;
         counts[B_U_READY] = counts[B_S_READY] = NSTATEW;
         for (int i = 0; i < NBAR; ++i) mbar_init(cx.bar + i, counts[i]);
         *cx.abort = 0u;
@@ -526,20 +531,16 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
         }
-    } else if (warp == W_PMMA) {
-        // ------------------------------------------- MMA: chunk-local products
+    } else if (warp == W_GMMA) {
+        // ------------------------------------------------- MMA: Gram products
         if (lane == 0) {
             const uint32_t idesc_g = idesc_bf16(128, 64, false, false);
-            const uint32_t idesc_wu = idesc_bf16(128, DK + DVT, false, true);
             for (int c = 0; c < NT; ++c) {
                 const int s = c & 1;
                 const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
                 if (!wait_bar(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
-                GDN_TRACE_AT(c, 10);
                 if (c >= 1 && !wait_bar(cx, B_G_EMPTY, (c - 1) & 1)) break;
-                GDN_TRACE_AT(c, 11);
                 tc_fence_after();
-                // G = [K;Q] K^T : A rows 0-63 = K, 64-127 = Q (K-major); B = K (K-major)
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * GRP + (kk & 3) * 32;
@@ -548,11 +549,18 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 mma_commit(cx.bar + B_G_FULL);
                 GDN_TRACE_AT(c, 8);
+            }
+        }
+    } else if (warp == W_PMMA) {
+        // --------------------------------------------------- MMA: WY products
+        if (lane == 0) {
+            const uint32_t idesc_wu = idesc_bf16(128, DK + DVT, false, true);
+            const uint32_t tt = smem_u32(base + SM_TT);
+            for (int c = 0; c < NT; ++c) {
+                const uint32_t st = smem_u32(base + SM_STAGE + (c & 1) * STAGE);
                 if (!wait_bar(cx, B_TT_FULL, c & 1)) break;
                 if (c >= 1 && !wait_bar(cx, B_WU_EMPTY, (c - 1) & 1)) break;
                 tc_fence_after();
-                // WU = [T'; T''] [K | V] : A K-major (K = 64 tokens), B MN-major
-                const uint32_t tt = smem_u32(base + SM_TT);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + TM_WU, desc_sw128(tt + kk * 32, 16, 1024),
@@ -622,32 +630,6 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // After the WY product: W rows (TMEM lanes 0-63) of chunk cc to its stage's
         // W slots (twin warps take one key block each), then release the WU
         // accumulator and publish the chunk.
-        const auto finish_chunk = [&](int cc) -> bool {
-            const int sc = cc & 1;
-            bool fine = warp_wait(cx, B_WU_FULL, cc & 1);
-            GDN_TRACE_WARP(cc, 5, 0);
-            tc_fence_after();
-            if (is_a) {
-                const int kb = hf;
-                float w0[16], w1[16], w2[16], w3[16];
-                tmem_ld16(lane_addr + TM_WU + 64 * kb, w0);
-                tmem_ld16(lane_addr + TM_WU + 64 * kb + 16, w1);
-                tmem_ld16(lane_addr + TM_WU + 64 * kb + 32, w2);
-                tmem_ld16(lane_addr + TM_WU + 64 * kb + 48, w3);
-                tmem_wait_ld();
-                uint8_t *wt = base + SM_STAGE + sc * STAGE + kb * GRP + OFF_W;
-                store16_bf16(wt, lrow, 0, w0);
-                store16_bf16(wt, lrow, 1, w1);
-                store16_bf16(wt, lrow, 2, w2);
-                store16_bf16(wt, lrow, 3, w3);
-                fence_async_smem();
-                tc_fence_before();
-                warp_arrive(cx, B_WU_EMPTY);
-            }
-            warp_arrive(cx, B_PREP_FULL + sc);
-            GDN_TRACE_WARP(cc, 6, 0);
-            return fine;
-        };
         bool ok = true;  // false once a wait has failed; the CTA is then aborting
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
@@ -668,6 +650,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_wait_ld();
                 tc_fence_before();
                 warp_arrive(cx, B_G_EMPTY);
+                GDN_TRACE_WARP(c, 22, 0);
                 if (is_a) {
                     gated_piece<true>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
                     gated_piece<true>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
@@ -678,9 +661,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hf + 16 + 4 * k) =
                             make_float4(v1[4 * k], v1[4 * k + 1], v1[4 * k + 2], v1[4 * k + 3]);
                     }
+                    GDN_TRACE_WARP(c, 23, 0);
                     // A complete (the four A warps) -> diagonal blocks of T
                     named_barrier(3, PREP_THREADS / 2);
+                    GDN_TRACE_WARP(c, 24, 0);
                     if (pt < 64) ut_diag(AF, TF, pt);
+                    GDN_TRACE_WARP(c, 25, 0);
                 } else {
                     gated_piece<false>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
                     gated_piece<false>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
@@ -691,9 +677,11 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             named_barrier(1, PREP_THREADS);
             GDN_TRACE_WARP(c, 2, 0);
-            ut_offdiag(AF, TF, NF, pt);
+            ut_offdiag(AF, TF, NF, pt, c);
             GDN_TRACE_WARP(c, 3, 0);
             // [T'; T''] : row rt, T'(r,i) = T(r,i) beta_i gamma_i, T''(r,i) = T(r,i) beta_i
+            // (the previous chunk's WY product must have read TT first)
+            if (c >= 1) ok &= warp_wait(cx, B_WU_FULL, (c - 1) & 1);
             {
                 const int rt = pt & 127, r = rt & 63;
                 const bool wgam = rt < 64;
@@ -719,7 +707,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 warp_arrive(cx, B_TT_FULL);
             }
             GDN_TRACE_WARP(c, 4, 0);
-            ok &= finish_chunk(c);
+            if (!is_a) warp_arrive(cx, B_PREP_FULL + (c & 1));
             // leave together: every prep thread sees the same decision
             if (named_barrier_or(1, PREP_THREADS, !ok || *cx.abort)) break;
         }
@@ -733,6 +721,28 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
         uint8_t *sbuf = base + SM_SB;
         const size_t head = (size_t)b * H + h;
+        const auto copy_w = [&](int cc) -> bool {
+            if (q >= 2) return true;
+            const bool fine = warp_wait(cx, B_WU_FULL, cc & 1);
+            tc_fence_after();
+            const int kb = hf;
+            float w0[16], w1[16], w2[16], w3[16];
+            tmem_ld16(lane_addr + TM_WU + 64 * kb, w0);
+            tmem_ld16(lane_addr + TM_WU + 64 * kb + 16, w1);
+            tmem_ld16(lane_addr + TM_WU + 64 * kb + 32, w2);
+            tmem_ld16(lane_addr + TM_WU + 64 * kb + 48, w3);
+            tmem_wait_ld();
+            uint8_t *wt = base + SM_STAGE + (cc & 1) * STAGE + kb * GRP + OFF_W;
+            store16_bf16(wt, lrow, 0, w0);
+            store16_bf16(wt, lrow, 1, w1);
+            store16_bf16(wt, lrow, 2, w2);
+            store16_bf16(wt, lrow, 3, w3);
+            fence_async_smem();
+            tc_fence_before();
+            warp_arrive(cx, B_WU_EMPTY);
+            warp_arrive(cx, B_PREP_FULL + (cc & 1));
+            return fine;
+        };
         // initial state: S^T row lrow = S0[v0 .. v0+63][lrow]; TMEM copy pre-scaled by gamma_last
         {
             const bool have = warp_wait(cx, B_IN_FULL + 0, 0);
@@ -754,6 +764,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             warp_arrive(cx, B_S_READY);
         }
+        if (NT > 0) copy_w(0);
         for (int c = 0; c < NT; ++c) {
             if (__any_sync(0xffffffffu, *cx.abort != 0u)) break;
             const int s = c & 1;
@@ -852,6 +863,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 GDN_TRACE_WARP(c, 21, NPREP);
                 if (!last && !have) break;
             }
+            if (c + 1 < NT) copy_w(c + 1);
             // chunk output rows (lanes 0-63)
             if (q < 2) {
                 if (!warp_wait(cx, B_Y_FULL, c & 1)) break;
