@@ -1,5 +1,5 @@
-// Fused chunkwise forward of the gated delta rule on sm_100a tensor cores
-// (tcgen05 + TMEM + TMA), bf16 q/k/v/o, float32 gates, state and accumulation.
+// Chunkwise forward of the gated delta rule on sm_100a tensor cores (tcgen05 +
+// TMEM + TMA), bf16 q/k/v/o, float32 gates, state and accumulation.
 //
 // Per chunk of C = 64 tokens (rows r), with g_r the running sum of log alpha
 // from the chunk start, gamma_r = exp(g_r), and S the state (Dv x Dk) entering
@@ -12,35 +12,41 @@
 //   U'  = U - W S^T                                                corrected values
 //   O   = diag(gamma) Q S^T + (Q K^T o exp(g_r - g_i) o [i <= r]) U'
 //   S  <- gamma_last S + U'^T diag(exp(g_last - g)) K
-// The first four lines do not depend on S and run one chunk ahead of the
-// sequential part.
 //
-// One CTA owns one (batch, head, 64-wide slice of value channels) and walks the
-// chunks of that head in order, with its slice of S^T (Dk x 64, float32)
-// resident in tensor memory for the whole sequence.  Warp roles:
-//   warps 0-3  PREP   gates and cumulative sums, A and P from the Gram matrix,
-//                     the UT solve (float32, CUDA cores), W to shared memory
-//   warps 4-7  STATE  U' = U - W S^T, the chunk output, the state hand-off
-//   warp 8     TMA    K, Q and V tiles into a two-stage ring
-//   warp 9     MMA    the sequential products (one elected thread)
-//   warp 10    MMA    the chunk-local products (one elected thread)
-// Every product is a tcgen05.mma with M = 128 (bf16 operands in 128-byte
-// swizzled shared memory, float32 accumulators in TMEM):
-//   G  = [K;Q] K^T            (prep)   rows 0-63 K K^T, rows 64-127 Q K^T
-//   WU = [T';T''] [K | V]     (prep)   T' = T diag(beta gamma), T'' = T diag(beta);
-//                                      W = rows 0-63 x K columns, U = rows 64-127 x V columns
-//   X  = [Q;W] S^T            (state)  rows 0-63 Q S^T, rows 64-127 W S^T
-//   Y  = [P;*] U'             (state)  rows 0-63 intra-chunk output
-//   S^T += K^T diag(exp(g_last - g)) U'   (state; S^T kept pre-scaled by gamma_last)
-// Shared-memory stage layout per 64-wide key block: K | Q | W (8 KiB each), so
-// that [K;Q] and [Q;W] are contiguous 128-row operands, and the K blocks and the
-// V tile sit 24 KiB apart so [K | V] is one MN-major operand of width Dk + 64.
+// Two kernels on one stream:
+//  1. gdn_ut_kernel, one CTA per (batch, head, chunk), all chunks in parallel:
+//     the Gram matrix (bf16 mma.sync, float32 accumulation), its gating, the
+//     UT solve in float32 and the bf16 tile [T'; T''] = [T diag(beta gamma);
+//     T diag(beta)] (128 x 64) into a workspace.  None of it depends on S, and
+//     the solve is a chain of small dependent steps: run wide, it is hidden by
+//     parallelism instead of sitting in front of the sequential pass.
+//  2. gdn_chunk_tc_kernel, one CTA per (batch, head, 64-wide slice of value
+//     channels), walking the chunks of that head in order with its slice of
+//     S^T (Dk x 64, float32) resident in tensor memory.  Warp roles:
+//       warp 0       TMA     K, Q, V and [T'; T''] into a two-stage ring, gate vectors
+//       warp 1       MMA     the sequential products; owns the TMEM allocation
+//       warps 2,3,6,7  P     the gated, masked Q K^T of each chunk (bf16)
+//       warp 4       MMA     G = [K;Q] K^T of each chunk
+//       warp 5       MMA     WU = [T';T''] [K | V] of each chunk
+//       warps 8-15   STATE   W to shared memory, U' = U - W S^T, the chunk
+//                            output, the state hand-off
+//     Every product is a tcgen05.mma with M = 128 (bf16 operands in 128-byte
+//     swizzled shared memory, float32 accumulators in TMEM):
+//       G  = [K;Q] K^T            rows 64-127 Q K^T (rows 0-63 unused)
+//       WU = [T';T''] [K | V]     W = rows 0-63 x K columns, U = rows 64-127 x V columns
+//       X  = [Q;W] S^T            rows 0-63 Q S^T, rows 64-127 W S^T
+//       Y  = [P;*] U'             rows 0-63 intra-chunk output
+//       S^T += K^T diag(exp(g_last - g)) U'   (S^T kept pre-scaled by gamma_last)
+//     Shared-memory stage layout per 64-wide key block: K | Q | W (8 KiB each),
+//     so that [K;Q] and [Q;W] are contiguous 128-row operands, and the K blocks
+//     and the V tile sit 24 KiB apart so [K | V] is one MN-major operand of
+//     width Dk + 64.
 //
-// Rows past the end of the sequence are loaded as zeros by TMA and get
-// beta = 0, log alpha = 0, which leaves the real rows' results unchanged.
-// Every mbarrier wait is bounded (about two seconds); on a timeout the CTA
-// records an error flag, stops all roles, waits for its outstanding copies and
-// releases its tensor memory.
+// Rows past the end of the sequence are loaded as zeros and get beta = 0,
+// log alpha = 0, which leaves the real rows' results unchanged.  Every mbarrier
+// wait is bounded (about two seconds); on a timeout the CTA records an error
+// flag, stops all roles, waits for its outstanding copies and releases its
+// tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -103,10 +109,9 @@ constexpr int KB = DK / 64;    // 64-wide key blocks
 constexpr int NSTAGE = 2;
 constexpr int BLK = 8192;      // one 64 x 64 bf16 tile (64 rows of 128 bytes)
 constexpr int GRP = 3 * BLK;   // K | Q | W of one key block
-constexpr int STAGE = KB * GRP + BLK;
-constexpr int OFF_K = 0, OFF_Q = BLK, OFF_W = 2 * BLK, OFF_V = KB * GRP;
+constexpr int STAGE = KB * GRP + 3 * BLK;  // + V tile + [T'; T''] (16 KiB)
+constexpr int OFF_K = 0, OFF_Q = BLK, OFF_W = 2 * BLK, OFF_V = KB * GRP, OFF_TT = KB * GRP + BLK;
 constexpr int LDA = 72;        // padded float32 row stride of A and T (16-B rows)
-constexpr int LDN = 20;        // padded row stride of the 16 x 16 N blocks
 
 // Per-stage gate vectors (float offsets), written by the TMA warp:
 constexpr int GV_G2 = 0;       // g_r log2(e), g_r = sum of log alpha over rows <= r
@@ -121,20 +126,21 @@ constexpr int GV_STRIDE = 640;
 // shared-memory map (bytes from the 1024-aligned base)
 constexpr int SM_STAGE = 0;
 constexpr int SM_SB = NSTAGE * STAGE;          // S^T bf16, DK rows x 128 B (MN-major B)
-constexpr int SM_UN = SM_SB + DK * 128;        // U' bf16, 64 rows (MN-major B)
+// P tiles for even / odd chunks.  The Y product reads its A operand as 128 rows
+// [P; *]: the 8 KiB after each P tile must be shared memory of this CTA (rows
+// 64-127 only feed accumulator lanes that are never read), hence U' follows.
+constexpr int SM_PT = SM_SB + DK * 128;
+constexpr int SM_UN = SM_PT + 2 * BLK;         // U' bf16, 64 rows (MN-major B)
 constexpr int SM_UP = SM_UN + BLK;             // diag(exp(g_last - g)) U' bf16
-constexpr int SM_PT = SM_UP + BLK;             // P tiles for even / odd chunks
-constexpr int SM_TT = SM_PT + 2 * BLK;         // [T'; T''] 128 rows (K-major A)
-constexpr int SM_AF = SM_TT + 2 * BLK;         // A, float32 64 x LDA
-constexpr int SM_TF = SM_AF + 64 * LDA * 4;    // T, float32 64 x LDA
-constexpr int SM_NF = SM_TF + 64 * LDA * 4;    // N_IJ = T_II A_IJ, six 16 x LDN float32 blocks
-constexpr int SM_GV = SM_NF + 6 * 16 * LDN * 4; // gate vectors, NSTAGE x GV_STRIDE floats
+constexpr int SM_GV = SM_UP + BLK;             // gate vectors, NSTAGE x GV_STRIDE floats
 constexpr int SM_BAR = SM_GV + NSTAGE * GV_STRIDE * 4;
 constexpr int NBAR = 20;
 constexpr int SM_MISC = SM_BAR + NBAR * 8;     // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr int SMEM_BYTES = SM_TOTAL + 1024;    // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(OFF_TT % 1024 == 0 && STAGE % 1024 == 0, "1024-byte aligned swizzled tiles");
+static_assert(SM_PT + (NSTAGE + 1) * BLK <= SM_GV, "[P; *] operand rows stay inside the P/U' tiles");
 static_assert(SM_BAR % 8 == 0, "mbarrier alignment");
 
 // TMEM columns
@@ -146,12 +152,11 @@ constexpr uint32_t TM_COLS = 512;
 enum {
     B_IN_FULL = 0,      // [2] TMA warp: gate vectors + tx bytes (1)
     B_IN_EMPTY = 2,     // [2] chain MMA commit after the last use of the stage (1)
-    B_G_FULL = 4,       // prep MMA commit (1)
-    B_G_EMPTY = 5,      // prep warps (8)
-    B_TT_FULL = 6,      // prep warps (8)
-    B_WU_FULL = 7,      // prep MMA commit (1)
-    B_WU_EMPTY = 8,     // prep warps on lanes 0-63 + state warps on lanes 64-127 (8)
-    B_PREP_FULL = 9,    // [2] prep warps (8)
+    B_G_FULL = 4,       // Gram MMA commit (1)
+    B_G_EMPTY = 5,      // P warps (4)
+    B_WU_FULL = 7,      // WY MMA commit (1)
+    B_WU_EMPTY = 8,     // state warps: W copied (lanes 0-63), U read (lanes 64-127) (8)
+    B_PREP_FULL = 9,    // [2] P warps (4) + state warps that copied W (4)
     B_PT_EMPTY = 11,    // [2] chain MMA commit (1)
     B_X_FULL = 13,      // chain MMA commit (1)
     B_U_READY = 14,     // state warps (8)
@@ -160,15 +165,16 @@ enum {
     B_S_READY = 17,     // state warps (8)
 };
 
-// warp roles
-constexpr int NPREP = 8;                  // warps 0-7: chunk preparation
-constexpr int NSTATEW = 8;                // warps 8-15: sequential state / output
-constexpr int W_TMA = NPREP + NSTATEW;    // 16: TMA loads and gate vectors
-constexpr int W_CHAIN = W_TMA + 1;        // 17: sequential MMAs, TMEM owner
-constexpr int W_PMMA = W_TMA + 2;         // 18: WY product of each chunk
-constexpr int W_GMMA = W_TMA + 3;         // 19: Gram product of each chunk
-constexpr int NTHREADS = 32 * (W_GMMA + 1);
-constexpr int PREP_THREADS = 32 * NPREP;
+// warp roles of the fused kernel (a warp reaches TMEM lanes 32 (warp % 4) .. + 31)
+constexpr int W_TMA = 0;                  // TMA loads and gate vectors
+constexpr int W_CHAIN = 1;                // sequential MMAs, TMEM owner
+constexpr int W_GMMA = 4;                 // Gram product of each chunk
+constexpr int W_PMMA = 5;                 // WY product of each chunk
+constexpr int NPW = 4;                    // P warps 2, 3, 6, 7 (TMEM lanes 64-127)
+constexpr int W_STATE0 = 8;               // warps 8-15: sequential state / output
+constexpr int NSTATEW = 8;
+constexpr int NTHREADS = 32 * (W_STATE0 + NSTATEW);
+
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -229,20 +235,34 @@ __device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
     }
 }
 
-// A wait on behalf of a whole warp: lane 0 polls (so waiting warps do not
-// compete with working warps for the shared-memory pipe) and the result is
-// broadcast, warp-uniform, so a timeout never splits a warp in front of a
-// warp-collective tcgen05 access.
-__device__ __forceinline__ bool warp_wait(const Ctx &cx, int idx, uint32_t parity) {
+// Slow path of warp_wait: lane 0 polls (so waiting warps do not compete with
+// working warps for the shared-memory pipe) and the result is broadcast.
+__device__ __noinline__ bool warp_wait_slow(const Ctx &cx, int idx, uint32_t parity) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = wait_bar(cx, idx, parity);
-    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();  // orders the other lanes' later accesses after lane 0's acquire
+    return ok;
 }
 
-// One arrival on behalf of a whole warp, after every lane's prior writes.
+// A wait on behalf of a whole warp.  The common case (the phase has already
+// completed) is one test and a vote, with no divergent branch; the result is
+// warp-uniform, so a timeout never splits a warp in front of a warp-collective
+// tcgen05 access.
+__device__ __forceinline__ bool warp_wait(const Ctx &cx, int idx, uint32_t parity) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(cx.bar + idx, parity))) return true;
+    return warp_wait_slow(cx, idx, parity);
+}
+
+// One arrival on behalf of a whole warp, after every lane's prior writes
+// (lane 0 arrives, predicated rather than branched).
 __device__ __forceinline__ void warp_arrive(const Ctx &cx, int idx) {
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(cx.bar + idx);
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %1, 0;\n\t"
+        "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(cx.bar + idx)),
+        "r"(threadIdx.x & 31u)
+        : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -271,7 +291,7 @@ __device__ __forceinline__ void tmem_ld16w(uint32_t taddr, float (&v)[16]) {
 // The UT transform T = (I + A)^-1 of the 64 x 64 strictly lower A (AF, float32,
 // stride LDA), blocked by 16 with D_I = I + A_II:
 //   T_II = D_I^-1                                   (ut_diag, forward substitution)
-//   N_IJ = T_II A_IJ,  I > J                        (ut_offdiag phase 1, all six blocks)
+//   N_IJ = T_II A_IJ,  I > J                        (ut_offdiag4 phase 1, all six blocks)
 //   T_IJ = -sum_{J <= K < I} N_IK T_KJ              (phases 2-4, by block diagonal)
 // TF receives the lower triangle and the diagonal; its strict upper part is not
 // written (and never read).
@@ -328,75 +348,214 @@ __device__ __forceinline__ void store16x16(const float (&acc)[2][4], float *__re
     }
 }
 
-// Off-diagonal blocks; all PREP_THREADS threads, one warp per 16 x 16 block
-// product.  NF block order: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
-__device__ __forceinline__ void ut_offdiag(const float *__restrict__ AF, float *__restrict__ TF,
-                                           float *__restrict__ NF, int p, int tc_trace_chunk = 0) {
-    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
-    const auto nf = [&](int blk) { return NF + blk * 16 * LDN; };
-    const auto tf = [&](int I, int J) { return TF + 16 * I * LDA + 16 * J; };
-    if (w < 6) {  // N_IJ = T_II A_IJ
-        const int I = (w == 0) ? 1 : (w < 3 ? 2 : 3);
-        const int J = (w == 0) ? 0 : (w < 3 ? w - 1 : w - 3);
-        float acc[2][4] = {};
-        mma16(acc, tf(I, I), LDA, AF + 16 * I * LDA + 16 * J, LDA, g, t);
-        store16x16(acc, nf(w), LDN, 1.f, g, t);
-    }
-    named_barrier(1, PREP_THREADS);
-    GDN_TRACE_WARP(tc_trace_chunk, 26, 0);
-    if (w < 3) {  // T_{J+1,J} = -N_{J+1,J} T_JJ
-        const int J = w;
-        float acc[2][4] = {};
-        mma16(acc, nf(J == 0 ? 0 : (J == 1 ? 2 : 5)), LDN, tf(J, J), LDA, g, t);
-        store16x16(acc, tf(J + 1, J), LDA, -1.f, g, t);
-    }
-    named_barrier(1, PREP_THREADS);
-    GDN_TRACE_WARP(tc_trace_chunk, 27, 0);
-    if (w < 2) {  // T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})
-        const int J = w;
-        float acc[2][4] = {};
-        mma16(acc, nf(J == 0 ? 1 : 4), LDN, tf(J, J), LDA, g, t);
-        mma16(acc, nf(J == 0 ? 2 : 5), LDN, tf(J + 1, J), LDA, g, t);
-        store16x16(acc, tf(J + 2, J), LDA, -1.f, g, t);
-    }
-    named_barrier(1, PREP_THREADS);
-    GDN_TRACE_WARP(tc_trace_chunk, 28, 0);
-    if (w == 0) {  // T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)
-        float acc[2][4] = {};
-        mma16(acc, nf(3), LDN, tf(0, 0), LDA, g, t);
-        mma16(acc, nf(4), LDN, tf(1, 0), LDA, g, t);
-        mma16(acc, nf(5), LDN, tf(2, 0), LDA, g, t);
-        store16x16(acc, tf(3, 0), LDA, -1.f, g, t);
-    }
-    named_barrier(1, PREP_THREADS);
-    GDN_TRACE_WARP(tc_trace_chunk, 29, 0);
-}
-
-// Gated Gram row, one 16-column piece at a time (columns i = 16 B + j): out[i] =
-// scale * Gamma(r, i) * gram[i] for i < r (kStrict) or i <= r, zero above, with
-// Gamma(r, i) = exp(g_r - g_i).  Off the row's diagonal 16-block R the decay
-// factors as u_r * w_R[i] (u_r = exp(g_r - g_{16R}), w_R[i] = exp(g_{16R} - g_i),
+// Gated, masked Q K^T row, one 16-column piece (columns i = 16 B + j) of row r:
+// out[i] = Gamma(r, i) gram[i] for i <= r, zero above, Gamma(r, i) = exp(g_r - g_i).
+// Off the row's diagonal 16-block R the decay factors as u_r * w_R[i] (u_r =
+// exp(g_r - g_{16R}), w_R[i] = exp(g_{16R} - g_i) for i < 16 R and 0 from 16 R on,
 // both <= 1, so nothing overflows); inside it, exp2 of the log2-domain
-// difference.
-template <bool kStrict>
-__device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float scale, float su,
+// difference.  kDiag: some lane of the warp has B == R (the exp2 path is then
+// evaluated for every lane and selected, so the warp never diverges).
+template <bool kDiag>
+__device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float su,
                                             const float *g2s, const float *w_all) {
     const int R = r >> 4;
-    if (B < R) {
-        const float *w = w_all + R * 64 + 16 * B;
+    const float *w = w_all + R * 64 + 16 * B;
+    const float gr = g2s[r];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] *= su * w[j];
-    } else if (B == R) {
-        const float gr = g2s[r];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int i = 16 * B + j;
-            const bool keep = kStrict ? (i < r) : (i <= r);
-            v[j] = keep ? scale * ex2(gr - g2s[i]) * v[j] : 0.f;
+    for (int j = 0; j < 16; ++j) {
+        const int i = 16 * B + j;
+        float f = su * w[j];
+        if (kDiag) {
+            const float e = ex2(gr - g2s[i]);
+            f = (B == R) ? ((i <= r) ? e : 0.f) : f;
         }
-    } else {
+        v[j] *= f;
+    }
+}
+
+// ------------------------------------------------------------- UT kernel --
+// One CTA of 4 warps per (chunk c, head h, batch b): [T'; T''] of that chunk,
+// bf16, 128 rows x 64 columns, row-major, at tt + ((b H + h) NT + c) 128 x 64.
+// Six CTAs fit on an SM (shared memory and registers), so six chunks are in
+// flight per SM and the solve's dependent steps overlap across chunks.
+constexpr int UT_THREADS = 128;
+constexpr int LDK = DK + 8;                        // bf16 row stride of the staged K chunk
+constexpr int UT_SM_KT = 0;                        // K chunk (64 x LDK bf16), then T (64 x LDA f32)
+constexpr int UT_SM_AF = C * LDA * 4;              // A (64 x LDA f32); N_IJ overwrite A_IJ
+constexpr int UT_SM_GT = UT_SM_AF + C * LDA * 4;   // g log2(e), beta, beta gamma (3 x 64)
+constexpr int UT_SMEM = UT_SM_GT + 3 * C * 4;
+constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
+static_assert(C * LDK * 2 <= UT_SM_AF, "K chunk fits in the T buffer");
+static_assert(UT_SM_AF % 16 == 0 && UT_SM_GT % 16 == 0, "16-byte aligned UT buffers");
+
+// Off-diagonal blocks of T with 4 warps, N_IJ = T_II A_IJ stored over A_IJ:
+//   phase 1  N for the six blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2), two rounds
+//   phase 2  T_{J+1,J} = -N_{J+1,J} T_JJ                              (3 warps)
+//   phase 3  T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})    (2 warps)
+//   phase 4  T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)              (1 warp)
+__device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__restrict__ TF,
+                                            int p) {
+    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    const auto blk = [&](float *M, int I, int J) { return M + 16 * I * LDA + 16 * J; };
+    constexpr int BI[6] = {1, 2, 2, 3, 3, 3}, BJ[6] = {0, 0, 1, 0, 1, 2};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+    for (int round = 0; round < 2; ++round) {
+        const int k = w + 4 * round;
+        if (k < 6) {
+            const int I = BI[k], J = BJ[k];
+            float acc[2][4] = {};
+            mma16(acc, blk(TF, I, I), LDA, blk(AF, I, J), LDA, g, t);
+            __syncwarp();
+            store16x16(acc, blk(AF, I, J), LDA, 1.f, g, t);
+        }
+    }
+    __syncthreads();
+    if (w < 3) {
+        float acc[2][4] = {};
+        mma16(acc, blk(AF, w + 1, w), LDA, blk(TF, w, w), LDA, g, t);
+        store16x16(acc, blk(TF, w + 1, w), LDA, -1.f, g, t);
+    }
+    __syncthreads();
+    if (w < 2) {
+        float acc[2][4] = {};
+        mma16(acc, blk(AF, w + 2, w), LDA, blk(TF, w, w), LDA, g, t);
+        mma16(acc, blk(AF, w + 2, w + 1), LDA, blk(TF, w + 1, w), LDA, g, t);
+        store16x16(acc, blk(TF, w + 2, w), LDA, -1.f, g, t);
+    }
+    __syncthreads();
+    if (w == 0) {
+        float acc[2][4] = {};
+        mma16(acc, blk(AF, 3, 0), LDA, blk(TF, 0, 0), LDA, g, t);
+        mma16(acc, blk(AF, 3, 1), LDA, blk(TF, 1, 0), LDA, g, t);
+        mma16(acc, blk(AF, 3, 2), LDA, blk(TF, 2, 0), LDA, g, t);
+        store16x16(acc, blk(TF, 3, 0), LDA, -1.f, g, t);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(UT_THREADS, 6)
+gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
+              const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt, int T, int H,
+              int NT) {
+    extern __shared__ __align__(16) uint8_t ut_smem[];
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int t0 = c * C;
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ut_smem + UT_SM_KT);
+    float *TF = reinterpret_cast<float *>(ut_smem + UT_SM_KT);
+    float *AF = reinterpret_cast<float *>(ut_smem + UT_SM_AF);
+    float *g2s = reinterpret_cast<float *>(ut_smem + UT_SM_GT);
+    float *bes = g2s + C, *bgs = g2s + 2 * C;
+
+    // K rows of the chunk (zeros past the end of the sequence): 16 x 16 B per row
+#pragma unroll
+    for (int m = 0; m < C * (DK / 8) / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int r = idx / (DK / 8), piece = idx % (DK / 8);
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (t0 + r < T)
+            val = __ldg(reinterpret_cast<const uint4 *>(
+                k + (((size_t)b * T + t0 + r) * H + h) * DK + 8 * piece));
+        *reinterpret_cast<uint4 *>(Ks + r * LDK + 8 * piece) = val;
+    }
+    if (warp == 0) {
+        // running sum of log alpha over rows lane and lane + 32, in log2 units
+        constexpr float LOG2E = 1.4426950408889634f;
+        float la[2], be[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            const bool in = t0 + r < T;
+            const size_t gi = ((size_t)b * T + t0 + r) * H + h;
+            la[hh] = in ? log_alpha[gi] : 0.f;
+            be[hh] = in ? beta[gi] : 0.f;
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, la[0], off);
+            const float y1 = __shfl_up_sync(0xffffffffu, la[1], off);
+            if (lane >= off) {
+                la[0] += y0;
+                la[1] += y1;
+            }
+        }
+        la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float g2 = la[hh] * LOG2E;
+            g2s[lane + 32 * hh] = g2;
+            bes[lane + 32 * hh] = be[hh];
+            bgs[lane + 32 * hh] = be[hh] * ex2(g2);
+        }
+    }
+    __syncthreads();
+
+    // Gram K K^T on and below the diagonal: warp w takes rows 16 w .. + 15 and the
+    // 2 w + 2 column tiles of 8 up to the diagonal, then gates it into A:
+    //   A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0
+    {
+        const int RB = warp, ntiles = 2 * RB + 2;
+        float acc[8][4] = {};
+        const __nv_bfloat16 *ar = Ks + (16 * RB + g) * LDK + 2 * t;
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+            const int k0 = 16 * ks;
+            const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(ar + k0),
+                                   *reinterpret_cast<const uint32_t *>(ar + 8 * LDK + k0),
+                                   *reinterpret_cast<const uint32_t *>(ar + k0 + 8),
+                                   *reinterpret_cast<const uint32_t *>(ar + 8 * LDK + k0 + 8)};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (j < ntiles) {
+                    const __nv_bfloat16 *br = Ks + (8 * j + g) * LDK + k0 + 2 * t;
+                    const uint32_t bb[2] = {*reinterpret_cast<const uint32_t *>(br),
+                                            *reinterpret_cast<const uint32_t *>(br + 8)};
+                    mma_bf16_16x8x16(acc[j], a, bb);
+                }
+            }
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = 16 * RB + g + 8 * hr;
+            const float gr = g2s[r], br = bes[r];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (j < ntiles) {
+                    const int i = 8 * j + 2 * t;
+                    const float a0 = (i < r) ? br * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
+                    const float a1 =
+                        (i + 1 < r) ? br * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1] : 0.f;
+                    *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
+                }
+            }
+        }
+    }
+    __syncthreads();  // A complete; K no longer read, its buffer becomes T
+    if (tid < C) ut_diag(AF, TF, tid);
+    __syncthreads();
+    ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
+
+    // [T'; T''] rows: T'(r, i) = T(r, i) beta_i gamma_i, T''(r, i) = T(r, i) beta_i
+    // for i <= r; thread -> (row, 8-column piece), 4 rows x 128 B per warp store
+    __nv_bfloat16 *dst = tt + ((size_t)((size_t)b * H + h) * NT + c) * TT_ELEMS;
+#pragma unroll
+    for (int m = 0; m < TT_ELEMS / 8 / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int rt = idx >> 3, i0 = 8 * (idx & 7), r = rt & (C - 1);
+        const float *sc = rt < C ? bgs : bes;
+        const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
+        const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
+        const float4 sa = *reinterpret_cast<const float4 *>(sc + i0);
+        const float4 sb = *reinterpret_cast<const float4 *>(sc + i0 + 4);
+        float x[8] = {ta.x * sa.x, ta.y * sa.y, ta.z * sa.z, ta.w * sa.w,
+                      tb.x * sb.x, tb.y * sb.y, tb.z * sb.z, tb.w * sb.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j > r) x[j] = 0.f;
+        *reinterpret_cast<uint4 *>(dst + rt * C + i0) =
+            make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                       pack_bf16(x[6], x[7]));
     }
 }
 
@@ -411,7 +570,8 @@ struct Params {
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tt,
+                    const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived by pointer arithmetic so that the compiler
     // keeps every access below in the shared address space
@@ -432,9 +592,9 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         int counts[NBAR];
         for (int i = 0; i < NBAR; ++i) counts[i] = 1;
         // one arrival per arriving warp
-        counts[B_G_EMPTY] = counts[B_TT_FULL] = NPREP;
+        counts[B_G_EMPTY] = NPW;
         counts[B_WU_EMPTY] = NSTATEW;
-        counts[B_PREP_FULL] = counts[B_PREP_FULL + 1] = NPREP / 2 + NSTATEW / 2;
+        counts[B_PREP_FULL] = counts[B_PREP_FULL + 1] = NPW + NSTATEW / 2;
         counts[B_U_READY] = counts[B_S_READY] = NSTATEW;
         for (int i = 0; i < NBAR; ++i) mbar_init(cx.bar + i, counts[i]);
         *cx.abort = 0u;
@@ -448,6 +608,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_tt);
     }
     tc_fence_before();
     __syncthreads();
@@ -456,22 +617,47 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (warp == W_TMA) {
         // ------------------------------------- TMA loads + per-chunk gate vectors
+        // The gate values of chunk c + 1 are fetched while chunk c is handled, and
+        // each stage's copies are started before its gate vectors are computed
+        // (the stage's barrier gets the byte count first and the warp's arrival
+        // after the vectors are written).
         constexpr float LOG2E = 1.4426950408889634f;
         int armed = 0;
-        for (int c = 0; c < NT; ++c) {
-            const int s = c & 1;
-            if (c >= 2 && !warp_wait(cx, B_IN_EMPTY + s, ((c - 2) >> 1) & 1)) break;
-            // rows lane (lo) and lane + 32 (hi); zero past the end of the sequence
-            const int t0 = c * C;
-            float la[2], be[2];
+        float nla[2], nbe[2];  // gate values of the next chunk (rows lane, lane + 32)
+        const auto fetch_gates = [&](int cc) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = lane + 32 * hh;
-                const bool in = t0 + r < T;
-                const size_t gi = ((size_t)b * T + t0 + r) * H + h;
-                la[hh] = in ? p.log_alpha[gi] : 0.f;
-                be[hh] = in ? p.beta[gi] : 0.f;
+                const bool in = cc * C + r < T;
+                const size_t gi = ((size_t)b * T + cc * C + r) * H + h;
+                nla[hh] = in ? p.log_alpha[gi] : 0.f;
+                nbe[hh] = in ? p.beta[gi] : 0.f;
             }
+        };
+        fetch_gates(0);
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            const int t0 = c * C;
+            float la[2] = {nla[0], nla[1]}, be[2] = {nbe[0], nbe[1]};
+            if (c + 1 < NT) fetch_gates(c + 1);
+            if (c >= 2 && !warp_wait(cx, B_IN_EMPTY + s, ((c - 2) >> 1) & 1)) break;
+            GDN_TRACE_WARP(c, 31, W_TMA);
+            if (lane == 0) {
+                uint8_t *st = base + SM_STAGE + s * STAGE;
+                mbar_expect_tx(cx.bar + B_IN_FULL + s, (2 * KB + 3) * BLK);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(st + kb * GRP + OFF_K, &tm_k, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
+                    tma_load_4d(st + kb * GRP + OFF_Q, &tm_q, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
+                }
+                tma_load_4d(st + OFF_V, &tm_v, cx.bar + B_IN_FULL + s, v0, h, t0, b);
+                tma_load_3d(st + OFF_TT, &tm_tt, cx.bar + B_IN_FULL + s, 0, 0,
+                            ((int)b * H + h) * NT + c);
+                GDN_TRACE_AT(c, 24);
+            }
+            armed = c + 1;
+            // running sums over rows lane (lo) and lane + 32 (hi); rows past the
+            // end of the sequence carry zeros
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y0 = __shfl_up_sync(0xffffffffu, la[0], off);
@@ -510,17 +696,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             gv[GV_W + 3 * 64 + 32 + lane] = lane < 16 ? ex2(g48 - g1) : 0.f;
             if (lane == 0) gv[GV_GL] = ex2(glast);
             __syncwarp();
-            if (lane == 0) {
-                uint8_t *st = base + SM_STAGE + s * STAGE;
-                mbar_arrive_expect_tx(cx.bar + B_IN_FULL + s, (2 * KB + 1) * BLK);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(st + kb * GRP + OFF_K, &tm_k, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
-                    tma_load_4d(st + kb * GRP + OFF_Q, &tm_q, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
-                }
-                tma_load_4d(st + OFF_V, &tm_v, cx.bar + B_IN_FULL + s, v0, h, t0, b);
-            }
-            armed = c + 1;
+            if (lane == 0) mbar_arrive(cx.bar + B_IN_FULL + s);
         }
         // never leave with copies in flight: wait for the last two stages
         if (lane == 0) {
@@ -555,10 +731,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // --------------------------------------------------- MMA: WY products
         if (lane == 0) {
             const uint32_t idesc_wu = idesc_bf16(128, DK + DVT, false, true);
-            const uint32_t tt = smem_u32(base + SM_TT);
             for (int c = 0; c < NT; ++c) {
                 const uint32_t st = smem_u32(base + SM_STAGE + (c & 1) * STAGE);
-                if (!wait_bar(cx, B_TT_FULL, c & 1)) break;
+                const uint32_t tt = st + OFF_TT;
+                if (!wait_bar(cx, B_IN_FULL + (c & 1), (c >> 1) & 1)) break;
                 if (c >= 1 && !wait_bar(cx, B_WU_EMPTY, (c - 1) & 1)) break;
                 tc_fence_after();
 #pragma unroll
@@ -581,8 +757,11 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int s = c & 1;
                 const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
                 if (!wait_bar(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
+                GDN_TRACE_AT(c, 5);
                 if (!wait_bar(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
+                GDN_TRACE_AT(c, 6);
                 if (!wait_bar(cx, B_S_READY, c & 1)) break;
+                GDN_TRACE_AT(c, 7);
                 tc_fence_after();
                 // X = [Q; W] S^T : A K-major (rows 0-63 Q, 64-127 W), B = S^T MN-major
 #pragma unroll
@@ -614,109 +793,55 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_commit(cx.bar + B_IN_EMPTY + s);
             }
         }
-    } else if (warp < NPREP) {
-        // ------------------------------------------------------------- PREP
-        // 8 warps; warp w reads TMEM lanes 32 (w % 4) .. + 31 and, with its twin
-        // w ^ 4, splits those lanes' columns in half (hf = w / 4).  Lanes 0-63
-        // carry the rows of K K^T (-> A), lanes 64-127 the rows of Q K^T (-> P).
-        const int pt = tid;                         // 0..255
-        const int q = warp & 3, hf = warp >> 2;
-        const int lrow = 32 * q + lane;             // TMEM lane of this thread
-        const bool is_a = q < 2;
-        float *AF = reinterpret_cast<float *>(base + SM_AF);
-        float *TF = reinterpret_cast<float *>(base + SM_TF);
-        float *NF = reinterpret_cast<float *>(base + SM_NF);
+    } else if (warp < W_STATE0) {
+        // ---------------------------------------------------------------- P
+        // warps 2, 3, 6, 7: TMEM lanes 64-127 of G hold Q K^T.  Warp w reads
+        // lanes 32 (w % 4) .. + 31 (chunk rows r = that lane - 64, 16-blocks
+        // 2 qr and 2 qr + 1) and the 16-column pieces hf and hf + 2 (hf = w / 4):
+        // every warp meets the diagonal in exactly one of its pieces (piece hf
+        // for qr = 0, piece hf + 2 for qr = 1).  P (bf16) goes to the chunk's P tile.
+        const int q = warp & 3, hf = warp >> 2, qr = q - 2;
+        const int r = 32 * q + lane - 64;
         const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
-        // After the WY product: W rows (TMEM lanes 0-63) of chunk cc to its stage's
-        // W slots (twin warps take one key block each), then release the WU
-        // accumulator and publish the chunk.
-        bool ok = true;  // false once a wait has failed; the CTA is then aborting
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
             const float *gv = gv_all + s * GV_STRIDE;
-            ok &= warp_wait(cx, B_IN_FULL + s, (c >> 1) & 1);
-            GDN_TRACE_WARP(c, 0, 0);
-            ok &= warp_wait(cx, B_G_FULL, c & 1);
-            GDN_TRACE_WARP(c, 1, 0);
+            if (!warp_wait(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
+            if (!warp_wait(cx, B_G_FULL, c & 1)) break;
+            GDN_TRACE_WARP(c, 22, 2);
+            if (c >= 2 && !warp_wait(cx, B_PT_EMPTY + s, ((c - 2) >> 1) & 1)) break;
+            GDN_TRACE_WARP(c, 3, 2);
             tc_fence_after();
-            {
-                const int r = lrow & 63;
-                if (!is_a && c >= 2) ok &= warp_wait(cx, B_PT_EMPTY + s, ((c - 2) >> 1) & 1);
-                const float scale = is_a ? gv[GV_BETA + r] : 1.f;
-                const float su = scale * gv[GV_U + r];
-                float v0[16], v1[16];
-                tmem_ld16(lane_addr + TM_G + 32 * hf, v0);
-                tmem_ld16(lane_addr + TM_G + 32 * hf + 16, v1);
-                tmem_wait_ld();
-                tc_fence_before();
-                warp_arrive(cx, B_G_EMPTY);
-                GDN_TRACE_WARP(c, 22, 0);
-                if (is_a) {
-                    gated_piece<true>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
-                    gated_piece<true>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hf + 4 * k) =
-                            make_float4(v0[4 * k], v0[4 * k + 1], v0[4 * k + 2], v0[4 * k + 3]);
-                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hf + 16 + 4 * k) =
-                            make_float4(v1[4 * k], v1[4 * k + 1], v1[4 * k + 2], v1[4 * k + 3]);
-                    }
-                    GDN_TRACE_WARP(c, 23, 0);
-                    // A complete (the four A warps) -> diagonal blocks of T
-                    named_barrier(3, PREP_THREADS / 2);
-                    GDN_TRACE_WARP(c, 24, 0);
-                    if (pt < 64) ut_diag(AF, TF, pt);
-                    GDN_TRACE_WARP(c, 25, 0);
-                } else {
-                    gated_piece<false>(v0, 2 * hf, r, scale, su, gv + GV_G2, gv + GV_W);
-                    gated_piece<false>(v1, 2 * hf + 1, r, scale, su, gv + GV_G2, gv + GV_W);
-                    store16_bf16(base + SM_PT + s * BLK, r, 2 * hf, v0);
-                    store16_bf16(base + SM_PT + s * BLK, r, 2 * hf + 1, v1);
-                    fence_async_smem();
-                }
+            const float su = gv[GV_U + r];
+            float v0[16], v1[16];
+            tmem_ld16(lane_addr + TM_G + 16 * hf, v0);
+            tmem_ld16(lane_addr + TM_G + 16 * hf + 32, v1);
+            tmem_wait_ld();
+            GDN_TRACE_WARP(c, 27, 2);
+            tc_fence_before();
+            warp_arrive(cx, B_G_EMPTY);
+            if (qr == 0) {
+                gated_piece<true>(v0, hf, r, su, gv + GV_G2, gv + GV_W);
+                gated_piece<false>(v1, hf + 2, r, su, gv + GV_G2, gv + GV_W);
+            } else {
+                gated_piece<false>(v0, hf, r, su, gv + GV_G2, gv + GV_W);
+                gated_piece<true>(v1, hf + 2, r, su, gv + GV_G2, gv + GV_W);
             }
-            named_barrier(1, PREP_THREADS);
-            GDN_TRACE_WARP(c, 2, 0);
-            ut_offdiag(AF, TF, NF, pt, c);
-            GDN_TRACE_WARP(c, 3, 0);
-            // [T'; T''] : row rt, T'(r,i) = T(r,i) beta_i gamma_i, T''(r,i) = T(r,i) beta_i
-            // (the previous chunk's WY product must have read TT first)
-            if (c >= 1) ok &= warp_wait(cx, B_WU_FULL, (c - 1) & 1);
-            {
-                const int rt = pt & 127, r = rt & 63;
-                const bool wgam = rt < 64;
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int B = 2 * (pt >> 7) + k;
-                    float v[16];
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const int i = 16 * B + 4 * qq;
-                        const float4 tv = *reinterpret_cast<const float4 *>(TF + r * LDA + i);
-                        const float4 bv = *reinterpret_cast<const float4 *>(gv + GV_BETA + i);
-                        float4 gv4 = make_float4(1.f, 1.f, 1.f, 1.f);
-                        if (wgam) gv4 = *reinterpret_cast<const float4 *>(gv + GV_GAM + i);
-                        v[4 * qq + 0] = (i + 0 <= r) ? tv.x * bv.x * gv4.x : 0.f;
-                        v[4 * qq + 1] = (i + 1 <= r) ? tv.y * bv.y * gv4.y : 0.f;
-                        v[4 * qq + 2] = (i + 2 <= r) ? tv.z * bv.z * gv4.z : 0.f;
-                        v[4 * qq + 3] = (i + 3 <= r) ? tv.w * bv.w * gv4.w : 0.f;
-                    }
-                    store16_bf16(base + SM_TT, rt, B, v);
-                }
-                fence_async_smem();
-                warp_arrive(cx, B_TT_FULL);
-            }
-            GDN_TRACE_WARP(c, 4, 0);
-            if (!is_a) warp_arrive(cx, B_PREP_FULL + (c & 1));
-            // leave together: every prep thread sees the same decision
-            if (named_barrier_or(1, PREP_THREADS, !ok || *cx.abort)) break;
+            GDN_TRACE_WARP(c, 28, 2);
+            store16_bf16(base + SM_PT + s * BLK, r, hf, v0);
+            store16_bf16(base + SM_PT + s * BLK, r, hf + 2, v1);
+            fence_async_smem();
+            GDN_TRACE_WARP(c, 29, 2);
+            warp_arrive(cx, B_PREP_FULL + s);
+            GDN_TRACE_WARP(c, 23, 2);
+            GDN_TRACE_WARP(c, 30, 7);
         }
     } else {
         // ------------------------------------------------------------ STATE
         // 8 warps; warp w reads TMEM lanes 32 (w % 4) .. + 31 (a key channel of
         // S^T, or a chunk row of X / Y) and handles half of that lane's 64
         // columns (hf), its twin the other half.
-        const int q = warp & 3, hf = (warp - NPREP) >> 2;
+        const int q = warp & 3, hf = (warp - W_STATE0) >> 2;
         const int lrow = 32 * q + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
         uint8_t *sbuf = base + SM_SB;
@@ -724,6 +849,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const auto copy_w = [&](int cc) -> bool {
             if (q >= 2) return true;
             const bool fine = warp_wait(cx, B_WU_FULL, cc & 1);
+            GDN_TRACE_WARP(cc, 25, W_STATE0);
             tc_fence_after();
             const int kb = hf;
             float w0[16], w1[16], w2[16], w3[16];
@@ -741,6 +867,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             warp_arrive(cx, B_WU_EMPTY);
             warp_arrive(cx, B_PREP_FULL + (cc & 1));
+            GDN_TRACE_WARP(cc, 26, W_STATE0);
             return fine;
         };
         // initial state: S^T row lrow = S0[v0 .. v0+63][lrow]; TMEM copy pre-scaled by gamma_last
@@ -771,7 +898,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int t0 = c * C;
             const float *gv = gv_all + s * GV_STRIDE;
             if (!warp_wait(cx, B_X_FULL, c & 1)) break;
-            GDN_TRACE_WARP(c, 16, NPREP);
+            GDN_TRACE_WARP(c, 16, W_STATE0);
             tc_fence_after();
             if (q >= 2) {
                 // U' = U - W S^T for chunk row r -> U' and diag(exp(g_last - g)) U' (bf16)
@@ -801,7 +928,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc_fence_before();
                 warp_arrive(cx, B_U_READY);
                 warp_arrive(cx, B_WU_EMPTY);
-                GDN_TRACE_WARP(c, 18, NPREP + 2);
+                GDN_TRACE_WARP(c, 18, W_STATE0 + 2);
             } else {
                 // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y; the
                 // intra-chunk MMA accumulates onto it
@@ -823,7 +950,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             // state hand-off: S^T (gamma-scaled + update) -> bf16 copy; TMEM pre-scaled
             if (!warp_wait(cx, B_ST_FULL, c & 1)) break;
-            GDN_TRACE_WARP(c, 20, NPREP);
+            GDN_TRACE_WARP(c, 20, W_STATE0);
             tc_fence_after();
             {
                 const bool last = c + 1 >= NT;
@@ -860,14 +987,15 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tc_fence_before();
                 warp_arrive(cx, B_S_READY);
-                GDN_TRACE_WARP(c, 21, NPREP);
+                GDN_TRACE_WARP(c, 21, W_STATE0);
+                GDN_TRACE_WARP(c, 4, W_STATE0 + 7);
                 if (!last && !have) break;
             }
             if (c + 1 < NT) copy_w(c + 1);
             // chunk output rows (lanes 0-63)
             if (q < 2) {
                 if (!warp_wait(cx, B_Y_FULL, c & 1)) break;
-                GDN_TRACE_WARP(c, 19, NPREP);
+                GDN_TRACE_WARP(c, 19, W_STATE0);
                 tc_fence_after();
                 float y0[16], y1[16];
                 tmem_ld16(lane_addr + TM_Y + 32 * hf, y0);
@@ -931,7 +1059,26 @@ bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Workspace of [T'; T''] tiles, [n_tiles, 128, 64] bf16: box of one whole tile, 128B swizzle.
+bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)(2 * C), (cuuint64_t)n_tiles};
+    cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)TT_ELEMS * 2};
+    cuuint32_t box[3] = {(cuuint32_t)C, (cuuint32_t)(2 * C), 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
+
+size_t tc_workspace_bytes(int B, int T, int H) {
+    const size_t NT = ((size_t)T + tc::C - 1) / tc::C;
+    return (size_t)B * H * NT * tc::TT_ELEMS * sizeof(__nv_bfloat16);
+}
 
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
     return bf16 && chunk == tc::C && Dk == tc::DK && Dv % tc::DVT == 0 && B >= 1 && T >= 1 &&
@@ -940,10 +1087,13 @@ bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
-                            int H, int Dk, int Dv, cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
+                            int H, int Dk, int Dv, void *workspace, cudaStream_t st) {
+    const int NT = (T + tc::C - 1) / tc::C;
+    auto *tt = static_cast<__nv_bfloat16 *>(workspace);
+    CUtensorMap mq, mk, mv, mt;
     if (!tc::make_map(&mq, q, B, T, H, Dk) || !tc::make_map(&mk, k, B, T, H, Dk) ||
-        !tc::make_map(&mv, v, B, T, H, Dv))
+        !tc::make_map(&mv, v, B, T, H, Dv) ||
+        !tc::make_map_tt(&mt, tt, (long long)B * H * NT))
         return cudaErrorInvalidValue;
     tc::Params p;
     p.log_alpha = log_alpha;
@@ -954,13 +1104,19 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     p.T = T;
     p.H = H;
     p.Dv = Dv;
-    p.NT = (T + tc::C - 1) / tc::C;
-    cudaError_t e = cudaFuncSetAttribute(tc::gdn_chunk_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::SMEM_BYTES);
+    p.NT = NT;
+    cudaError_t e = cudaFuncSetAttribute(tc::gdn_ut_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::UT_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc::gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    tc::gdn_ut_kernel<<<dim3(NT, H, B), tc::UT_THREADS, tc::UT_SMEM, st>>>(
+        static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, T, H, NT);
+    e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     tc::gdn_chunk_tc_kernel<<<dim3(Dv / tc::DVT, H, B), tc::NTHREADS, tc::SMEM_BYTES, st>>>(
-        mq, mk, mv, p);
+        mq, mk, mv, mt, p);
     return cudaPeekAtLastError();
 }
 

@@ -54,8 +54,10 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype
 
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
                                     gdn_dtype_t dtype) {
-    if (gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype) != GDN_PATH_SIMT) return 0;
-    return gdn::simt_workspace_bytes(B, T, H, chunk);
+    const int path = gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype);
+    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H);
+    if (path == GDN_PATH_SIMT) return gdn::simt_workspace_bytes(B, T, H, chunk);
+    return 0;
 }
 
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -90,12 +92,25 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
         return GDN_ERR_INVALID_ARG;
 
     const bool bf16 = dtype == GDN_BF16;
+    const bool tc = gdn::tc_supported(B, T, H, Dk, Dv, chunk, bf16);
+    const size_t need = tc ? gdn::tc_workspace_bytes(B, T, H)
+                           : gdn::simt_workspace_bytes(B, T, H, chunk);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    // the workspace is scratch written by the kernels: it must not alias anything else
+    if (overlaps(workspace, need, q, n_tok * Dk * esz) ||
+        overlaps(workspace, need, k, n_tok * Dk * esz) ||
+        overlaps(workspace, need, v, n_tok * Dv * esz) ||
+        overlaps(workspace, need, log_alpha, n_tok * sizeof(float)) ||
+        overlaps(workspace, need, beta, n_tok * sizeof(float)) ||
+        overlaps(workspace, need, o, o_bytes) ||
+        (S0 && overlaps(workspace, need, S0, state_bytes)) ||
+        (S_T && overlaps(workspace, need, S_T, state_bytes)))
+        return GDN_ERR_INVALID_ARG;
     cudaError_t e;
-    if (gdn::tc_supported(B, T, H, Dk, Dv, chunk, bf16)) {
-        e = gdn::launch_chunk_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, st);
+    if (tc) {
+        e = gdn::launch_chunk_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, workspace,
+                                 st);
     } else {
-        const size_t need = gdn::simt_workspace_bytes(B, T, H, chunk);
-        if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
         e = gdn::launch_chunk_simt(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk,
                                    bf16, workspace, st);
     }

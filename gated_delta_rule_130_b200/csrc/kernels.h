@@ -20,11 +20,13 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               int T, int H, int Dk, int Dv, int chunk, bool bf16, void *workspace,
                               cudaStream_t st);
 
-// Fused tcgen05 chunkwise forward: chunk_tc.cu.
+// tcgen05 chunkwise forward (bf16, Dk = 128, chunk 64): chunk_tc.cu.  The
+// workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of every head.
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
+size_t tc_workspace_bytes(int B, int T, int H);
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
-                            int H, int Dk, int Dv, cudaStream_t st);
+                            int H, int Dk, int Dv, void *workspace, cudaStream_t st);
 
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).

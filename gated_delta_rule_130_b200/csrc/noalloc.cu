@@ -3,9 +3,8 @@
 // run the layer: engines that plan every buffer once at start-up and forbid
 // allocation afterwards, code paths where cudaMalloc's implicit device-wide
 // synchronisation is not acceptable, and hosts that own the device's memory
-// and hand the library none.  For them the workspace the CUDA-core path needs
-// lives in a fixed array compiled into this library instead of a buffer they
-// pass in.
+// and hand the library none.  For them the workspace lives in a fixed array
+// compiled into this library instead of a buffer they pass in.
 //
 // The array is a file-scope __device__ array of kScratchBytes (8 MiB); every
 // GPU that loads the library holds it until the process exits.  Its device

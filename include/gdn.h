@@ -62,7 +62,10 @@ typedef enum {
     GDN_PATH_NONE = 0,     /* empty problem: nothing (or only a state copy) runs */
     GDN_PATH_SIMT = 1,     /* two CUDA-core kernels: chunk preparation, then the
                               sequential state/output pass; needs a workspace */
-    GDN_PATH_TCGEN05 = 2   /* one fused tcgen05 tensor-core kernel, no workspace */
+    GDN_PATH_TCGEN05 = 2   /* bf16, Dk = 128, chunk 64, Dv a multiple of 64: the
+                              per-chunk UT transform for all chunks in parallel
+                              (into the workspace), then one tcgen05 tensor-core
+                              kernel for the sequential pass; needs a workspace */
 } gdn_path_t;
 
 /* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0
@@ -86,7 +89,9 @@ typedef enum {
  *   o   : output [B,T,H,Dv] in `dtype` (required; must not overlap an input).
  *   S_T : final state per head, or NULL if not wanted.
  *   workspace / workspace_bytes : device scratch of at least
- *         gdn_chunk_fwd_workspace_size(...) bytes (NULL/0 when that is 0).
+ *         gdn_chunk_fwd_workspace_size(...) bytes (NULL/0 when that is 0),
+ *         16-byte aligned, overlapping no other argument; its contents on
+ *         entry do not matter and are undefined on return.
  */
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
@@ -95,8 +100,9 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v,
                            gdn_dtype_t dtype, void *workspace,
                            size_t workspace_bytes, void *stream);
 
-/* Bytes of device workspace gdn_chunk_fwd needs for these sizes (0 for the
- * fused tensor-core path and for empty problems). */
+/* Bytes of device workspace gdn_chunk_fwd needs for these sizes (0 for empty
+ * problems): on the tensor-core path 16 KiB per 64-token chunk of every
+ * (batch, head), on the CUDA-core path (2 chunk^2 + chunk) floats per chunk. */
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv,
                                     int chunk, gdn_dtype_t dtype);
 
@@ -113,10 +119,9 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk,
  * counterpart: this is a property of the library, not of the method.
  *
  * Same arguments and results as gdn_chunk_fwd, minus the workspace.  The
- * CUDA-core path's scratch is a fixed 8 MiB array inside the library (held on
- * every GPU that loads it until exit); sizes whose workspace
- * (gdn_chunk_fwd_workspace_size) exceeds 8 MiB return GDN_ERR_UNSUPPORTED with
- * nothing launched.  The first call on a device looks up the array's address
+ * scratch is a fixed 8 MiB array inside the library (held on every GPU that
+ * loads it until exit); sizes whose workspace (gdn_chunk_fwd_workspace_size)
+ * exceeds 8 MiB return GDN_ERR_UNSUPPORTED with nothing launched.  The first call on a device looks up the array's address
  * (with that device current) and must come before any stream capture.  All
  * calls share the array: calls whose work overlaps on the GPU race and must be
  * serialised by the caller.  Allocates nothing.

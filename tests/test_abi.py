@@ -64,7 +64,7 @@ def test_path_selection_and_workspace(lib):
 
 def _chunk(lib, **kw):
     a = dict(q=16, k=16, v=16, la=16, beta=16, S0=None, o=4096, S_T=None, B=1, T=8, H=1, Dk=16,
-             Dv=16, chunk=16, dtype=0, ws=16, ws_bytes=1 << 30, stream=None)
+             Dv=16, chunk=16, dtype=0, ws=1 << 40, ws_bytes=1 << 30, stream=None)
     a.update(kw)
     return lib.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["o"],
                              a["S_T"], a["B"], a["T"], a["H"], a["Dk"], a["Dv"], a["chunk"],
@@ -77,6 +77,7 @@ def _chunk(lib, **kw):
     (dict(chunk=48), 2), (dict(chunk=128), 2), (dict(Dk=272), 2), (dict(Dv=528), 2),
     (dict(q=24), 1), (dict(S_T=4100), 1),                 # misaligned pointers
     (dict(ws=None), 1), (dict(ws_bytes=64), 1),           # short workspace
+    (dict(ws=4096), 1), (dict(ws=32), 1),                 # workspace overlaps o / an input
     (dict(o=16), 1),                                      # output overlaps an input
     (dict(B=0), 0), (dict(H=0), 0),                       # empty: nothing to do
 ])

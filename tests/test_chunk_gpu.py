@@ -67,6 +67,29 @@ def test_gate_laws_bf16_small(gdn, gate_law):
     _full_check(gdn, I.chunk_inputs(w), 64, TOL_BF16)
 
 
+def test_tc_path_workspace(gdn):
+    # one bf16 [T'; T''] tile (128 x 64) per chunk of every (batch, head)
+    B, T, H = 2, 130, 3
+    assert gdn.chunk_fwd_path(B, T, H, 128, 128, 64, torch.bfloat16) == "tcgen05"
+    assert gdn.chunk_fwd_workspace_size(B, T, H, 128, 128, 64, torch.bfloat16) == \
+        B * H * 3 * 128 * 64 * 2
+
+
+def test_tc_path_ignores_workspace_contents(gdn):
+    # the workspace is scratch: garbage (NaN) on entry leaves the results unchanged
+    w = I.workload("bf16_T2k", B=1, H=2, T=200, s0_law="normal002", seed=11)
+    inp = I.chunk_inputs(w)
+    dev = {n: (t.cuda() if t is not None else None) for n, t in inp.items()}
+    need = gdn.chunk_fwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16)
+    outs = []
+    for fill in (0.0, float("nan")):
+        ws = torch.full((need // 4,), fill, dtype=torch.float32, device="cuda")
+        outs.append(gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                  dev["S0"], chunk=64, workspace=ws))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
 def test_chunk_size_invariance_f32(gdn):
     w = I.workload("tiny_f32", T=96, B=1, H=2, Dk=32, Dv=32, s0_law="normal002", seed=3)
     inp = I.chunk_inputs(w)
