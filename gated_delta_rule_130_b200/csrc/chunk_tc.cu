@@ -107,6 +107,7 @@ constexpr int DVT = 64;        // value channels per CTA
 constexpr int DK = 128;        // key channels
 constexpr int KB = DK / 64;    // 64-wide key blocks
 constexpr int NSTAGE = 2;
+constexpr int L2_AHEAD = 2;    // chunks between a tile's L2 prefetch and its shared-memory load
 constexpr int BLK = 8192;      // one 64 x 64 bf16 tile (64 rows of 128 bytes)
 constexpr int GRP = 3 * BLK;   // K | Q | W of one key block
 constexpr int STAGE = KB * GRP + 3 * BLK;  // + V tile + [T'; T''] (16 KiB)
@@ -654,6 +655,17 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tma_load_3d(st + OFF_TT, &tm_tt, cx.bar + B_IN_FULL + s, 0, 0,
                             ((int)b * H + h) * NT + c);
                 GDN_TRACE_AT(c, 24);
+                // the tiles of a later chunk start streaming from DRAM into L2 now,
+                // so that its shared-memory load, once a stage is free, hits L2
+                for (int cq = (c == 0 ? 1 : c + L2_AHEAD); cq <= c + L2_AHEAD && cq < NT; ++cq) {
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_prefetch_l2_4d(&tm_k, kb * 64, h, cq * C, b);
+                        tma_prefetch_l2_4d(&tm_q, kb * 64, h, cq * C, b);
+                    }
+                    tma_prefetch_l2_4d(&tm_v, v0, h, cq * C, b);
+                    tma_prefetch_l2_3d(&tm_tt, 0, 0, ((int)b * H + h) * NT + cq);
+                }
             }
             armed = c + 1;
             // running sums over rows lane (lo) and lane + 32 (hi); rows past the
@@ -709,14 +721,15 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == W_GMMA) {
         // ------------------------------------------------- MMA: Gram products
-        if (lane == 0) {
-            const uint32_t idesc_g = idesc_bf16(128, 64, false, false);
-            for (int c = 0; c < NT; ++c) {
-                const int s = c & 1;
-                const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
-                if (!wait_bar(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
-                if (c >= 1 && !wait_bar(cx, B_G_EMPTY, (c - 1) & 1)) break;
-                tc_fence_after();
+        // the whole warp waits (fast path: a test and a vote); lane 0 issues
+        const uint32_t idesc_g = idesc_bf16(128, 64, false, false);
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
+            if (!warp_wait(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
+            if (c >= 1 && !warp_wait(cx, B_G_EMPTY, (c - 1) & 1)) break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * GRP + (kk & 3) * 32;
@@ -726,17 +739,18 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_commit(cx.bar + B_G_FULL);
                 GDN_TRACE_AT(c, 8);
             }
+            __syncwarp();
         }
     } else if (warp == W_PMMA) {
         // --------------------------------------------------- MMA: WY products
-        if (lane == 0) {
-            const uint32_t idesc_wu = idesc_bf16(128, DK + DVT, false, true);
-            for (int c = 0; c < NT; ++c) {
-                const uint32_t st = smem_u32(base + SM_STAGE + (c & 1) * STAGE);
-                const uint32_t tt = st + OFF_TT;
-                if (!wait_bar(cx, B_IN_FULL + (c & 1), (c >> 1) & 1)) break;
-                if (c >= 1 && !wait_bar(cx, B_WU_EMPTY, (c - 1) & 1)) break;
-                tc_fence_after();
+        const uint32_t idesc_wu = idesc_bf16(128, DK + DVT, false, true);
+        for (int c = 0; c < NT; ++c) {
+            const uint32_t st = smem_u32(base + SM_STAGE + (c & 1) * STAGE);
+            const uint32_t tt = st + OFF_TT;
+            if (!warp_wait(cx, B_IN_FULL + (c & 1), (c >> 1) & 1)) break;
+            if (c >= 1 && !warp_wait(cx, B_WU_EMPTY, (c - 1) & 1)) break;
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + TM_WU, desc_sw128(tt + kk * 32, 16, 1024),
@@ -744,26 +758,27 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_commit(cx.bar + B_WU_FULL);
                 GDN_TRACE_AT(c, 9);
             }
+            __syncwarp();
         }
     } else if (warp == W_CHAIN) {
         // ---------------------------------------------- MMA: sequential chain
-        if (lane == 0) {
-            const uint32_t idesc_x = idesc_bf16(128, DVT, false, true);
-            const uint32_t idesc_y = idesc_bf16(128, DVT, false, true);
-            const uint32_t idesc_s = idesc_bf16(128, DVT, true, true);
-            const uint32_t sb = smem_u32(base + SM_SB), un = smem_u32(base + SM_UN),
-                           up = smem_u32(base + SM_UP);
-            for (int c = 0; c < NT; ++c) {
-                const int s = c & 1;
-                const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
-                if (!wait_bar(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
-                GDN_TRACE_AT(c, 5);
-                if (!wait_bar(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
-                GDN_TRACE_AT(c, 6);
-                if (!wait_bar(cx, B_S_READY, c & 1)) break;
-                GDN_TRACE_AT(c, 7);
-                tc_fence_after();
-                // X = [Q; W] S^T : A K-major (rows 0-63 Q, 64-127 W), B = S^T MN-major
+        const uint32_t idesc_x = idesc_bf16(128, DVT, false, true);
+        const uint32_t idesc_y = idesc_bf16(128, DVT, false, true);
+        const uint32_t idesc_s = idesc_bf16(128, DVT, true, true);
+        const uint32_t sb = smem_u32(base + SM_SB), un = smem_u32(base + SM_UN),
+                       up = smem_u32(base + SM_UP);
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
+            if (!warp_wait(cx, B_IN_FULL + s, (c >> 1) & 1)) break;
+            GDN_TRACE_WARP(c, 5, W_CHAIN);
+            if (!warp_wait(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
+            GDN_TRACE_WARP(c, 6, W_CHAIN);
+            if (!warp_wait(cx, B_S_READY, c & 1)) break;
+            GDN_TRACE_WARP(c, 7, W_CHAIN);
+            tc_fence_after();
+            // X = [Q; W] S^T : A K-major (rows 0-63 Q, 64-127 W), B = S^T MN-major
+            if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * GRP + (kk & 3) * 32;
@@ -772,9 +787,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 mma_commit(cx.bar + B_X_FULL);
                 GDN_TRACE_AT(c, 12);
-                if (!wait_bar(cx, B_U_READY, c & 1)) break;
-                GDN_TRACE_AT(c, 13);
-                tc_fence_after();
+            }
+            __syncwarp();
+            if (!warp_wait(cx, B_U_READY, c & 1)) break;
+            GDN_TRACE_WARP(c, 13, W_CHAIN);
+            tc_fence_after();
+            if (lane == 0) {
                 // S^T += K^T (decay U') : A = K^T (MN-major, key blocks GRP apart).
                 // Issued first: the next chunk waits on it.
 #pragma unroll
@@ -782,6 +800,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     mma_bf16(tmem + TM_ST, desc_sw128(st + OFF_K + kk * 2048, GRP, 1024),
                              desc_sw128(up + kk * 2048, 16, 1024), idesc_s, 1u);
                 mma_commit(cx.bar + B_ST_FULL);
+                // the stage (K, Q, W) is not read after MMA3 and MMA1
+                mma_commit(cx.bar + B_IN_EMPTY + s);
                 // Y += [P; *] U'  (Y holds diag(gamma) Q S^T; rows 64-127 of A unused)
                 const uint32_t pt = smem_u32(base + SM_PT + s * BLK);
 #pragma unroll
@@ -790,8 +810,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                              desc_sw128(un + kk * 2048, 16, 1024), idesc_y, 1u);
                 mma_commit(cx.bar + B_Y_FULL);
                 mma_commit(cx.bar + B_PT_EMPTY + s);
-                mma_commit(cx.bar + B_IN_EMPTY + s);
             }
+            __syncwarp();
         }
     } else if (warp < W_STATE0) {
         // ---------------------------------------------------------------- P
