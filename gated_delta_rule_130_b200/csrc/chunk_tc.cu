@@ -398,12 +398,11 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
                                             int p) {
     const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
     const auto blk = [&](float *M, int I, int J) { return M + 16 * I * LDA + 16 * J; };
-    constexpr int BI[6] = {1, 2, 2, 3, 3, 3}, BJ[6] = {0, 0, 1, 0, 1, 2};
 #pragma unroll
     for (int round = 0; round < 2; ++round) {
-        const int k = w + 4 * round;
+        const int k = w + 4 * round;  // block (I, J) in the order listed above
         if (k < 6) {
-            const int I = BI[k], J = BJ[k];
+            const int I = k == 0 ? 1 : (k < 3 ? 2 : 3), J = k == 0 ? 0 : (k < 3 ? k - 1 : k - 3);
             float acc[2][4] = {};
             mma16(acc, blk(TF, I, I), LDA, blk(AF, I, J), LDA, g, t);
             __syncwarp();
@@ -449,16 +448,14 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     float *g2s = reinterpret_cast<float *>(ut_smem + UT_SM_GT);
     float *bes = g2s + C, *bgs = g2s + 2 * C;
 
-    // K rows of the chunk (zeros past the end of the sequence): 16 x 16 B per row
+    // K rows of the chunk (zero-filled past the end of the sequence): 16 x 16 B per row
 #pragma unroll
     for (int m = 0; m < C * (DK / 8) / UT_THREADS; ++m) {
         const int idx = tid + UT_THREADS * m;
         const int r = idx / (DK / 8), piece = idx % (DK / 8);
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (t0 + r < T)
-            val = __ldg(reinterpret_cast<const uint4 *>(
-                k + (((size_t)b * T + t0 + r) * H + h) * DK + 8 * piece));
-        *reinterpret_cast<uint4 *>(Ks + r * LDK + 8 * piece) = val;
+        const bool in = t0 + r < T;
+        const __nv_bfloat16 *src = k + (((size_t)b * T + (in ? t0 + r : 0)) * H + h) * DK + 8 * piece;
+        cp_async16(Ks + r * LDK + 8 * piece, src, in ? 16u : 0u);
     }
     if (warp == 0) {
         // running sum of log alpha over rows lane and lane + 32, in log2 units
@@ -490,6 +487,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
             bgs[lane + 32 * hh] = be[hh] * ex2(g2);
         }
     }
+    cp_async_wait_all();
     __syncthreads();
 
     // Gram K K^T on and below the diagonal: warp w takes rows 16 w .. + 15 and the
@@ -498,21 +496,24 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     {
         const int RB = warp, ntiles = 2 * RB + 2;
         float acc[8][4] = {};
-        const __nv_bfloat16 *ar = Ks + (16 * RB + g) * LDK + 2 * t;
+        // ldmatrix row addresses: A (rows 16 RB.., matrices [rows 0-7 | 8-15] x
+        // [cols 0-7 | 8-15]) and B (a pair of 8-row tiles x [cols 0-7 | 8-15])
+        const int mi = lane >> 3, ri = lane & 7;
+        const __nv_bfloat16 *arow = Ks + (16 * RB + ri + 8 * (mi & 1)) * LDK + 8 * (mi >> 1);
+        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi >> 1)) * LDK + 8 * (mi & 1);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
             const int k0 = 16 * ks;
-            const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(ar + k0),
-                                   *reinterpret_cast<const uint32_t *>(ar + 8 * LDK + k0),
-                                   *reinterpret_cast<const uint32_t *>(ar + k0 + 8),
-                                   *reinterpret_cast<const uint32_t *>(ar + 8 * LDK + k0 + 8)};
+            uint32_t a[4];
+            ldmatrix_x4(a, arow + k0);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j < ntiles) {
-                    const __nv_bfloat16 *br = Ks + (8 * j + g) * LDK + k0 + 2 * t;
-                    const uint32_t bb[2] = {*reinterpret_cast<const uint32_t *>(br),
-                                            *reinterpret_cast<const uint32_t *>(br + 8)};
-                    mma_bf16_16x8x16(acc[j], a, bb);
+            for (int jp = 0; jp < 4; ++jp) {
+                if (2 * jp < ntiles) {
+                    uint32_t bq[4];
+                    ldmatrix_x4(bq, brow + 16 * jp * LDK + k0);
+                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+                    mma_bf16_16x8x16(acc[2 * jp], a, b0);
+                    mma_bf16_16x8x16(acc[2 * jp + 1], a, b1);
                 }
             }
         }
@@ -538,25 +539,19 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
 
     // [T'; T''] rows: T'(r, i) = T(r, i) beta_i gamma_i, T''(r, i) = T(r, i) beta_i
-    // for i <= r; thread -> (row, 8-column piece), 4 rows x 128 B per warp store
+    // for i <= r; thread -> (row, 4-column piece): 16 threads read one T row with
+    // no bank conflict and write its 128 bytes
     __nv_bfloat16 *dst = tt + ((size_t)((size_t)b * H + h) * NT + c) * TT_ELEMS;
-#pragma unroll
-    for (int m = 0; m < TT_ELEMS / 8 / UT_THREADS; ++m) {
+#pragma unroll 4
+    for (int m = 0; m < TT_ELEMS / 4 / UT_THREADS; ++m) {
         const int idx = tid + UT_THREADS * m;
-        const int rt = idx >> 3, i0 = 8 * (idx & 7), r = rt & (C - 1);
+        const int rt = idx >> 4, i0 = 4 * (idx & 15), r = rt & (C - 1);
         const float *sc = rt < C ? bgs : bes;
-        const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
-        const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
-        const float4 sa = *reinterpret_cast<const float4 *>(sc + i0);
-        const float4 sb = *reinterpret_cast<const float4 *>(sc + i0 + 4);
-        float x[8] = {ta.x * sa.x, ta.y * sa.y, ta.z * sa.z, ta.w * sa.w,
-                      tb.x * sb.x, tb.y * sb.y, tb.z * sb.z, tb.w * sb.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (i0 + j > r) x[j] = 0.f;
-        *reinterpret_cast<uint4 *>(dst + rt * C + i0) =
-            make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                       pack_bf16(x[6], x[7]));
+        const float4 tv = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
+        const float4 sv = *reinterpret_cast<const float4 *>(sc + i0);
+        const float x0 = i0 + 0 <= r ? tv.x * sv.x : 0.f, x1 = i0 + 1 <= r ? tv.y * sv.y : 0.f;
+        const float x2 = i0 + 2 <= r ? tv.z * sv.z : 0.f, x3 = i0 + 3 <= r ? tv.w * sv.w : 0.f;
+        *reinterpret_cast<uint2 *>(dst + rt * C + i0) = make_uint2(pack_bf16(x0, x1), pack_bf16(x2, x3));
     }
 }
 

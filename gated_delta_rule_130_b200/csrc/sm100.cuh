@@ -216,6 +216,26 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// 16-byte asynchronous global -> shared copy; bytes past src_bytes (0 or 16) are
+// zero-filled.  Completion: cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Four 8 x 8 bf16 matrices from shared memory; lane l gives the address of row
+// l % 8 of matrix l / 8 and receives, in r[m], elements 2 (l % 4) and 2 (l % 4) + 1
+// of row l / 4 of matrix m.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_ptr)));
+}
+
 // D (16 x 8, f32) += A (16 x 16, bf16, row-major) B (16 x 8, bf16, column-major).
 // Lane (g = lane / 4, t = lane % 4) holds a = {A[g][2t..], A[g+8][2t..],
 // A[g][2t+8..], A[g+8][2t+8..]} and b = {B[2t..][g], B[2t+8..][g]} as bf16
