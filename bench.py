@@ -318,58 +318,60 @@ def run_ours(args):
                        "frac": tflops / tc_peak, "flops": F,
                        "peak_source": f"{pk_kind} bf16_tflops (burst)"}}
 
-    # decode step: batch 256, H 16, d 128, 1000 steps, state resident in HBM
-    wd = I.workload("decode_b256")
-    S = I.decode_state(wd, device=device)
-    dec_in = [{n: t.to(device) for n, t in I.decode_step_inputs(wd, t).items()} for t in range(8)]
-    od = torch.empty((wd.B, wd.H, wd.Dv), dtype=wd.torch_dtype, device=device)
-    it = [0]
+    decode, e2e = None, None
+    if not args.chunk_only:  # (--chunk-only: the chunkwise step alone, for profiling)
+        # decode step: batch 256, H 16, d 128, 1000 steps, state resident in HBM
+        wd = I.workload("decode_b256")
+        S = I.decode_state(wd, device=device)
+        dec_in = [{n: t.to(device) for n, t in I.decode_step_inputs(wd, t).items()} for t in range(8)]
+        od = torch.empty((wd.B, wd.H, wd.Dv), dtype=wd.torch_dtype, device=device)
+        it = [0]
 
-    def dstep():
-        x = dec_in[it[0] % len(dec_in)]
-        it[0] += 1
-        G.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=od)
+        def dstep():
+            x = dec_in[it[0] % len(dec_in)]
+            it[0] += 1
+            G.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=od)
 
-    for _ in range(20):
-        dstep()
-    dms = time_loop(dstep, wd.steps, stream, world)
-    dms_max = _max_over_ranks(dms, world, device)
-    d_us = 1e3 * dms / wd.steps
-    d_gbs = decode_bytes(wd) / (d_us * 1e-6) / 1e9
-    decode = {"workload": f"decode_b256: batch={wd.B} H={wd.H} Dk={wd.Dk} Dv={wd.Dv} bf16 "
-                          f"q/k/v/o, f32 state in place, {wd.steps} steps",
-              "us_per_step": 1e3 * dms_max / wd.steps, "achieved": d_gbs, "unit": "GB/s",
-              "peak": hbm_peak, "frac": d_gbs / hbm_peak, "bytes_per_step": decode_bytes(wd),
-              "gpu_launches": wd.steps}
+        for _ in range(20):
+            dstep()
+        dms = time_loop(dstep, wd.steps, stream, world)
+        dms_max = _max_over_ranks(dms, world, device)
+        d_us = 1e3 * dms / wd.steps
+        d_gbs = decode_bytes(wd) / (d_us * 1e-6) / 1e9
+        decode = {"workload": f"decode_b256: batch={wd.B} H={wd.H} Dk={wd.Dk} Dv={wd.Dv} bf16 "
+                              f"q/k/v/o, f32 state in place, {wd.steps} steps",
+                  "us_per_step": 1e3 * dms_max / wd.steps, "achieved": d_gbs, "unit": "GB/s",
+                  "peak": hbm_peak, "frac": d_gbs / hbm_peak, "bytes_per_step": decode_bytes(wd),
+                  "gpu_launches": wd.steps}
 
-    # end to end through the public API with host buffers: pinned host inputs
-    # copied in, the call, o and S_T copied back, every step
-    host = {n: (t.pin_memory() if t is not None else None) for n, t in inp_cpu.items()}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    s_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
-    dev_bufs = {n: (torch.empty_like(t, device=device) if t is not None else None)
-                for n, t in host.items()}
+        # end to end through the public API with host buffers: pinned host inputs
+        # copied in, the call, o and S_T copied back, every step
+        host = {n: (t.pin_memory() if t is not None else None) for n, t in inp_cpu.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        s_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+        dev_bufs = {n: (torch.empty_like(t, device=device) if t is not None else None)
+                    for n, t in host.items()}
 
-    def e2e_step():
-        for n, t in host.items():
-            if t is not None:
-                dev_bufs[n].copy_(t, non_blocking=True)
-        G.chunk_fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["log_alpha"],
-                    dev_bufs["beta"], dev_bufs["S0"], chunk=w.chunk, out=o, S_T=S_T, workspace=ws)
-        o_h.copy_(o, non_blocking=True)
-        s_h.copy_(S_T, non_blocking=True)
+        def e2e_step():
+            for n, t in host.items():
+                if t is not None:
+                    dev_bufs[n].copy_(t, non_blocking=True)
+            G.chunk_fwd(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["log_alpha"],
+                        dev_bufs["beta"], dev_bufs["S0"], chunk=w.chunk, out=o, S_T=S_T, workspace=ws)
+            o_h.copy_(o, non_blocking=True)
+            s_h.copy_(S_T, non_blocking=True)
 
-    e2e_steps = max(3, min(steps, 30))
-    for _ in range(3):
-        e2e_step()
-    ems = _max_over_ranks(time_loop(e2e_step, e2e_steps, stream, world), world, device)
-    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
-    e2e = {"value": world * tokens / (ems / e2e_steps * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        e2e_steps = max(3, min(steps, 30))
+        for _ in range(3):
+            e2e_step()
+        ems = _max_over_ranks(time_loop(e2e_step, e2e_steps, stream, world), world, device)
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+        e2e = {"value": world * tokens / (ems / e2e_steps * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
 
     if rank == 0:
@@ -399,6 +401,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chunk-only", action="store_true",
+                    help="time the chunkwise forward only (no decode, end-to-end or CPU legs)")
     args = ap.parse_args()
     if args.impl == "reference":
         if args.steps is None:

@@ -438,6 +438,9 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
               const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt, int T, int H,
               int NT) {
     extern __shared__ __align__(16) uint8_t ut_smem[];
+    // the sequential kernel that follows on the stream may be scheduled now (it
+    // waits for this grid's completion before it reads the tiles)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -631,6 +634,9 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         };
         fetch_gates(0);
+        // the [T'; T''] tiles come from the UT kernel launched just before this
+        // one (programmatic dependent launch): wait for its completion first
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
             const int t0 = c * C;
@@ -1130,8 +1136,20 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
         static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, T, H, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
-    tc::gdn_chunk_tc_kernel<<<dim3(Dv / tc::DVT, H, B), tc::NTHREADS, tc::SMEM_BYTES, st>>>(
-        mq, mk, mv, mt, p);
+    // programmatic dependent launch: the CTAs may start (TMEM, barriers, the initial
+    // state) while the UT kernel drains; the TMA warp waits for it before loading
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Dv / tc::DVT, H, B);
+    cfg.blockDim = dim3(tc::NTHREADS);
+    cfg.dynamicSmemBytes = tc::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tc::gdn_chunk_tc_kernel, mq, mk, mv, mt, p);
+    if (e != cudaSuccess) return e;
     return cudaPeekAtLastError();
 }
 
