@@ -45,16 +45,16 @@ def peaks():
 
 
 def measured_traffic(path: str):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None if the kernel sources changed since the capture."""
+    """DRAM bytes of one call (both tcgen05-path kernels) from the committed ncu
+    summary, or None if the kernel sources changed since the capture."""
     import hashlib
-    f = os.path.join(ROOT, "profiles", "traffic_gdn_chunk_tc_kernel.txt")
+    f = os.path.join(ROOT, "profiles", "traffic_gdn_chunk_fwd_tc.txt")
     if path != "tcgen05" or not os.path.exists(f):
         return None
     value, ok = None, True
     for line in open(f):
         line = line.strip()
-        if line.startswith("dram_bytes_per_launch:"):
+        if line.startswith("dram_bytes_per_call:"):
             value = float(line.split(":", 1)[1])
         elif line.startswith("sha256 "):
             rel, digest = line[len("sha256 "):].split(":", 1)
