@@ -43,6 +43,14 @@ def _load():
     lib.gdn_chunk_fwd_path.restype = I
     lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, vp]
     lib.gdn_decode_step.restype = I
+    U = ctypes.c_uint
+    lib.gdn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, I, U, vp,
+                                     Z, vp]
+    lib.gdn_chunk_fwd_ex.restype = I
+    lib.gdn_chunk_fwd_workspace_size_ex.argtypes = [I, I, I, I, I, I, I, U]
+    lib.gdn_chunk_fwd_workspace_size_ex.restype = Z
+    lib.gdn_decode_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, U, vp]
+    lib.gdn_decode_step_ex.restype = I
     lib.gdn_check_device_status.argtypes = []
     lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]
@@ -87,9 +95,20 @@ def check_device_status():
     _check(int(LIB.gdn_check_device_status()), "gdn_check_device_status")
 
 
-def chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> int:
+# Input prologue flags of the _ex entry points (gdn_flag_t in include/gdn.h).
+GDN_FLAG_L2NORM_QK = 1
+GDN_FLAG_GATE_LOGITS = 2
+
+
+def _flags(l2norm_qk: bool, gate_logits: bool) -> int:
+    return (GDN_FLAG_L2NORM_QK if l2norm_qk else 0) | (GDN_FLAG_GATE_LOGITS if gate_logits else 0)
+
+
+def chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16,
+                             l2norm_qk: bool = False, gate_logits: bool = False) -> int:
     code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
-    return int(LIB.gdn_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+    return int(LIB.gdn_chunk_fwd_workspace_size_ex(B, T, H, Dk, Dv, chunk, code,
+                                                   _flags(l2norm_qk, gate_logits)))
 
 
 def chunk_fwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
@@ -101,13 +120,18 @@ def chunk_fwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=None,
-              return_state: bool = True, workspace=None):
+              return_state: bool = True, workspace=None, l2norm_qk: bool = False,
+              gate_logits: bool = False):
     """Chunkwise forward: returns (o [B,T,H,Dv], S_T [B,H,Dv,Dk] float32 or None).
 
     q, k [B,T,H,Dk] and v [B,T,H,Dv] in float32 or bfloat16 (same type);
     log_alpha, beta [B,T,H] float32; S0 [B,H,Dv,Dk] float32 or None (zeros).
     ``S_T`` may be passed (and may be ``S0`` itself for in-place continuation).
+    ``l2norm_qk``: q and k are raw and get normalised per token and head in the
+    kernels; ``gate_logits``: log_alpha and beta hold logits (log alpha =
+    -softplus(x), beta = sigmoid(y)).
     """
+    flags = _flags(l2norm_qk, gate_logits)
     if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
         raise GdnError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
     B, T, H, Dk = q.shape
@@ -137,22 +161,25 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=
         args.append(_dev(S_T, "S_T", torch.float32, dev))
     else:
         args.append(None)
-    need = int(LIB.gdn_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+    need = int(LIB.gdn_chunk_fwd_workspace_size_ex(B, T, H, Dk, Dv, chunk, code, flags))
     ws_ptr, ws_bytes = None, 0
     if need:
         if workspace is None or workspace.numel() * workspace.element_size() < need:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    st = LIB.gdn_chunk_fwd(*args, B, T, H, Dk, Dv, chunk, code, ws_ptr, ws_bytes, _stream_ptr(dev))
+    st = LIB.gdn_chunk_fwd_ex(*args, B, T, H, Dk, Dv, chunk, code, flags, ws_ptr, ws_bytes,
+                              _stream_ptr(dev))
     _check(st, "gdn_chunk_fwd")
     return o, S_T
 
 
-def decode_step(q, k, v, log_alpha, beta, S, out=None):
+def decode_step(q, k, v, log_alpha, beta, S, out=None, l2norm_qk: bool = False,
+                gate_logits: bool = False):
     """One recurrent step for every (b,h); S [B,H,Dv,Dk] float32 is updated in place.
 
     q, k [B,H,Dk], v [B,H,Dv] float32 or bfloat16; log_alpha, beta [B,H] float32.
-    Returns o [B,H,Dv] in q's dtype.
+    Returns o [B,H,Dv] in q's dtype.  ``l2norm_qk`` / ``gate_logits``: the input
+    prologue, as in ``chunk_fwd``.
     """
     if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
         raise GdnError("q, k must be [B,H,Dk] and v [B,H,Dv]")
@@ -163,10 +190,10 @@ def decode_step(q, k, v, log_alpha, beta, S, out=None):
     if log_alpha.shape != (B, H) or beta.shape != (B, H) or S.shape != (B, H, Dv, Dk):
         raise GdnError("log_alpha, beta must be [B,H] and S [B,H,Dv,Dk]")
     o = out if out is not None else torch.empty((B, H, Dv), dtype=q.dtype, device=dev)
-    st = LIB.gdn_decode_step(
+    st = LIB.gdn_decode_step_ex(
         _dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
         _dev(log_alpha, "log_alpha", torch.float32, dev), _dev(beta, "beta", torch.float32, dev),
         _dev(S, "S", torch.float32, dev), _dev(o, "out", q.dtype, dev), B, H, Dk, Dv, code,
-        _stream_ptr(dev))
+        _flags(l2norm_qk, gate_logits), _stream_ptr(dev))
     _check(st, "gdn_decode_step")
     return o

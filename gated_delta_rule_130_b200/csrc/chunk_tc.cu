@@ -122,7 +122,9 @@ constexpr int GV_DCY = 192;    // exp(g_last - g_r)
 constexpr int GV_U = 256;      // exp(g_r - g_{16 R(r)})            (R(r) = r / 16)
 constexpr int GV_W = 320;      // [R][i]: exp(g_{16R} - g_i) for i < 16R, else 0
 constexpr int GV_GL = 576;     // gamma_last = exp(g_last)
-constexpr int GV_STRIDE = 640;
+constexpr int GV_RK = 640;     // 1/|k_r| (1 unless q and k are L2-normalised in the kernel)
+constexpr int GV_RQ = 704;     // 1/|q_r| (written by the P warps)
+constexpr int GV_STRIDE = 768;
 
 // shared-memory map (bytes from the 1024-aligned base)
 constexpr int SM_STAGE = 0;
@@ -383,8 +385,8 @@ constexpr int UT_THREADS = 128;
 constexpr int LDK = DK + 8;                        // bf16 row stride of the staged K chunk
 constexpr int UT_SM_KT = 0;                        // K chunk (64 x LDK bf16), then T (64 x LDA f32)
 constexpr int UT_SM_AF = C * LDA * 4;              // A (64 x LDA f32); N_IJ overwrite A_IJ
-constexpr int UT_SM_GT = UT_SM_AF + C * LDA * 4;   // g log2(e), beta, beta gamma (3 x 64)
-constexpr int UT_SMEM = UT_SM_GT + 3 * C * 4;
+constexpr int UT_SM_GT = UT_SM_AF + C * LDA * 4;   // g log2(e), beta, beta gamma |k|^-1, |k|^-1
+constexpr int UT_SMEM = UT_SM_GT + 4 * C * 4;
 constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
 static_assert(C * LDK * 2 <= UT_SM_AF, "K chunk fits in the T buffer");
 static_assert(UT_SM_AF % 16 == 0 && UT_SM_GT % 16 == 0, "16-byte aligned UT buffers");
@@ -435,8 +437,8 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
 
 __global__ void __launch_bounds__(UT_THREADS, 6)
 gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
-              const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt, int T, int H,
-              int NT) {
+              const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt,
+              float *__restrict__ rk_out, int T, int H, int NT, unsigned flags) {
     extern __shared__ __align__(16) uint8_t ut_smem[];
     // the sequential kernel that follows on the stream may be scheduled now (it
     // waits for this grid's completion before it reads the tiles)
@@ -449,7 +451,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     float *TF = reinterpret_cast<float *>(ut_smem + UT_SM_KT);
     float *AF = reinterpret_cast<float *>(ut_smem + UT_SM_AF);
     float *g2s = reinterpret_cast<float *>(ut_smem + UT_SM_GT);
-    float *bes = g2s + C, *bgs = g2s + 2 * C;
+    float *bes = g2s + C, *bgs = g2s + 2 * C, *rks = g2s + 3 * C;
 
     // K rows of the chunk (zero-filled past the end of the sequence): 16 x 16 B per row
 #pragma unroll
@@ -469,8 +471,9 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
             const int r = lane + 32 * hh;
             const bool in = t0 + r < T;
             const size_t gi = ((size_t)b * T + t0 + r) * H + h;
-            la[hh] = in ? log_alpha[gi] : 0.f;
-            be[hh] = in ? beta[gi] : 0.f;
+            const float2 gp = in ? gate_pair(log_alpha[gi], beta[gi], flags) : make_float2(0.f, 0.f);
+            la[hh] = gp.x;
+            be[hh] = gp.y;
         }
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -491,6 +494,33 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
         }
     }
     cp_async_wait_all();
+    __syncthreads();
+    // 1/|k_r| per row (two threads a row), folded into the Gram rows and the
+    // columns of T'; kept in the workspace for the sequential kernel
+    if (flags & kFlagL2Norm) {
+        const int r = tid >> 1, half = tid & 1;
+        const uint4 *row = reinterpret_cast<const uint4 *>(Ks + r * LDK + 64 * half);
+        float ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint4 u = row[m];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                ss += f.x * f.x + f.y * f.y;
+            }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (half == 0) {
+            const float rkv = rsqrtf(ss + kNormEps);
+            rks[r] = rkv;
+            bgs[r] *= rkv;
+            rk_out[((size_t)((size_t)b * H + h) * NT + c) * C + r] = rkv;
+        }
+    } else if (tid < C) {
+        rks[tid] = 1.f;
+    }
     __syncthreads();
 
     // Gram K K^T on and below the diagonal: warp w takes rows 16 w .. + 15 and the
@@ -523,14 +553,16 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int r = 16 * RB + g + 8 * hr;
-            const float gr = g2s[r], br = bes[r];
+            const float gr = g2s[r], br = bes[r] * rks[r];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (j < ntiles) {
                     const int i = 8 * j + 2 * t;
-                    const float a0 = (i < r) ? br * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
-                    const float a1 =
-                        (i + 1 < r) ? br * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1] : 0.f;
+                    const float a0 =
+                        (i < r) ? br * rks[i] * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
+                    const float a1 = (i + 1 < r)
+                                         ? br * rks[i + 1] * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1]
+                                         : 0.f;
                     *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
                 }
             }
@@ -541,7 +573,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     __syncthreads();
     ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
 
-    // [T'; T''] rows: T'(r, i) = T(r, i) beta_i gamma_i, T''(r, i) = T(r, i) beta_i
+    // [T'; T''] rows: T'(r, i) = T(r, i) beta_i gamma_i / |k_i|, T''(r, i) = T(r, i) beta_i
     // for i <= r; thread -> (row, 4-column piece): 16 threads read one T row with
     // no bank conflict and write its 128 bytes
     __nv_bfloat16 *dst = tt + ((size_t)((size_t)b * H + h) * NT + c) * TT_ELEMS;
@@ -564,7 +596,9 @@ struct Params {
     const float *S0;
     __nv_bfloat16 *o;
     float *S_T;
+    const float *rk;       // 1/|k| per token from the UT kernel (L2-normalising only)
     int T, H, Dv, NT;
+    unsigned flags;        // input prologue (kFlagL2Norm, kFlagGateLogits)
 };
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -622,7 +656,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // after the vectors are written).
         constexpr float LOG2E = 1.4426950408889634f;
         int armed = 0;
-        float nla[2], nbe[2];  // gate values of the next chunk (rows lane, lane + 32)
+        float nla[2], nbe[2], nrk[2];  // gate values of the next chunk (rows lane, lane + 32)
+        const bool l2n = (p.flags & kFlagL2Norm) != 0;
         const auto fetch_gates = [&](int cc) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -631,16 +666,26 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const size_t gi = ((size_t)b * T + cc * C + r) * H + h;
                 nla[hh] = in ? p.log_alpha[gi] : 0.f;
                 nbe[hh] = in ? p.beta[gi] : 0.f;
+                nrk[hh] = l2n ? p.rk[((size_t)((size_t)b * H + h) * NT + cc) * C + r] : 1.f;
             }
         };
-        fetch_gates(0);
-        // the [T'; T''] tiles come from the UT kernel launched just before this
-        // one (programmatic dependent launch): wait for its completion first
+        // the [T'; T''] tiles (and 1/|k|) come from the UT kernel launched just
+        // before this one (programmatic dependent launch): wait for its completion
         asm volatile("griddepcontrol.wait;" ::: "memory");
+        fetch_gates(0);
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
             const int t0 = c * C;
-            float la[2] = {nla[0], nla[1]}, be[2] = {nbe[0], nbe[1]};
+            float la[2], be[2];
+            const float rk2[2] = {nrk[0], nrk[1]};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                // rows past the end keep log alpha = beta = 0
+                const bool in = t0 + lane + 32 * hh < T;
+                const float2 gp = in ? gate_pair(nla[hh], nbe[hh], p.flags) : make_float2(0.f, 0.f);
+                la[hh] = gp.x;
+                be[hh] = gp.y;
+            }
             if (c + 1 < NT) fetch_gates(c + 1);
             if (c >= 2 && !warp_wait(cx, B_IN_EMPTY + s, ((c - 2) >> 1) & 1)) break;
             GDN_TRACE_WARP(c, 31, W_TMA);
@@ -693,6 +738,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             gv[GV_G2 + 32 + lane] = g1;
             gv[GV_BETA + lane] = be[0];
             gv[GV_BETA + 32 + lane] = be[1];
+            gv[GV_RK + lane] = rk2[0];
+            gv[GV_RK + 32 + lane] = rk2[1];
             gv[GV_GAM + lane] = ex2(g0);
             gv[GV_GAM + 32 + lane] = ex2(g1);
             gv[GV_DCY + lane] = ex2(glast - g0);
@@ -848,6 +895,37 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 gated_piece<false>(v0, hf, r, su, gv + GV_G2, gv + GV_W);
                 gated_piece<true>(v1, hf + 2, r, su, gv + GV_G2, gv + GV_W);
             }
+            if (p.flags & kFlagL2Norm) {
+                // P_ri = Gamma_ri (q_r . k_i) / (|q_r| |k_i|): 1/|q_r| from this row of
+                // the chunk's Q tile (both key blocks, 128-byte swizzled rows), 1/|k_i|
+                // from the gate vectors; the twin warp computes the same row norm
+                const uint8_t *st = base + SM_STAGE + s * STAGE;
+                float ss = 0.f;
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(
+                            st + kb * GRP + OFF_Q + sw128_offset(r, 16 * m));
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f =
+                                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                            ss += f.x * f.x + f.y * f.y;
+                        }
+                    }
+                }
+                const float rq = rsqrtf(ss + kNormEps);
+                if (hf == 0) gv_all[s * GV_STRIDE + GV_RQ + r] = rq;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    v0[j] *= rq * gv[GV_RK + 16 * hf + j];
+                    v1[j] *= rq * gv[GV_RK + 16 * (hf + 2) + j];
+                }
+            } else if (hf == 0) {
+                gv_all[s * GV_STRIDE + GV_RQ + r] = 1.f;
+            }
             GDN_TRACE_WARP(c, 28, 2);
             store16_bf16(base + SM_PT + s * BLK, r, hf, v0);
             store16_bf16(base + SM_PT + s * BLK, r, hf + 2, v1);
@@ -924,7 +1002,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (q >= 2) {
                 // U' = U - W S^T for chunk row r -> U' and diag(exp(g_last - g)) U' (bf16)
                 const int r = lrow - 64;
-                const float dc = gv[GV_DCY + r];
+                // K enters the state update normalised: scale U' rows by 1/|k_r| too
+                const float dc = gv[GV_DCY + r] * gv[GV_RK + r];
                 float x0[16], x1[16], u0[16], u1[16];
                 tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
                 tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
@@ -953,7 +1032,9 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             } else {
                 // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y; the
                 // intra-chunk MMA accumulates onto it
-                const float gr = gv[GV_GAM + lrow];
+                // 1/|q_r| comes from the P warps (published with this chunk's P tile)
+                if ((p.flags & kFlagL2Norm) && !warp_wait(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
+                const float gr = gv[GV_GAM + lrow] * gv[GV_RQ + lrow];
                 float x0[16], x1[16];
                 tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
                 tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
@@ -1096,9 +1177,10 @@ bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 
 }  // namespace tc
 
-size_t tc_workspace_bytes(int B, int T, int H) {
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags) {
     const size_t NT = ((size_t)T + tc::C - 1) / tc::C;
-    return (size_t)B * H * NT * tc::TT_ELEMS * sizeof(__nv_bfloat16);
+    const size_t tiles = (size_t)B * H * NT * tc::TT_ELEMS * sizeof(__nv_bfloat16);
+    return tiles + ((flags & kFlagL2Norm) ? (size_t)B * H * NT * tc::C * sizeof(float) : 0);
 }
 
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
@@ -1108,9 +1190,13 @@ bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
-                            int H, int Dk, int Dv, void *workspace, cudaStream_t st) {
+                            int H, int Dk, int Dv, unsigned flags, void *workspace,
+                            cudaStream_t st) {
     const int NT = (T + tc::C - 1) / tc::C;
     auto *tt = static_cast<__nv_bfloat16 *>(workspace);
+    float *rk = (flags & kFlagL2Norm)
+                    ? reinterpret_cast<float *>(tt + (size_t)B * H * NT * tc::TT_ELEMS)
+                    : nullptr;
     CUtensorMap mq, mk, mv, mt;
     if (!tc::make_map(&mq, q, B, T, H, Dk) || !tc::make_map(&mk, k, B, T, H, Dk) ||
         !tc::make_map(&mv, v, B, T, H, Dv) ||
@@ -1126,6 +1212,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     p.H = H;
     p.Dv = Dv;
     p.NT = NT;
+    p.rk = rk;
+    p.flags = flags;
     cudaError_t e = cudaFuncSetAttribute(tc::gdn_ut_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::UT_SMEM);
     if (e != cudaSuccess) return e;
@@ -1133,7 +1221,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                              tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     tc::gdn_ut_kernel<<<dim3(NT, H, B), tc::UT_THREADS, tc::UT_SMEM, st>>>(
-        static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, T, H, NT);
+        static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, rk, T, H, NT, flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the CTAs may start (TMEM, barriers, the initial

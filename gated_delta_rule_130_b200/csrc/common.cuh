@@ -31,4 +31,23 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// Optional input prologue (gdn_flag_t bits of the _ex entry points): q and k
+// divided by sqrt(|x|^2 + kNormEps) per token and head; gates given as logits,
+// log alpha = -softplus(x), beta = sigmoid(y).
+constexpr unsigned kFlagL2Norm = 1u, kFlagGateLogits = 2u;
+constexpr float kNormEps = 1e-6f;
+
+// -softplus(x) = -(max(x, 0) + log(1 + e^-|x|)): no overflow on either side.
+__device__ __forceinline__ float neg_softplus(float x) {
+    return -(fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+}
+// 1 / (1 + e^-y); saturates to 0 or 1 without producing NaN.
+__device__ __forceinline__ float sigmoid(float y) { return 1.f / (1.f + expf(-y)); }
+
+// The gate pair of one token and head as the kernels use it: (log alpha, beta).
+__device__ __forceinline__ float2 gate_pair(float la, float be, unsigned flags) {
+    return (flags & kFlagGateLogits) ? make_float2(neg_softplus(la), sigmoid(be))
+                                     : make_float2(la, be);
+}
+
 }  // namespace gdn

@@ -31,6 +31,9 @@ gdn_status_t check_sizes(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dty
 
 bool empty_problem(int B, int T, int H) { return B == 0 || H == 0 || T == 0; }
 
+constexpr unsigned kKnownFlags = GDN_FLAG_L2NORM_QK | GDN_FLAG_GATE_LOGITS;
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
 }  // namespace
 
 extern "C" {
@@ -52,20 +55,40 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype
     return GDN_PATH_SIMT;
 }
 
+size_t gdn_chunk_fwd_workspace_size_ex(int B, int T, int H, int Dk, int Dv, int chunk,
+                                       gdn_dtype_t dtype, unsigned flags) {
+    const int path = gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype);
+    if (flags & ~kKnownFlags) return 0;
+    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H, flags);
+    if (path == GDN_PATH_SIMT) {
+        const size_t base = gdn::simt_workspace_bytes(B, T, H, chunk);
+        return flags ? align256(base) + gdn::prologue_bytes(B, T, H, Dk, dtype == GDN_BF16, flags)
+                     : base;
+    }
+    return 0;
+}
+
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
                                     gdn_dtype_t dtype) {
-    const int path = gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype);
-    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H);
-    if (path == GDN_PATH_SIMT) return gdn::simt_workspace_bytes(B, T, H, chunk);
-    return 0;
+    return gdn_chunk_fwd_workspace_size_ex(B, T, H, Dk, Dv, chunk, dtype, 0u);
 }
 
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
                            const float *beta, const float *S0, void *o, float *S_T, int B, int T,
                            int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype, void *workspace,
                            size_t workspace_bytes, void *stream) {
+    return gdn_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, dtype,
+                            0u, workspace, workspace_bytes, stream);
+}
+
+gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta, const float *S0, void *o,
+                              float *S_T, int B, int T, int H, int Dk, int Dv, int chunk,
+                              gdn_dtype_t dtype, unsigned flags, void *workspace,
+                              size_t workspace_bytes, void *stream) {
     const gdn_status_t sz = check_sizes(B, T, H, Dk, Dv, chunk, dtype);
     if (sz != GDN_OK) return sz;
+    if (flags & ~kKnownFlags) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t esz = dtype == GDN_BF16 ? 2 : 4;
     const size_t n_tok = (size_t)B * T * H;
@@ -93,8 +116,7 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
 
     const bool bf16 = dtype == GDN_BF16;
     const bool tc = gdn::tc_supported(B, T, H, Dk, Dv, chunk, bf16);
-    const size_t need = tc ? gdn::tc_workspace_bytes(B, T, H)
-                           : gdn::simt_workspace_bytes(B, T, H, chunk);
+    const size_t need = gdn_chunk_fwd_workspace_size_ex(B, T, H, Dk, Dv, chunk, dtype, flags);
     if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
     // the workspace is scratch written by the kernels: it must not alias anything else
     if (overlaps(workspace, need, q, n_tok * Dk * esz) ||
@@ -108,11 +130,20 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
         return GDN_ERR_INVALID_ARG;
     cudaError_t e;
     if (tc) {
-        e = gdn::launch_chunk_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, workspace,
-                                 st);
+        e = gdn::launch_chunk_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, flags,
+                                 workspace, st);
     } else {
-        e = gdn::launch_chunk_simt(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk,
-                                   bf16, workspace, st);
+        // the prologue's output sits after the CUDA-core path's own scratch
+        gdn::Prepared in{q, k, log_alpha, beta};
+        e = cudaSuccess;
+        if (flags)
+            e = gdn::launch_prologue(
+                q, k, log_alpha, beta, B, T, H, Dk, bf16, flags,
+                static_cast<uint8_t *>(workspace) + align256(gdn::simt_workspace_bytes(B, T, H, chunk)),
+                &in, st);
+        if (e == cudaSuccess)
+            e = gdn::launch_chunk_simt(in.q, in.k, v, in.log_alpha, in.beta, S0, o, S_T, B, T, H,
+                                       Dk, Dv, chunk, bf16, workspace, st);
     }
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -127,7 +158,15 @@ gdn_status_t gdn_check_device_status(void) {
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                              const float *beta, float *S, void *o, int B, int H, int Dk, int Dv,
                              gdn_dtype_t dtype, void *stream) {
+    return gdn_decode_step_ex(q, k, v, log_alpha, beta, S, o, B, H, Dk, Dv, dtype, 0u, stream);
+}
+
+gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, float *S, void *o,
+                                int B, int H, int Dk, int Dv, gdn_dtype_t dtype, unsigned flags,
+                                void *stream) {
     if (B < 0 || H < 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (flags & ~kKnownFlags) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (Dk > kMaxDk || Dv > kMaxDv) return GDN_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return GDN_OK;
@@ -140,7 +179,8 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const 
     if (overlaps(o, heads * Dv * esz, S, heads * Dv * Dk * sizeof(float)))
         return GDN_ERR_INVALID_ARG;
     const cudaError_t e = gdn::launch_decode(q, k, v, log_alpha, beta, S, o, B, H, Dk, Dv,
-                                             dtype == GDN_BF16, static_cast<cudaStream_t>(stream));
+                                             dtype == GDN_BF16, flags,
+                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

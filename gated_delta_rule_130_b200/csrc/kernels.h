@@ -9,9 +9,22 @@
 namespace gdn {
 
 // Recurrent step over every (b,h): decode.cu.
+// (flags: input prologue bits, see common.cuh.)
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *o, int B, int H, int Dk, int Dv,
-                          bool bf16, cudaStream_t st);
+                          bool bf16, unsigned flags, cudaStream_t st);
+
+// Input prologue for the CUDA-core path: prologue.cu.  Writes the prepared q, k
+// (if L2-normalising) and gates (if given as logits) into `ws` and points `out`
+// at the arrays to use (the originals where the flags leave them alone).
+struct Prepared {
+    const void *q, *k;
+    const float *log_alpha, *beta;
+};
+size_t prologue_bytes(int B, int T, int H, int Dk, bool bf16, unsigned flags);
+cudaError_t launch_prologue(const void *q, const void *k, const float *la, const float *be,
+                            int B, int T, int H, int Dk, bool bf16, unsigned flags, void *ws,
+                            Prepared *out, cudaStream_t st);
 
 // CUDA-core chunkwise forward (any supported size, f32 or bf16): chunk_simt.cu.
 size_t simt_workspace_bytes(int B, int T, int H, int chunk);
@@ -22,11 +35,13 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
 
 // tcgen05 chunkwise forward (bf16, Dk = 128, chunk 64): chunk_tc.cu.  The
 // workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of every head.
+// With the L2-normalisation flag the workspace also holds 1/|k| per token.
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
-size_t tc_workspace_bytes(int B, int T, int H);
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags);
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
-                            int H, int Dk, int Dv, void *workspace, cudaStream_t st);
+                            int H, int Dk, int Dv, unsigned flags, void *workspace,
+                            cudaStream_t st);
 
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).

@@ -103,6 +103,42 @@ def chunk_inputs(w: Workload, seed: int | None = None, device="cpu"):
     return out
 
 
+def raw_chunk_inputs(w: Workload, seed: int | None = None, device="cpu"):
+    """Inputs for the library's optional input prologue (per-token L2 normalisation
+    of q and k, gate activations): q, k ~ 2 N(0,1) rounded to the dtype and NOT
+    normalised; v as in ``chunk_inputs``; the two gate arrays hold logits ~ N(0,1)
+    (decay logit in ``log_alpha``, write logit in ``beta``); S0 per the workload."""
+    gen = torch.Generator().manual_seed((w.seed if seed is None else seed) + 500_000)
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    q = (2.0 * torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    k = (2.0 * torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    v = torch.randn((B, T, H, Dv), generator=gen).to(w.torch_dtype)
+    x = torch.randn((B, T, H), generator=gen)
+    y = torch.randn((B, T, H), generator=gen)
+    S0 = None
+    if w.s0_law == "normal002":
+        S0 = 0.02 * torch.randn((B, H, Dv, Dk), generator=gen)
+    out = dict(q=q, k=k, v=v, log_alpha=x, beta=y, S0=S0)
+    if device != "cpu":
+        out = {n: (t.to(device) if t is not None else None) for n, t in out.items()}
+    return out
+
+
+def raw_decode_step_inputs(w: Workload, step: int, device="cpu"):
+    """Token ``step`` of a decode run for the input prologue: raw q, k (2 N(0,1)),
+    v, and the decay / write logits ~ N(0,1) in ``log_alpha`` / ``beta``."""
+    gen = torch.Generator().manual_seed(w.seed * 1_000_003 + step + 7_000_001)
+    B, H, Dk, Dv = w.B, w.H, w.Dk, w.Dv
+    q = (2.0 * torch.randn((B, H, Dk), generator=gen)).to(w.torch_dtype)
+    k = (2.0 * torch.randn((B, H, Dk), generator=gen)).to(w.torch_dtype)
+    v = torch.randn((B, H, Dv), generator=gen).to(w.torch_dtype)
+    out = dict(q=q, k=k, v=v, log_alpha=torch.randn((B, H), generator=gen),
+               beta=torch.randn((B, H), generator=gen))
+    if device != "cpu":
+        out = {n: t.to(device) for n, t in out.items()}
+    return out
+
+
 def decode_state(w: Workload, device="cpu"):
     """Initial decode state S0 [B,H,Dv,Dk] f32."""
     gen = torch.Generator().manual_seed(w.seed)

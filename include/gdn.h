@@ -72,6 +72,23 @@ typedef enum {
  * (a zero size is an empty problem and is not an error). */
 
 /*
+ * Optional input prologue of the _ex entry points, applied inside the kernels
+ * (bit flags, may be combined).  The pages fix neither a normalisation of q and
+ * k nor a parameterisation of the gates; these are the plain readings (exact
+ * write-over S_t k_t = v_t, the "Critical Insight" section of "Gated DeltaNet:
+ * Harmonizing Gating and the Delta Rule ...", holds for unit keys):
+ *   GDN_FLAG_L2NORM_QK   q and k are divided by sqrt(|x|^2 + 1e-6), per token
+ *                        and head, before use (the caller passes raw q, k);
+ *   GDN_FLAG_GATE_LOGITS log_alpha holds a logit x and beta a logit y:
+ *                        log alpha = -softplus(x) = -log(1 + e^x), beta = 1 / (1 + e^-y).
+ */
+typedef enum {
+    GDN_FLAG_NONE = 0,
+    GDN_FLAG_L2NORM_QK = 1,
+    GDN_FLAG_GATE_LOGITS = 2
+} gdn_flag_t;
+
+/*
  * Chunkwise forward over a whole sequence (training / prefill form).
  *
  * Each sequence is cut into chunks of `chunk` tokens (the last one may be
@@ -105,6 +122,23 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v,
  * (batch, head), on the CUDA-core path (2 chunk^2 + chunk) floats per chunk. */
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int Dk, int Dv,
                                     int chunk, gdn_dtype_t dtype);
+
+/*
+ * gdn_chunk_fwd with the input prologue selected by `flags` (gdn_flag_t bits;
+ * 0 is exactly gdn_chunk_fwd).  q, k, log_alpha and beta are read as the flags
+ * say and are not modified.  The workspace must hold
+ * gdn_chunk_fwd_workspace_size_ex(..., flags) bytes (the tensor-core path keeps
+ * 1/|k| per token there, the CUDA-core path the prepared inputs).  Unknown flag
+ * bits: GDN_ERR_INVALID_ARG.
+ */
+gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              const float *S0, void *o, float *S_T,
+                              int B, int T, int H, int Dk, int Dv, int chunk,
+                              gdn_dtype_t dtype, unsigned flags, void *workspace,
+                              size_t workspace_bytes, void *stream);
+size_t gdn_chunk_fwd_workspace_size_ex(int B, int T, int H, int Dk, int Dv,
+                                       int chunk, gdn_dtype_t dtype, unsigned flags);
 
 /* The path gdn_chunk_fwd takes for these sizes (a gdn_path_t), or -1 if the
  * sizes are invalid or unsupported. */
@@ -146,6 +180,13 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v,
                              const float *log_alpha, const float *beta,
                              float *S, void *o, int B, int H, int Dk, int Dv,
                              gdn_dtype_t dtype, void *stream);
+
+/* gdn_decode_step with the input prologue selected by `flags` (gdn_flag_t bits,
+ * applied in the kernel; 0 is exactly gdn_decode_step). */
+gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                float *S, void *o, int B, int H, int Dk, int Dv,
+                                gdn_dtype_t dtype, unsigned flags, void *stream);
 
 /*
  * Synchronise the current device and report whether a fused tensor-core

@@ -108,3 +108,30 @@ def test_binding_fails_loudly_without_library(tmp_path):
             "    print('RAISED', e)\n") % str(tmp_path)
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, timeout=120)
     assert "RAISED" in out.stdout and "libgdn.so not found" in out.stdout
+
+
+def test_prologue_flags_checked_before_launch(lib):
+    # unknown flag bits are rejected on the host (nothing is dereferenced)
+    f = lib.gdn_chunk_fwd_ex
+    f.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 7 + [ctypes.c_uint, ctypes.c_void_p,
+                                                                 ctypes.c_size_t, ctypes.c_void_p]
+    assert f(16, 16, 16, 16, 16, None, 4096, None, 1, 8, 1, 16, 16, 16, 0, 4, 1 << 40, 1 << 30,
+             None) == 1
+    d = lib.gdn_decode_step_ex
+    d.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int] * 5 + [ctypes.c_uint, ctypes.c_void_p]
+    assert d(16, 16, 16, 16, 16, 1 << 20, 16, 2, 2, 16, 16, 1, 8, None) == 1
+    assert d(16, 16, 16, 16, 16, 1 << 20, 16, 0, 2, 16, 16, 1, 3, None) == 0  # empty: nothing to do
+
+
+def test_prologue_workspace_size_on_the_cuda_core_path(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    C, NT, rows, Dk = 16, 4, 64 * 2, 16
+    base = 2 * NT * (2 * C * C + C) * 4                     # 16896, a multiple of 256
+    assert b.chunk_fwd_workspace_size(1, 64, 2, Dk, 16, C, torch.float32) == base
+    # prepared q, k (float32) and gates follow the path's own scratch
+    assert b.chunk_fwd_workspace_size(1, 64, 2, Dk, 16, C, torch.float32, l2norm_qk=True) == \
+        base + 2 * rows * Dk * 4
+    assert b.chunk_fwd_workspace_size(1, 64, 2, Dk, 16, C, torch.float32, gate_logits=True) == \
+        base + 1024
+    assert b.chunk_fwd_workspace_size(1, 64, 2, Dk, 16, C, torch.float32, True, True) == \
+        base + 2 * rows * Dk * 4 + 2 * rows * 4
