@@ -370,6 +370,43 @@ def run_ours(args):
         e2e = {"value": world * tokens / (ems / e2e_steps * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
+    # the optional input prologue (q, k L2-normalised and gates given as logits),
+    # fused into the kernels, against the plain call and against preparing the
+    # inputs in a separate pass (torch device ops) before the plain call
+    prologue = None
+    if not args.chunk_only:
+        raw = {n: (t.to(device) if t is not None else None)
+               for n, t in I.raw_chunk_inputs(w, seed=w.seed + rank).items()}
+        ws_p = torch.empty(max(G.chunk_fwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                          w.torch_dtype, True, True), 1),
+                           dtype=torch.uint8, device=device)
+
+        def fused_step():
+            G.chunk_fwd(raw["q"], raw["k"], raw["v"], raw["log_alpha"], raw["beta"], raw["S0"],
+                        chunk=w.chunk, out=o, S_T=S_T, workspace=ws_p, l2norm_qk=True,
+                        gate_logits=True)
+
+        def unfused_step():
+            F = torch.nn.functional
+            qn = F.normalize(raw["q"].float(), dim=-1, eps=1e-6).to(w.torch_dtype)
+            kn = F.normalize(raw["k"].float(), dim=-1, eps=1e-6).to(w.torch_dtype)
+            la = -F.softplus(raw["log_alpha"])
+            be = torch.sigmoid(raw["beta"])
+            G.chunk_fwd(qn, kn, raw["v"], la, be, raw["S0"], chunk=w.chunk, out=o, S_T=S_T,
+                        workspace=ws)
+
+        n_p = max(20, min(steps, 400))
+        for _ in range(3):
+            fused_step()
+            unfused_step()
+        f_ms = _max_over_ranks(time_loop(fused_step, n_p, stream, world), world, device) / n_p
+        u_ms = _max_over_ranks(time_loop(unfused_step, n_p, stream, world), world, device) / n_p
+        prologue = {"what": "raw q, k and gate logits; normalisation and activations fused into "
+                            "the kernels (l2norm_qk, gate_logits)",
+                    "fused_ms_per_step": f_ms, "plain_ms_per_step": ms_step,
+                    "unfused_prepass_ms_per_step": u_ms,
+                    "fused_tokens_per_s": world * tokens / (f_ms * 1e-3), "steps": n_p}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
@@ -387,6 +424,7 @@ def run_ours(args):
                        "path": path},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
+            "prologue": prologue,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

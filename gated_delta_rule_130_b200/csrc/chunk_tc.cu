@@ -147,8 +147,11 @@ static_assert(SM_PT + (NSTAGE + 1) * BLK <= SM_GV, "[P; *] operand rows stay ins
 static_assert(SM_BAR % 8 == 0, "mbarrier alignment");
 
 // TMEM columns
-constexpr uint32_t TM_ST = 0, TM_X = 64, TM_Y = 128, TM_G = 192, TM_WU = 256;
+// G is 128 columns wide when q and k are normalised in the kernel ([K;Q][K;Q]^T:
+// the diagonal of Q Q^T gives |q|^2), 64 otherwise.
+constexpr uint32_t TM_ST = 0, TM_X = 64, TM_G = 128, TM_WU = 256, TM_Y = 448;
 constexpr uint32_t TM_U = TM_WU + DK;
+static_assert(TM_G + 128 <= TM_WU && TM_U + DVT <= TM_Y && TM_Y + DVT == 512, "TMEM columns");
 constexpr uint32_t TM_COLS = 512;
 
 // barrier indices (arrivals)
@@ -386,7 +389,8 @@ constexpr int LDK = DK + 8;                        // bf16 row stride of the sta
 constexpr int UT_SM_KT = 0;                        // K chunk (64 x LDK bf16), then T (64 x LDA f32)
 constexpr int UT_SM_AF = C * LDA * 4;              // A (64 x LDA f32); N_IJ overwrite A_IJ
 constexpr int UT_SM_GT = UT_SM_AF + C * LDA * 4;   // g log2(e), beta, beta gamma |k|^-1, |k|^-1
-constexpr int UT_SMEM = UT_SM_GT + 4 * C * 4;
+// shared memory of the plain / the normalising instantiation (the latter keeps 1/|k|)
+constexpr int ut_smem_bytes(bool norm) { return UT_SM_GT + (norm ? 4 : 3) * C * 4; }
 constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
 static_assert(C * LDK * 2 <= UT_SM_AF, "K chunk fits in the T buffer");
 static_assert(UT_SM_AF % 16 == 0 && UT_SM_GT % 16 == 0, "16-byte aligned UT buffers");
@@ -435,6 +439,9 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
     __syncthreads();
 }
 
+// kNorm: q and k are L2-normalised inside the kernels (1/|k| folded into the
+// Gram rows and T', and written to rk_out); without it the kernel is unchanged.
+template <bool kNorm>
 __global__ void __launch_bounds__(UT_THREADS, 6)
 gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
               const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt,
@@ -497,7 +504,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     __syncthreads();
     // 1/|k_r| per row (two threads a row), folded into the Gram rows and the
     // columns of T'; kept in the workspace for the sequential kernel
-    if (flags & kFlagL2Norm) {
+    if constexpr (kNorm) {
         const int r = tid >> 1, half = tid & 1;
         const uint4 *row = reinterpret_cast<const uint4 *>(Ks + r * LDK + 64 * half);
         float ss = 0.f;
@@ -518,10 +525,8 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
             bgs[r] *= rkv;
             rk_out[((size_t)((size_t)b * H + h) * NT + c) * C + r] = rkv;
         }
-    } else if (tid < C) {
-        rks[tid] = 1.f;
+        __syncthreads();
     }
-    __syncthreads();
 
     // Gram K K^T on and below the diagonal: warp w takes rows 16 w .. + 15 and the
     // 2 w + 2 column tiles of 8 up to the diagonal, then gates it into A:
@@ -553,16 +558,15 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int r = 16 * RB + g + 8 * hr;
-            const float gr = g2s[r], br = bes[r] * rks[r];
+            const float gr = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (j < ntiles) {
                     const int i = 8 * j + 2 * t;
-                    const float a0 =
-                        (i < r) ? br * rks[i] * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
-                    const float a1 = (i + 1 < r)
-                                         ? br * rks[i + 1] * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1]
-                                         : 0.f;
+                    const float s0 = kNorm ? br * rks[i] : br, s1 = kNorm ? br * rks[i + 1] : br;
+                    const float a0 = (i < r) ? s0 * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
+                    const float a1 =
+                        (i + 1 < r) ? s1 * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1] : 0.f;
                     *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
                 }
             }
@@ -601,6 +605,9 @@ struct Params {
     unsigned flags;        // input prologue (kFlagL2Norm, kFlagGateLogits)
 };
 
+// kNorm: as for gdn_ut_kernel (G widens to [K;Q][K;Q]^T, whose Q Q^T diagonal
+// gives |q|^2, and 1/|k|, 1/|q| scale P and the U' epilogue).
+template <bool kNorm>
 __global__ void __launch_bounds__(NTHREADS, 1)
 gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tt,
@@ -657,7 +664,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr float LOG2E = 1.4426950408889634f;
         int armed = 0;
         float nla[2], nbe[2], nrk[2];  // gate values of the next chunk (rows lane, lane + 32)
-        const bool l2n = (p.flags & kFlagL2Norm) != 0;
+        constexpr bool l2n = kNorm;
         const auto fetch_gates = [&](int cc) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -738,8 +745,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             gv[GV_G2 + 32 + lane] = g1;
             gv[GV_BETA + lane] = be[0];
             gv[GV_BETA + 32 + lane] = be[1];
-            gv[GV_RK + lane] = rk2[0];
-            gv[GV_RK + 32 + lane] = rk2[1];
+            if constexpr (kNorm) {
+                gv[GV_RK + lane] = rk2[0];
+                gv[GV_RK + 32 + lane] = rk2[1];
+            }
             gv[GV_GAM + lane] = ex2(g0);
             gv[GV_GAM + 32 + lane] = ex2(g1);
             gv[GV_DCY + lane] = ex2(glast - g0);
@@ -770,7 +779,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     } else if (warp == W_GMMA) {
         // ------------------------------------------------- MMA: Gram products
         // the whole warp waits (fast path: a test and a vote); lane 0 issues
-        const uint32_t idesc_g = idesc_bf16(128, 64, false, false);
+        // B = K, or [K; Q] (contiguous per key block) when |q| is needed too
+        const uint32_t idesc_g = idesc_bf16(128, kNorm ? 128 : 64, false, false);
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
             const uint32_t st = smem_u32(base + SM_STAGE + s * STAGE);
@@ -884,6 +894,13 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float v0[16], v1[16];
             tmem_ld16(lane_addr + TM_G + 16 * hf, v0);
             tmem_ld16(lane_addr + TM_G + 16 * hf + 32, v1);
+            // with normalisation: this warp's 32 x 32 diagonal block of Q Q^T (its
+            // lane l needs column l), read before G is released
+            float d0[16], d1[16];
+            if constexpr (kNorm) {
+                tmem_ld16(lane_addr + TM_G + 64 + 32 * qr, d0);
+                tmem_ld16(lane_addr + TM_G + 64 + 32 * qr + 16, d1);
+            }
             tmem_wait_ld();
             GDN_TRACE_WARP(c, 27, 2);
             tc_fence_before();
@@ -895,36 +912,22 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 gated_piece<false>(v0, hf, r, su, gv + GV_G2, gv + GV_W);
                 gated_piece<true>(v1, hf + 2, r, su, gv + GV_G2, gv + GV_W);
             }
-            if (p.flags & kFlagL2Norm) {
-                // P_ri = Gamma_ri (q_r . k_i) / (|q_r| |k_i|): 1/|q_r| from this row of
-                // the chunk's Q tile (both key blocks, 128-byte swizzled rows), 1/|k_i|
-                // from the gate vectors; the twin warp computes the same row norm
-                const uint8_t *st = base + SM_STAGE + s * STAGE;
-                float ss = 0.f;
+            if constexpr (kNorm) {
+                // P_ri = Gamma_ri (q_r . k_i) / (|q_r| |k_i|): |q_r|^2 is the diagonal of
+                // Q Q^T (G columns 64 + r), 1/|k_i| comes with the gate vectors
+                float qq = 0.f;
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const uint4 u = *reinterpret_cast<const uint4 *>(
-                            st + kb * GRP + OFF_Q + sw128_offset(r, 16 * m));
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f =
-                                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                            ss += f.x * f.x + f.y * f.y;
-                        }
-                    }
+                for (int j = 0; j < 16; ++j) {
+                    qq = (lane == j) ? d0[j] : qq;
+                    qq = (lane == 16 + j) ? d1[j] : qq;
                 }
-                const float rq = rsqrtf(ss + kNormEps);
+                const float rq = rsqrtf(fmaxf(qq, 0.f) + kNormEps);
                 if (hf == 0) gv_all[s * GV_STRIDE + GV_RQ + r] = rq;
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     v0[j] *= rq * gv[GV_RK + 16 * hf + j];
                     v1[j] *= rq * gv[GV_RK + 16 * (hf + 2) + j];
                 }
-            } else if (hf == 0) {
-                gv_all[s * GV_STRIDE + GV_RQ + r] = 1.f;
             }
             GDN_TRACE_WARP(c, 28, 2);
             store16_bf16(base + SM_PT + s * BLK, r, hf, v0);
@@ -1003,7 +1006,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // U' = U - W S^T for chunk row r -> U' and diag(exp(g_last - g)) U' (bf16)
                 const int r = lrow - 64;
                 // K enters the state update normalised: scale U' rows by 1/|k_r| too
-                const float dc = gv[GV_DCY + r] * gv[GV_RK + r];
+                const float dc = kNorm ? gv[GV_DCY + r] * gv[GV_RK + r] : gv[GV_DCY + r];
                 float x0[16], x1[16], u0[16], u1[16];
                 tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
                 tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
@@ -1033,8 +1036,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y; the
                 // intra-chunk MMA accumulates onto it
                 // 1/|q_r| comes from the P warps (published with this chunk's P tile)
-                if ((p.flags & kFlagL2Norm) && !warp_wait(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
-                const float gr = gv[GV_GAM + lrow] * gv[GV_RQ + lrow];
+                if (kNorm && !warp_wait(cx, B_PREP_FULL + s, (c >> 1) & 1)) break;
+                const float gr = kNorm ? gv[GV_GAM + lrow] * gv[GV_RQ + lrow] : gv[GV_GAM + lrow];
                 float x0[16], x1[16];
                 tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
                 tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
@@ -1214,13 +1217,15 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     p.NT = NT;
     p.rk = rk;
     p.flags = flags;
-    cudaError_t e = cudaFuncSetAttribute(tc::gdn_ut_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::UT_SMEM);
+    const bool norm = (flags & kFlagL2Norm) != 0;
+    auto *ut = norm ? tc::gdn_ut_kernel<true> : tc::gdn_ut_kernel<false>;
+    auto *seq = norm ? tc::gdn_chunk_tc_kernel<true> : tc::gdn_chunk_tc_kernel<false>;
+    const int ut_smem = tc::ut_smem_bytes(norm);
+    cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize, ut_smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc::gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::SMEM_BYTES);
+    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    tc::gdn_ut_kernel<<<dim3(NT, H, B), tc::UT_THREADS, tc::UT_SMEM, st>>>(
+    ut<<<dim3(NT, H, B), tc::UT_THREADS, ut_smem, st>>>(
         static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, rk, T, H, NT, flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
@@ -1236,7 +1241,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tc::gdn_chunk_tc_kernel, mq, mk, mv, mt, p);
+    e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mt, p);
     if (e != cudaSuccess) return e;
     return cudaPeekAtLastError();
 }

@@ -55,8 +55,10 @@ decode_rows_vec(const T *__restrict__ q, const T *__restrict__ k, const T *__res
         sk += s[j].x * kk[j].x + s[j].y * kk[j].y + s[j].z * kk[j].z + s[j].w * kk[j].w;
         sq += s[j].x * qq[j].x + s[j].y * qq[j].y + s[j].z * qq[j].z + s[j].w * qq[j].w;
         kq += kk[j].x * qq[j].x + kk[j].y * qq[j].y + kk[j].z * qq[j].z + kk[j].w * qq[j].w;
-        kk2 += kk[j].x * kk[j].x + kk[j].y * kk[j].y + kk[j].z * kk[j].z + kk[j].w * kk[j].w;
-        qq2 += qq[j].x * qq[j].x + qq[j].y * qq[j].y + qq[j].z * qq[j].z + qq[j].w * qq[j].w;
+        if (flags & kFlagL2Norm) {
+            kk2 += kk[j].x * kk[j].x + kk[j].y * kk[j].y + kk[j].z * kk[j].z + kk[j].w * kk[j].w;
+            qq2 += qq[j].x * qq[j].x + qq[j].y * qq[j].y + qq[j].z * qq[j].z + qq[j].w * qq[j].w;
+        }
     }
 #pragma unroll
     for (int off = L / 2; off > 0; off >>= 1) {
