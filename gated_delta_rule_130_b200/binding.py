@@ -51,6 +51,11 @@ def _load():
     lib.gdn_chunk_fwd_workspace_size_ex.restype = Z
     lib.gdn_decode_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, U, vp]
     lib.gdn_decode_step_ex.restype = I
+    lib.gdn_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, I, I, I, I, I, I,
+                                         U, vp, Z, vp]
+    lib.gdn_chunk_fwd_varlen.restype = I
+    lib.gdn_chunk_fwd_varlen_workspace_size.argtypes = [vp, I, I, I, I, I, I, U]
+    lib.gdn_chunk_fwd_varlen_workspace_size.restype = Z
     lib.gdn_check_device_status.argtypes = []
     lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]
@@ -170,6 +175,78 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=
     st = LIB.gdn_chunk_fwd_ex(*args, B, T, H, Dk, Dv, chunk, code, flags, ws_ptr, ws_bytes,
                               _stream_ptr(dev))
     _check(st, "gdn_chunk_fwd")
+    return o, S_T
+
+
+def _host_offsets(cu_seqlens) -> torch.Tensor:
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
+    if cu.dim() != 1 or cu.numel() < 1:
+        raise GdnError("cu_seqlens must be a 1-D list of N + 1 offsets")
+    return cu
+
+
+def chunk_fwd_varlen_workspace_size(cu_seqlens, H, Dk, Dv, chunk=64, dtype=torch.bfloat16,
+                                    l2norm_qk: bool = False, gate_logits: bool = False) -> int:
+    cu = _host_offsets(cu_seqlens)
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(LIB.gdn_chunk_fwd_varlen_workspace_size(cu.data_ptr(), cu.numel() - 1, H, Dk, Dv,
+                                                       chunk, code, _flags(l2norm_qk, gate_logits)))
+
+
+def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk: int = 64, out=None,
+                     S_T=None, return_state: bool = True, workspace=None, l2norm_qk: bool = False,
+                     gate_logits: bool = False):
+    """Chunkwise forward over N variable-length sequences packed without padding.
+
+    q, k [total, H, Dk], v [total, H, Dv], log_alpha, beta [total, H]; ``cu_seqlens``
+    the N + 1 token offsets (host list or tensor; sequence n is tokens
+    cu_seqlens[n] .. cu_seqlens[n + 1] - 1).  S0 / S_T are [N, H, Dv, Dk] float32.
+    Returns (o [total, H, Dv], S_T or None).
+    """
+    cu = _host_offsets(cu_seqlens)
+    N = cu.numel() - 1
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise GdnError("q, k must be [total,H,Dk] and v [total,H,Dv]")
+    total, H, Dk = q.shape
+    Dv = v.shape[2]
+    if int(cu[-1]) != total:
+        raise GdnError("cu_seqlens[-1] must equal the number of packed tokens")
+    dev = q.device
+    code = _dtype_code(q)
+    flags = _flags(l2norm_qk, gate_logits)
+    if log_alpha.shape != (total, H) or beta.shape != (total, H):
+        raise GdnError("log_alpha and beta must be [total,H]")
+    args = [_dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
+            _dev(log_alpha, "log_alpha", torch.float32, dev), _dev(beta, "beta", torch.float32, dev)]
+    if S0 is not None:
+        if S0.shape != (N, H, Dv, Dk):
+            raise GdnError("S0 must be [N,H,Dv,Dk]")
+        args.append(_dev(S0, "S0", torch.float32, dev))
+    else:
+        args.append(None)
+    o = out if out is not None else torch.empty((total, H, Dv), dtype=q.dtype, device=dev)
+    if o.shape != (total, H, Dv):
+        raise GdnError("out must be [total,H,Dv]")
+    args.append(_dev(o, "out", q.dtype, dev))
+    if S_T is None and return_state:
+        S_T = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        if S_T.shape != (N, H, Dv, Dk):
+            raise GdnError("S_T must be [N,H,Dv,Dk]")
+        args.append(_dev(S_T, "S_T", torch.float32, dev))
+    else:
+        args.append(None)
+    cu_dev = cu.to(dev)
+    need = int(LIB.gdn_chunk_fwd_varlen_workspace_size(cu.data_ptr(), N, H, Dk, Dv, chunk, code,
+                                                       flags))
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    st = LIB.gdn_chunk_fwd_varlen(*args, cu_dev.data_ptr(), cu.data_ptr(), N, H, Dk, Dv, chunk,
+                                  code, flags, ws_ptr, ws_bytes, _stream_ptr(dev))
+    _check(st, "gdn_chunk_fwd_varlen")
     return o, S_T
 
 

@@ -379,9 +379,56 @@ __device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float 
     }
 }
 
+// ------------------------------------------------------------- sequences --
+// Where each sequence lives in the packed token dimension ([tokens, H, D] rows):
+// a fixed-length batch (cu == nullptr: sequence b is tokens [b T, b T + T)) or
+// variable lengths (tokens cu[b] .. cu[b + 1]).  Chunks are numbered globally,
+// sequence by sequence: sequence b owns chunks chunk0 .. chunk0 + ceil(len / C).
+struct Seqs {
+    const int *cu;         // n + 1 token offsets (device), or null
+    const int *cu_chunks;  // n + 1 chunk offsets (device), or null
+    int T;                 // the common length when cu is null
+    int n;                 // number of sequences
+};
+
+struct Span {
+    int off, len, chunk0;
+};
+
+__device__ __forceinline__ Span seq_span(const Seqs &q, int b) {
+    if (q.cu) return Span{q.cu[b], q.cu[b + 1] - q.cu[b], q.cu_chunks[b]};
+    return Span{b * q.T, q.T, b * ((q.T + C - 1) / C)};
+}
+
+// The sequence a global chunk index belongs to: the last b with cu_chunks[b] <= g
+// (empty sequences share their start with the next one and are skipped).
+__device__ __forceinline__ int seq_of_chunk(const Seqs &q, int g) {
+    if (!q.cu) return g / ((q.T + C - 1) / C);
+    int lo = 0, hi = q.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (q.cu_chunks[mid] <= g) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// cu_chunks[b] = sum over earlier sequences of ceil(len / C) (one thread; the
+// sequence count is small next to the work of a call)
+__global__ void seq_chunk_offsets(const int *__restrict__ cu, int n, int *__restrict__ cu_chunks) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        int acc = 0;
+        for (int b = 0; b < n; ++b) {
+            cu_chunks[b] = acc;
+            acc += (cu[b + 1] - cu[b] + C - 1) / C;
+        }
+        cu_chunks[n] = acc;
+    }
+}
+
 // ------------------------------------------------------------- UT kernel --
-// One CTA of 4 warps per (chunk c, head h, batch b): [T'; T''] of that chunk,
-// bf16, 128 rows x 64 columns, row-major, at tt + ((b H + h) NT + c) 128 x 64.
+// One CTA of 4 warps per (global chunk g, head h): [T'; T''] of that chunk,
+// bf16, 128 rows x 64 columns, row-major, at tt + (g H + h) 128 x 64.
 // Six CTAs fit on an SM (shared memory and registers), so six chunks are in
 // flight per SM and the solve's dependent steps overlap across chunks.
 constexpr int UT_THREADS = 128;
@@ -445,12 +492,16 @@ template <bool kNorm>
 __global__ void __launch_bounds__(UT_THREADS, 6)
 gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
               const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt,
-              float *__restrict__ rk_out, int T, int H, int NT, unsigned flags) {
+              float *__restrict__ rk_out, const Seqs sq, int H, unsigned flags) {
     extern __shared__ __align__(16) uint8_t ut_smem[];
     // the sequential kernel that follows on the stream may be scheduled now (it
     // waits for this grid's completion before it reads the tiles)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // global chunk g of head h: chunk c of sequence b, whose tokens start at sp.off
+    const int gch = blockIdx.x, h = blockIdx.y;
+    const int b = seq_of_chunk(sq, gch);
+    const Span sp = seq_span(sq, b);
+    const int c = gch - sp.chunk0, T = sp.len;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int t0 = c * C;
@@ -466,7 +517,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
         const int idx = tid + UT_THREADS * m;
         const int r = idx / (DK / 8), piece = idx % (DK / 8);
         const bool in = t0 + r < T;
-        const __nv_bfloat16 *src = k + (((size_t)b * T + (in ? t0 + r : 0)) * H + h) * DK + 8 * piece;
+        const __nv_bfloat16 *src = k + ((size_t)(sp.off + (in ? t0 + r : 0)) * H + h) * DK + 8 * piece;
         cp_async16(Ks + r * LDK + 8 * piece, src, in ? 16u : 0u);
     }
     if (warp == 0) {
@@ -477,7 +528,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
         for (int hh = 0; hh < 2; ++hh) {
             const int r = lane + 32 * hh;
             const bool in = t0 + r < T;
-            const size_t gi = ((size_t)b * T + t0 + r) * H + h;
+            const size_t gi = (size_t)(sp.off + t0 + r) * H + h;
             const float2 gp = in ? gate_pair(log_alpha[gi], beta[gi], flags) : make_float2(0.f, 0.f);
             la[hh] = gp.x;
             be[hh] = gp.y;
@@ -523,7 +574,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
             const float rkv = rsqrtf(ss + kNormEps);
             rks[r] = rkv;
             bgs[r] *= rkv;
-            rk_out[((size_t)((size_t)b * H + h) * NT + c) * C + r] = rkv;
+            rk_out[((size_t)gch * H + h) * C + r] = rkv;
         }
         __syncthreads();
     }
@@ -580,7 +631,7 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     // [T'; T''] rows: T'(r, i) = T(r, i) beta_i gamma_i / |k_i|, T''(r, i) = T(r, i) beta_i
     // for i <= r; thread -> (row, 4-column piece): 16 threads read one T row with
     // no bank conflict and write its 128 bytes
-    __nv_bfloat16 *dst = tt + ((size_t)((size_t)b * H + h) * NT + c) * TT_ELEMS;
+    __nv_bfloat16 *dst = tt + ((size_t)gch * H + h) * TT_ELEMS;
 #pragma unroll 4
     for (int m = 0; m < TT_ELEMS / 4 / UT_THREADS; ++m) {
         const int idx = tid + UT_THREADS * m;
@@ -601,7 +652,8 @@ struct Params {
     __nv_bfloat16 *o;
     float *S_T;
     const float *rk;       // 1/|k| per token from the UT kernel (L2-normalising only)
-    int T, H, Dv, NT;
+    Seqs sq;               // the sequences (one per blockIdx.z)
+    int H, Dv;
     unsigned flags;        // input prologue (kFlagL2Norm, kFlagGateLogits)
 };
 
@@ -626,7 +678,19 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int vt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int v0 = vt * DVT;
-    const int T = p.T, H = p.H, NT = p.NT;
+    const int H = p.H;
+    // sequence b: tokens sp.off .. sp.off + T of the packed rows, chunks sp.chunk0 ..
+    const Span sp = seq_span(p.sq, b);
+    const int T = sp.len, NT = (T + C - 1) / C;
+    if (NT == 0) {
+        // an empty sequence: the final state is the initial one (this CTA's slice)
+        if (p.S_T)
+            for (int e = threadIdx.x; e < DVT * DK; e += NTHREADS) {
+                const size_t idx = ((size_t)b * H + h) * p.Dv * DK + (size_t)v0 * DK + e;
+                p.S_T[idx] = p.S0 ? p.S0[idx] : 0.f;
+            }
+        return;
+    }
 
     if (tid == 0) {
         int counts[NBAR];
@@ -670,10 +734,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = lane + 32 * hh;
                 const bool in = cc * C + r < T;
-                const size_t gi = ((size_t)b * T + cc * C + r) * H + h;
+                const size_t gi = (size_t)(sp.off + cc * C + r) * H + h;
                 nla[hh] = in ? p.log_alpha[gi] : 0.f;
                 nbe[hh] = in ? p.beta[gi] : 0.f;
-                nrk[hh] = l2n ? p.rk[((size_t)((size_t)b * H + h) * NT + cc) * C + r] : 1.f;
+                nrk[hh] = l2n ? p.rk[((size_t)(sp.chunk0 + cc) * H + h) * C + r] : 1.f;
             }
         };
         // the [T'; T''] tiles (and 1/|k|) come from the UT kernel launched just
@@ -701,23 +765,25 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mbar_expect_tx(cx.bar + B_IN_FULL + s, (2 * KB + 3) * BLK);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(st + kb * GRP + OFF_K, &tm_k, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
-                    tma_load_4d(st + kb * GRP + OFF_Q, &tm_q, cx.bar + B_IN_FULL + s, kb * 64, h, t0, b);
+                    tma_load_4d(st + kb * GRP + OFF_K, &tm_k, cx.bar + B_IN_FULL + s, kb * 64, h,
+                                sp.off + t0, 0);
+                    tma_load_4d(st + kb * GRP + OFF_Q, &tm_q, cx.bar + B_IN_FULL + s, kb * 64, h,
+                                sp.off + t0, 0);
                 }
-                tma_load_4d(st + OFF_V, &tm_v, cx.bar + B_IN_FULL + s, v0, h, t0, b);
+                tma_load_4d(st + OFF_V, &tm_v, cx.bar + B_IN_FULL + s, v0, h, sp.off + t0, 0);
                 tma_load_3d(st + OFF_TT, &tm_tt, cx.bar + B_IN_FULL + s, 0, 0,
-                            ((int)b * H + h) * NT + c);
+                            (sp.chunk0 + c) * H + h);
                 GDN_TRACE_AT(c, 24);
                 // the tiles of a later chunk start streaming from DRAM into L2 now,
                 // so that its shared-memory load, once a stage is free, hits L2
                 for (int cq = (c == 0 ? 1 : c + L2_AHEAD); cq <= c + L2_AHEAD && cq < NT; ++cq) {
 #pragma unroll
                     for (int kb = 0; kb < KB; ++kb) {
-                        tma_prefetch_l2_4d(&tm_k, kb * 64, h, cq * C, b);
-                        tma_prefetch_l2_4d(&tm_q, kb * 64, h, cq * C, b);
+                        tma_prefetch_l2_4d(&tm_k, kb * 64, h, sp.off + cq * C, 0);
+                        tma_prefetch_l2_4d(&tm_q, kb * 64, h, sp.off + cq * C, 0);
                     }
-                    tma_prefetch_l2_4d(&tm_v, v0, h, cq * C, b);
-                    tma_prefetch_l2_3d(&tm_tt, 0, 0, ((int)b * H + h) * NT + cq);
+                    tma_prefetch_l2_4d(&tm_v, v0, h, sp.off + cq * C, 0);
+                    tma_prefetch_l2_3d(&tm_tt, 0, 0, (sp.chunk0 + cq) * H + h);
                 }
             }
             armed = c + 1;
@@ -1108,7 +1174,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_wait_ld();
                 if (t0 + lrow < T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
-                        p.o + (((size_t)b * T + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
+                        p.o + ((size_t)(sp.off + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
                         dst[k] = make_uint4(pack_bf16(y0[8 * k + 0], y0[8 * k + 1]),
@@ -1180,10 +1246,22 @@ bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 
 }  // namespace tc
 
+// Workspace: [chunk offsets of the sequences, variable lengths only, padded to
+// 256 B][one [T'; T''] tile per chunk and head][1/|k| per token, normalising only].
+static size_t tc_offsets_bytes(int n_seq, bool varlen) {
+    return varlen ? (((size_t)n_seq + 1) * sizeof(int) + 255) & ~size_t(255) : 0;
+}
+
+size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
+                               unsigned flags) {
+    const size_t tiles = (size_t)total_chunks * H * tc::TT_ELEMS * sizeof(__nv_bfloat16);
+    const size_t rk = (flags & kFlagL2Norm) ? (size_t)total_chunks * H * tc::C * sizeof(float) : 0;
+    return tc_offsets_bytes(n_seq, varlen) + tiles + rk;
+}
+
 size_t tc_workspace_bytes(int B, int T, int H, unsigned flags) {
-    const size_t NT = ((size_t)T + tc::C - 1) / tc::C;
-    const size_t tiles = (size_t)B * H * NT * tc::TT_ELEMS * sizeof(__nv_bfloat16);
-    return tiles + ((flags & kFlagL2Norm) ? (size_t)B * H * NT * tc::C * sizeof(float) : 0);
+    const long long NT = ((long long)T + tc::C - 1) / tc::C;
+    return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags);
 }
 
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
@@ -1191,30 +1269,38 @@ bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
            H >= 1 && tc::encode_fn() != nullptr;
 }
 
-cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
-                            const float *beta, const float *S0, void *o, float *S_T, int B, int T,
-                            int H, int Dk, int Dv, unsigned flags, void *workspace,
-                            cudaStream_t st) {
-    const int NT = (T + tc::C - 1) / tc::C;
-    auto *tt = static_cast<__nv_bfloat16 *>(workspace);
+cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
+                                 const int *cu_seqlens, long long total_chunks, int H, int Dk,
+                                 int Dv, unsigned flags, void *workspace, cudaStream_t st) {
+    const bool varlen = cu_seqlens != nullptr;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
+    auto *tt = reinterpret_cast<__nv_bfloat16 *>(ws + tc_offsets_bytes(n_seq, varlen));
     float *rk = (flags & kFlagL2Norm)
-                    ? reinterpret_cast<float *>(tt + (size_t)B * H * NT * tc::TT_ELEMS)
+                    ? reinterpret_cast<float *>(tt + (size_t)total_chunks * H * tc::TT_ELEMS)
                     : nullptr;
     CUtensorMap mq, mk, mv, mt;
-    if (!tc::make_map(&mq, q, B, T, H, Dk) || !tc::make_map(&mk, k, B, T, H, Dk) ||
-        !tc::make_map(&mv, v, B, T, H, Dv) ||
-        !tc::make_map_tt(&mt, tt, (long long)B * H * NT))
+    if (!tc::make_map(&mq, q, 1, (int)total_T, H, Dk) ||
+        !tc::make_map(&mk, k, 1, (int)total_T, H, Dk) ||
+        !tc::make_map(&mv, v, 1, (int)total_T, H, Dv) ||
+        !tc::make_map_tt(&mt, tt, total_chunks > 0 ? total_chunks * H : 1))
         return cudaErrorInvalidValue;
+    if (varlen) {
+        tc::seq_chunk_offsets<<<1, 32, 0, st>>>(cu_seqlens, n_seq, cu_chunks);
+        const cudaError_t e0 = cudaPeekAtLastError();
+        if (e0 != cudaSuccess) return e0;
+    }
     tc::Params p;
     p.log_alpha = log_alpha;
     p.beta = beta;
     p.S0 = S0;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.S_T = S_T;
-    p.T = T;
+    p.sq = tc::Seqs{cu_seqlens, cu_chunks, T_fixed, n_seq};
     p.H = H;
     p.Dv = Dv;
-    p.NT = NT;
     p.rk = rk;
     p.flags = flags;
     const bool norm = (flags & kFlagL2Norm) != 0;
@@ -1225,14 +1311,15 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    ut<<<dim3(NT, H, B), tc::UT_THREADS, ut_smem, st>>>(
-        static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, rk, T, H, NT, flags);
+    if (total_chunks > 0)
+        ut<<<dim3((unsigned)total_chunks, H, 1), tc::UT_THREADS, ut_smem, st>>>(
+            static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, rk, p.sq, H, flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the CTAs may start (TMEM, barriers, the initial
     // state) while the UT kernel drains; the TMA warp waits for it before loading
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(Dv / tc::DVT, H, B);
+    cfg.gridDim = dim3(Dv / tc::DVT, H, n_seq);
     cfg.blockDim = dim3(tc::NTHREADS);
     cfg.dynamicSmemBytes = tc::SMEM_BYTES;
     cfg.stream = st;
@@ -1244,6 +1331,16 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mt, p);
     if (e != cudaSuccess) return e;
     return cudaPeekAtLastError();
+}
+
+cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *S0, void *o, float *S_T, int B, int T,
+                            int H, int Dk, int Dv, unsigned flags, void *workspace,
+                            cudaStream_t st) {
+    // a fixed-length batch is B packed sequences of length T
+    const long long NT = ((long long)T + tc::C - 1) / tc::C;
+    return launch_chunk_tc_seqs(q, k, v, log_alpha, beta, S0, o, S_T, B, T, (long long)B * T,
+                                nullptr, (long long)B * NT, H, Dk, Dv, flags, workspace, st);
 }
 
 #ifdef GDN_TRACE

@@ -34,6 +34,23 @@ bool empty_problem(int B, int T, int H) { return B == 0 || H == 0 || T == 0; }
 constexpr unsigned kKnownFlags = GDN_FLAG_L2NORM_QK | GDN_FLAG_GATE_LOGITS;
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
+// Packed-sequence offsets: N + 1 ints from 0, non-decreasing, total below 2^31.
+struct Offsets {
+    long long total = 0, chunks64 = 0;  // tokens; chunks of 64 tokens over all sequences
+    int max_len = 0;
+};
+bool read_offsets(const int *cu, int N, Offsets *out) {
+    if (!cu || N < 0 || cu[0] != 0) return false;
+    for (int n = 0; n < N; ++n) {
+        const long long len = (long long)cu[n + 1] - cu[n];
+        if (len < 0) return false;
+        out->chunks64 += (len + 63) / 64;
+        if (len > out->max_len) out->max_len = (int)len;
+    }
+    out->total = cu[N];
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -144,6 +161,110 @@ gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
         if (e == cudaSuccess)
             e = gdn::launch_chunk_simt(in.q, in.k, v, in.log_alpha, in.beta, S0, o, S_T, B, T, H,
                                        Dk, Dv, chunk, bf16, workspace, st);
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+size_t gdn_chunk_fwd_varlen_workspace_size(const int *cu_seqlens_host, int N, int H, int Dk,
+                                           int Dv, int chunk, gdn_dtype_t dtype, unsigned flags) {
+    Offsets off;
+    if ((flags & ~kKnownFlags) || !read_offsets(cu_seqlens_host, N, &off)) return 0;
+    if (check_sizes(N, off.max_len, H, Dk, Dv, chunk, dtype) != GDN_OK) return 0;
+    if (N == 0 || H == 0 || off.total == 0) return 0;
+    const bool bf16 = dtype == GDN_BF16;
+    if (gdn::tc_supported(N, off.max_len, H, Dk, Dv, chunk, bf16))
+        return gdn::tc_workspace_bytes_seqs(N, off.chunks64, H, true, flags);
+    // CUDA-core path: one sequence at a time (scratch for the longest), prologue once
+    const size_t base = gdn::simt_workspace_bytes(1, off.max_len, H, chunk);
+    return flags ? align256(base) +
+                       gdn::prologue_bytes(1, (int)off.total, H, Dk, bf16, flags)
+                 : base;
+}
+
+gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  void *o, float *S_T, const int *cu_seqlens,
+                                  const int *cu_seqlens_host, int N, int H, int Dk, int Dv,
+                                  int chunk, gdn_dtype_t dtype, unsigned flags, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    if (flags & ~kKnownFlags) return GDN_ERR_INVALID_ARG;
+    Offsets off;
+    if (!read_offsets(cu_seqlens_host, N, &off)) return GDN_ERR_INVALID_ARG;
+    const gdn_status_t sz = check_sizes(N, off.max_len, H, Dk, Dv, chunk, dtype);
+    if (sz != GDN_OK) return sz;
+    if (off.total > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4;
+    const size_t n_tok = (size_t)off.total * H;
+    const size_t head_state = (size_t)H * Dv * Dk;  // floats of one sequence's state
+    const size_t state_bytes = (size_t)N * head_state * sizeof(float);
+    if (N == 0 || H == 0) return GDN_OK;
+    if (S_T && (!aligned16(S_T) || (S0 && !aligned16(S0)))) return GDN_ERR_INVALID_ARG;
+    if (S_T && S0 && S_T != S0 && overlaps(S_T, state_bytes, S0, state_bytes))
+        return GDN_ERR_INVALID_ARG;
+    const auto copy_state = [&](int n) -> cudaError_t {  // empty sequence n: S_T = S0
+        if (!S_T) return cudaSuccess;
+        float *dst = S_T + (size_t)n * head_state;
+        if (!S0) return cudaMemsetAsync(dst, 0, head_state * sizeof(float), st);
+        const float *src = S0 + (size_t)n * head_state;
+        return src == dst ? cudaSuccess
+                          : cudaMemcpyAsync(dst, src, head_state * sizeof(float),
+                                            cudaMemcpyDeviceToDevice, st);
+    };
+    if (off.total == 0) {
+        for (int n = 0; n < N; ++n)
+            if (copy_state(n) != cudaSuccess) return GDN_ERR_CUDA;
+        return GDN_OK;
+    }
+    if (!q || !k || !v || !log_alpha || !beta || !o || !cu_seqlens) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, o, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t o_bytes = n_tok * Dv * esz;
+    if (overlaps(o, o_bytes, q, n_tok * Dk * esz) || overlaps(o, o_bytes, k, n_tok * Dk * esz) ||
+        overlaps(o, o_bytes, v, n_tok * Dv * esz))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need =
+        gdn_chunk_fwd_varlen_workspace_size(cu_seqlens_host, N, H, Dk, Dv, chunk, dtype, flags);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    if (overlaps(workspace, need, q, n_tok * Dk * esz) ||
+        overlaps(workspace, need, k, n_tok * Dk * esz) ||
+        overlaps(workspace, need, v, n_tok * Dv * esz) ||
+        overlaps(workspace, need, log_alpha, n_tok * sizeof(float)) ||
+        overlaps(workspace, need, beta, n_tok * sizeof(float)) ||
+        overlaps(workspace, need, o, o_bytes) ||
+        (S0 && overlaps(workspace, need, S0, state_bytes)) ||
+        (S_T && overlaps(workspace, need, S_T, state_bytes)) ||
+        overlaps(workspace, need, cu_seqlens, ((size_t)N + 1) * sizeof(int)))
+        return GDN_ERR_INVALID_ARG;
+    const bool bf16 = dtype == GDN_BF16;
+    cudaError_t e = cudaSuccess;
+    if (gdn::tc_supported(N, off.max_len, H, Dk, Dv, chunk, bf16)) {
+        e = gdn::launch_chunk_tc_seqs(q, k, v, log_alpha, beta, S0, o, S_T, N, 0, off.total,
+                                      cu_seqlens, off.chunks64, H, Dk, Dv, flags, workspace, st);
+    } else {
+        // the CUDA-core path, one sequence at a time on the caller's stream (they reuse
+        // the scratch in turn); the prologue runs once over all tokens
+        gdn::Prepared in{q, k, log_alpha, beta};
+        const size_t base = align256(gdn::simt_workspace_bytes(1, off.max_len, H, chunk));
+        if (flags)
+            e = gdn::launch_prologue(q, k, log_alpha, beta, 1, (int)off.total, H, Dk, bf16, flags,
+                                     static_cast<uint8_t *>(workspace) + base, &in, st);
+        for (int n = 0; n < N && e == cudaSuccess; ++n) {
+            const int t0 = cu_seqlens_host[n], len = cu_seqlens_host[n + 1] - t0;
+            if (len == 0) {
+                e = copy_state(n);
+                continue;
+            }
+            const size_t tk = (size_t)t0 * H;
+            e = gdn::launch_chunk_simt(
+                static_cast<const uint8_t *>(in.q) + tk * Dk * esz,
+                static_cast<const uint8_t *>(in.k) + tk * Dk * esz,
+                static_cast<const uint8_t *>(v) + tk * Dv * esz, in.log_alpha + tk, in.beta + tk,
+                S0 ? S0 + (size_t)n * head_state : nullptr, static_cast<uint8_t *>(o) + tk * Dv * esz,
+                S_T ? S_T + (size_t)n * head_state : nullptr, 1, len, H, Dk, Dv, chunk, bf16,
+                workspace, st);
+        }
     }
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -42,6 +42,17 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
                             int H, int Dk, int Dv, unsigned flags, void *workspace,
                             cudaStream_t st);
+// The same over n_seq sequences packed along the token dimension: fixed length
+// T_fixed (cu_seqlens == nullptr) or the device offsets cu_seqlens (n_seq + 1);
+// total_chunks = sum of ceil(length / 64).  The workspace then starts with the
+// per-sequence chunk offsets (computed on the device).
+size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
+                               unsigned flags);
+cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
+                                 const int *cu_seqlens, long long total_chunks, int H, int Dk,
+                                 int Dv, unsigned flags, void *workspace, cudaStream_t st);
 
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).

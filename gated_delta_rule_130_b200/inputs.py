@@ -139,6 +139,44 @@ def raw_decode_step_inputs(w: Workload, step: int, device="cpu"):
     return out
 
 
+def varlen_lengths(n: int, total: int, seed: int, min_len: int = 1):
+    """n sequence lengths summing to ``total``: a seeded log-uniform mix (a few long
+    prompts, many short ones, ragged ends), each at least ``min_len``."""
+    gen = torch.Generator().manual_seed(seed)
+    w = torch.exp(torch.rand(n, generator=gen) * 4.0)          # spread of e^4 ~ 55x
+    raw = (w / w.sum() * (total - n * min_len)).floor().long() + min_len
+    raw[0] += total - int(raw.sum())                            # exact total
+    return [int(x) for x in raw]
+
+
+def varlen_inputs(lengths, H: int, Dk: int, Dv: int, dtype: str = "bf16",
+                  gate_law: str = "slow_softplus", s0_law: str = "zero", seed: int = 2001,
+                  device="cpu"):
+    """Sequences of the given lengths packed along the token dimension: q, k
+    [total, H, Dk] (unit rows), v [total, H, Dv], log_alpha, beta [total, H] f32,
+    S0 [N, H, Dv, Dk] f32 or None, and cu_seqlens (N + 1 int offsets, a list).
+    Same draw recipe as ``chunk_inputs`` with B = 1 and T = total."""
+    total = int(sum(lengths))
+    w = Workload("varlen", 1, H, total, Dk, Dv, 64, dtype, gate_law, "zero", seed)
+    d = chunk_inputs(w)
+    out = {n: d[n][0] for n in ("q", "k", "v", "log_alpha", "beta")}
+    gen = torch.Generator().manual_seed(seed + 77)
+    out["S0"] = (0.02 * torch.randn((len(lengths), H, Dv, Dk), generator=gen)
+                 if s0_law == "normal002" else None)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    if device != "cpu":
+        out = {n: (t.to(device) if t is not None else None) for n, t in out.items()}
+    out["cu_seqlens"] = cu
+    return out
+
+
+# Serving-shaped prefill batch: 12 sequences of mixed lengths, 16,384 tokens in all
+# (the headline's token count), H 16, d 128, bf16.
+VARLEN_SERVING = dict(n=12, total=16384, seed=2002, H=16, Dk=128, Dv=128)
+
+
 def decode_state(w: Workload, device="cpu"):
     """Initial decode state S0 [B,H,Dv,Dk] f32."""
     gen = torch.Generator().manual_seed(w.seed)

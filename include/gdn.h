@@ -146,6 +146,32 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk,
                        gdn_dtype_t dtype);
 
 /*
+ * Chunkwise forward over N variable-length sequences packed along the token
+ * dimension without padding (the serving / prefill form; the pages say nothing
+ * about batching, this is the plain reading): q, k [total, H, Dk], v and o
+ * [total, H, Dv], log_alpha and beta [total, H], with total = cu_seqlens[N].
+ * Sequence n is tokens cu_seqlens[n] .. cu_seqlens[n + 1] - 1 and has its own
+ * state, S0 and S_T [N, H, Dv, Dk] (NULL S0: zeros; an empty sequence gets
+ * S_T = S0).  The offsets (N + 1 ints, starting at 0, non-decreasing) are given
+ * twice: `cu_seqlens` in device memory, read by the kernels, and
+ * `cu_seqlens_host` in host memory, read before anything is launched for the
+ * sizes and the checks; both must hold the same values.  Everything else is as
+ * for gdn_chunk_fwd_ex; the workspace must hold
+ * gdn_chunk_fwd_varlen_workspace_size(...) bytes.  Bad offsets:
+ * GDN_ERR_INVALID_ARG; N above 65535: GDN_ERR_UNSUPPORTED.
+ */
+gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta,
+                                  const float *S0, void *o, float *S_T,
+                                  const int *cu_seqlens, const int *cu_seqlens_host,
+                                  int N, int H, int Dk, int Dv, int chunk,
+                                  gdn_dtype_t dtype, unsigned flags, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+size_t gdn_chunk_fwd_varlen_workspace_size(const int *cu_seqlens_host, int N, int H,
+                                           int Dk, int Dv, int chunk, gdn_dtype_t dtype,
+                                           unsigned flags);
+
+/*
  * gdn_chunk_fwd without a caller workspace, for callers that cannot allocate
  * device memory (engines that plan all buffers at start-up and forbid
  * allocation later, paths where cudaMalloc's implicit synchronisation is not

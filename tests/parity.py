@@ -35,3 +35,22 @@ def head_slices(o, S, units, H):
         if S is not None:
             ss.append(S[b, h])
     return np.stack(os_), (np.stack(ss) if S is not None else None)
+
+
+def oracle_varlen(inp, units=None):
+    """Oracle forward of packed variable-length sequences (a dict from
+    inputs.varlen_inputs): each sequence on its own, outputs packed back.  With
+    ``units`` (heads) only those heads are computed (NaN elsewhere)."""
+    cu = inp["cu_seqlens"]
+    H, Dv, Dk = inp["q"].shape[1], inp["v"].shape[2], inp["q"].shape[2]
+    o = np.full((cu[-1], H, Dv), np.nan)
+    S = np.full((len(cu) - 1, H, Dv, Dk), np.nan)
+    for n in range(len(cu) - 1):
+        a, b = cu[n], cu[n + 1]
+        sl = lambda t: t[a:b].unsqueeze(0)
+        S0 = inp["S0"][n:n + 1] if inp["S0"] is not None else None
+        on, Sn = O.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_alpha"]),
+                           sl(inp["beta"]), S0, units=units)
+        o[a:b] = on[0]
+        S[n] = Sn[0]
+    return o, S

@@ -135,3 +135,59 @@ def test_prologue_workspace_size_on_the_cuda_core_path(lib):
         base + 1024
     assert b.chunk_fwd_workspace_size(1, 64, 2, Dk, 16, C, torch.float32, True, True) == \
         base + 2 * rows * Dk * 4 + 2 * rows * 4
+
+
+def _varlen(lib, cu, **kw):
+    a = dict(q=16, k=16, v=16, la=16, beta=16, S0=None, o=1 << 24, S_T=None, cu_dev=1 << 28, H=1,
+             Dk=16, Dv=16, chunk=16, dtype=0, flags=0, ws=1 << 40, ws_bytes=1 << 30)
+    a.update(kw)
+    N = a.pop("N") if "N" in a else len(cu) - 1
+    host = (ctypes.c_int * len(cu))(*cu) if cu is not None else None
+    return lib.gdn_chunk_fwd_varlen(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["o"],
+                                    a["S_T"], a["cu_dev"], ctypes.cast(host, ctypes.c_void_p)
+                                    if host is not None else None, N, a["H"], a["Dk"], a["Dv"],
+                                    a["chunk"], a["dtype"], a["flags"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("cu,kw,status", [
+    ([1, 4, 8], {}, 1),                       # offsets must start at 0
+    ([0, 6, 4, 9], {}, 1),                    # and never decrease
+    (None, dict(N=2), 1),                     # no host offsets
+    ([0, 4, 8], dict(N=-1), 1),
+    ([0, 4, 8], dict(flags=8), 1),            # unknown prologue flag
+    ([0, 4, 8], dict(q=None), 1),
+    ([0, 4, 8], dict(cu_dev=None), 1),        # device offsets missing
+    ([0, 4, 8], dict(ws=None), 1), ([0, 4, 8], dict(ws_bytes=16), 1),
+    ([0, 4, 8], dict(o=16), 1),               # output overlaps q
+    ([0, 4, 8], dict(ws=1 << 28), 1),         # workspace overlaps the device offsets
+    ([0, 4, 8], dict(chunk=48), 2), ([0, 4, 8], dict(Dk=272), 2),
+    ([0], {}, 0),                             # no sequences: nothing to do
+    ([0, 0, 0], {}, 0),                       # empty sequences, no state asked for
+    ([0] * 65537, {}, 2),                     # more sequences than one grid dimension holds
+])
+def test_chunk_fwd_varlen_rejects_before_launch(lib, cu, kw, status):
+    assert _varlen(lib, cu, **kw) == status
+
+
+def test_varlen_workspace_sizes(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    # CUDA-core path: scratch for the longest sequence, reused by each in turn
+    C, H = 16, 2
+    cu = [0, 5, 45, 62]                       # lengths 5, 40, 17: longest has 3 chunks
+    assert b.chunk_fwd_varlen_workspace_size(cu, H, 16, 16, C, torch.float32) == \
+        H * 3 * (2 * C * C + C) * 4
+    a256 = lambda n: (n + 255) // 256 * 256   # each part starts on a 256-byte boundary
+    assert b.chunk_fwd_varlen_workspace_size(cu, H, 16, 16, C, torch.float32, True, True) == \
+        a256(H * 3 * (2 * C * C + C) * 4) + a256(2 * 62 * H * 16 * 4 + 2 * 62 * H * 4)
+    assert b.chunk_fwd_varlen_workspace_size([0, 0], H, 16, 16, C, torch.float32) == 0
+    assert b.chunk_fwd_varlen_workspace_size([0, 3, 1], H, 16, 16, C, torch.float32) == 0
+
+
+def test_varlen_binding_checks_the_offsets():
+    from gated_delta_rule_130_b200 import binding as b
+    q = torch.zeros(10, 2, 16)
+    la = torch.zeros(10, 2)
+    with pytest.raises(b.GdnError):          # offsets end before the packed tokens do
+        b.chunk_fwd_varlen(q, q, q, la, la, [0, 4, 8])
+    with pytest.raises(b.GdnError):
+        b.chunk_fwd_varlen(q, q, q, la, la, [[0, 10]])
