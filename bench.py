@@ -407,6 +407,37 @@ def run_ours(args):
                     "unfused_prepass_ms_per_step": u_ms,
                     "fused_tokens_per_s": world * tokens / (f_ms * 1e-3), "steps": n_p}
 
+    # packed variable-length batch of the same token count: 12 sequences of mixed
+    # lengths (the serving form), one call over all of them
+    varlen = None
+    if not args.chunk_only:
+        c = I.VARLEN_SERVING
+        lengths = I.varlen_lengths(c["n"], c["total"], c["seed"])
+        vin = I.varlen_inputs(lengths, c["H"], c["Dk"], c["Dv"], "bf16", seed=c["seed"] + rank,
+                              device=device)
+        cu = vin["cu_seqlens"]
+        cu_d = torch.tensor(cu, dtype=torch.int32, device=device)
+        vo = torch.empty((c["total"], c["H"], c["Dv"]), dtype=torch.bfloat16, device=device)
+        vS = torch.empty((c["n"], c["H"], c["Dv"], c["Dk"]), dtype=torch.float32, device=device)
+        vws = torch.empty(max(G.chunk_fwd_varlen_workspace_size(cu, c["H"], c["Dk"], c["Dv"]), 1),
+                          dtype=torch.uint8, device=device)
+
+        def varlen_step():
+            G.chunk_fwd_varlen(vin["q"], vin["k"], vin["v"], vin["log_alpha"], vin["beta"], cu,
+                               out=vo, S_T=vS, workspace=vws, cu_seqlens_device=cu_d)
+
+        n_v = max(20, min(steps, 400))
+        for _ in range(3):
+            varlen_step()
+        v_ms = _max_over_ranks(time_loop(varlen_step, n_v, stream, world), world, device) / n_v
+        varlen = {"workload": f"{c['n']} packed sequences, {c['total']} tokens (lengths "
+                              f"{min(lengths)}..{max(lengths)}), H={c['H']} Dk={c['Dk']} "
+                              f"Dv={c['Dv']} bf16, S0=0",
+                  "lengths": lengths, "ms_per_step": v_ms,
+                  "tokens_per_s": world * c["total"] / (v_ms * 1e-3), "steps": n_v,
+                  "path": "tcgen05" if G.chunk_fwd_path(1, max(lengths), c["H"], c["Dk"], c["Dv"])
+                  == "tcgen05" else "simt"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
@@ -424,7 +455,7 @@ def run_ours(args):
                        "path": path},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
-            "prologue": prologue,
+            "prologue": prologue, "varlen": varlen,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

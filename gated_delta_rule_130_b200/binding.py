@@ -195,12 +195,14 @@ def chunk_fwd_varlen_workspace_size(cu_seqlens, H, Dk, Dv, chunk=64, dtype=torch
 
 def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk: int = 64, out=None,
                      S_T=None, return_state: bool = True, workspace=None, l2norm_qk: bool = False,
-                     gate_logits: bool = False):
+                     gate_logits: bool = False, cu_seqlens_device=None):
     """Chunkwise forward over N variable-length sequences packed without padding.
 
     q, k [total, H, Dk], v [total, H, Dv], log_alpha, beta [total, H]; ``cu_seqlens``
     the N + 1 token offsets (host list or tensor; sequence n is tokens
     cu_seqlens[n] .. cu_seqlens[n + 1] - 1).  S0 / S_T are [N, H, Dv, Dk] float32.
+    ``cu_seqlens_device``: the same offsets as an int32 tensor on q's device (else
+    they are copied there on every call, a synchronous copy).
     Returns (o [total, H, Dv], S_T or None).
     """
     cu = _host_offsets(cu_seqlens)
@@ -236,7 +238,13 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk: int =
         args.append(_dev(S_T, "S_T", torch.float32, dev))
     else:
         args.append(None)
-    cu_dev = cu.to(dev)
+    if cu_seqlens_device is not None:
+        if cu_seqlens_device.shape != cu.shape:
+            raise GdnError("cu_seqlens_device must hold the N + 1 offsets")
+        _dev(cu_seqlens_device, "cu_seqlens_device", torch.int32, dev)
+        cu_dev = cu_seqlens_device
+    else:
+        cu_dev = cu.to(dev)
     need = int(LIB.gdn_chunk_fwd_varlen_workspace_size(cu.data_ptr(), N, H, Dk, Dv, chunk, code,
                                                        flags))
     ws_ptr, ws_bytes = None, 0

@@ -387,6 +387,7 @@ __device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float 
 struct Seqs {
     const int *cu;         // n + 1 token offsets (device), or null
     const int *cu_chunks;  // n + 1 chunk offsets (device), or null
+    const int *order;      // launch order of the sequences (device), or null
     int T;                 // the common length when cu is null
     int n;                 // number of sequences
 };
@@ -413,16 +414,75 @@ __device__ __forceinline__ int seq_of_chunk(const Seqs &q, int g) {
     return lo;
 }
 
-// cu_chunks[b] = sum over earlier sequences of ceil(len / C) (one thread; the
-// sequence count is small next to the work of a call)
-__global__ void seq_chunk_offsets(const int *__restrict__ cu, int n, int *__restrict__ cu_chunks) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        int acc = 0;
-        for (int b = 0; b < n; ++b) {
-            cu_chunks[b] = acc;
-            acc += (cu[b + 1] - cu[b] + C - 1) / C;
+// Bucket of a sequence by its chunk count on a quarter-octave scale (exact below
+// 4 chunks, then 4 buckets per power of two): non-decreasing in the count.
+constexpr int kLenBuckets = 128;
+__device__ __forceinline__ int len_bucket(int chunks) {
+    if (chunks < 4) return chunks;
+    const int msb = 31 - __clz(chunks);
+    return min(kLenBuckets - 1, 4 * msb - 4 + ((chunks >> (msb - 2)) & 3));
+}
+
+// Sequence schedule, one block: cu_chunks[b] = sum over earlier sequences of
+// ceil(len / C) (cu_chunks[n] = all chunks), and order[] = the sequences longest
+// first (by bucket; ties in any order).  The sequential kernel takes sequence
+// order[blockIdx.z], so the CTAs of the longest sequences, which set the
+// critical path, are dispatched in the first wave.
+constexpr int kScheduleThreads = 1024;
+__global__ void __launch_bounds__(kScheduleThreads)
+seq_schedule(const int *__restrict__ cu, int n, int *__restrict__ cu_chunks,
+             int *__restrict__ order) {
+    __shared__ int hist[kLenBuckets];
+    __shared__ int warp_sum[kScheduleThreads / 32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    constexpr int NW = kScheduleThreads / 32;
+    for (int i = tid; i < kLenBuckets; i += kScheduleThreads) hist[i] = 0;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += kScheduleThreads) {
+        const int b = base + tid;
+        const int nc = b < n ? (cu[b + 1] - cu[b] + C - 1) / C : 0;
+        if (b < n) atomicAdd(&hist[len_bucket(nc)], 1);
+        int x = nc;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
         }
-        cu_chunks[n] = acc;
+        if (lane == 31) warp_sum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {  // exclusive scan of the warp totals
+            const int t = warp_sum[lane];
+            int y = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int z = __shfl_up_sync(0xffffffffu, y, o);
+                if (lane >= o) y += z;
+            }
+            warp_sum[lane] = y - t;
+        }
+        __syncthreads();
+        const int excl = carry + warp_sum[warp] + x - nc;
+        if (b < n) cu_chunks[b] = excl;
+        __syncthreads();  // every thread has read carry
+        if (tid == kScheduleThreads - 1) carry = excl + nc;
+        __syncthreads();
+    }
+    static_assert(NW == 32, "one warp scans the warp totals");
+    if (tid == 0) {
+        cu_chunks[n] = carry;
+        int acc = 0;  // bucket starts, longest bucket first
+        for (int k = kLenBuckets - 1; k >= 0; --k) {
+            const int c = hist[k];
+            hist[k] = acc;
+            acc += c;
+        }
+    }
+    __syncthreads();
+    for (int b = tid; b < n; b += kScheduleThreads) {
+        const int nc = (cu[b + 1] - cu[b] + C - 1) / C;
+        order[atomicAdd(&hist[len_bucket(nc)], 1)] = b;
     }
 }
 
@@ -676,7 +736,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float *gv_all = reinterpret_cast<float *>(base + SM_GV);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int vt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int vt = blockIdx.x, h = blockIdx.y;
+    const int b = p.sq.order ? p.sq.order[blockIdx.z] : (int)blockIdx.z;
     const int v0 = vt * DVT;
     const int H = p.H;
     // sequence b: tokens sp.off .. sp.off + T of the packed rows, chunks sp.chunk0 ..
@@ -1248,8 +1309,9 @@ bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 
 // Workspace: [chunk offsets of the sequences, variable lengths only, padded to
 // 256 B][one [T'; T''] tile per chunk and head][1/|k| per token, normalising only].
+// chunk offsets (n + 1) and launch order (n) of the sequences
 static size_t tc_offsets_bytes(int n_seq, bool varlen) {
-    return varlen ? (((size_t)n_seq + 1) * sizeof(int) + 255) & ~size_t(255) : 0;
+    return varlen ? ((2 * (size_t)n_seq + 1) * sizeof(int) + 255) & ~size_t(255) : 0;
 }
 
 size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
@@ -1288,7 +1350,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
         !tc::make_map_tt(&mt, tt, total_chunks > 0 ? total_chunks * H : 1))
         return cudaErrorInvalidValue;
     if (varlen) {
-        tc::seq_chunk_offsets<<<1, 32, 0, st>>>(cu_seqlens, n_seq, cu_chunks);
+        tc::seq_schedule<<<1, tc::kScheduleThreads, 0, st>>>(cu_seqlens, n_seq, cu_chunks,
+                                                             cu_chunks + n_seq + 1);
         const cudaError_t e0 = cudaPeekAtLastError();
         if (e0 != cudaSuccess) return e0;
     }
@@ -1298,7 +1361,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
     p.S0 = S0;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.S_T = S_T;
-    p.sq = tc::Seqs{cu_seqlens, cu_chunks, T_fixed, n_seq};
+    p.sq = tc::Seqs{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
+                    n_seq};
     p.H = H;
     p.Dv = Dv;
     p.rk = rk;

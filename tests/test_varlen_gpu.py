@@ -127,3 +127,17 @@ def test_varlen_tcgen05_workspace_size(gdn):
     # with L2 normalisation the per-row key scales (float32) follow the tiles
     assert gdn.chunk_fwd_varlen_workspace_size([0, 1, 66], 4, 128, 128, 64, torch.bfloat16,
                                                l2norm_qk=True) == 256 + 3 * tile + 3 * 4 * 64 * 4
+
+
+def test_varlen_device_offsets_give_the_same_bits(gdn):
+    lengths = [100, 3, 64]
+    inp = I.varlen_inputs(lengths, 2, 128, 128, "bf16", s0_law="normal002", seed=8,
+                          device="cuda")
+    cu = inp["cu_seqlens"]
+    args = [inp[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+    o1, S1 = gdn.chunk_fwd_varlen(*args, cu, S0=inp["S0"])
+    o2, S2 = gdn.chunk_fwd_varlen(*args, cu, S0=inp["S0"],
+                                  cu_seqlens_device=torch.tensor(cu, dtype=torch.int32,
+                                                                 device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
