@@ -220,3 +220,202 @@ int gdn_oracle_decode(const double *q, const double *k, const double *v,
     j.units = units; j.n_units = n_units; j.mode = 1;
     return run_job(&j, nthreads);
 }
+
+/*
+ * Backward: the exact reverse-mode derivative of (1) and (2) for a scalar loss
+ * L with given dL/do_t (d_o) and dL/dS_T (dS_T, NULL for zero).  The pages name
+ * the parallel (chunkwise) training algorithm but print no backward; the plain
+ * reading is the gradient of the forward above, taken token by token in reverse.
+ * With G the gradient of S_t (all later uses), A_t = alpha (I - beta k k^T):
+ *
+ *   G      += do_t q_t^T                          (from o_t = S_t q_t)
+ *   dq_t    = S_t^T do_t
+ *   dv_t    = beta G k
+ *   dbeta_t = (v - alpha S_{t-1} k) . (G k)
+ *   dalpha  = <G, S_{t-1}> - beta (S_{t-1} k) . (G k),  dlog_alpha_t = alpha dalpha
+ *   dk_t    = beta G^T v - alpha beta (G^T S_{t-1} k + S_{t-1}^T G k)
+ *   G      <- G A_t = alpha (G - beta (G k) k^T)  (the gradient of S_{t-1})
+ *
+ * and dS0 is G after token 0.  S_{t-1} is needed in reverse order: the states at
+ * every CKPT-th token are kept from a forward sweep and each block of tokens is
+ * swept forward again from its checkpoint before it is walked backwards.
+ */
+#define CKPT 64
+
+typedef struct {
+    const double *q, *k, *v, *la, *beta, *S0, *d_o, *dS_T;
+    double *dq, *dk, *dv, *dla, *dbeta, *dS0;
+    long B, T, H, Dk, Dv;
+    const int *units;
+    int n_units, n_threads, thread_id;
+    int status;
+} bjob_t;
+
+static void bwd_unit(bjob_t *j, long u)
+{
+    const long b = u / j->H, h = u % j->H, T = j->T, H = j->H, Dk = j->Dk, Dv = j->Dv;
+    const long SZ = Dv * Dk;
+    const long nblk = (T + CKPT - 1) / CKPT;
+    /* ck[c]: state before token c*CKPT; st[i]: state after token blk*CKPT+i-1 */
+    double *ck = (double *)malloc(sizeof(double) * (size_t)((nblk > 0 ? nblk : 1) * SZ));
+    double *st = (double *)malloc(sizeof(double) * (size_t)((CKPT + 1) * SZ));
+    double *G = (double *)malloc(sizeof(double) * (size_t)SZ);
+    double *o_scratch = (double *)malloc(sizeof(double) * (size_t)Dv);
+    double *sk = (double *)malloc(sizeof(double) * (size_t)Dv);
+    double *Gk = (double *)malloc(sizeof(double) * (size_t)Dv);
+    if (!ck || !st || !G || !o_scratch || !sk || !Gk) {
+        j->status = -2;
+        free(ck); free(st); free(G); free(o_scratch); free(sk); free(Gk);
+        return;
+    }
+#define QK(t) (((b * T + (t)) * H + h) * Dk)
+#define VV(t) (((b * T + (t)) * H + h) * Dv)
+#define GG(t) ((b * T + (t)) * H + h)
+    /* forward sweep keeping the checkpoints */
+    double *S = st;
+    if (j->S0)
+        memcpy(S, j->S0 + u * SZ, sizeof(double) * (size_t)SZ);
+    else
+        memset(S, 0, sizeof(double) * (size_t)SZ);
+    for (long t = 0; t < T; ++t) {
+        if (t % CKPT == 0)
+            memcpy(ck + (t / CKPT) * SZ, S, sizeof(double) * (size_t)SZ);
+        gdn_token(S, j->q + QK(t), j->k + QK(t), j->v + VV(t), j->la[GG(t)], j->beta[GG(t)],
+                  o_scratch, Dk, Dv);
+    }
+    if (j->dS_T)
+        memcpy(G, j->dS_T + u * SZ, sizeof(double) * (size_t)SZ);
+    else
+        memset(G, 0, sizeof(double) * (size_t)SZ);
+    for (long blk = nblk - 1; blk >= 0; --blk) {
+        const long t0 = blk * CKPT, t1 = (t0 + CKPT < T) ? t0 + CKPT : T;
+        memcpy(st, ck + blk * SZ, sizeof(double) * (size_t)SZ);
+        for (long t = t0; t < t1; ++t) {
+            double *nxt = st + (t - t0 + 1) * SZ;
+            memcpy(nxt, st + (t - t0) * SZ, sizeof(double) * (size_t)SZ);
+            gdn_token(nxt, j->q + QK(t), j->k + QK(t), j->v + VV(t), j->la[GG(t)],
+                      j->beta[GG(t)], o_scratch, Dk, Dv);
+        }
+        for (long t = t1 - 1; t >= t0; --t) {
+            const double *Sp = st + (t - t0) * SZ;     /* S_{t-1} */
+            const double *Sc = st + (t - t0 + 1) * SZ; /* S_t */
+            const double *q = j->q + QK(t), *k = j->k + QK(t), *v = j->v + VV(t);
+            const double *dout = j->d_o + VV(t);
+            const double alpha = exp(j->la[GG(t)]), beta = j->beta[GG(t)];
+            double *dq = j->dq + QK(t), *dk = j->dk + QK(t), *dv = j->dv + VV(t);
+            for (long i = 0; i < Dv; ++i)
+                for (long m = 0; m < Dk; ++m)
+                    G[i * Dk + m] += dout[i] * q[m];
+            for (long m = 0; m < Dk; ++m) {
+                double a = 0.0;
+                for (long i = 0; i < Dv; ++i)
+                    a += Sc[i * Dk + m] * dout[i];
+                dq[m] = a;
+            }
+            double dbeta = 0.0, dalpha = 0.0;
+            for (long i = 0; i < Dv; ++i) {
+                double a = 0.0, c = 0.0;
+                for (long m = 0; m < Dk; ++m) {
+                    a += Sp[i * Dk + m] * k[m];
+                    c += G[i * Dk + m] * k[m];
+                    dalpha += G[i * Dk + m] * Sp[i * Dk + m];
+                }
+                sk[i] = a;
+                Gk[i] = c;
+                dv[i] = beta * c;
+                dbeta += (v[i] - alpha * a) * c;
+                dalpha -= beta * a * c;
+            }
+            for (long m = 0; m < Dk; ++m) {
+                double gv = 0.0, gs = 0.0, sg = 0.0;
+                for (long i = 0; i < Dv; ++i) {
+                    gv += G[i * Dk + m] * v[i];
+                    gs += G[i * Dk + m] * sk[i];
+                    sg += Sp[i * Dk + m] * Gk[i];
+                }
+                dk[m] = beta * gv - alpha * beta * (gs + sg);
+            }
+            j->dbeta[GG(t)] = dbeta;
+            j->dla[GG(t)] = alpha * dalpha;
+            for (long i = 0; i < Dv; ++i)
+                for (long m = 0; m < Dk; ++m)
+                    G[i * Dk + m] = alpha * (G[i * Dk + m] - beta * Gk[i] * k[m]);
+        }
+    }
+    memcpy(j->dS0 + u * SZ, G, sizeof(double) * (size_t)SZ);
+#undef QK
+#undef VV
+#undef GG
+    free(ck); free(st); free(G); free(o_scratch); free(sk); free(Gk);
+}
+
+static void *bwd_worker(void *arg)
+{
+    bjob_t *j = (bjob_t *)arg;
+    const long n = j->units ? j->n_units : j->B * j->H;
+    for (long i = j->thread_id; i < n; i += j->n_threads)
+        bwd_unit(j, j->units ? (long)j->units[i] : i);
+    return NULL;
+}
+
+/*
+ * Gradients of every input for the units listed (all when units is NULL):
+ * dq, dk [B,T,H,Dk], dv [B,T,H,Dv], dlog_alpha, dbeta [B,T,H], dS0 [B,H,Dv,Dk].
+ * S0 and dS_T may be NULL (zero).  Only the listed units' slices are written.
+ * Returns 0, -1 on a bad argument, -2 on allocation failure.
+ */
+int gdn_oracle_backward(const double *q, const double *k, const double *v,
+                        const double *log_alpha, const double *beta, const double *S0,
+                        const double *d_o, const double *dS_T,
+                        double *dq, double *dk, double *dv, double *dlog_alpha,
+                        double *dbeta, double *dS0,
+                        long B, long T, long H, long Dk, long Dv,
+                        const int *units, int n_units, int nthreads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk || !dv || !dlog_alpha ||
+        !dbeta || !dS0)
+        return -1;
+    if (B <= 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0)
+        return -1;
+    if (check_units(units, n_units, B * H))
+        return -1;
+    const long n = units ? n_units : B * H;
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > n)
+        nthreads = (int)(n > 0 ? n : 1);
+    bjob_t *jobs = (bjob_t *)malloc(sizeof(bjob_t) * (size_t)nthreads);
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!jobs || !tid) {
+        free(jobs);
+        free(tid);
+        return -2;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        bjob_t *j = &jobs[i];
+        memset(j, 0, sizeof(*j));
+        j->q = q; j->k = k; j->v = v; j->la = log_alpha; j->beta = beta; j->S0 = S0;
+        j->d_o = d_o; j->dS_T = dS_T;
+        j->dq = dq; j->dk = dk; j->dv = dv; j->dla = dlog_alpha; j->dbeta = dbeta; j->dS0 = dS0;
+        j->B = B; j->T = T; j->H = H; j->Dk = Dk; j->Dv = Dv;
+        j->units = units; j->n_units = n_units; j->n_threads = nthreads; j->thread_id = i;
+    }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&tid[i], NULL, bwd_worker, &jobs[i]) != 0)
+            break;
+        started = i;
+    }
+    bwd_worker(&jobs[0]);
+    for (int i = 1; i <= started; ++i)
+        pthread_join(tid[i], NULL);
+    for (int i = started + 1; i < nthreads; ++i)
+        bwd_worker(&jobs[i]);
+    int status = 0;
+    for (int i = 0; i < nthreads; ++i)
+        if (jobs[i].status)
+            status = jobs[i].status;
+    free(jobs);
+    free(tid);
+    return status;
+}

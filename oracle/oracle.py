@@ -6,7 +6,8 @@ executes anything in this directory, and this module imports nothing from it.
 
 The oracle is the gated delta rule applied token by token in float64,
     S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T)) + beta_t v_t k_t^T,  o_t = S_t q_t,
-see the header of ``gdn_oracle.c`` for the pages it follows and the readings taken.
+and its exact reverse-mode gradient (``backward``); see the header of
+``gdn_oracle.c`` for the pages it follows and the readings taken.
 """
 from __future__ import annotations
 
@@ -46,6 +47,9 @@ def _bind(path: str):
     lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp, L, L, L, L, L,
                                       ip, ctypes.c_int, ctypes.c_int]
     lib.gdn_oracle_decode.restype = ctypes.c_int
+    lib.gdn_oracle_backward.argtypes = [dp] * 14 + [L, L, L, L, L, ip, ctypes.c_int,
+                                                    ctypes.c_int]
+    lib.gdn_oracle_backward.restype = ctypes.c_int
     return lib
 
 
@@ -133,6 +137,37 @@ def decode(q, k, v, log_alpha, beta, S, units=None, nthreads=None, lib=None):
     if rc != 0:
         raise RuntimeError(f"gdn_oracle_decode failed ({rc})")
     return o, s
+
+
+def backward(q, k, v, log_alpha, beta, S0, d_o, dS_T=None, units=None, nthreads=None, lib=None):
+    """Exact gradients of a scalar loss through the whole-sequence recurrence.
+
+    Inputs as for ``forward`` plus d_o = dL/do [B,T,H,Dv] and dS_T = dL/dS_T
+    [B,H,Dv,Dk] (None: zero).  Returns (dq, dk, dv, dlog_alpha, dbeta, dS0) as
+    float64 arrays in the layouts of q, k, v, log_alpha, beta and S0.  With
+    ``units`` only those heads are computed (NaN elsewhere).
+    """
+    q, k, v, la, be, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_o))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, T, H) or la.shape != (B, T, H) \
+            or be.shape != (B, T, H) or do.shape != v.shape:
+        raise ValueError("shape mismatch")
+    s0 = None if S0 is None else _f64(S0)
+    ds = None if dS_T is None else _f64(dS_T)
+    for x, n in ((s0, "S0"), (ds, "dS_T")):
+        if x is not None and x.shape != (B, H, Dv, Dk):
+            raise ValueError(f"{n} must be [B,H,Dv,Dk]")
+    fill = np.nan if units is not None else 0.0
+    out = [np.full(q.shape, fill), np.full(q.shape, fill), np.full(v.shape, fill),
+           np.full(la.shape, fill), np.full(la.shape, fill), np.full((B, H, Dv, Dk), fill)]
+    up, nu, _keep = _units(units, B * H)
+    rc = (lib or _load()).gdn_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(s0), _ptr(do), _ptr(ds),
+        *(_ptr(a) for a in out), B, T, H, Dk, Dv, up, nu, int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_backward failed ({rc})")
+    return tuple(out)
 
 
 def load_variant(path: str):
