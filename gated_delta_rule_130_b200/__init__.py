@@ -9,7 +9,8 @@ first such use raises if ``libgdn.so`` is missing -- there is no fallback.
 
 _BINDING_NAMES = {
     "chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_varlen_workspace_size", "decode_step",
-    "chunk_fwd_workspace_size", "chunk_fwd_path", "library_path",
+    "chunk_fwd_workspace_size", "chunk_fwd_path", "library_path", "chunk_bwd",
+    "chunk_bwd_workspace_size",
     "GdnError", "check_device_status",
 }
 

@@ -56,6 +56,11 @@ def _load():
     lib.gdn_chunk_fwd_varlen.restype = I
     lib.gdn_chunk_fwd_varlen_workspace_size.argtypes = [vp, I, I, I, I, I, I, U]
     lib.gdn_chunk_fwd_varlen_workspace_size.restype = Z
+    lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, I, I, I,
+                                  I, I, I, I, vp, Z, vp]
+    lib.gdn_chunk_bwd.restype = I
+    lib.gdn_chunk_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_bwd_workspace_size.restype = Z
     lib.gdn_check_device_status.argtypes = []
     lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]
@@ -176,6 +181,56 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=
                               _stream_ptr(dev))
     _check(st, "gdn_chunk_fwd")
     return o, S_T
+
+
+def chunk_bwd_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> int:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(LIB.gdn_chunk_bwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, S0, d_o, dS_T=None, chunk: int = 64, workspace=None,
+              want_dS0: bool = True):
+    """Chunkwise backward of ``chunk_fwd`` (plain gates, no prologue).
+
+    Given the forward's inputs and d_o = dL/do [B,T,H,Dv] (q's dtype), dS_T =
+    dL/dS_T [B,H,Dv,Dk] float32 or None, returns (dq, dk, dv, dlog_alpha, dbeta,
+    dS0): dq, dk, dv in q's dtype, the rest float32 (dS0 None unless want_dS0).
+    """
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise GdnError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[3]
+    dev = q.device
+    code = _dtype_code(q)
+    if log_alpha.shape != (B, T, H) or beta.shape != (B, T, H):
+        raise GdnError("log_alpha and beta must be [B,T,H]")
+    if d_o.shape != v.shape:
+        raise GdnError("d_o must be [B,T,H,Dv]")
+    state = (B, H, Dv, Dk)
+    for x, n in ((S0, "S0"), (dS_T, "dS_T")):
+        if x is not None and x.shape != state:
+            raise GdnError(f"{n} must be [B,H,Dv,Dk]")
+    opt = lambda x, n: _dev(x, n, torch.float32, dev) if x is not None else None
+    args = [_dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
+            _dev(log_alpha, "log_alpha", torch.float32, dev),
+            _dev(beta, "beta", torch.float32, dev), opt(S0, "S0"),
+            _dev(d_o, "d_o", q.dtype, dev), opt(dS_T, "dS_T")]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    dbe = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    dS0 = torch.empty(state, dtype=torch.float32, device=dev) if want_dS0 else None
+    args += [dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dla.data_ptr(), dbe.data_ptr(),
+             dS0.data_ptr() if dS0 is not None else None]
+    need = int(LIB.gdn_chunk_bwd_workspace_size(B, T, H, Dk, Dv, chunk, code))
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    st = LIB.gdn_chunk_bwd(*args, B, T, H, Dk, Dv, chunk, code, ws_ptr, ws_bytes,
+                           _stream_ptr(dev))
+    _check(st, "gdn_chunk_bwd")
+    return dq, dk, dv, dla, dbe, dS0
 
 
 def _host_offsets(cu_seqlens) -> torch.Tensor:

@@ -35,7 +35,8 @@ size_t simt_workspace_bytes(int B, int T, int H, int C) {
     return (size_t)B * H * NT * per_chunk_floats(C) * sizeof(float);
 }
 
-template <typename T>
+// kPT: write P' = P T (the forward's read-out); else P itself (the backward's).
+template <typename T, bool kPT>
 __global__ void __launch_bounds__(256)
 chunk_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
            const float *__restrict__ beta, float *__restrict__ ws, int Tlen, int H, int Dk, int C,
@@ -119,9 +120,10 @@ chunk_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__rest
     for (int idx = threadIdx.x; idx < C * C; idx += blockDim.x) {
         const int r = idx / C, j = idx - r * C;
         float acc = 0.f;  // (P T)[r][j]; both factors lower triangular
-        for (int i = j; i <= r; ++i) acc += P[r * C + i] * Tm[i * C + j];
+        if (kPT)
+            for (int i = j; i <= r; ++i) acc += P[r * C + i] * Tm[i * C + j];
         out[idx] = Tm[idx];
-        out[C * C + idx] = acc;
+        out[C * C + idx] = kPT ? acc : P[idx];
     }
     if (threadIdx.x < C) out[2 * C * C + threadIdx.x] = g[threadIdx.x];
 }
@@ -130,8 +132,8 @@ template <typename T, int DVT>
 __global__ void __launch_bounds__(256)
 chunk_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
             const float *__restrict__ beta, const float *__restrict__ S0, T *__restrict__ o,
-            float *__restrict__ S_T, const float *__restrict__ ws, int Tlen, int H, int Dk, int Dv,
-            int C, int NT) {
+            float *__restrict__ S_T, const float *__restrict__ ws, float *__restrict__ S_hist,
+            int Tlen, int H, int Dk, int Dv, int C, int NT) {
     extern __shared__ float sm[];
     const int v0 = blockIdx.x * DVT, h = blockIdx.y, b = blockIdx.z;
     const int nv = min(DVT, Dv - v0);
@@ -158,6 +160,13 @@ chunk_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restric
         const int t0 = c * C, n = min(C, Tlen - t0);
         const float *wsc = ws + (head * NT + c) * per_chunk_floats(C);
         __syncthreads();  // previous chunk has finished with every buffer
+        if (S_hist) {     // the state entering chunk c (the backward recomputes it)
+            float *dst = S_hist + ((head * NT + c) * Dv + v0) * Dk;
+            for (int idx = threadIdx.x; idx < nv * Dk; idx += blockDim.x) {
+                const int i = idx / Dk, j = idx - i * Dk;
+                dst[idx] = Ss[i * ldk + j];
+            }
+        }
         for (int idx = threadIdx.x; idx < C * Dk; idx += blockDim.x) {
             const int r = idx / Dk, j = idx - r * Dk;
             float kv = 0.f, qv = 0.f;
@@ -210,7 +219,7 @@ chunk_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restric
                 y += Pp[r * C + m] * rr;
             }
             Un[r * ldv + i] = u;
-            if (r < n && i < nv)
+            if (o && r < n && i < nv)
                 o[(((size_t)b * Tlen + t0 + r) * H + h) * Dv + v0 + i] =
                     from_f32<T>(Xq[r * ldv + i] + y);
         }
@@ -245,20 +254,65 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
                                2 * (size_t)C * C + 3 * (size_t)C * (DVT + 1) + 3 * C + 1) *
                               sizeof(float);
     cudaError_t e;
-    e = cudaFuncSetAttribute(chunk_prep<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_prep<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_prep);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_state<T, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    chunk_prep<T><<<dim3(NT, H, B), 256, smem_prep, st>>>(
+    chunk_prep<T, true><<<dim3(NT, H, B), 256, smem_prep, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws, Tlen, H, Dk, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), 256, smem_state, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0,
-        static_cast<T *>(o), S_T, ws, Tlen, H, Dk, Dv, C, NT);
+        static_cast<T *>(o), S_T, ws, nullptr, Tlen, H, Dk, Dv, C, NT);
     return cudaPeekAtLastError();
+}
+
+// The backward's recomputation: T, P and g of every chunk into ws_prep, and the
+// state entering every chunk into S_hist ([B, H, NT, Dv, Dk] float32).
+template <typename T, int DVT>
+static cudaError_t launch_recompute_t(const void *q, const void *k, const void *v,
+                                      const float *la, const float *beta, const float *S0,
+                                      int B, int Tlen, int H, int Dk, int Dv, int C,
+                                      float *ws_prep, float *S_hist, cudaStream_t st) {
+    const int NT = (Tlen + C - 1) / C;
+    const size_t smem_prep = (2 * (size_t)C * (Dk + 1) + 3 * (size_t)C * C + 2 * C) * sizeof(float);
+    const size_t smem_state = ((size_t)DVT * (Dk + 1) + 2 * (size_t)C * (Dk + 1) +
+                               2 * (size_t)C * C + 3 * (size_t)C * (DVT + 1) + 3 * C + 1) *
+                              sizeof(float);
+    cudaError_t e;
+    e = cudaFuncSetAttribute(chunk_prep<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_prep);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_state<T, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_state);
+    if (e != cudaSuccess) return e;
+    chunk_prep<T, false><<<dim3(NT, H, B), 256, smem_prep, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws_prep, Tlen, H, Dk, C,
+        NT);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), 256, smem_state, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0,
+        nullptr, nullptr, ws_prep, S_hist, Tlen, H, Dk, Dv, C, NT);
+    return cudaPeekAtLastError();
+}
+
+cudaError_t launch_bwd_recompute(const void *q, const void *k, const void *v, const float *la,
+                                 const float *beta, const float *S0, int B, int T, int H, int Dk,
+                                 int Dv, int chunk, bool bf16, float *ws_prep, float *S_hist,
+                                 cudaStream_t st) {
+    if (Dk > 128)
+        return bf16 ? launch_recompute_t<__nv_bfloat16, 16>(q, k, v, la, beta, S0, B, T, H, Dk,
+                                                            Dv, chunk, ws_prep, S_hist, st)
+                    : launch_recompute_t<float, 16>(q, k, v, la, beta, S0, B, T, H, Dk, Dv, chunk,
+                                                    ws_prep, S_hist, st);
+    return bf16 ? launch_recompute_t<__nv_bfloat16, 32>(q, k, v, la, beta, S0, B, T, H, Dk, Dv,
+                                                        chunk, ws_prep, S_hist, st)
+                : launch_recompute_t<float, 32>(q, k, v, la, beta, S0, B, T, H, Dk, Dv, chunk,
+                                                ws_prep, S_hist, st);
 }
 
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *la,

@@ -269,6 +269,73 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
+                                    gdn_dtype_t dtype) {
+    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::bwd_supported(Dk, chunk))
+        return 0;
+    if (empty_problem(B, T, H)) return 0;
+    return gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk);
+}
+
+gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *S0, const void *d_o,
+                           const float *dS_T, void *dq, void *dk, void *dv, float *dlog_alpha,
+                           float *dbeta, float *dS0, int B, int T, int H, int Dk, int Dv,
+                           int chunk, gdn_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    const gdn_status_t sz = check_sizes(B, T, H, Dk, Dv, chunk, dtype);
+    if (sz != GDN_OK) return sz;
+    if (!gdn::bwd_supported(Dk, chunk)) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4;
+    const size_t n_tok = (size_t)B * T * H;
+    const size_t state_bytes = (size_t)B * H * Dv * Dk * sizeof(float);
+    if (B == 0 || H == 0) return GDN_OK;
+    if (T == 0) {  // no tokens: dS0 = dS_T
+        if (!dS0) return GDN_OK;
+        if (!aligned16(dS0) || (dS_T && !aligned16(dS_T))) return GDN_ERR_INVALID_ARG;
+        if (dS_T && dS_T != dS0 && overlaps(dS0, state_bytes, dS_T, state_bytes))
+            return GDN_ERR_INVALID_ARG;
+        cudaError_t e = dS_T ? (dS_T == dS0 ? cudaSuccess
+                                            : cudaMemcpyAsync(dS0, dS_T, state_bytes,
+                                                              cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(dS0, 0, state_bytes, st);
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+    if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk || !dv || !dlog_alpha ||
+        !dbeta)
+        return GDN_ERR_INVALID_ARG;
+    const struct { const void *p; size_t n; } in[] = {
+        {q, n_tok * Dk * esz}, {k, n_tok * Dk * esz}, {v, n_tok * Dv * esz},
+        {log_alpha, n_tok * sizeof(float)}, {beta, n_tok * sizeof(float)}, {S0, state_bytes},
+        {d_o, n_tok * Dv * esz}, {dS_T, state_bytes}};
+    const struct { const void *p; size_t n; } out[] = {
+        {dq, n_tok * Dk * esz}, {dk, n_tok * Dk * esz}, {dv, n_tok * Dv * esz},
+        {dlog_alpha, n_tok * sizeof(float)}, {dbeta, n_tok * sizeof(float)}, {dS0, state_bytes}};
+    for (const auto &a : in)
+        if (a.p && !aligned16(a.p)) return GDN_ERR_INVALID_ARG;
+    for (const auto &a : out)
+        if (a.p && !aligned16(a.p)) return GDN_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    // outputs alias neither an input nor one another
+    for (size_t i = 0; i < sizeof(out) / sizeof(out[0]); ++i) {
+        for (const auto &a : in)
+            if (overlaps(out[i].p, out[i].n, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+        for (size_t j = i + 1; j < sizeof(out) / sizeof(out[0]); ++j)
+            if (overlaps(out[i].p, out[i].n, out[j].p, out[j].n)) return GDN_ERR_INVALID_ARG;
+    }
+    const size_t need = gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    for (const auto &a : in)
+        if (overlaps(workspace, need, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+    for (const auto &a : out)
+        if (overlaps(workspace, need, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_chunk_bwd(q, k, v, log_alpha, beta, S0, d_o, dS_T, dq, dk, dv,
+                                                dlog_alpha, dbeta, dS0, B, T, H, Dk, Dv, chunk,
+                                                dtype == GDN_BF16, workspace, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status_t gdn_check_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
     unsigned int flag = 0;

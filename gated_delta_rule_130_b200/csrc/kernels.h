@@ -33,6 +33,24 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               int T, int H, int Dk, int Dv, int chunk, bool bf16, void *workspace,
                               cudaStream_t st);
 
+// The backward's recomputation on the CUDA-core path (chunk_simt.cu): T, P, g
+// per chunk into ws_prep ([B,H,NT] x (2 C^2 + C) floats) and the state entering
+// every chunk into S_hist ([B,H,NT,Dv,Dk] floats).
+cudaError_t launch_bwd_recompute(const void *q, const void *k, const void *v, const float *la,
+                                 const float *beta, const float *S0, int B, int T, int H, int Dk,
+                                 int Dv, int chunk, bool bf16, float *ws_prep, float *S_hist,
+                                 cudaStream_t st);
+
+// CUDA-core chunkwise backward (Dk <= 128): chunk_bwd.cu.  Workspace: the
+// recomputed T, P, g, the chunk states and the state gradients.
+bool bwd_supported(int Dk, int chunk);
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk);
+cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la,
+                             const float *beta, const float *S0, const void *d_o,
+                             const float *dS_T, void *dq, void *dk, void *dv, float *dla,
+                             float *dbeta, float *dS0, int B, int T, int H, int Dk, int Dv,
+                             int chunk, bool bf16, void *workspace, cudaStream_t st);
+
 // tcgen05 chunkwise forward (bf16, Dk = 128, chunk 64): chunk_tc.cu.  The
 // workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of every head.
 // With the L2-normalisation flag the workspace also holds 1/|k| per token.

@@ -215,6 +215,41 @@ gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v,
                                 gdn_dtype_t dtype, unsigned flags, void *stream);
 
 /*
+ * Chunkwise backward: the gradients of a scalar loss L through gdn_chunk_fwd,
+ * given dL/do and dL/dS_T.  The pages name the parallel (chunkwise) training
+ * algorithm ("Gated Delta Networks: Improving Mamba2 with Delta Rule", section
+ * "Approach"; "Gated DeltaNet: Harmonizing Gating and the Delta Rule ...",
+ * section "Hardware-Efficient Training") but print no backward; this is the
+ * exact derivative of the forward (plain gates: log_alpha and beta as given,
+ * no prologue), computed chunk by chunk through the WY/UT form.
+ *
+ *   inputs  q, k [B,T,H,Dk], v [B,T,H,Dv] in `dtype`; log_alpha, beta [B,T,H]
+ *           float32; S0 [B,H,Dv,Dk] float32 or NULL (zeros) -- as for the forward;
+ *           d_o [B,T,H,Dv] in `dtype`; dS_T [B,H,Dv,Dk] float32 or NULL (zeros).
+ *   outputs dq, dk [B,T,H,Dk] and dv [B,T,H,Dv] in `dtype`; dlog_alpha, dbeta
+ *           [B,T,H] float32; dS0 [B,H,Dv,Dk] float32 or NULL (not written).
+ *
+ * Arithmetic is float32 on the CUDA cores (bf16 inputs are widened; bf16
+ * gradients are rounded once at the end).  Three launches: the forward's
+ * per-chunk T, P, g and chunk states are recomputed into the workspace
+ * (gdn_chunk_bwd_workspace_size bytes: (2 C^2 + C + 2 Dv Dk) floats per chunk
+ * and head), the state gradient is walked back over the chunks, and the
+ * per-chunk gradients are formed in parallel.  Limits as for the forward plus
+ * Dk <= 128 (GDN_ERR_UNSUPPORTED otherwise).  Outputs must not overlap any
+ * input or each other; the workspace must not overlap anything.  T = 0 only
+ * sets dS0 = dS_T.  Enqueued on `stream`.
+ */
+gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta, const float *S0,
+                           const void *d_o, const float *dS_T,
+                           void *dq, void *dk, void *dv, float *dlog_alpha, float *dbeta,
+                           float *dS0, int B, int T, int H, int Dk, int Dv, int chunk,
+                           gdn_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                           void *stream);
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
+                                    gdn_dtype_t dtype);
+
+/*
  * Synchronise the current device and report whether a fused tensor-core
  * kernel gave up since the last check: its pipeline waits are bounded (about
  * two seconds each); a CTA that times out stops, records a flag and leaves its

@@ -191,3 +191,38 @@ def test_varlen_binding_checks_the_offsets():
         b.chunk_fwd_varlen(q, q, q, la, la, [0, 4, 8])
     with pytest.raises(b.GdnError):
         b.chunk_fwd_varlen(q, q, q, la, la, [[0, 10]])
+
+
+def _bwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, la=16, beta=16, S0=None, do=1 << 20, dS_T=None, dq=1 << 24,
+             dk=1 << 25, dv=1 << 26, dla=1 << 27, dbeta=1 << 28, dS0=None, B=1, T=8, H=1, Dk=16,
+             Dv=16, chunk=16, dtype=0, ws=1 << 40, ws_bytes=1 << 30)
+    a.update(kw)
+    return lib.gdn_chunk_bwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["do"],
+                             a["dS_T"], a["dq"], a["dk"], a["dv"], a["dla"], a["dbeta"], a["dS0"],
+                             a["B"], a["T"], a["H"], a["Dk"], a["Dv"], a["chunk"], a["dtype"],
+                             a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(do=None), 1), (dict(dq=None), 1), (dict(dbeta=None), 1),
+    (dict(Dk=0), 1), (dict(dtype=3), 1), (dict(chunk=48), 2),
+    (dict(Dk=144), 2),                                     # the backward takes Dk <= 128
+    (dict(dq=24), 1),                                      # misaligned
+    (dict(dq=16), 1),                                      # a gradient overlaps q
+    (dict(dk=1 << 24), 1),                                 # two gradients overlap
+    (dict(ws=None), 1), (dict(ws_bytes=64), 1), (dict(ws=1 << 20), 1),
+    (dict(B=0), 0), (dict(H=0), 0), (dict(T=0), 0),        # nothing to do (dS0 not asked)
+])
+def test_chunk_bwd_rejects_before_launch(lib, kw, status):
+    assert _bwd(lib, **kw) == status
+
+
+def test_chunk_bwd_workspace_size(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    # recomputed T, P (C x C) and g (C), the chunk state and its gradient (Dv x Dk)
+    C, NT, H, Dk, Dv = 16, 3, 2, 32, 8
+    assert b.chunk_bwd_workspace_size(1, 40, H, Dk, Dv, C, torch.float32) == \
+        H * NT * (2 * C * C + C + 2 * Dv * Dk) * 4
+    assert b.chunk_bwd_workspace_size(1, 40, H, 256, Dv, C, torch.float32) == 0
+    assert b.chunk_bwd_workspace_size(1, 0, H, Dk, Dv, C, torch.float32) == 0
