@@ -83,6 +83,16 @@ def chunk_bytes(w, has_s0: bool) -> float:
     return tok * (esz * (2 * w.Dk + 2 * w.Dv) + 8) + state * (2 if has_s0 else 1)
 
 
+def bwd_bytes(w, has_s0: bool) -> float:
+    """Compulsory HBM bytes of one chunkwise backward: q, k, v and d_o read and dq,
+    dk, dv written once in the element type, both gates read and both gate
+    gradients written (float32); S0 (if given) and dS_T read, dS0 written."""
+    esz = 2 if w.dtype == "bf16" else 4
+    tok = w.B * w.T * w.H
+    state = w.B * w.H * w.Dv * w.Dk * 4
+    return tok * (esz * (4 * w.Dk + 3 * w.Dv) + 16) + state * (3 if has_s0 else 2)
+
+
 def decode_bytes(w) -> float:
     """Compulsory HBM bytes of one decode step: the float32 state read and written,
     q, k, v read and o written in the element type, the two gates read."""
@@ -438,6 +448,34 @@ def run_ours(args):
                   "path": "tcgen05" if G.chunk_fwd_path(1, max(lengths), c["H"], c["Dk"], c["Dv"])
                   == "tcgen05" else "simt"}
 
+    # chunkwise backward of the headline call (given dL/do and dL/dS_T)
+    backward = None
+    if not args.chunk_only:
+        gen = torch.Generator().manual_seed(w.seed + 99 + rank)
+        bdo = torch.randn((w.B, w.T, w.H, w.Dv), generator=gen).to(w.torch_dtype).to(device)
+        bdS = torch.randn((w.B, w.H, w.Dv, w.Dk), generator=gen).to(device)
+        bws = torch.empty(max(G.chunk_bwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                         w.torch_dtype), 1),
+                          dtype=torch.uint8, device=device)
+
+        def bwd_step():
+            G.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                        bdo, bdS, chunk=w.chunk, workspace=bws)
+
+        for _ in range(3):
+            bwd_step()
+        n_b = 20
+        b_ms = _max_over_ranks(time_loop(bwd_step, n_b, stream, world), world, device) / n_b
+        bb = bwd_bytes(w, inp["S0"] is not None)
+        b_gbs = bb / (b_ms * 1e-3) / 1e9
+        backward = {"workload": "headline_T4k backward: dq, dk, dv, dlog_alpha, dbeta, dS0 "
+                                "from d_o and dS_T",
+                    "path": "CUDA cores, float32 arithmetic (4 launches per call)",
+                    "ms_per_step": b_ms, "tokens_per_s": world * tokens / (b_ms * 1e-3),
+                    "achieved": b_gbs, "unit": "GB/s", "peak": hbm_peak,
+                    "frac": b_gbs / hbm_peak, "algorithmic_bytes": bb, "steps": n_b,
+                    "gpu_launches": 4 * n_b}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
@@ -455,7 +493,7 @@ def run_ours(args):
                        "path": path},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
-            "prologue": prologue, "varlen": varlen,
+            "prologue": prologue, "varlen": varlen, "backward": backward,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
