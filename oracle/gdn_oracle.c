@@ -419,3 +419,127 @@ int gdn_oracle_backward(const double *q, const double *k, const double *v,
     free(tid);
     return status;
 }
+
+/*
+ * Channel-wise gates (Gated DeltaNet-2, "Gated DeltaNet-2: Decoupling Erase and
+ * Write in Linear Attention", abstract): a decay per key channel alpha_t in
+ * (0,1]^Dk (given as log alpha, as above), a channel-wise erase gate b_t
+ * (Dk, on the key side) and a channel-wise write gate w_t (Dv, on the value
+ * side).  The pages give the roles and the reductions but not the formula; the
+ * reading taken keeps one rank-one edit per token:
+ *
+ *   S_t = S_{t-1} Diag(alpha_t) ( I - (b_t o k_t) k_t^T ) + (w_t o v_t) k_t^T   (3)
+ *   o_t = S_t q_t
+ *
+ * which is the rule (1) when alpha_t, b_t and w_t are all the scalar alpha_t,
+ * beta_t, beta_t ("reducing to KDA when both gates collapse to the same scalar
+ * and to Gated DeltaNet when the decay also collapses").  Row i of (3):
+ *   d_j = alpha_j S[i][j];  e = sum_j d_j b_j k_j;
+ *   S[i][j] = d_j - e k_j + w_i v_i k_j
+ */
+static void gdn2_token(double *S, const double *q, const double *k, const double *v,
+                       const double *log_alpha, const double *b, const double *w,
+                       double *o, long Dk, long Dv)
+{
+    for (long i = 0; i < Dv; ++i) {
+        double *row = S + i * Dk;
+        double e = 0.0;
+        for (long j = 0; j < Dk; ++j) {
+            row[j] = exp(log_alpha[j]) * row[j];
+            e += row[j] * b[j] * k[j];
+        }
+        for (long j = 0; j < Dk; ++j)
+            row[j] = row[j] - e * k[j] + w[i] * v[i] * k[j];
+        double oi = 0.0;
+        for (long j = 0; j < Dk; ++j)
+            oi += q[j] * row[j];
+        o[i] = oi;
+    }
+}
+
+typedef struct {
+    const double *q, *k, *v, *la, *b, *w;
+    double *o, *S;
+    long B, T, H, Dk, Dv;
+    const int *units;
+    int n_units, n_threads, thread_id;
+} cwjob_t;
+
+static void *cw_worker(void *arg)
+{
+    const cwjob_t *j = (const cwjob_t *)arg;
+    const long n = j->units ? j->n_units : j->B * j->H;
+    for (long ii = j->thread_id; ii < n; ii += j->n_threads) {
+        const long u = j->units ? (long)j->units[ii] : ii;
+        const long b = u / j->H, h = u % j->H;
+        double *S = j->S + u * j->Dv * j->Dk;
+        for (long t = 0; t < j->T; ++t) {
+            const long row = (b * j->T + t) * j->H + h; /* token row of [B,T,H,*] */
+            gdn2_token(S, j->q + row * j->Dk, j->k + row * j->Dk, j->v + row * j->Dv,
+                       j->la + row * j->Dk, j->b + row * j->Dk, j->w + row * j->Dv,
+                       j->o + row * j->Dv, j->Dk, j->Dv);
+        }
+    }
+    return NULL;
+}
+
+/*
+ * Whole-sequence recurrence (3): q,k,log_alpha,b [B,T,H,Dk]; v,w [B,T,H,Dv];
+ * S0 [B,H,Dv,Dk] or NULL; o [B,T,H,Dv]; S_T [B,H,Dv,Dk].  units as for
+ * gdn_oracle_forward.  Returns 0, -1 on a bad argument, -2 on allocation failure.
+ */
+int gdn_oracle_forward_cw(const double *q, const double *k, const double *v,
+                          const double *log_alpha, const double *b, const double *w,
+                          const double *S0, double *o, double *S_T,
+                          long B, long T, long H, long Dk, long Dv,
+                          const int *units, int n_units, int nthreads)
+{
+    if (!q || !k || !v || !log_alpha || !b || !w || !o || !S_T)
+        return -1;
+    if (B <= 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0)
+        return -1;
+    if (check_units(units, n_units, B * H))
+        return -1;
+    const long n = units ? n_units : B * H;
+    for (long i = 0; i < n; ++i) {
+        const long u = units ? units[i] : i;
+        double *dst = S_T + u * Dv * Dk;
+        if (S0)
+            memcpy(dst, S0 + u * Dv * Dk, sizeof(double) * (size_t)(Dv * Dk));
+        else
+            memset(dst, 0, sizeof(double) * (size_t)(Dv * Dk));
+    }
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > n)
+        nthreads = (int)(n > 0 ? n : 1);
+    cwjob_t *jobs = (cwjob_t *)malloc(sizeof(cwjob_t) * (size_t)nthreads);
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!jobs || !tid) {
+        free(jobs);
+        free(tid);
+        return -2;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        cwjob_t *j = &jobs[i];
+        memset(j, 0, sizeof(*j));
+        j->q = q; j->k = k; j->v = v; j->la = log_alpha; j->b = b; j->w = w;
+        j->o = o; j->S = S_T;
+        j->B = B; j->T = T; j->H = H; j->Dk = Dk; j->Dv = Dv;
+        j->units = units; j->n_units = n_units; j->n_threads = nthreads; j->thread_id = i;
+    }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&tid[i], NULL, cw_worker, &jobs[i]) != 0)
+            break;
+        started = i;
+    }
+    cw_worker(&jobs[0]);
+    for (int i = 1; i <= started; ++i)
+        pthread_join(tid[i], NULL);
+    for (int i = started + 1; i < nthreads; ++i)
+        cw_worker(&jobs[i]);
+    free(jobs);
+    free(tid);
+    return 0;
+}

@@ -50,6 +50,9 @@ def _bind(path: str):
     lib.gdn_oracle_backward.argtypes = [dp] * 14 + [L, L, L, L, L, ip, ctypes.c_int,
                                                     ctypes.c_int]
     lib.gdn_oracle_backward.restype = ctypes.c_int
+    lib.gdn_oracle_forward_cw.argtypes = [dp] * 9 + [L, L, L, L, L, ip, ctypes.c_int,
+                                                     ctypes.c_int]
+    lib.gdn_oracle_forward_cw.restype = ctypes.c_int
     return lib
 
 
@@ -168,6 +171,34 @@ def backward(q, k, v, log_alpha, beta, S0, d_o, dS_T=None, units=None, nthreads=
     if rc != 0:
         raise RuntimeError(f"gdn_oracle_backward failed ({rc})")
     return tuple(out)
+
+
+def forward_cw(q, k, v, log_alpha, b, w, S0=None, units=None, nthreads=None, lib=None):
+    """Channel-wise gates (Gated DeltaNet-2 reading, see gdn_oracle.c):
+    S_t = S_{t-1} Diag(alpha_t) (I - (b_t o k_t) k_t^T) + (w_t o v_t) k_t^T, o_t = S_t q_t.
+
+    q, k, log_alpha, b [B,T,H,Dk]; v, w [B,T,H,Dv]; S0 [B,H,Dv,Dk] or None.
+    Returns (o [B,T,H,Dv], S_T [B,H,Dv,Dk]) in float64 (NaN outside ``units``).
+    """
+    q, k, v, la, bb, ww = (_f64(x) for x in (q, k, v, log_alpha, b, w))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if k.shape != q.shape or la.shape != q.shape or bb.shape != q.shape or \
+            v.shape[:3] != (B, T, H) or ww.shape != v.shape:
+        raise ValueError("shape mismatch")
+    s0 = None if S0 is None else _f64(S0)
+    if s0 is not None and s0.shape != (B, H, Dv, Dk):
+        raise ValueError("S0 must be [B,H,Dv,Dk]")
+    fill = np.nan if units is not None else 0.0
+    o = np.full((B, T, H, Dv), fill)
+    st = np.full((B, H, Dv, Dk), fill)
+    up, nu, _keep = _units(units, B * H)
+    rc = (lib or _load()).gdn_oracle_forward_cw(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(bb), _ptr(ww), _ptr(s0), _ptr(o), _ptr(st),
+        B, T, H, Dk, Dv, up, nu, int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_forward_cw failed ({rc})")
+    return o, st
 
 
 def load_variant(path: str):
