@@ -10,7 +10,7 @@ first such use raises if ``libgdn.so`` is missing -- there is no fallback.
 _BINDING_NAMES = {
     "chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_varlen_workspace_size", "decode_step",
     "chunk_fwd_workspace_size", "chunk_fwd_path", "library_path", "chunk_bwd",
-    "chunk_bwd_workspace_size",
+    "chunk_bwd_workspace_size", "chunk_fwd_cw", "chunk_fwd_cw_workspace_size", "decode_step_cw",
     "GdnError", "check_device_status",
 }
 

@@ -61,6 +61,13 @@ def _load():
     lib.gdn_chunk_bwd.restype = I
     lib.gdn_chunk_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.gdn_chunk_bwd_workspace_size.restype = Z
+    lib.gdn_chunk_fwd_cw.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, I, I, I, I, I, I, I, vp,
+                                     Z, vp]
+    lib.gdn_chunk_fwd_cw.restype = I
+    lib.gdn_chunk_fwd_cw_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_fwd_cw_workspace_size.restype = Z
+    lib.gdn_decode_step_cw.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, I, I, I, I, I, vp]
+    lib.gdn_decode_step_cw.restype = I
     lib.gdn_check_device_status.argtypes = []
     lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]
@@ -231,6 +238,77 @@ def chunk_bwd(q, k, v, log_alpha, beta, S0, d_o, dS_T=None, chunk: int = 64, wor
                            _stream_ptr(dev))
     _check(st, "gdn_chunk_bwd")
     return dq, dk, dv, dla, dbe, dS0
+
+
+def chunk_fwd_cw_workspace_size(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> int:
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return int(LIB.gdn_chunk_fwd_cw_workspace_size(B, T, H, Dk, Dv, chunk, code))
+
+
+def chunk_fwd_cw(q, k, v, log_alpha, b, w, S0=None, chunk: int = 64, out=None, S_T=None,
+                 return_state: bool = True, workspace=None):
+    """Channel-wise gates: S_t = S_{t-1} Diag(alpha_t)(I - (b_t o k_t) k_t^T) + (w_t o v_t) k_t^T.
+
+    q, k [B,T,H,Dk], v [B,T,H,Dv] (float32 or bfloat16); log_alpha, b
+    [B,T,H,Dk] and w [B,T,H,Dv] float32; S0 [B,H,Dv,Dk] float32 or None.
+    Returns (o [B,T,H,Dv], S_T or None).
+    """
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise GdnError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[3]
+    dev = q.device
+    code = _dtype_code(q)
+    if log_alpha.shape != q.shape or b.shape != q.shape or w.shape != v.shape:
+        raise GdnError("log_alpha and b must be [B,T,H,Dk] and w [B,T,H,Dv]")
+    args = [_dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
+            _dev(log_alpha, "log_alpha", torch.float32, dev), _dev(b, "b", torch.float32, dev),
+            _dev(w, "w", torch.float32, dev)]
+    state = (B, H, Dv, Dk)
+    if S0 is not None and S0.shape != state:
+        raise GdnError("S0 must be [B,H,Dv,Dk]")
+    args.append(_dev(S0, "S0", torch.float32, dev) if S0 is not None else None)
+    o = out if out is not None else torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
+    if o.shape != (B, T, H, Dv):
+        raise GdnError("out must be [B,T,H,Dv]")
+    args.append(_dev(o, "out", q.dtype, dev))
+    if S_T is None and return_state:
+        S_T = torch.empty(state, dtype=torch.float32, device=dev)
+    if S_T is not None and S_T.shape != state:
+        raise GdnError("S_T must be [B,H,Dv,Dk]")
+    args.append(_dev(S_T, "S_T", torch.float32, dev) if S_T is not None else None)
+    need = int(LIB.gdn_chunk_fwd_cw_workspace_size(B, T, H, Dk, Dv, chunk, code))
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    st = LIB.gdn_chunk_fwd_cw(*args, B, T, H, Dk, Dv, chunk, code, ws_ptr, ws_bytes,
+                              _stream_ptr(dev))
+    _check(st, "gdn_chunk_fwd_cw")
+    return o, S_T
+
+
+def decode_step_cw(q, k, v, log_alpha, b, w, S, out=None):
+    """One channel-wise-gate step for every (b, h); S [B,H,Dv,Dk] updated in place.
+    q, k, log_alpha, b [B,H,Dk]; v, w [B,H,Dv].  Returns o [B,H,Dv]."""
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise GdnError("q, k must be [B,H,Dk] and v [B,H,Dv]")
+    B, H, Dk = q.shape
+    Dv = v.shape[2]
+    dev = q.device
+    if log_alpha.shape != q.shape or b.shape != q.shape or w.shape != v.shape:
+        raise GdnError("log_alpha and b must be [B,H,Dk] and w [B,H,Dv]")
+    if S.shape != (B, H, Dv, Dk):
+        raise GdnError("S must be [B,H,Dv,Dk]")
+    o = out if out is not None else torch.empty((B, H, Dv), dtype=q.dtype, device=dev)
+    st = LIB.gdn_decode_step_cw(
+        _dev(q, "q", q.dtype, dev), _dev(k, "k", q.dtype, dev), _dev(v, "v", q.dtype, dev),
+        _dev(log_alpha, "log_alpha", torch.float32, dev), _dev(b, "b", torch.float32, dev),
+        _dev(w, "w", torch.float32, dev), _dev(S, "S", torch.float32, dev),
+        _dev(o, "out", q.dtype, dev), B, H, Dk, Dv, _dtype_code(q), _stream_ptr(dev))
+    _check(st, "gdn_decode_step_cw")
+    return o
 
 
 def _host_offsets(cu_seqlens) -> torch.Tensor:

@@ -336,6 +336,95 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+size_t gdn_chunk_fwd_cw_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
+                                       gdn_dtype_t dtype) {
+    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::cw_supported(Dk, chunk))
+        return 0;
+    if (empty_problem(B, T, H)) return 0;
+    return gdn::cw_workspace_bytes(B, T, H, Dk, chunk);
+}
+
+gdn_status_t gdn_chunk_fwd_cw(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *b, const float *w,
+                              const float *S0, void *o, float *S_T, int B, int T, int H, int Dk,
+                              int Dv, int chunk, gdn_dtype_t dtype, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    const gdn_status_t sz = check_sizes(B, T, H, Dk, Dv, chunk, dtype);
+    if (sz != GDN_OK) return sz;
+    if (!gdn::cw_supported(Dk, chunk)) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4;
+    const size_t n_tok = (size_t)B * T * H;
+    const size_t state_bytes = (size_t)B * H * Dv * Dk * sizeof(float);
+    if (B == 0 || H == 0) return GDN_OK;
+    if (T == 0) {  // no tokens: the final state is the initial one
+        if (!S_T) return GDN_OK;
+        if (!aligned16(S_T) || (S0 && !aligned16(S0))) return GDN_ERR_INVALID_ARG;
+        if (S0 && S0 != S_T && overlaps(S_T, state_bytes, S0, state_bytes))
+            return GDN_ERR_INVALID_ARG;
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, state_bytes,
+                                                          cudaMemcpyDeviceToDevice, st))
+                           : cudaMemsetAsync(S_T, 0, state_bytes, st);
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+    if (!q || !k || !v || !log_alpha || !b || !w || !o) return GDN_ERR_INVALID_ARG;
+    const struct { const void *p; size_t n; } in[] = {
+        {q, n_tok * Dk * esz}, {k, n_tok * Dk * esz}, {v, n_tok * Dv * esz},
+        {log_alpha, n_tok * Dk * sizeof(float)}, {b, n_tok * Dk * sizeof(float)},
+        {w, n_tok * Dv * sizeof(float)}, {S0, state_bytes}};
+    for (const auto &a : in)
+        if (a.p && !aligned16(a.p)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(o) || (S_T && !aligned16(S_T)) || (workspace && !aligned16(workspace)))
+        return GDN_ERR_INVALID_ARG;
+    const size_t o_bytes = n_tok * Dv * esz;
+    for (const auto &a : in) {
+        if (overlaps(o, o_bytes, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+        // S_T may be S0 itself (in-place continuation), nothing else
+        if (S_T && a.p != S0 && overlaps(S_T, state_bytes, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+    }
+    if (S_T && S0 && S_T != S0 && overlaps(S_T, state_bytes, S0, state_bytes))
+        return GDN_ERR_INVALID_ARG;
+    if (S_T && overlaps(S_T, state_bytes, o, o_bytes)) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::cw_workspace_bytes(B, T, H, Dk, chunk);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    for (const auto &a : in)
+        if (overlaps(workspace, need, a.p, a.n)) return GDN_ERR_INVALID_ARG;
+    if (overlaps(workspace, need, o, o_bytes) ||
+        (S_T && overlaps(workspace, need, S_T, state_bytes)))
+        return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_chunk_cw(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, Dk,
+                                               Dv, chunk, dtype == GDN_BF16, workspace, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_decode_step_cw(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *b, const float *w, float *S,
+                                void *o, int B, int H, int Dk, int Dv, gdn_dtype_t dtype,
+                                void *stream) {
+    const gdn_status_t sz = check_sizes(B, 1, H, Dk, Dv, 16, dtype);
+    if (sz != GDN_OK) return sz;
+    if (B == 0 || H == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !b || !w || !S || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, b, w, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t esz = dtype == GDN_BF16 ? 2 : 4, heads = (size_t)B * H;
+    const size_t s_bytes = heads * Dv * Dk * sizeof(float), o_bytes = heads * Dv * esz;
+    const struct { const void *p; size_t n; } in[] = {
+        {q, heads * Dk * esz}, {k, heads * Dk * esz}, {v, heads * Dv * esz},
+        {log_alpha, heads * Dk * sizeof(float)}, {b, heads * Dk * sizeof(float)},
+        {w, heads * Dv * sizeof(float)}};
+    for (const auto &a : in)
+        if (overlaps(o, o_bytes, a.p, a.n) || overlaps(S, s_bytes, a.p, a.n))
+            return GDN_ERR_INVALID_ARG;
+    if (overlaps(o, o_bytes, S, s_bytes)) return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_decode_cw(q, k, v, log_alpha, b, w, S, o, B, H, Dk, Dv,
+                                                dtype == GDN_BF16,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status_t gdn_check_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
     unsigned int flag = 0;

@@ -51,6 +51,19 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              float *dbeta, float *dS0, int B, int T, int H, int Dk, int Dv,
                              int chunk, bool bf16, void *workspace, cudaStream_t st);
 
+// Channel-wise gates (decay per key channel, erase gate b on the key side,
+// write gate w on the value side; CUDA cores, Dk <= 128): chunk_cw.cu.
+// log alpha and b are [B,T,H,Dk] float32, w is [B,T,H,Dv] float32.
+bool cw_supported(int Dk, int chunk);
+size_t cw_workspace_bytes(int B, int T, int H, int Dk, int chunk);
+cudaError_t launch_chunk_cw(const void *q, const void *k, const void *v, const float *la,
+                            const float *bg, const float *wg, const float *S0, void *o, float *S_T,
+                            int B, int T, int H, int Dk, int Dv, int chunk, bool bf16,
+                            void *workspace, cudaStream_t st);
+cudaError_t launch_decode_cw(const void *q, const void *k, const void *v, const float *la,
+                             const float *bg, const float *wg, float *S, void *o, int B, int H,
+                             int Dk, int Dv, bool bf16, cudaStream_t st);
+
 // tcgen05 chunkwise forward (bf16, Dk = 128, chunk 64): chunk_tc.cu.  The
 // workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of every head.
 // With the L2-normalisation flag the workspace also holds 1/|k| per token.

@@ -103,6 +103,27 @@ def chunk_inputs(w: Workload, seed: int | None = None, device="cpu"):
     return out
 
 
+def cw_inputs(w: Workload, seed: int | None = None, device="cpu"):
+    """Inputs with channel-wise gates: as ``chunk_inputs`` (same q, k, v and S0
+    draws for the same seed), with log_alpha [B,T,H,Dk] drawn by the workload's
+    gate law per key channel, an erase gate b = sigmoid(N) [B,T,H,Dk] and a write
+    gate w = sigmoid(N) [B,T,H,Dv], all float32."""
+    gen = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    q = _unit_rows(torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    k = _unit_rows(torch.randn((B, T, H, Dk), generator=gen)).to(w.torch_dtype)
+    v = torch.randn((B, T, H, Dv), generator=gen).to(w.torch_dtype)
+    la, b = _gates(gen, (B, T, H, Dk), w.gate_law)
+    wg = torch.sigmoid(torch.randn((B, T, H, Dv), generator=gen)).contiguous()
+    S0 = None
+    if w.s0_law == "normal002":
+        S0 = 0.02 * torch.randn((B, H, Dv, Dk), generator=gen)
+    out = dict(q=q, k=k, v=v, log_alpha=la, b=b, w=wg, S0=S0)
+    if device != "cpu":
+        out = {n: (t.to(device) if t is not None else None) for n, t in out.items()}
+    return out
+
+
 def raw_chunk_inputs(w: Workload, seed: int | None = None, device="cpu"):
     """Inputs for the library's optional input prologue (per-token L2 normalisation
     of q and k, gate activations): q, k ~ 2 N(0,1) rounded to the dtype and NOT

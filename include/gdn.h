@@ -250,6 +250,47 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chu
                                     gdn_dtype_t dtype);
 
 /*
+ * Channel-wise gates.  "Gated DeltaNet-2: Decoupling Erase and Write in Linear
+ * Attention" (abstract) gives each key channel its own decay (as KDA does) and
+ * splits the scalar beta into a channel-wise erase gate b_t on the key side and
+ * a channel-wise write gate w_t on the value side; it reduces to the scalar
+ * rule when the three collapse.  The pages give no formula; the reading taken
+ * keeps one rank-one edit per token:
+ *
+ *   S_t = S_{t-1} Diag(alpha_t) (I - (b_t o k_t) k_t^T) + (w_t o v_t) k_t^T,
+ *   o_t = S_t q_t,   alpha_t = exp(log_alpha_t) per key channel.
+ *
+ *   q, k [B,T,H,Dk] and v, o [B,T,H,Dv] in `dtype`; log_alpha and b [B,T,H,Dk]
+ *   float32; w [B,T,H,Dv] float32; S0 (or NULL), S_T (or NULL) [B,H,Dv,Dk]
+ *   float32, S_T may equal S0.  With log_alpha, b and w constant over their
+ *   channels (log alpha, beta, beta) this is gdn_chunk_fwd.
+ *
+ * Chunkwise on the CUDA cores (float32 arithmetic): the channel-wise decay
+ * between two rows of a chunk enters each key product as exp(Lam_r - Lam_i)
+ * per channel.  Limits as for gdn_chunk_fwd plus Dk <= 128
+ * (GDN_ERR_UNSUPPORTED).  Workspace: gdn_chunk_fwd_cw_workspace_size bytes
+ * ((2 C^2 + C Dk) floats per chunk and head).  Enqueued on `stream`.
+ */
+gdn_status_t gdn_chunk_fwd_cw(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *b, const float *w,
+                              const float *S0, void *o, float *S_T,
+                              int B, int T, int H, int Dk, int Dv, int chunk,
+                              gdn_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                              void *stream);
+size_t gdn_chunk_fwd_cw_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
+                                       gdn_dtype_t dtype);
+
+/*
+ * One recurrent step of the channel-wise rule above for every (b, h), the
+ * state updated in place: q, k, log_alpha, b [B,H,Dk]; v, w, o [B,H,Dv];
+ * S [B,H,Dv,Dk] float32.  All required; o must not overlap S or an input.
+ */
+gdn_status_t gdn_decode_step_cw(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *b, const float *w,
+                                float *S, void *o, int B, int H, int Dk, int Dv,
+                                gdn_dtype_t dtype, void *stream);
+
+/*
  * Synchronise the current device and report whether a fused tensor-core
  * kernel gave up since the last check: its pipeline waits are bounded (about
  * two seconds each); a CTA that times out stops, records a flag and leaves its

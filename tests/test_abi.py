@@ -226,3 +226,25 @@ def test_chunk_bwd_workspace_size(lib):
         H * NT * (2 * C * C + C + 2 * Dv * Dk) * 4
     assert b.chunk_bwd_workspace_size(1, 40, H, 256, Dv, C, torch.float32) == 0
     assert b.chunk_bwd_workspace_size(1, 0, H, Dk, Dv, C, torch.float32) == 0
+
+
+def test_chunk_fwd_cw_checks(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    f = lib.gdn_chunk_fwd_cw
+    args = lambda **kw: dict(dict(q=16, k=16, v=16, la=16, bg=16, w=16, S0=None, o=1 << 24,
+                                  S_T=None, B=1, T=8, H=1, Dk=16, Dv=16, chunk=16, dtype=0,
+                                  ws=1 << 40, ws_bytes=1 << 30), **kw)
+    call = lambda a: f(a["q"], a["k"], a["v"], a["la"], a["bg"], a["w"], a["S0"], a["o"],
+                       a["S_T"], a["B"], a["T"], a["H"], a["Dk"], a["Dv"], a["chunk"],
+                       a["dtype"], a["ws"], a["ws_bytes"], None)
+    assert call(args(bg=None)) == 1 and call(args(w=None)) == 1
+    assert call(args(Dk=144)) == 2 and call(args(chunk=48)) == 2
+    assert call(args(o=16)) == 1 and call(args(ws=None)) == 1 and call(args(ws_bytes=8)) == 1
+    assert call(args(B=0)) == 0 and call(args(T=0)) == 0
+    # T, P' (C x C) and the running log-decay sums (C x Dk) per chunk and head
+    assert b.chunk_fwd_cw_workspace_size(2, 40, 3, 16, 8, 16, torch.float32) == \
+        2 * 3 * 3 * (2 * 16 * 16 + 16 * 16) * 4
+    d = lib.gdn_decode_step_cw
+    assert d(16, 16, 16, 16, 16, None, 1 << 20, 16, 1, 1, 16, 16, 0, None) == 1
+    assert d(16, 16, 16, 16, 16, 16, 1 << 20, 16, 1, 1, 16, 16, 0, None) == 1   # o overlaps q
+    assert d(16, 16, 16, 16, 16, 16, 1 << 20, 1 << 24, 0, 1, 16, 16, 0, None) == 0
