@@ -476,6 +476,56 @@ def run_ours(args):
                     "frac": b_gbs / hbm_peak, "algorithmic_bytes": bb, "steps": n_b,
                     "gpu_launches": 4 * n_b}
 
+    # channel-wise gates (decay per key channel, erase and write gates) on the
+    # headline shape, and their decode step at batch 256
+    channel_wise = None
+    if not args.chunk_only:
+        cin = I.cw_inputs(w, seed=w.seed + rank, device=device)
+        cws = torch.empty(max(G.chunk_fwd_cw_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                            w.torch_dtype), 1),
+                          dtype=torch.uint8, device=device)
+
+        def cw_step():
+            G.chunk_fwd_cw(cin["q"], cin["k"], cin["v"], cin["log_alpha"], cin["b"], cin["w"],
+                           cin["S0"], chunk=w.chunk, out=o, S_T=S_T, workspace=cws)
+
+        for _ in range(3):
+            cw_step()
+        n_c = 10
+        c_ms = _max_over_ranks(time_loop(cw_step, n_c, stream, world), world, device) / n_c
+        esz = 2
+        c_bytes = w.B * w.T * w.H * (esz * (2 * w.Dk + 2 * w.Dv) + 4 * (2 * w.Dk + w.Dv)) + \
+            w.B * w.H * w.Dv * w.Dk * 4
+        wd = I.workload("decode_b256")
+        dcin = I.cw_inputs(I.workload("decode_b256", T=1, s0_law="normal002"), device=device)
+        one = lambda x: x[:, 0].contiguous()
+        xq, xk, xv, xl, xb, xw = (one(dcin[n]) for n in ("q", "k", "v", "log_alpha", "b", "w"))
+        Sd = dcin["S0"].clone()
+        od_cw = torch.empty((wd.B, wd.H, wd.Dv), dtype=wd.torch_dtype, device=device)
+
+        def cw_dstep():
+            G.decode_step_cw(xq, xk, xv, xl, xb, xw, Sd, out=od_cw)
+
+        for _ in range(10):
+            cw_dstep()
+        n_d = 200
+        cd_us = 1e3 * _max_over_ranks(time_loop(cw_dstep, n_d, stream, world), world,
+                                      device) / n_d
+        cd_bytes = wd.B * wd.H * (8 * wd.Dv * wd.Dk + esz * (2 * wd.Dk + 2 * wd.Dv) +
+                                  4 * (2 * wd.Dk + wd.Dv))
+        channel_wise = {
+            "workload": "headline_T4k shape with a decay and an erase gate per key channel and "
+                        "a write gate per value channel (float32 gates)",
+            "path": "CUDA cores, float32 arithmetic (2 launches per call)",
+            "ms_per_step": c_ms, "tokens_per_s": world * tokens / (c_ms * 1e-3),
+            "achieved": c_bytes / (c_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "frac": c_bytes / (c_ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": c_bytes,
+            "steps": n_c,
+            "decode": {"workload": "batch 256, H 16, d 128, bf16, state in place",
+                       "us_per_step": cd_us, "achieved": cd_bytes / (cd_us * 1e-6) / 1e9,
+                       "unit": "GB/s", "frac": cd_bytes / (cd_us * 1e-6) / 1e9 / hbm_peak,
+                       "bytes_per_step": cd_bytes, "steps": n_d}}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
@@ -494,6 +544,7 @@ def run_ours(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
             "prologue": prologue, "varlen": varlen, "backward": backward,
+            "channel_wise": channel_wise,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
