@@ -35,13 +35,16 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
+// The sequential (chunk-walking) kernels run one CTA per SM; 16 warps hide more
+// of their shared-memory latency than 8.
+constexpr int kSeqThreads = 512;
 
 // Per (b, h, chunk) floats of the recomputed T, P and g.
 __host__ __device__ inline size_t prep_floats(int C) { return 2 * (size_t)C * C + C; }
 
 // dS, walked backwards over the chunks of one head, DVT rows per CTA.
 template <typename T, int DVT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kSeqThreads)
 bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ beta,
           const T *__restrict__ d_o, const float *__restrict__ dS_T, float *__restrict__ dS0,
           const float *__restrict__ ws_prep, float *__restrict__ dS_hist, int Tlen, int H, int Dk,
@@ -64,7 +67,7 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
     float *gl = dc + C;             // 1 : exp(g_last)
     const size_t head = (size_t)b * H + h;
 
-    for (int idx = threadIdx.x; idx < DVT * Dk; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < DVT * Dk; idx += kSeqThreads) {
         const int i = idx / Dk, j = idx - i * Dk;
         dS[i * ldk + j] = (i < nv && dS_T) ? dS_T[(head * Dv + v0 + i) * Dk + j] : 0.f;
     }
@@ -74,12 +77,12 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
         __syncthreads();
         {   // dS' of this chunk (the gradient of the state it hands on)
             float *dst = dS_hist + ((head * NT + c) * Dv + v0) * Dk;
-            for (int idx = threadIdx.x; idx < nv * Dk; idx += kThreads) {
+            for (int idx = threadIdx.x; idx < nv * Dk; idx += kSeqThreads) {
                 const int i = idx / Dk, j = idx - i * Dk;
                 dst[idx] = dS[i * ldk + j];
             }
         }
-        for (int idx = threadIdx.x; idx < C * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * Dk; idx += kSeqThreads) {
             const int r = idx / Dk, j = idx - r * Dk;
             float kv = 0.f, qv = 0.f;
             if (r < n) {
@@ -90,11 +93,11 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
             Ks[r * ldk + j] = kv;
             Qs[r * ldk + j] = qv;
         }
-        for (int idx = threadIdx.x; idx < C * C; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * C; idx += kSeqThreads) {
             Tm[idx] = wsc[idx];
             Pm[idx] = wsc[C * C + idx];
         }
-        for (int idx = threadIdx.x; idx < C * DVT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * DVT; idx += kSeqThreads) {
             const int r = idx / DVT, i = idx - r * DVT;
             dO[r * ldv + i] = (r < n && i < nv)
                                   ? to_f32(d_o[(((size_t)b * Tlen + t0 + r) * H + h) * Dv + v0 + i])
@@ -112,7 +115,7 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
         __syncthreads();
 
         // dU' = P^T dO + D K dS^T
-        for (int idx = threadIdx.x; idx < C * DVT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * DVT; idx += kSeqThreads) {
             const int r = idx / DVT, i = idx - r * DVT;
             float a = 0.f, kd = 0.f;
             for (int m = r; m < C; ++m) a += Pm[m * C + r] * dO[m * ldv + i];
@@ -121,7 +124,7 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
         }
         __syncthreads();
         // Z = T^T dU'
-        for (int idx = threadIdx.x; idx < C * DVT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * DVT; idx += kSeqThreads) {
             const int r = idx / DVT, i = idx - r * DVT;
             float a = 0.f;
             for (int m = r; m < C; ++m) a += Tm[m * C + r] * dU[m * ldv + i];
@@ -129,7 +132,7 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
         }
         __syncthreads();
         // dS <- exp(g_last) dS + dO^T diag(exp g) Q - Z^T diag(beta exp g) K
-        for (int idx = threadIdx.x; idx < DVT * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < DVT * Dk; idx += kSeqThreads) {
             const int i = idx / Dk, j = idx - i * Dk;
             float a = 0.f;
             for (int r = 0; r < C; ++r)
@@ -139,7 +142,7 @@ bwd_state(const T *__restrict__ q, const T *__restrict__ k, const float *__restr
     }
     __syncthreads();
     if (dS0) {
-        for (int idx = threadIdx.x; idx < nv * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < nv * Dk; idx += kSeqThreads) {
             const int i = idx / Dk, j = idx - i * Dk;
             dS0[(head * Dv + v0 + i) * Dk + j] = dS[i * ldk + j];
         }
@@ -473,6 +476,17 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     }
 }
 
+// Workspace: [T, P, g per chunk | S_hist | dS_hist | (tensor-core recompute:
+// its tile workspace | a scratch output)].
+size_t base_floats(int B, int T, int H, int Dk, int Dv, int C) {
+    const size_t NT = ((size_t)T + C - 1) / C;
+    return (size_t)B * H * NT * (prep_floats(C) + 2 * (size_t)Dv * Dk);
+}
+
+bool tc_recompute(int B, int T, int H, int Dk, int Dv, int C, bool bf16) {
+    return tc_supported(B, T, H, Dk, Dv, C, bf16);
+}
+
 template <typename T>
 cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const float *la,
                          const float *beta, const float *S0, const void *d_o, const float *dS_T,
@@ -484,8 +498,21 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
     float *ws_prep = static_cast<float *>(workspace);
     float *S_hist = ws_prep + (size_t)B * H * NT * prep_floats(C);
     float *dS_hist = S_hist + (size_t)B * H * NT * Dv * Dk;
-    cudaError_t e = launch_bwd_recompute(q, k, v, la, beta, S0, B, Tlen, H, Dk, Dv, C,
-                                         sizeof(T) == 2, ws_prep, S_hist, st);
+    const bool bf16 = sizeof(T) == 2;
+    cudaError_t e;
+    if (tc_recompute(B, Tlen, H, Dk, Dv, C, bf16)) {
+        // T, P, g on the CUDA cores; the chunk states from the tensor-core forward
+        uint8_t *tail = reinterpret_cast<uint8_t *>(ws_prep + base_floats(B, Tlen, H, Dk, Dv, C));
+        void *o_scratch = tail + ((tc_workspace_bytes(B, Tlen, H, 0) + 255) & ~size_t(255));
+        e = launch_bwd_recompute(q, k, v, la, beta, S0, B, Tlen, H, Dk, Dv, C, bf16, ws_prep,
+                                 nullptr, st);
+        if (e != cudaSuccess) return e;
+        e = launch_chunk_tc(q, k, v, la, beta, S0, o_scratch, nullptr, B, Tlen, H, Dk, Dv, 0u,
+                            tail, st, S_hist);
+    } else {
+        e = launch_bwd_recompute(q, k, v, la, beta, S0, B, Tlen, H, Dk, Dv, C, bf16, ws_prep,
+                                 S_hist, st);
+    }
     if (e != cudaSuccess) return e;
     const size_t smem_s = bwd_state_smem_floats<DVT>(C, Dk) * sizeof(float);
     const size_t smem_g = bwd_grads_smem_floats(C, Dk) * sizeof(float);
@@ -495,7 +522,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
     e = cudaFuncSetAttribute(bwd_grads<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_g);
     if (e != cudaSuccess) return e;
-    bwd_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kThreads, smem_s, st>>>(
+    bwd_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kSeqThreads, smem_s, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), beta, static_cast<const T *>(d_o),
         dS_T, dS0, ws_prep, dS_hist, Tlen, H, Dk, Dv, C, NT);
     e = cudaPeekAtLastError();
@@ -509,9 +536,12 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
 
 }  // namespace
 
-size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk) {
-    const size_t NT = ((size_t)T + chunk - 1) / chunk;
-    return (size_t)B * H * NT * (prep_floats(chunk) + 2 * (size_t)Dv * Dk) * sizeof(float);
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
+    size_t n = base_floats(B, T, H, Dk, Dv, chunk) * sizeof(float);
+    if (tc_recompute(B, T, H, Dk, Dv, chunk, bf16))
+        n += ((tc_workspace_bytes(B, T, H, 0) + 255) & ~size_t(255)) +
+             (size_t)B * T * H * Dv * sizeof(__nv_bfloat16);
+    return n;
 }
 
 bool bwd_supported(int Dk, int chunk) {

@@ -29,6 +29,9 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
+// The sequential (chunk-walking) kernels run one CTA per SM; 16 warps hide more
+// of their shared-memory latency than 8.
+constexpr int kSeqThreads = 512;
 
 __host__ __device__ inline size_t cw_chunk_floats(int C, int Dk) {
     return 2 * (size_t)C * C + (size_t)C * Dk;
@@ -119,7 +122,7 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
 }
 
 template <typename T, int DVT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kSeqThreads)
 cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
          const float *__restrict__ bg, const float *__restrict__ wg, const float *__restrict__ S0,
          T *__restrict__ o, float *__restrict__ S_T, const float *__restrict__ ws, int Tlen, int H,
@@ -140,7 +143,7 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
     float *ln = Un + C * ldv;       // Dk : exp(Lam_last)
     const size_t head = (size_t)b * H + h;
 
-    for (int idx = threadIdx.x; idx < DVT * Dk; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < DVT * Dk; idx += kSeqThreads) {
         const int i = idx / Dk, j = idx - i * Dk;
         Ss[i * ldk + j] = (i < nv && S0) ? S0[(head * Dv + v0 + i) * Dk + j] : 0.f;
     }
@@ -150,7 +153,7 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
         const float *wsc = ws + (head * NT + c) * cw_chunk_floats(C, Dk);
         const float *Lam = wsc + 2 * C * C;
         __syncthreads();  // the previous chunk has finished with every buffer
-        for (int idx = threadIdx.x; idx < C * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * Dk; idx += kSeqThreads) {
             const int r = idx / Dk, j = idx - r * Dk;
             float kv = 0.f, qv = 0.f, bv = 0.f;
             if (r < n) {
@@ -166,13 +169,13 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
             KD[r * ldk + j] = kv * expf(ll - lr);
             if (r == 0) ln[j] = expf(ll);
         }
-        for (int idx = threadIdx.x; idx < C * C; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * C; idx += kSeqThreads) {
             Tm[idx] = wsc[idx];
             Pp[idx] = wsc[C * C + idx];
         }
         __syncthreads();
         // R = w o V - BL S^T,  Xq = QL S^T
-        for (int idx = threadIdx.x; idx < C * DVT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * DVT; idx += kSeqThreads) {
             const int r = idx / DVT, i = idx - r * DVT;
             float xb = 0.f, xq = 0.f;
             for (int j = 0; j < Dk; ++j) {
@@ -190,7 +193,7 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
         }
         __syncthreads();
         // U = T R,  O = Xq + P' R
-        for (int idx = threadIdx.x; idx < C * DVT; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < C * DVT; idx += kSeqThreads) {
             const int r = idx / DVT, i = idx - r * DVT;
             float u = 0.f, y = 0.f;
             for (int m = 0; m <= r; ++m) {
@@ -204,7 +207,7 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
         }
         __syncthreads();
         // S <- S Diag(exp(Lam_last)) + U^T KD
-        for (int idx = threadIdx.x; idx < DVT * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < DVT * Dk; idx += kSeqThreads) {
             const int i = idx / Dk, j = idx - i * Dk;
             float acc = 0.f;
             for (int r = 0; r < C; ++r) acc += Un[r * ldv + i] * KD[r * ldk + j];
@@ -213,7 +216,7 @@ cw_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__
     }
     __syncthreads();
     if (S_T) {
-        for (int idx = threadIdx.x; idx < nv * Dk; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < nv * Dk; idx += kSeqThreads) {
             const int i = idx / Dk, j = idx - i * Dk;
             S_T[(head * Dv + v0 + i) * Dk + j] = Ss[i * ldk + j];
         }
@@ -256,6 +259,71 @@ decode_cw(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     if (lane == 0) o[row] = from_f32<T>(acc);
 }
 
+// The same step with the row in registers: NPL = Dk / 32 consecutive channels
+// per lane (16-byte accesses), ROWS rows of one head per warp so that the
+// head's gates are loaded once per warp.  The state row is read and written once.
+template <typename T, int NPL, int ROWS>
+__global__ void __launch_bounds__(kThreads)
+decode_cw_vec(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+              const float *__restrict__ la, const float *__restrict__ bg,
+              const float *__restrict__ wg, float *__restrict__ S, T *__restrict__ o,
+              long long rows, int Dv) {
+    constexpr int Dk = 32 * NPL;
+    const long long row0 = (((long long)blockIdx.x * kThreads + threadIdx.x) / 32) * ROWS;
+    const int lane = threadIdx.x % 32;
+    if (row0 >= rows) return;  // whole warp leaves together (rows is a multiple of ROWS)
+    const long long head = row0 / Dv;
+    const int j0 = lane * NPL;
+    float al[NPL], bk[NPL], kk[NPL], qq[NPL];
+#pragma unroll
+    for (int m = 0; m < NPL; m += 4) {
+        const float4 l4 = load4(la + head * Dk + j0 + m), b4 = load4(bg + head * Dk + j0 + m);
+        const float4 k4 = load4(k + head * Dk + j0 + m), q4 = load4(q + head * Dk + j0 + m);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            al[m + u] = expf(lv[u]);
+            kk[m + u] = kv[u];
+            bk[m + u] = bv[u] * kv[u];
+            qq[m + u] = qv[u];
+        }
+    }
+#pragma unroll
+    for (int rr = 0; rr < ROWS; ++rr) {
+        const long long row = row0 + rr;
+        const int i = (int)(row - head * Dv);
+        float *s = S + row * Dk + j0;
+        float d[NPL];
+        float e = 0.f;
+#pragma unroll
+        for (int m = 0; m < NPL; m += 4) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(s + m);
+            d[m] = al[m] * s4.x;
+            d[m + 1] = al[m + 1] * s4.y;
+            d[m + 2] = al[m + 2] * s4.z;
+            d[m + 3] = al[m + 3] * s4.w;
+        }
+#pragma unroll
+        for (int m = 0; m < NPL; ++m) e += d[m] * bk[m];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
+        const float c = wg[head * Dv + i] * to_f32(v[head * Dv + i]) - e;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < NPL; ++m) {
+            d[m] += c * kk[m];
+            acc += d[m] * qq[m];
+        }
+#pragma unroll
+        for (int m = 0; m < NPL; m += 4)
+            *reinterpret_cast<float4 *>(s + m) = make_float4(d[m], d[m + 1], d[m + 2], d[m + 3]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) o[row] = from_f32<T>(acc);
+    }
+}
+
 template <typename T>
 cudaError_t launch_cw_t(const void *q, const void *k, const void *v, const float *la,
                         const float *bg, const float *wg, const float *S0, void *o, float *S_T,
@@ -278,7 +346,7 @@ cudaError_t launch_cw_t(const void *q, const void *k, const void *v, const float
         static_cast<const T *>(q), static_cast<const T *>(k), la, bg, ws, Tlen, H, Dk, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
-    cw_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kThreads, smem_state, st>>>(
+    cw_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kSeqThreads, smem_state, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), bg, wg,
         S0, static_cast<T *>(o), S_T, ws, Tlen, H, Dk, Dv, C, NT);
     return cudaPeekAtLastError();
@@ -309,6 +377,24 @@ cudaError_t launch_decode_cw(const void *q, const void *k, const void *v, const 
                              const float *bg, const float *wg, float *S, void *o, int B, int H,
                              int Dk, int Dv, bool bf16, cudaStream_t st) {
     const long long rows = (long long)B * H * Dv;
+    constexpr int ROWS = 4;
+    if ((Dk == 128 || Dk == 256) && Dv % ROWS == 0) {
+        const long long warps = rows / ROWS;
+        const unsigned blocks = (unsigned)((warps * 32 + kThreads - 1) / kThreads);
+#define GDN_CW_VEC(TT, NPL)                                                                    \
+    decode_cw_vec<TT, NPL, ROWS><<<blocks, kThreads, 0, st>>>(                                  \
+        static_cast<const TT *>(q), static_cast<const TT *>(k), static_cast<const TT *>(v), la, \
+        bg, wg, S, static_cast<TT *>(o), rows, Dv)
+        if (bf16) {
+            if (Dk == 128) GDN_CW_VEC(__nv_bfloat16, 4);
+            else GDN_CW_VEC(__nv_bfloat16, 8);
+        } else {
+            if (Dk == 128) GDN_CW_VEC(float, 4);
+            else GDN_CW_VEC(float, 8);
+        }
+#undef GDN_CW_VEC
+        return cudaPeekAtLastError();
+    }
     const unsigned blocks = (unsigned)((rows * 32 + kThreads - 1) / kThreads);
     if (bf16)
         decode_cw<__nv_bfloat16><<<blocks, kThreads, 0, st>>>(

@@ -30,6 +30,10 @@ namespace gdn {
 
 __host__ __device__ inline size_t per_chunk_floats(int C) { return 2 * (size_t)C * C + C; }
 
+// The sequential pass runs one CTA per SM (shared memory); 16 warps hide more of
+// its shared-memory latency than 8.
+constexpr int kSeqThreads = 512;
+
 size_t simt_workspace_bytes(int B, int T, int H, int C) {
     const size_t NT = ((size_t)T + C - 1) / C;
     return (size_t)B * H * NT * per_chunk_floats(C) * sizeof(float);
@@ -129,7 +133,7 @@ chunk_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__rest
 }
 
 template <typename T, int DVT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kSeqThreads)
 chunk_state(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
             const float *__restrict__ beta, const float *__restrict__ S0, T *__restrict__ o,
             float *__restrict__ S_T, const float *__restrict__ ws, float *__restrict__ S_hist,
@@ -264,7 +268,7 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
         static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws, Tlen, H, Dk, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
-    chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), 256, smem_state, st>>>(
+    chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kSeqThreads, smem_state, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0,
         static_cast<T *>(o), S_T, ws, nullptr, Tlen, H, Dk, Dv, C, NT);
     return cudaPeekAtLastError();
@@ -293,8 +297,8 @@ static cudaError_t launch_recompute_t(const void *q, const void *k, const void *
         static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws_prep, Tlen, H, Dk, C,
         NT);
     e = cudaPeekAtLastError();
-    if (e != cudaSuccess) return e;
-    chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), 256, smem_state, st>>>(
+    if (e != cudaSuccess || !S_hist) return e;
+    chunk_state<T, DVT><<<dim3((Dv + DVT - 1) / DVT, H, B), kSeqThreads, smem_state, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0,
         nullptr, nullptr, ws_prep, S_hist, Tlen, H, Dk, Dv, C, NT);
     return cudaPeekAtLastError();

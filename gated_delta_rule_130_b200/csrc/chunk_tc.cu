@@ -713,6 +713,8 @@ struct Params {
     float *S_T;
     const float *rk;       // 1/|k| per token from the UT kernel (L2-normalising only)
     Seqs sq;               // the sequences (one per blockIdx.z)
+    float *S_hist;         // optional (fixed-length batches): the state entering every
+                           // chunk, [B*H][NT][Dv][Dk] float32, for the backward
     int H, Dv;
     unsigned flags;        // input prologue (kFlagL2Norm, kFlagGateLogits)
 };
@@ -1110,6 +1112,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + 16 * B + j) * DK + lrow] : 0.f;
+                if (p.S_hist)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        p.S_hist[((size_t)head * NT * p.Dv + v0 + 16 * B + j) * DK + lrow] = sv[j];
                 store16_bf16(sbuf, lrow, B, sv);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) sv[j] *= gl;
@@ -1199,6 +1205,14 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!last) {
                     store16_bf16(sbuf, lrow, 2 * hf, s0);
                     store16_bf16(sbuf, lrow, 2 * hf + 1, s1);
+                    if (p.S_hist) {  // the state entering chunk c + 1
+                        float *dst = p.S_hist + (((size_t)head * NT + c + 1) * p.Dv + v0 + 32 * hf) * DK + lrow;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            dst[j * DK] = s0[j];
+                            dst[(16 + j) * DK] = s1[j];
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         s0[j] *= gl;
@@ -1335,7 +1349,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
-                                 int Dv, unsigned flags, void *workspace, cudaStream_t st) {
+                                 int Dv, unsigned flags, void *workspace, cudaStream_t st,
+                                 float *S_hist) {
     const bool varlen = cu_seqlens != nullptr;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
@@ -1367,6 +1382,7 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
     p.Dv = Dv;
     p.rk = rk;
     p.flags = flags;
+    p.S_hist = varlen ? nullptr : S_hist;
     const bool norm = (flags & kFlagL2Norm) != 0;
     auto *ut = norm ? tc::gdn_ut_kernel<true> : tc::gdn_ut_kernel<false>;
     auto *seq = norm ? tc::gdn_chunk_tc_kernel<true> : tc::gdn_chunk_tc_kernel<false>;
@@ -1400,11 +1416,12 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
                             int H, int Dk, int Dv, unsigned flags, void *workspace,
-                            cudaStream_t st) {
+                            cudaStream_t st, float *S_hist) {
     // a fixed-length batch is B packed sequences of length T
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
     return launch_chunk_tc_seqs(q, k, v, log_alpha, beta, S0, o, S_T, B, T, (long long)B * T,
-                                nullptr, (long long)B * NT, H, Dk, Dv, flags, workspace, st);
+                                nullptr, (long long)B * NT, H, Dk, Dv, flags, workspace, st,
+                                S_hist);
 }
 
 #ifdef GDN_TRACE

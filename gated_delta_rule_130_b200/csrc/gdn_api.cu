@@ -274,7 +274,7 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chu
     if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::bwd_supported(Dk, chunk))
         return 0;
     if (empty_problem(B, T, H)) return 0;
-    return gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk);
+    return gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16);
 }
 
 gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -324,7 +324,7 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
         for (size_t j = i + 1; j < sizeof(out) / sizeof(out[0]); ++j)
             if (overlaps(out[i].p, out[i].n, out[j].p, out[j].n)) return GDN_ERR_INVALID_ARG;
     }
-    const size_t need = gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk);
+    const size_t need = gdn::bwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16);
     if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
     for (const auto &a : in)
         if (overlaps(workspace, need, a.p, a.n)) return GDN_ERR_INVALID_ARG;

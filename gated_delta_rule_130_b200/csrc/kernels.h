@@ -36,6 +36,7 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
 // The backward's recomputation on the CUDA-core path (chunk_simt.cu): T, P, g
 // per chunk into ws_prep ([B,H,NT] x (2 C^2 + C) floats) and the state entering
 // every chunk into S_hist ([B,H,NT,Dv,Dk] floats).
+// (S_hist == nullptr: T, P, g only.)
 cudaError_t launch_bwd_recompute(const void *q, const void *k, const void *v, const float *la,
                                  const float *beta, const float *S0, int B, int T, int H, int Dk,
                                  int Dv, int chunk, bool bf16, float *ws_prep, float *S_hist,
@@ -43,8 +44,10 @@ cudaError_t launch_bwd_recompute(const void *q, const void *k, const void *v, co
 
 // CUDA-core chunkwise backward (Dk <= 128): chunk_bwd.cu.  Workspace: the
 // recomputed T, P, g, the chunk states and the state gradients.
+// bf16 sizes the tensor-core forward takes recompute the chunk states with it
+// (its [T'; T''] tiles and a scratch output then also live in the workspace).
 bool bwd_supported(int Dk, int chunk);
-size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk);
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
 cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la,
                              const float *beta, const float *S0, const void *d_o,
                              const float *dS_T, void *dq, void *dk, void *dv, float *dla,
@@ -69,10 +72,11 @@ cudaError_t launch_decode_cw(const void *q, const void *k, const void *v, const 
 // With the L2-normalisation flag the workspace also holds 1/|k| per token.
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
 size_t tc_workspace_bytes(int B, int T, int H, unsigned flags);
+// S_hist (optional): the state entering every chunk, [B*H][NT][Dv][Dk] float32.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
                             int H, int Dk, int Dv, unsigned flags, void *workspace,
-                            cudaStream_t st);
+                            cudaStream_t st, float *S_hist = nullptr);
 // The same over n_seq sequences packed along the token dimension: fixed length
 // T_fixed (cu_seqlens == nullptr) or the device offsets cu_seqlens (n_seq + 1);
 // total_chunks = sum of ceil(length / 64).  The workspace then starts with the
@@ -83,7 +87,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
-                                 int Dv, unsigned flags, void *workspace, cudaStream_t st);
+                                 int Dv, unsigned flags, void *workspace, cudaStream_t st,
+                                 float *S_hist = nullptr);
 
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).

@@ -100,7 +100,8 @@ def test_cw_no_tokens_and_in_place_state(gdn):
     assert torch.equal(S_T, d["S0"])
 
 
-@pytest.mark.parametrize("Dk,Dv,dtype", [(128, 128, "f32"), (128, 128, "bf16"), (48, 20, "f32")])
+@pytest.mark.parametrize("Dk,Dv,dtype", [(128, 128, "f32"), (128, 128, "bf16"), (256, 36, "f32"),
+                                         (256, 64, "bf16"), (48, 20, "f32"), (128, 30, "f32")])
 def test_cw_decode(gdn, Dk, Dv, dtype):
     w = I.workload("tiny_f32", B=3, H=2, T=12, Dk=Dk, Dv=Dv, dtype=dtype, s0_law="normal002",
                    seed=Dk + Dv)
