@@ -34,7 +34,6 @@ namespace gdn {
 
 namespace {
 
-constexpr int kThreads = 256;
 // The sequential (chunk-walking) kernels run one CTA per SM; 16 warps hide more
 // of their shared-memory latency than 8.
 constexpr int kSeqThreads = 512;
@@ -156,7 +155,9 @@ constexpr size_t bwd_state_smem_floats(int C, int Dk) {
 }
 
 constexpr int DVS = 16;        // value channels per pass of bwd_grads
-constexpr int kMaxCols = 32;   // key channels per thread: Dk / (kThreads / C) <= 128 / 4
+constexpr int kGradThreads = 512;
+constexpr int kMaxCols = 16;   // key channels per thread: Dk / (kGradThreads / C) <= 128 / 8
+static_assert(kGradThreads / 16 <= 32, "a row's threads share one warp (C >= 16)");
 
 __host__ __device__ constexpr int region_floats(int C, int Dk) {
     return (2 * DVS * (Dk + 1) + 7 * C * (DVS + 1)) > C * (Dk + 1)
@@ -169,10 +170,10 @@ __host__ __device__ constexpr size_t bwd_grads_smem_floats(int C, int Dk) {
 }
 
 // Every input gradient of one chunk of one head.  The thread layout for the
-// C x Dk results: kThreads / C consecutive threads share a row, each owning the
-// key channels j = sub, sub + kThreads / C, ...
+// C x Dk results: kGradThreads / C consecutive threads share a row, each owning
+// the key channels j = sub, sub + kGradThreads / C, ...
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kGradThreads)
 bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
           const float *__restrict__ beta, const T *__restrict__ d_o,
           const float *__restrict__ ws_prep, const float *__restrict__ S_hist,
@@ -214,10 +215,10 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     const float *Sc = S_hist + (head * NT + c) * (size_t)Dv * Dk;
     const float *dSc = dS_hist + (head * NT + c) * (size_t)Dv * Dk;
     const int tid = threadIdx.x;
-    const int TPR = kThreads / C, row = tid / TPR, sub = tid - row * TPR;
+    const int TPR = kGradThreads / C, row = tid / TPR, sub = tid - row * TPR;
     const size_t tok = (size_t)b * Tlen + t0;  // first token of the chunk
 
-    for (int idx = tid; idx < C * Dk; idx += kThreads) {
+    for (int idx = tid; idx < C * Dk; idx += kGradThreads) {
         const int r = idx / Dk, j = idx - r * Dk;
         float kv = 0.f, qv = 0.f;
         if (r < n) {
@@ -228,7 +229,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         Ks[r * ldk + j] = kv;
         Qs[r * ldk + j] = qv;
     }
-    for (int idx = tid; idx < C * C; idx += kThreads) {
+    for (int idx = tid; idx < C * C; idx += kGradThreads) {
         Tm[idx] = wsc[idx];
         Pm[idx] = wsc[C * C + idx];
         dP[idx] = 0.f;
@@ -247,7 +248,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
     }
     __syncthreads();
-    for (int idx = tid; idx < C * Dk; idx += kThreads) {
+    for (int idx = tid; idx < C * Dk; idx += kGradThreads) {
         const int r = idx / Dk, j = idx - r * Dk;
         float a = 0.f;
         for (int m = 0; m <= r; ++m) a += Tm[r * C + m] * bt[m] * eg[m] * Ks[m * ldk + j];
@@ -260,12 +261,12 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
 
     for (int v0 = 0; v0 < Dv; v0 += DVS) {
         const int nv = min(DVS, Dv - v0);
-        for (int idx = tid; idx < DVS * Dk; idx += kThreads) {
+        for (int idx = tid; idx < DVS * Dk; idx += kGradThreads) {
             const int i = idx / Dk, j = idx - i * Dk;
             Ss[i * ldk + j] = i < nv ? Sc[(size_t)(v0 + i) * Dk + j] : 0.f;
             dSs[i * ldk + j] = i < nv ? dSc[(size_t)(v0 + i) * Dk + j] : 0.f;
         }
-        for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        for (int idx = tid; idx < C * DVS; idx += kGradThreads) {
             const int r = idx / DVS, i = idx - r * DVS;
             const bool in = r < n && i < nv;
             const size_t off = ((tok + r) * H + h) * Dv + v0 + i;
@@ -274,7 +275,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         __syncthreads();
         // U = T diag(beta) V,  U' = U - W S^T,  K dS'^T
-        for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        for (int idx = tid; idx < C * DVS; idx += kGradThreads) {
             const int r = idx / DVS, i = idx - r * DVS;
             float u = 0.f, w = 0.f, kd = 0.f;
             for (int m = 0; m <= r; ++m) u += Tm[r * C + m] * bt[m] * Vs[m * lds + i];
@@ -288,7 +289,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         __syncthreads();
         // dU' = P^T dO + D K dS'^T
-        for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        for (int idx = tid; idx < C * DVS; idx += kGradThreads) {
             const int r = idx / DVS, i = idx - r * DVS;
             float a = 0.f;
             for (int m = r; m < C; ++m) a += Pm[m * C + r] * dOs[m * lds + i];
@@ -296,7 +297,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         __syncthreads();
         // Z = T^T dU',  dV = diag(beta) Z
-        for (int idx = tid; idx < C * DVS; idx += kThreads) {
+        for (int idx = tid; idx < C * DVS; idx += kGradThreads) {
             const int r = idx / DVS, i = idx - r * DVS;
             float z = 0.f;
             for (int m = r; m < C; ++m) z += Tm[m * C + r] * dUs[m * lds + i];
@@ -305,7 +306,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         __syncthreads();
         // this slice's share of dP = dO U'^T, Z U^T and the row and scalar sums
-        for (int idx = tid; idx < C * C; idx += kThreads) {
+        for (int idx = tid; idx < C * C; idx += kGradThreads) {
             const int r = idx / C, i = idx - r * C;
             if (i <= r) {
                 float a = 0.f, z = 0.f;
@@ -328,7 +329,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         {
             float p = 0.f;
-            for (int idx = tid; idx < DVS * Dk; idx += kThreads) {
+            for (int idx = tid; idx < DVS * Dk; idx += kGradThreads) {
                 const int i = idx / Dk, j = idx - i * Dk;
                 p += Ss[i * ldk + j] * dSs[i * ldk + j];
             }
@@ -390,7 +391,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         if (j < Dk) DW[row * ldk + j] = aW[m];
     }
     // the read-out's gating: dg from dP o P, and dP <- dP o Gamma (masked)
-    for (int idx = tid; idx < C * C; idx += kThreads) {
+    for (int idx = tid; idx < C * C; idx += kGradThreads) {
         const int r = idx / C, i = idx - r * C;
         float d = 0.f;
         if (i <= r) {
@@ -406,7 +407,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     }
     __syncthreads();
     // dA = strictly-lower(-(Y W^T + Z U^T)); its dg and dbeta terms; E into Pm
-    for (int idx = tid; idx < C * C; idx += kThreads) {
+    for (int idx = tid; idx < C * C; idx += kGradThreads) {
         const int r = idx / C, i = idx - r * C;
         float e = 0.f;
         if (i < r) {
@@ -527,7 +528,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
         dS_T, dS0, ws_prep, dS_hist, Tlen, H, Dk, Dv, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
-    bwd_grads<T><<<dim3(NT, H, B), kThreads, smem_g, st>>>(
+    bwd_grads<T><<<dim3(NT, H, B), kGradThreads, smem_g, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta,
         static_cast<const T *>(d_o), ws_prep, S_hist, dS_hist, static_cast<T *>(dq),
         static_cast<T *>(dk), static_cast<T *>(dv), dla, dbeta, Tlen, H, Dk, Dv, C, NT);
