@@ -141,3 +141,22 @@ def test_varlen_device_offsets_give_the_same_bits(gdn):
                                                                  device="cuda"))
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_varlen_cuda_core_path_with_prologue_and_state_in_place(gdn):
+    lengths = [37, 0, 90, 16]
+    inp = I.varlen_inputs(lengths, 2, 32, 24, "f32", s0_law="normal002", seed=31)
+    gen = torch.Generator().manual_seed(5)
+    for n in ("q", "k"):   # raw rows: scale each by a random factor
+        inp[n] = inp[n] * torch.empty(inp[n].shape[:2] + (1,)).uniform_(0.5, 3.0, generator=gen)
+    d = {n: (t.cuda() if isinstance(t, torch.Tensor) else t) for n, t in inp.items()}
+    S = d["S0"].clone()
+    o, _ = gdn.chunk_fwd_varlen(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                inp["cu_seqlens"], S0=S, S_T=S, chunk=32, l2norm_qk=True,
+                                gate_logits=True)
+    torch.cuda.synchronize()
+    q, k, la, be = PR.apply(inp["q"].double().numpy(), inp["k"].double().numpy(),
+                            inp["log_alpha"].numpy(), inp["beta"].numpy(), True, True)
+    ref = dict(inp, q=torch.from_numpy(q), k=torch.from_numpy(k), log_alpha=torch.from_numpy(la),
+               beta=torch.from_numpy(be))
+    _check(o, S, ref, TOL_F32)
