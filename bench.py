@@ -565,6 +565,38 @@ def run_ours(args):
                        "unit": "GB/s", "frac": cd_bytes / (cd_us * 1e-6) / 1e9 / hbm_peak,
                        "bytes_per_step": cd_bytes, "steps": n_d}}
 
+    # the other chunkwise-forward shapes: d = 128 at T = 2K, one 32K-token sequence
+    # (S0 != 0, strong decay) and the wide heads (Dk 256, Dv 512)
+    configs = None
+    if not args.chunk_only:
+        configs = []
+        for name, n_steps in (("bf16_T2k", 50), ("long_T32k", 20), ("wide_dk256_dv512", 3)):
+            wc = I.workload(name)
+            cin = I.chunk_inputs(wc, seed=wc.seed + rank, device=device)
+            co = torch.empty((wc.B, wc.T, wc.H, wc.Dv), dtype=wc.torch_dtype, device=device)
+            cS = torch.empty((wc.B, wc.H, wc.Dv, wc.Dk), dtype=torch.float32, device=device)
+            cw_ = torch.empty(max(G.chunk_fwd_workspace_size(wc.B, wc.T, wc.H, wc.Dk, wc.Dv,
+                                                             wc.chunk, wc.torch_dtype), 1),
+                              dtype=torch.uint8, device=device)
+
+            def cstep():
+                G.chunk_fwd(cin["q"], cin["k"], cin["v"], cin["log_alpha"], cin["beta"],
+                            cin["S0"], chunk=wc.chunk, out=co, S_T=cS, workspace=cw_)
+
+            for _ in range(3):
+                cstep()
+            c_ms = _max_over_ranks(time_loop(cstep, n_steps, stream, world), world,
+                                   device) / n_steps
+            cb, cf = chunk_bytes(wc, cin["S0"] is not None), chunk_flops(wc)
+            configs.append({
+                "workload": f"{name}: B={wc.B} H={wc.H} T={wc.T} Dk={wc.Dk} Dv={wc.Dv} "
+                            f"chunk={wc.chunk} bf16, gates {wc.gate_law}, S0 {wc.s0_law}",
+                "path": G.chunk_fwd_path(wc.B, wc.T, wc.H, wc.Dk, wc.Dv, wc.chunk, wc.torch_dtype),
+                "ms_per_step": c_ms, "tokens_per_s": world * wc.B * wc.T / (c_ms * 1e-3),
+                "hbm_frac": cb / (c_ms * 1e-3) / 1e9 / hbm_peak,
+                "tc_frac": cf / (c_ms * 1e-3) / 1e12 / tc_peak, "steps": n_steps})
+            del cin, co, cS, cw_
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.chunk_only:
         cpu = cpu_baseline(w, inp_cpu)
@@ -583,7 +615,7 @@ def run_ours(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
             "prologue": prologue, "varlen": varlen, "backward": backward,
-            "channel_wise": channel_wise,
+            "channel_wise": channel_wise, "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -298,7 +298,7 @@ __device__ __forceinline__ void tmem_ld16w(uint32_t taddr, float (&v)[16]) {
 // stride LDA), blocked by 16 with D_I = I + A_II:
 //   T_II = D_I^-1                                   (ut_diag, forward substitution)
 //   N_IJ = T_II A_IJ,  I > J                        (ut_offdiag4 phase 1, all six blocks)
-//   T_IJ = -sum_{J <= K < I} N_IK T_KJ              (phases 2-4, by block diagonal)
+//   T_IJ = -sum_{J <= K < I} N_IK T_KJ              (phase 2, one warp per block column)
 // TF receives the lower triangle and the diagonal; its strict upper part is not
 // written (and never read).
 
@@ -523,25 +523,17 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
         }
     }
     __syncthreads();
+    // block column J of T needs only its own earlier blocks and the N blocks:
+    // warp J walks down it, T_IJ = -sum_{K=J}^{I-1} N_IK T_KJ, with no CTA barrier
     if (w < 3) {
-        float acc[2][4] = {};
-        mma16(acc, blk(AF, w + 1, w), LDA, blk(TF, w, w), LDA, g, t);
-        store16x16(acc, blk(TF, w + 1, w), LDA, -1.f, g, t);
-    }
-    __syncthreads();
-    if (w < 2) {
-        float acc[2][4] = {};
-        mma16(acc, blk(AF, w + 2, w), LDA, blk(TF, w, w), LDA, g, t);
-        mma16(acc, blk(AF, w + 2, w + 1), LDA, blk(TF, w + 1, w), LDA, g, t);
-        store16x16(acc, blk(TF, w + 2, w), LDA, -1.f, g, t);
-    }
-    __syncthreads();
-    if (w == 0) {
-        float acc[2][4] = {};
-        mma16(acc, blk(AF, 3, 0), LDA, blk(TF, 0, 0), LDA, g, t);
-        mma16(acc, blk(AF, 3, 1), LDA, blk(TF, 1, 0), LDA, g, t);
-        mma16(acc, blk(AF, 3, 2), LDA, blk(TF, 2, 0), LDA, g, t);
-        store16x16(acc, blk(TF, 3, 0), LDA, -1.f, g, t);
+        const int J = w;
+        for (int I = J + 1; I < 4; ++I) {
+            float acc[2][4] = {};
+            for (int K = J; K < I; ++K)
+                mma16(acc, blk(AF, I, K), LDA, blk(TF, K, J), LDA, g, t);
+            store16x16(acc, blk(TF, I, J), LDA, -1.f, g, t);
+            __syncwarp();
+        }
     }
     __syncthreads();
 }
