@@ -494,7 +494,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
                          void *dq, void *dk, void *dv, float *dla, float *dbeta, float *dS0, int B,
                          int Tlen, int H, int Dk, int Dv, int C, void *workspace,
                          cudaStream_t st) {
-    constexpr int DVT = 32;
+    constexpr int DVT = 64;  // one CTA per SM (shared memory): fewer, busier CTAs
     const int NT = (Tlen + C - 1) / C;
     float *ws_prep = static_cast<float *>(workspace);
     float *S_hist = ws_prep + (size_t)B * H * NT * prep_floats(C);

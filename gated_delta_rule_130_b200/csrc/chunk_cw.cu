@@ -19,7 +19,7 @@
 // Rows past a ragged end are zero tokens (k = q = b = w = 0, log alpha = 0).
 //
 // Kernels: cw_prep (one CTA per chunk) writes T, P' and Lam; cw_state (one CTA
-// per head and 32 value channels) runs the chunks in order with its slice of S
+// per head and 64 value channels) runs the chunks in order with its slice of S
 // in shared memory; decode_cw is the single-token step, one warp per state row.
 #include "common.cuh"
 #include "kernels.h"
@@ -329,7 +329,7 @@ cudaError_t launch_cw_t(const void *q, const void *k, const void *v, const float
                         const float *bg, const float *wg, const float *S0, void *o, float *S_T,
                         int B, int Tlen, int H, int Dk, int Dv, int C, void *workspace,
                         cudaStream_t st) {
-    constexpr int DVT = 32;
+    constexpr int DVT = 64;  // one CTA per SM (shared memory): fewer, busier CTAs
     const int NT = (Tlen + C - 1) / C;
     float *ws = static_cast<float *>(workspace);
     const size_t smem_prep = (4 * (size_t)C * (Dk + 1) + 3 * (size_t)C * C) * sizeof(float);

@@ -313,9 +313,9 @@ cudaError_t launch_bwd_recompute(const void *q, const void *k, const void *v, co
                                                             Dv, chunk, ws_prep, S_hist, st)
                     : launch_recompute_t<float, 16>(q, k, v, la, beta, S0, B, T, H, Dk, Dv, chunk,
                                                     ws_prep, S_hist, st);
-    return bf16 ? launch_recompute_t<__nv_bfloat16, 32>(q, k, v, la, beta, S0, B, T, H, Dk, Dv,
+    return bf16 ? launch_recompute_t<__nv_bfloat16, 64>(q, k, v, la, beta, S0, B, T, H, Dk, Dv,
                                                         chunk, ws_prep, S_hist, st)
-                : launch_recompute_t<float, 32>(q, k, v, la, beta, S0, B, T, H, Dk, Dv, chunk,
+                : launch_recompute_t<float, 64>(q, k, v, la, beta, S0, B, T, H, Dk, Dv, chunk,
                                                 ws_prep, S_hist, st);
 }
 
@@ -323,16 +323,18 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               const float *beta, const float *S0, void *o, float *S_T, int B,
                               int T, int H, int Dk, int Dv, int chunk, bool bf16, void *workspace,
                               cudaStream_t st) {
-    // Narrower value slices for wide keys keep the shared-memory footprint under
-    // the per-CTA limit (Dk = 256, C = 64: about 195 KB).
+    // 64 value rows per CTA for Dk <= 128 (one CTA per SM by shared memory, about
+    // 182 KB at C = 64: fewer, busier CTAs, one wave for B H Dv / 64 <= 148);
+    // narrower slices for wide keys keep the footprint under the per-CTA limit
+    // (Dk = 256, C = 64: about 195 KB).
     if (Dk > 128)
         return bf16 ? launch_simt_t<__nv_bfloat16, 16>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk,
                                                        Dv, chunk, workspace, st)
                     : launch_simt_t<float, 16>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk, Dv,
                                                chunk, workspace, st);
-    return bf16 ? launch_simt_t<__nv_bfloat16, 32>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk, Dv,
+    return bf16 ? launch_simt_t<__nv_bfloat16, 64>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk, Dv,
                                                    chunk, workspace, st)
-                : launch_simt_t<float, 32>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk,
+                : launch_simt_t<float, 64>(q, k, v, la, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk,
                                            workspace, st);
 }
 
