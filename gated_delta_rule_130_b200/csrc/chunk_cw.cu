@@ -29,8 +29,8 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
-// The sequential (chunk-walking) kernels run one CTA per SM; 16 warps hide more
-// of their shared-memory latency than 8.
+// The chunk kernels (prep and the sequential pass) run one CTA per SM; 16 warps
+// hide more of their shared-memory latency than 8.
 constexpr int kSeqThreads = 512;
 
 __host__ __device__ inline size_t cw_chunk_floats(int C, int Dk) {
@@ -38,7 +38,7 @@ __host__ __device__ inline size_t cw_chunk_floats(int C, int Dk) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kSeqThreads)
 cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
         const float *__restrict__ bg, float *__restrict__ ws, int Tlen, int H, int Dk, int C,
         int NT) {
@@ -55,7 +55,7 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
     const int t0 = c * C, n = min(C, Tlen - t0);
     const size_t tok = (size_t)b * Tlen + t0;
 
-    for (int idx = threadIdx.x; idx < C * Dk; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C * Dk; idx += kSeqThreads) {
         const int r = idx / Dk, j = idx - r * Dk;
         float kv = 0.f, qv = 0.f, bv = 0.f, lv = 0.f;
         if (r < n) {
@@ -71,7 +71,7 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
         Lm[r * ldk + j] = lv;
     }
     __syncthreads();
-    for (int j = threadIdx.x; j < Dk; j += kThreads) {  // running sums, one channel per thread
+    for (int j = threadIdx.x; j < Dk; j += kSeqThreads) {  // running sums, one channel per thread
         float acc = 0.f;
         for (int r = 0; r < C; ++r) {
             acc += Lm[r * ldk + j];
@@ -79,7 +79,7 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < C * C; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C * C; idx += kSeqThreads) {
         const int r = idx / C, i = idx - r * C;
         float a = 0.f, p = 0.f;
         if (i <= r) {
@@ -95,7 +95,7 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
     }
     __syncthreads();
     // T = (I + A)^-1 by forward substitution, one column per thread
-    for (int j = threadIdx.x; j < C; j += kThreads) {
+    for (int j = threadIdx.x; j < C; j += kSeqThreads) {
         for (int r = 0; r < C; ++r) {
             float val = (r == j) ? 1.f : 0.f;
             if (r > j) {
@@ -108,14 +108,14 @@ cw_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restric
     }
     __syncthreads();
     float *out = ws + (((size_t)b * H + h) * NT + c) * cw_chunk_floats(C, Dk);
-    for (int idx = threadIdx.x; idx < C * C; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C * C; idx += kSeqThreads) {
         const int r = idx / C, j = idx - r * C;
         float acc = 0.f;  // (P T)[r][j]
         for (int i = j; i <= r; ++i) acc += P[r * C + i] * Tm[i * C + j];
         out[idx] = Tm[idx];
         out[C * C + idx] = acc;
     }
-    for (int idx = threadIdx.x; idx < C * Dk; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C * Dk; idx += kSeqThreads) {
         const int r = idx / Dk, j = idx - r * Dk;
         out[2 * C * C + idx] = Lm[r * ldk + j];
     }
@@ -342,7 +342,7 @@ cudaError_t launch_cw_t(const void *q, const void *k, const void *v, const float
     e = cudaFuncSetAttribute(cw_state<T, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    cw_prep<T><<<dim3(NT, H, B), kThreads, smem_prep, st>>>(
+    cw_prep<T><<<dim3(NT, H, B), kSeqThreads, smem_prep, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), la, bg, ws, Tlen, H, Dk, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;

@@ -30,8 +30,8 @@ namespace gdn {
 
 __host__ __device__ inline size_t per_chunk_floats(int C) { return 2 * (size_t)C * C + C; }
 
-// The sequential pass runs one CTA per SM (shared memory); 16 warps hide more of
-// its shared-memory latency than 8.
+// Both kernels run one CTA per SM (shared memory); 16 warps hide more of their
+// shared-memory latency than 8.
 constexpr int kSeqThreads = 512;
 
 size_t simt_workspace_bytes(int B, int T, int H, int C) {
@@ -41,7 +41,7 @@ size_t simt_workspace_bytes(int B, int T, int H, int C) {
 
 // kPT: write P' = P T (the forward's read-out); else P itself (the backward's).
 template <typename T, bool kPT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kSeqThreads)
 chunk_prep(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
            const float *__restrict__ beta, float *__restrict__ ws, int Tlen, int H, int Dk, int C,
            int NT) {
@@ -264,7 +264,7 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
     e = cudaFuncSetAttribute(chunk_state<T, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    chunk_prep<T, true><<<dim3(NT, H, B), 256, smem_prep, st>>>(
+    chunk_prep<T, true><<<dim3(NT, H, B), kSeqThreads, smem_prep, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws, Tlen, H, Dk, C, NT);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
@@ -293,7 +293,7 @@ static cudaError_t launch_recompute_t(const void *q, const void *k, const void *
     e = cudaFuncSetAttribute(chunk_state<T, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    chunk_prep<T, false><<<dim3(NT, H, B), 256, smem_prep, st>>>(
+    chunk_prep<T, false><<<dim3(NT, H, B), kSeqThreads, smem_prep, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), la, beta, ws_prep, Tlen, H, Dk, C,
         NT);
     e = cudaPeekAtLastError();
