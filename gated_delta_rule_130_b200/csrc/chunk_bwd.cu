@@ -166,7 +166,18 @@ __host__ __device__ constexpr int region_floats(int C, int Dk) {
 }
 
 __host__ __device__ constexpr size_t bwd_grads_smem_floats(int C, int Dk) {
-    return 3 * (size_t)C * (Dk + 1) + 4 * (size_t)C * C + region_floats(C, Dk) + 8 * (size_t)C + 2;
+    return 3 * (size_t)C * (Dk + 1) + 2 * (size_t)C * C + 2 * (size_t)C * (C + 1) +
+           region_floats(C, Dk) + 8 * (size_t)C + 2;
+}
+
+// The t-th element (row-major) of the lower triangle with the diagonal:
+// r (r + 1) / 2 <= t < (r + 1) (r + 2) / 2, i = t - r (r + 1) / 2.
+__device__ __forceinline__ void lower_incl(int t, int &r, int &i) {
+    int rr = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while (rr * (rr + 1) / 2 > t) --rr;
+    while ((rr + 1) * (rr + 2) / 2 <= t) ++rr;
+    r = rr;
+    i = t - rr * (rr + 1) / 2;
 }
 
 // Every input gradient of one chunk of one head.  The thread layout for the
@@ -189,9 +200,12 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     float *Ks = Qs + C * ldk;            // C x ldk
     float *Ws = Ks + C * ldk;            // C x ldk : W = T diag(beta exp g) K
     float *Tm = Ws + C * ldk;            // C x C
-    float *Pm = Tm + C * C;              // C x C : P, later E
-    float *dP = Pm + C * C;              // C x C : dO U'^T, later (dP o Gamma)
-    float *ZU = dP + C * C;              // C x C : Z U^T
+    // P (later E) and dP are read along rows by the threads of several rows at
+    // once: a row stride of C + 1 keeps those reads on distinct banks
+    const int ldc = C + 1;
+    float *Pm = Tm + C * C;              // C x ldc : P, later E
+    float *dP = Pm + C * ldc;            // C x ldc : dO U'^T, later (dP o Gamma)
+    float *ZU = dP + C * ldc;            // C x C : Z U^T
     float *R = ZU + C * C;               // the value-slice buffers, later dW then Y
     float *gv = R + region_floats(C, Dk);  // C : g
     float *eg = gv + C;                  // C : exp(g)
@@ -230,9 +244,10 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         Qs[r * ldk + j] = qv;
     }
     for (int idx = tid; idx < C * C; idx += kGradThreads) {
+        const int r = idx / C, i = idx - r * C;
         Tm[idx] = wsc[idx];
-        Pm[idx] = wsc[C * C + idx];
-        dP[idx] = 0.f;
+        Pm[r * ldc + i] = wsc[C * C + idx];
+        dP[r * ldc + i] = 0.f;
         ZU[idx] = 0.f;
     }
     if (tid < C) {
@@ -292,7 +307,7 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         for (int idx = tid; idx < C * DVS; idx += kGradThreads) {
             const int r = idx / DVS, i = idx - r * DVS;
             float a = 0.f;
-            for (int m = r; m < C; ++m) a += Pm[m * C + r] * dOs[m * lds + i];
+            for (int m = r; m < C; ++m) a += Pm[m * ldc + r] * dOs[m * lds + i];
             dUs[r * lds + i] = a + dc[r] * KdS[r * lds + i];
         }
         __syncthreads();
@@ -306,17 +321,16 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         }
         __syncthreads();
         // this slice's share of dP = dO U'^T, Z U^T and the row and scalar sums
-        for (int idx = tid; idx < C * C; idx += kGradThreads) {
-            const int r = idx / C, i = idx - r * C;
-            if (i <= r) {
-                float a = 0.f, z = 0.f;
-                for (int u = 0; u < DVS; ++u) {
-                    a += dOs[r * lds + u] * Ups[i * lds + u];
-                    z += Zs[r * lds + u] * Us[i * lds + u];
-                }
-                dP[idx] += a;
-                if (i < r) ZU[idx] += z;
+        for (int t = tid; t < C * (C + 1) / 2; t += kGradThreads) {  // i <= r only
+            int r, i;
+            lower_incl(t, r, i);
+            float a = 0.f, z = 0.f;
+            for (int u = 0; u < DVS; ++u) {
+                a += dOs[r * lds + u] * Ups[i * lds + u];
+                z += Zs[r * lds + u] * Us[i * lds + u];
             }
+            dP[r * ldc + i] += a;
+            if (i < r) ZU[r * C + i] += z;
         }
         if (tid < C) {
             float a = 0.f, e = 0.f;
@@ -390,41 +404,38 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
         const int j = sub + TPR * m;
         if (j < Dk) DW[row * ldk + j] = aW[m];
     }
-    // the read-out's gating: dg from dP o P, and dP <- dP o Gamma (masked)
-    for (int idx = tid; idx < C * C; idx += kGradThreads) {
-        const int r = idx / C, i = idx - r * C;
-        float d = 0.f;
-        if (i <= r) {
-            const float dp = dP[idx];
-            if (i < r) {
-                const float dG = dp * Pm[idx];
-                atomicAdd(&dg[r], dG);
-                atomicAdd(&dg[i], -dG);
-            }
-            d = dp * expf(gv[r] - gv[i]);
+    // the read-out's gating: dg from dP o P, and dP <- dP o Gamma (i <= r; the
+    // upper triangle stays zero and is never read)
+    for (int t = tid; t < C * (C + 1) / 2; t += kGradThreads) {
+        int r, i;
+        lower_incl(t, r, i);
+        const float dp = dP[r * ldc + i];
+        if (i < r) {
+            const float dG = dp * Pm[r * ldc + i];
+            atomicAdd(&dg[r], dG);
+            atomicAdd(&dg[i], -dG);
         }
-        dP[idx] = d;
+        dP[r * ldc + i] = dp * expf(gv[r] - gv[i]);
     }
     __syncthreads();
     // dA = strictly-lower(-(Y W^T + Z U^T)); its dg and dbeta terms; E into Pm
-    for (int idx = tid; idx < C * C; idx += kGradThreads) {
-        const int r = idx / C, i = idx - r * C;
-        float e = 0.f;
-        if (i < r) {
-            float yw = 0.f, kk = 0.f;
-            for (int j = 0; j < Dk; ++j) {
-                yw += DW[r * ldk + j] * Ws[i * ldk + j];
-                kk += Ks[r * ldk + j] * Ks[i * ldk + j];
-            }
-            const float da = -(yw + ZU[idx]);
-            const float G = expf(gv[r] - gv[i]);
-            const float a = bt[r] * G * kk;  // A[r][i]
-            atomicAdd(&dg[r], da * a);
-            atomicAdd(&dg[i], -da * a);
-            atomicAdd(&db[r], da * G * kk);
-            e = bt[r] * da * G;
+    // (i < r only; Pm keeps P elsewhere, which is never read as E)
+    for (int t = tid; t < C * (C - 1) / 2; t += kGradThreads) {
+        int r, i;
+        lower_incl(t, r, i);
+        r += 1;  // the strictly lower pairs of C rows are the pairs i <= r of C - 1 rows
+        float yw = 0.f, kk = 0.f;
+        for (int j = 0; j < Dk; ++j) {
+            yw += DW[r * ldk + j] * Ws[i * ldk + j];
+            kk += Ks[r * ldk + j] * Ks[i * ldk + j];
         }
-        Pm[idx] = e;
+        const float da = -(yw + ZU[r * C + i]);
+        const float G = expf(gv[r] - gv[i]);
+        const float a = bt[r] * G * kk;  // A[r][i]
+        atomicAdd(&dg[r], da * a);
+        atomicAdd(&dg[i], -da * a);
+        atomicAdd(&db[r], da * G * kk);
+        Pm[r * ldc + i] = bt[r] * da * G;
     }
     __syncthreads();
     // dQ = dQ1 + (dP o Gamma) K
@@ -435,17 +446,35 @@ bwd_grads(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     for (int m = 0; m < kMaxCols; ++m) {
         const int j = sub + TPR * m;
         if (j < Dk) {
-            float dq_ = aQ[m];
-            for (int i = 0; i <= row; ++i) dq_ += dP[row * C + i] * Ks[i * ldk + j];
             const float y = DW[row * ldk + j];
-            float dk_ = aK[m] + btr * egr * y;
-            for (int rr = row; rr < C; ++rr) dk_ += dP[rr * C + row] * Qs[rr * ldk + j];
-            for (int i = 0; i < row; ++i) dk_ += Pm[row * C + i] * Ks[i * ldk + j];
-            for (int rr = row + 1; rr < C; ++rr) dk_ += Pm[rr * C + row] * Ks[rr * ldk + j];
+            aK[m] += btr * egr * y;
             yk += y * Ks[row * ldk + j];
-            if (row < n) {
-                dq[qk_row + j] = from_f32<T>(dq_);
-                dk[qk_row + j] = from_f32<T>(dk_);
+        }
+    }
+    // one pass over the chunk rows i: (dP o Gamma) along this row (dQ) and down
+    // this column (dK), E along the row and down the column (dK); each matrix
+    // element is loaded once for all of the thread's key channels
+    for (int i = 0; i < C; ++i) {
+        const float pr = i <= row ? dP[row * ldc + i] : 0.f;
+        const float pc = i >= row ? dP[i * ldc + row] : 0.f;
+        const float e = (i < row ? Pm[row * ldc + i] : 0.f) + (i > row ? Pm[i * ldc + row] : 0.f);
+#pragma unroll
+        for (int m = 0; m < kMaxCols; ++m) {
+            const int j = sub + TPR * m;
+            if (j < Dk) {
+                const float kij = Ks[i * ldk + j];
+                aQ[m] += pr * kij;
+                aK[m] += pc * Qs[i * ldk + j] + e * kij;
+            }
+        }
+    }
+    if (row < n) {
+#pragma unroll
+        for (int m = 0; m < kMaxCols; ++m) {
+            const int j = sub + TPR * m;
+            if (j < Dk) {
+                dq[qk_row + j] = from_f32<T>(aQ[m]);
+                dk[qk_row + j] = from_f32<T>(aK[m]);
             }
         }
     }
