@@ -18,6 +18,7 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 }
 
 constexpr int kMaxDk = 256, kMaxDv = 512, kMaxGrid = 65535;
+constexpr unsigned long long kMaxTokenHeads = 1ull << 40;
 
 // 0 = fine, otherwise the status to return.
 gdn_status_t check_sizes(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
@@ -26,6 +27,10 @@ gdn_status_t check_sizes(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dty
     if (Dk > kMaxDk || Dv > kMaxDv) return GDN_ERR_UNSUPPORTED;
     if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
     if (B > kMaxGrid || H > kMaxGrid) return GDN_ERR_UNSUPPORTED;
+    // bound the token-head count so that every byte count derived from the sizes
+    // (tensors, states, workspaces) stays far inside size_t
+    if ((unsigned long long)B * (unsigned long long)H * ((unsigned long long)T + 64) > kMaxTokenHeads)
+        return GDN_ERR_UNSUPPORTED;
     return GDN_OK;
 }
 

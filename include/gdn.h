@@ -69,7 +69,9 @@ typedef enum {
 } gdn_path_t;
 
 /* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0
- * (a zero size is an empty problem and is not an error). */
+ * (a zero size is an empty problem and is not an error); B, H <= 65535 and
+ * B * H * (T + 64) <= 2^40 (so that no byte count derived from the sizes can
+ * overflow); beyond these GDN_ERR_UNSUPPORTED. */
 
 /*
  * Optional input prologue of the _ex entry points, applied inside the kernels

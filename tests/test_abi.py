@@ -248,3 +248,17 @@ def test_chunk_fwd_cw_checks(lib):
     assert d(16, 16, 16, 16, 16, None, 1 << 20, 16, 1, 1, 16, 16, 0, None) == 1
     assert d(16, 16, 16, 16, 16, 16, 1 << 20, 16, 1, 1, 16, 16, 0, None) == 1   # o overlaps q
     assert d(16, 16, 16, 16, 16, 16, 1 << 20, 1 << 24, 0, 1, 16, 16, 0, None) == 0
+
+
+def test_sizes_whose_byte_counts_would_overflow_are_refused(lib):
+    from gated_delta_rule_130_b200 import binding as b
+    B, H, T = 65535, 65535, 2 ** 31 - 1            # B H (T + 64) far above 2^40
+    assert _chunk(lib, B=B, H=H, T=T) == 2
+    assert _bwd(lib, B=B, H=H, T=T) == 2
+    assert b.chunk_fwd_workspace_size(B, T, H, 16, 16, 16, torch.float32) == 0
+    assert b.chunk_bwd_workspace_size(B, T, H, 16, 16, 16, torch.float32) == 0
+    assert b.chunk_fwd_cw_workspace_size(B, T, H, 16, 16, 16, torch.float32) == 0
+    with pytest.raises(b.GdnError):
+        b.chunk_fwd_path(B, T, H, 16, 16, 16, torch.float32)
+    # just inside the bound the checks pass on to the workspace test (short: 1)
+    assert _chunk(lib, B=1, H=1, T=2 ** 31 - 1, ws_bytes=16) == 1
