@@ -262,3 +262,28 @@ def test_sizes_whose_byte_counts_would_overflow_are_refused(lib):
         b.chunk_fwd_path(B, T, H, 16, 16, 16, torch.float32)
     # just inside the bound the checks pass on to the workspace test (short: 1)
     assert _chunk(lib, B=1, H=1, T=2 ** 31 - 1, ws_bytes=16) == 1
+
+
+def test_binding_shape_checks_of_the_newer_entry_points():
+    """Mismatched shapes are refused by the binding before any device work."""
+    from gated_delta_rule_130_b200 import binding as b
+    q = torch.zeros(1, 8, 2, 16)
+    v = torch.zeros(1, 8, 2, 12)
+    g = torch.zeros(1, 8, 2)
+    with pytest.raises(b.GdnError):                      # d_o must be shaped like v
+        b.chunk_bwd(q, q, v, g, g, None, torch.zeros(1, 8, 2, 16))
+    with pytest.raises(b.GdnError):                      # dS_T must be [B,H,Dv,Dk]
+        b.chunk_bwd(q, q, v, g, g, None, v, torch.zeros(1, 2, 16, 12))
+    with pytest.raises(b.GdnError):                      # gates must be [B,T,H]
+        b.chunk_bwd(q, q, v, torch.zeros(1, 8, 3), g, None, v)
+    with pytest.raises(b.GdnError):                      # channel-wise decay is per key channel
+        b.chunk_fwd_cw(q, q, v, g, q, v)
+    with pytest.raises(b.GdnError):                      # the write gate is per value channel
+        b.chunk_fwd_cw(q, q, v, q, q, q)
+    with pytest.raises(b.GdnError):
+        b.chunk_fwd_cw(q, q, v, q, q, v, S0=torch.zeros(1, 2, 16, 12))
+    with pytest.raises(b.GdnError):                      # decode state must be [B,H,Dv,Dk]
+        b.decode_step_cw(q[:, 0], q[:, 0], v[:, 0], q[:, 0], q[:, 0], v[:, 0],
+                         torch.zeros(1, 2, 16, 12))
+    with pytest.raises(b.GdnError):                      # packed q, k, v are [total,H,D]
+        b.chunk_fwd_varlen(q, q, v, g, g, [0, 8])
