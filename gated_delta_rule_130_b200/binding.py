@@ -68,6 +68,8 @@ def _load():
     lib.gdn_chunk_fwd_cw_workspace_size.restype = Z
     lib.gdn_decode_step_cw.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, I, I, I, I, I, vp]
     lib.gdn_decode_step_cw.restype = I
+    lib.gdn_debug_withhold_first_arrival.argtypes = [I]
+    lib.gdn_debug_withhold_first_arrival.restype = I
     lib.gdn_check_device_status.argtypes = []
     lib.gdn_check_device_status.restype = I
     lib.gdn_status_string.argtypes = [I]

@@ -56,14 +56,22 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace gdn {
 
 // Set by a fused-kernel CTA that gave up waiting (read with gdn_check_device_status).
 __device__ unsigned int g_tc_error = 0;
 
+// Test hook of the bounded waits (gdn_debug_withhold_first_arrival): when set,
+// the TMA warp of every sequential-kernel CTA withholds its arrival on the first
+// stage, so every role's first wait runs out and the CTA takes its abort path
+// (flag set, roles stopped, copies drained, tensor memory released).
+__device__ unsigned int g_tc_withhold_first = 0;
+
 // Optional per-role timeline of CTA (0,0,0) for performance work: build with
-// -DGDN_TRACE and read with gdn_trace_read().  Compiled out otherwise.
+// -DGDN_TRACE; that build alone exports gdn_trace_read() and gdn_tracew_read()
+// (end of this file) to copy the timelines out.  Compiled out otherwise.
 #ifdef GDN_TRACE
 __device__ unsigned long long g_trace[64 * 32];
 __device__ unsigned long long g_tracew[16 * 32 * 20];
@@ -102,7 +110,6 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int C = 64;          // chunk length (tokens)
 constexpr int DVT = 64;        // value channels per CTA
 constexpr int DK = 128;        // key channels
 constexpr int KB = DK / 64;    // 64-wide key blocks
@@ -112,7 +119,6 @@ constexpr int BLK = 8192;      // one 64 x 64 bf16 tile (64 rows of 128 bytes)
 constexpr int GRP = 3 * BLK;   // K | Q | W of one key block
 constexpr int STAGE = KB * GRP + 3 * BLK;  // + V tile + [T'; T''] (16 KiB)
 constexpr int OFF_K = 0, OFF_Q = BLK, OFF_W = 2 * BLK, OFF_V = KB * GRP, OFF_TT = KB * GRP + BLK;
-constexpr int LDA = 72;        // padded float32 row stride of A and T (16-B rows)
 
 // Per-stage gate vectors (float offsets), written by the TMA warp:
 constexpr int GV_G2 = 0;       // g_r log2(e), g_r = sum of log alpha over rows <= r
@@ -181,179 +187,6 @@ constexpr int W_STATE0 = 8;               // warps 8-15: sequential state / outp
 constexpr int NSTATEW = 8;
 constexpr int NTHREADS = 32 * (W_STATE0 + NSTATEW);
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;
-
-__device__ __forceinline__ uint64_t now_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// 2^x (hardware approximation, relative error about 2^-22)
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-struct Ctx {
-    uint8_t *base;
-    uint64_t *bar;
-    volatile uint32_t *abort;
-};
-
-// Bounded wait; false (and the CTA-wide abort flag set) on timeout or abort.
-__device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
-    uint64_t *b = cx.bar + idx;
-#ifdef GDN_WAIT_TEST_SLEEP_NS
-    {
-        if (mbar_test_wait(b, parity)) return true;
-        const uint64_t t0 = now_ns();
-        for (uint32_t it = 1;; ++it) {
-            __nanosleep(GDN_WAIT_TEST_SLEEP_NS);
-            if (mbar_test_wait(b, parity)) return true;
-            if ((it & 63u) == 0) {
-                if (*cx.abort) return false;
-                if (now_ns() - t0 > kTimeoutNs) {
-                    *cx.abort = 1u;
-                    atomicOr(&g_tc_error, 1u);
-                    return false;
-                }
-            }
-        }
-    }
-#endif
-    if (mbar_try_wait(b, parity)) return true;
-    const uint64_t t0 = now_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(b, parity)) return true;
-#ifdef GDN_WAIT_BACKOFF_NS
-        if (it > 32) __nanosleep(GDN_WAIT_BACKOFF_NS);
-#endif
-        if ((it & 255u) == 0) {
-            if (*cx.abort) return false;
-            if (now_ns() - t0 > kTimeoutNs) {
-                *cx.abort = 1u;
-                atomicOr(&g_tc_error, 1u);
-                return false;
-            }
-        }
-    }
-}
-
-// Slow path of warp_wait: lane 0 polls (so waiting warps do not compete with
-// working warps for the shared-memory pipe) and the result is broadcast.
-__device__ __noinline__ bool warp_wait_slow(const Ctx &cx, int idx, uint32_t parity) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(cx, idx, parity);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();  // orders the other lanes' later accesses after lane 0's acquire
-    return ok;
-}
-
-// A wait on behalf of a whole warp.  The common case (the phase has already
-// completed) is one test and a vote, with no divergent branch; the result is
-// warp-uniform, so a timeout never splits a warp in front of a warp-collective
-// tcgen05 access.
-__device__ __forceinline__ bool warp_wait(const Ctx &cx, int idx, uint32_t parity) {
-    if (__all_sync(0xffffffffu, mbar_try_wait(cx.bar + idx, parity))) return true;
-    return warp_wait_slow(cx, idx, parity);
-}
-
-// One arrival on behalf of a whole warp, after every lane's prior writes
-// (lane 0 arrives, predicated rather than branched).
-__device__ __forceinline__ void warp_arrive(const Ctx &cx, int idx) {
-    __syncwarp();
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %1, 0;\n\t"
-        "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(cx.bar + idx)),
-        "r"(threadIdx.x & 31u)
-        : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<const uint32_t *>(&h);
-}
-
-// Columns [16 piece, 16 piece + 16) of bf16 row `row` of a 128B-swizzled tile.
-__device__ __forceinline__ void store16_bf16(uint8_t *tile, int row, int piece, const float (&v)[16]) {
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        uint4 q;
-        q.x = pack_bf16(v[8 * k + 0], v[8 * k + 1]);
-        q.y = pack_bf16(v[8 * k + 2], v[8 * k + 3]);
-        q.z = pack_bf16(v[8 * k + 4], v[8 * k + 5]);
-        q.w = pack_bf16(v[8 * k + 6], v[8 * k + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw128_offset(row, (2 * piece + k) * 16)) = q;
-    }
-}
-
-__device__ __forceinline__ void tmem_ld16w(uint32_t taddr, float (&v)[16]) {
-    tmem_ld16(taddr, v);
-    tmem_wait_ld();
-}
-
-// The UT transform T = (I + A)^-1 of the 64 x 64 strictly lower A (AF, float32,
-// stride LDA), blocked by 16 with D_I = I + A_II:
-//   T_II = D_I^-1                                   (ut_diag, forward substitution)
-//   N_IJ = T_II A_IJ,  I > J                        (ut_offdiag4 phase 1, all six blocks)
-//   T_IJ = -sum_{J <= K < I} N_IK T_KJ              (phase 2, one warp per block column)
-// TF receives the lower triangle and the diagonal; its strict upper part is not
-// written (and never read).
-
-// Column j of T_II for block I = p / 16 (p < 64).
-__device__ __forceinline__ void ut_diag(const float *__restrict__ AF, float *__restrict__ TF, int p) {
-    const int I = p >> 4, j = p & 15, o = 16 * I;
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        float a[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = *reinterpret_cast<const float4 *>(AF + (o + r) * LDA + o + 4 * q);
-            a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
-        }
-        float acc0 = 0.f, acc1 = 0.f;  // two partial sums: shorter dependency chains
-#pragma unroll
-        for (int i = 0; i < r; ++i) {
-            if (i & 1) acc1 = fmaf(a[i], x[i], acc1);
-            else acc0 = fmaf(a[i], x[i], acc0);
-        }
-        x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -(acc0 + acc1));
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) TF[(o + r) * LDA + o + j] = x[r];
-}
-
-// acc (16 x 16 as two 16 x 8 mma tiles) += Ablk (16 x 16, stride lda) * Bblk
-// (16 x 16, stride ldb), TF32 tensor-core products with float32 accumulation;
-// one warp.
-__device__ __forceinline__ void mma16(float (&acc)[2][4], const float *__restrict__ A, int lda,
-                                      const float *__restrict__ B, int ldb, int g, int t) {
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const int k0 = 8 * ks;
-        const uint32_t a[4] = {to_tf32(A[g * lda + k0 + t]), to_tf32(A[(g + 8) * lda + k0 + t]),
-                               to_tf32(A[g * lda + k0 + t + 4]), to_tf32(A[(g + 8) * lda + k0 + t + 4])};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t bb[2] = {to_tf32(B[(k0 + t) * ldb + 8 * nt + g]),
-                                    to_tf32(B[(k0 + t + 4) * ldb + 8 * nt + g])};
-            mma_tf32_16x8x8(acc[nt], a, bb);
-        }
-    }
-}
-
-__device__ __forceinline__ void store16x16(const float (&acc)[2][4], float *__restrict__ D, int ld,
-                                           float sign, int g, int t) {
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        *reinterpret_cast<float2 *>(D + g * ld + 8 * nt + 2 * t) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
-        *reinterpret_cast<float2 *>(D + (g + 8) * ld + 8 * nt + 2 * t) = make_float2(sign * acc[nt][2], sign * acc[nt][3]);
-    }
-}
-
 // Gated, masked Q K^T row, one 16-column piece (columns i = 16 B + j) of row r:
 // out[i] = Gamma(r, i) gram[i] for i <= r, zero above, Gamma(r, i) = exp(g_r - g_i).
 // Off the row's diagonal 16-block R the decay factors as u_r * w_R[i] (u_r =
@@ -377,41 +210,6 @@ __device__ __forceinline__ void gated_piece(float (&v)[16], int B, int r, float 
         }
         v[j] *= f;
     }
-}
-
-// ------------------------------------------------------------- sequences --
-// Where each sequence lives in the packed token dimension ([tokens, H, D] rows):
-// a fixed-length batch (cu == nullptr: sequence b is tokens [b T, b T + T)) or
-// variable lengths (tokens cu[b] .. cu[b + 1]).  Chunks are numbered globally,
-// sequence by sequence: sequence b owns chunks chunk0 .. chunk0 + ceil(len / C).
-struct Seqs {
-    const int *cu;         // n + 1 token offsets (device), or null
-    const int *cu_chunks;  // n + 1 chunk offsets (device), or null
-    const int *order;      // launch order of the sequences (device), or null
-    int T;                 // the common length when cu is null
-    int n;                 // number of sequences
-};
-
-struct Span {
-    int off, len, chunk0;
-};
-
-__device__ __forceinline__ Span seq_span(const Seqs &q, int b) {
-    if (q.cu) return Span{q.cu[b], q.cu[b + 1] - q.cu[b], q.cu_chunks[b]};
-    return Span{b * q.T, q.T, b * ((q.T + C - 1) / C)};
-}
-
-// The sequence a global chunk index belongs to: the last b with cu_chunks[b] <= g
-// (empty sequences share their start with the next one and are skipped).
-__device__ __forceinline__ int seq_of_chunk(const Seqs &q, int g) {
-    if (!q.cu) return g / ((q.T + C - 1) / C);
-    int lo = 0, hi = q.n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (q.cu_chunks[mid] <= g) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
 }
 
 // Bucket of a sequence by its chunk count on a quarter-octave scale (exact below
@@ -501,42 +299,6 @@ constexpr int ut_smem_bytes(bool norm) { return UT_SM_GT + (norm ? 4 : 3) * C * 
 constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
 static_assert(C * LDK * 2 <= UT_SM_AF, "K chunk fits in the T buffer");
 static_assert(UT_SM_AF % 16 == 0 && UT_SM_GT % 16 == 0, "16-byte aligned UT buffers");
-
-// Off-diagonal blocks of T with 4 warps, N_IJ = T_II A_IJ stored over A_IJ:
-//   phase 1  N for the six blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2), two rounds
-//   phase 2  T_{J+1,J} = -N_{J+1,J} T_JJ                              (3 warps)
-//   phase 3  T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})    (2 warps)
-//   phase 4  T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)              (1 warp)
-__device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__restrict__ TF,
-                                            int p) {
-    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
-    const auto blk = [&](float *M, int I, int J) { return M + 16 * I * LDA + 16 * J; };
-#pragma unroll
-    for (int round = 0; round < 2; ++round) {
-        const int k = w + 4 * round;  // block (I, J) in the order listed above
-        if (k < 6) {
-            const int I = k == 0 ? 1 : (k < 3 ? 2 : 3), J = k == 0 ? 0 : (k < 3 ? k - 1 : k - 3);
-            float acc[2][4] = {};
-            mma16(acc, blk(TF, I, I), LDA, blk(AF, I, J), LDA, g, t);
-            __syncwarp();
-            store16x16(acc, blk(AF, I, J), LDA, 1.f, g, t);
-        }
-    }
-    __syncthreads();
-    // block column J of T needs only its own earlier blocks and the N blocks:
-    // warp J walks down it, T_IJ = -sum_{K=J}^{I-1} N_IK T_KJ, with no CTA barrier
-    if (w < 3) {
-        const int J = w;
-        for (int I = J + 1; I < 4; ++I) {
-            float acc[2][4] = {};
-            for (int K = J; K < I; ++K)
-                mma16(acc, blk(AF, I, K), LDA, blk(TF, K, J), LDA, g, t);
-            store16x16(acc, blk(TF, I, J), LDA, -1.f, g, t);
-            __syncwarp();
-        }
-    }
-    __syncthreads();
-}
 
 // kNorm: q and k are L2-normalised inside the kernels (1/|k| folded into the
 // Gram rows and T', and written to rk_out); without it the kernel is unchanged.
@@ -727,6 +489,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     cx.bar = reinterpret_cast<uint64_t *>(base + SM_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + SM_MISC);
     cx.abort = reinterpret_cast<volatile uint32_t *>(base + SM_MISC + 4);
+    cx.err = &g_tc_error;
     float *gv_all = reinterpret_cast<float *>(base + SM_GV);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -798,6 +561,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // the [T'; T''] tiles (and 1/|k|) come from the UT kernel launched just
         // before this one (programmatic dependent launch): wait for its completion
         asm volatile("griddepcontrol.wait;" ::: "memory");
+        const bool withhold = *reinterpret_cast<volatile unsigned int *>(&g_tc_withhold_first) != 0u;
         fetch_gates(0);
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1;
@@ -886,7 +650,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             gv[GV_W + 3 * 64 + 32 + lane] = lane < 16 ? ex2(g48 - g1) : 0.f;
             if (lane == 0) gv[GV_GL] = ex2(glast);
             __syncwarp();
-            if (lane == 0) mbar_arrive(cx.bar + B_IN_FULL + s);
+            if (lane == 0 && !(withhold && c == 0)) mbar_arrive(cx.bar + B_IN_FULL + s);
         }
         // never leave with copies in flight: wait for the last two stages
         if (lane == 0) {
@@ -1424,6 +1188,11 @@ extern "C" int gdn_tracew_read(unsigned long long *dst) {
     return (int)cudaMemcpyFromSymbol(dst, g_tracew, sizeof(g_tracew));
 }
 #endif
+
+cudaError_t set_withhold_first_arrival(bool on) {
+    const unsigned int v = on ? 1u : 0u;
+    return cudaMemcpyToSymbol(g_tc_withhold_first, &v, sizeof(v));
+}
 
 cudaError_t read_and_clear_device_error(unsigned int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_tc_error, sizeof(unsigned int));

@@ -430,6 +430,10 @@ gdn_status_t gdn_decode_step_cw(const void *q, const void *k, const void *v,
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status_t gdn_debug_withhold_first_arrival(int enable) {
+    return gdn::set_withhold_first_arrival(enable != 0) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status_t gdn_check_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
     unsigned int flag = 0;

@@ -93,5 +93,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).
 cudaError_t read_and_clear_device_error(unsigned int *flag);
+// Test hook: the sequential tcgen05 kernel withholds its first stage's arrival
+// (every CTA then times out, about two seconds, and sets that flag).
+cudaError_t set_withhold_first_arrival(bool on);
 
 }  // namespace gdn

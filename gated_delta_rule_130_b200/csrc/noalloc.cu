@@ -10,10 +10,14 @@
 // GPU that loads the library holds it until the process exits.  Its device
 // address is looked up once per device (the first call on that device, with
 // that device current), so that first call must come before any stream capture.
-// All calls share the one array and it keeps the last call's contents: the
-// kernels write every workspace element before they read it, so nothing needs
-// clearing, but calls whose work overlaps on the GPU (different streams, or
-// threads) race on it and must be serialised by the caller.
+// All calls share the one array and it keeps the last call's contents.  The
+// two paths that use it write their scratch before reading it (the CUDA-core
+// path's per-chunk T, P and gate sums; the tcgen05 path's [T'; T''] tiles, and
+// with the prologue flags off there is nothing else), so nothing needs
+// clearing; calls whose work overlaps on the GPU (different streams, or
+// threads) race on it and must be serialised by the caller.  The address is
+// cached for the life of the process: after a cudaDeviceReset the cached value
+// is stale, and the entry point must not be used on that device again.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -16,9 +16,11 @@
  *
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    allocates nothing, keeps no state between calls, and only enqueues work on
- *    `stream` (a cudaStream_t; NULL means the legacy default stream).  Calls
- *    return as soon as the work is enqueued.
+ *    allocates nothing and only enqueues work on `stream` (a cudaStream_t; NULL
+ *    means the legacy default stream).  Calls return as soon as the work is
+ *    enqueued.  No entry point keeps state between calls, except
+ *    gdn_chunk_fwd_noalloc, whose fixed scratch array and cached address are
+ *    described at its declaration.
  *  - Layouts are dense row-major (C order), no strides:
  *        q, k      [B, T, H, Dk]     (decode: [B, H, Dk])
  *        v, o      [B, T, H, Dv]     (decode: [B, H, Dv])
@@ -182,11 +184,16 @@ size_t gdn_chunk_fwd_varlen_workspace_size(const int *cu_seqlens_host, int N, in
  *
  * Same arguments and results as gdn_chunk_fwd, minus the workspace.  The
  * scratch is a fixed 8 MiB array inside the library (held on every GPU that
- * loads it until exit); sizes whose workspace (gdn_chunk_fwd_workspace_size)
- * exceeds 8 MiB return GDN_ERR_UNSUPPORTED with nothing launched.  The first call on a device looks up the array's address
- * (with that device current) and must come before any stream capture.  All
- * calls share the array: calls whose work overlaps on the GPU race and must be
- * serialised by the caller.  Allocates nothing.
+ * loads it until exit).  The size limit is checked first: sizes whose workspace
+ * (gdn_chunk_fwd_workspace_size) exceeds 8 MiB return GDN_ERR_UNSUPPORTED with
+ * nothing launched and no pointer looked at; the other checks are those of
+ * gdn_chunk_fwd.  The first call on a device looks up the array's address
+ * (with that device current) and must come before any stream capture; the
+ * address is kept for the life of the process, so a cudaDeviceReset makes this
+ * entry point unusable on that device until the process restarts.  All calls
+ * share the array and it keeps the last call's contents (every path that uses
+ * it writes its scratch before reading it): calls whose work overlaps on the
+ * GPU race and must be serialised by the caller.  Allocates nothing.
  */
 gdn_status_t gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                    const float *log_alpha, const float *beta,
@@ -300,6 +307,18 @@ gdn_status_t gdn_decode_step_cw(const void *q, const void *k, const void *v,
  * it) or if synchronising failed, GDN_OK otherwise.
  */
 gdn_status_t gdn_check_device_status(void);
+
+/*
+ * Test hook of that failure detection (the pages have no counterpart).  With
+ * `enable` != 0 the sequential tensor-core kernel of every later
+ * gdn_chunk_fwd* call on the current device withholds the arrival that
+ * publishes its first stage of inputs: every warp's first wait runs out (about
+ * two seconds), each CTA records the flag above, stops, drains its copies and
+ * frees its tensor memory, and the call's outputs are left incomplete.  Nothing
+ * faults and the context stays usable.  enable = 0 restores normal operation.
+ * Synchronous; returns GDN_ERR_CUDA if the flag could not be written.
+ */
+gdn_status_t gdn_debug_withhold_first_arrival(int enable);
 
 /* Static, human-readable name of a status code. */
 const char *gdn_status_string(gdn_status_t status);
