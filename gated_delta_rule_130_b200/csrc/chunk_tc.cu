@@ -1080,25 +1080,32 @@ bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 // Workspace: [chunk offsets of the sequences, variable lengths only, padded to
 // 256 B][one [T'; T''] tile per chunk and head][1/|k| per token, normalising only].
 // chunk offsets (n + 1) and launch order (n) of the sequences
-static size_t tc_offsets_bytes(int n_seq, bool varlen) {
+size_t tc_offsets_bytes(int n_seq, bool varlen) {
     return varlen ? ((2 * (size_t)n_seq + 1) * sizeof(int) + 255) & ~size_t(255) : 0;
 }
 
 size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                               unsigned flags) {
+                               unsigned flags, int Dk) {
+    if (Dk == tcw_dk) return tcw_workspace_bytes_seqs(n_seq, total_chunks, H, varlen, flags);
     const size_t tiles = (size_t)total_chunks * H * tc::TT_ELEMS * sizeof(__nv_bfloat16);
     const size_t rk = (flags & kFlagL2Norm) ? (size_t)total_chunks * H * tc::C * sizeof(float) : 0;
     return tc_offsets_bytes(n_seq, varlen) + tiles + rk;
 }
 
-size_t tc_workspace_bytes(int B, int T, int H, unsigned flags) {
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk) {
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
-    return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags);
+    return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags, Dk);
 }
 
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
-    return bf16 && chunk == tc::C && Dk == tc::DK && Dv % tc::DVT == 0 && B >= 1 && T >= 1 &&
-           H >= 1 && tc::encode_fn() != nullptr;
+    return bf16 && chunk == tc::C && (Dk == tc::DK || Dk == tcw_dk) && Dv % tc::DVT == 0 &&
+           B >= 1 && T >= 1 && H >= 1 && tc::encode_fn() != nullptr;
+}
+
+cudaError_t launch_seq_schedule(const int *cu_seqlens, int n_seq, int *cu_chunks, int *order,
+                                cudaStream_t st) {
+    tc::seq_schedule<<<1, tc::kScheduleThreads, 0, st>>>(cu_seqlens, n_seq, cu_chunks, order);
+    return cudaPeekAtLastError();
 }
 
 cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
@@ -1107,6 +1114,11 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
                                  int Dv, unsigned flags, void *workspace, cudaStream_t st,
                                  float *S_hist) {
+    if (Dk == tcw_dk) {
+        if (S_hist) return cudaErrorInvalidValue;  // the state history is a Dk = 128 feature
+        return launch_chunk_tcw_seqs(q, k, v, log_alpha, beta, S0, o, S_T, n_seq, T_fixed, total_T,
+                                     cu_seqlens, total_chunks, H, Dv, flags, workspace, st);
+    }
     const bool varlen = cu_seqlens != nullptr;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
@@ -1121,9 +1133,8 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
         !tc::make_map_tt(&mt, tt, total_chunks > 0 ? total_chunks * H : 1))
         return cudaErrorInvalidValue;
     if (varlen) {
-        tc::seq_schedule<<<1, tc::kScheduleThreads, 0, st>>>(cu_seqlens, n_seq, cu_chunks,
-                                                             cu_chunks + n_seq + 1);
-        const cudaError_t e0 = cudaPeekAtLastError();
+        const cudaError_t e0 = launch_seq_schedule(cu_seqlens, n_seq, cu_chunks,
+                                                   cu_chunks + n_seq + 1, st);
         if (e0 != cudaSuccess) return e0;
     }
     tc::Params p;

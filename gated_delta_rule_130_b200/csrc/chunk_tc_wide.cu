@@ -1,0 +1,886 @@
+// Chunkwise forward of the gated delta rule on sm_100a tensor cores for wide
+// heads: Dk = 256, Dv any multiple of 64 (the 1.3B-parameter layer shape has
+// Dv = 512), bf16 q/k/v/o, float32 gates, state and accumulation.
+//
+// The chunk algebra is the one of chunk_tc.cu (the gated WY/UT form of "Gated
+// Delta Networks: Improving Mamba2 with Delta Rule", section "Approach"; "Gated
+// DeltaNet: Harmonizing Gating and the Delta Rule ...", section
+// "Hardware-Efficient Training"), per chunk of C = 64 tokens with g_r the
+// running sum of log alpha from the chunk start and gamma_r = exp(g_r):
+//   A   = strictly-lower( beta_r exp(g_r - g_i) k_r . k_i ),   T = (I + A)^-1
+//   P   = Q K^T o exp(g_r - g_i) o [i <= r]
+//   W   = T diag(beta gamma) K,   U = T diag(beta) V,   U' = U - W S^T
+//   O   = diag(gamma) Q S^T + P U'
+//   S  <- gamma_last S + U'^T diag(exp(g_last - g)) K
+// At Dk = 256 a chunk's key-side tiles (Q, K and W, 32 KiB each) and a 256-row
+// slice of the state leave no room in one SM for chunk_tc.cu's in-kernel Gram
+// and WY products next to a two-stage ring, so the key-side work moves to the
+// parallel kernel:
+//  1. gdn_utw_kernel, one CTA per (chunk, head), all chunks in parallel: the
+//     Gram matrix and Q K^T (bf16 mma.sync, float32 accumulation), the gating,
+//     the blocked UT solve, and W = T diag(beta gamma) K; it writes the bf16
+//     tiles [P; T''] (128 x 64, T'' = T diag(beta)) and W (64 x 256) of each
+//     chunk to the workspace.  None of it depends on the state, and it is
+//     formed once per head instead of once per value slice.
+//  2. gdn_chunk_tcw_kernel, one CTA per (sequence, head, 64 value channels),
+//     walking the chunks in order with S^T (256 x 64, float32, as two 128-lane
+//     halves) resident in tensor memory.  Products (tcgen05.mma, M = 128, bf16
+//     operands in 128-byte-swizzled shared memory, float32 in TMEM):
+//       X     = [Q;W] S^T             rows 0-63 Q S^T, rows 64-127 W S^T (K = 256)
+//       U     = [P;T''] V             rows 64-127 U (rows 0-63 unused)     (K = 64)
+//       S^T_h += K_h^T diag(exp(g_last - g)) U'   for the key halves h     (K = 64)
+//       Y     = [P;T''] U'            rows 0-63 P U', Y preloaded with gamma Q S^T
+//     Warp roles: 0 TMA (and gate vectors), 1 the sequential products (TMEM
+//     owner), 2 the U product, 4-11 the state warps (U' = U - W S^T, the
+//     output, the state hand-off).  [Q;W] and K are single-buffered and
+//     refilled as soon as the product that last reads them completes; V,
+//     [P;T''] and the gate vectors use a two-stage ring.
+// Rows past the end of a sequence are loaded as zeros and get beta = 0 and
+// log alpha = 0, which leaves the real rows' results unchanged.  Every mbarrier
+// wait is bounded (about two seconds); a CTA that times out sets an error flag
+// (gdn_check_device_status), stops, waits for its copies and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+
+// Set by a CTA of gdn_chunk_tcw_kernel that gave up waiting.
+__device__ unsigned int g_tcw_error = 0;
+
+namespace tcw {
+
+using namespace sm100;
+using tc::C;
+using tc::Ctx;
+using tc::LDA;
+using tc::Seqs;
+using tc::Span;
+
+constexpr int DK = 256;
+constexpr int KB = DK / 64;        // 64-key blocks
+constexpr int DVT = 64;            // value channels per CTA of the sequential kernel
+constexpr float LOG2E = 1.4426950408889634f;
+
+// ------------------------------------------------------------- UT kernel --
+// One CTA of 4 warps per (global chunk g, head h).  Outputs at tile index
+// g H + h: [P; T''] (128 x 64 bf16, row-major), W (64 x 256 bf16, row-major) and,
+// when normalising, 1/|q| and 1/|k| of the chunk's rows (2 x 64 float32).
+constexpr int UT_THREADS = 128;
+constexpr int LDKW = DK + 8;                       // bf16 row stride of staged K, Q and W
+constexpr int LDB = C + 8;                         // bf16 row stride of P and T'
+constexpr int SM_K = 0;                            // K chunk (64 x LDKW bf16)
+constexpr int SM_Q = SM_K + C * LDKW * 2;          // Q chunk; then T (f32); then W staging
+constexpr int SM_A = SM_Q + C * LDKW * 2;          // A (f32, 64 x LDA); then T' (bf16)
+constexpr int SM_P = SM_A + C * LDA * 4;           // P (bf16, 64 x LDB)
+constexpr int SM_G = SM_P + C * LDB * 2;           // 5 x 64 floats of per-row gates and norms
+constexpr int UT_SMEM = SM_G + 5 * C * 4;
+constexpr int PT_ELEMS = 2 * C * C;
+constexpr int W_ELEMS = C * DK;
+static_assert(C * LDA * 4 <= C * LDKW * 2, "T fits in the Q buffer");
+static_assert(C * LDB * 2 <= C * LDA * 4, "T' fits in the A buffer");
+static_assert(SM_Q % 16 == 0 && SM_A % 16 == 0 && SM_P % 16 == 0 && SM_G % 16 == 0,
+              "16-byte aligned buffers");
+
+template <bool kNorm>
+__global__ void __launch_bounds__(UT_THREADS, 2)
+gdn_utw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+               const float *__restrict__ log_alpha, const float *__restrict__ beta,
+               __nv_bfloat16 *__restrict__ pt, __nv_bfloat16 *__restrict__ wt,
+               float *__restrict__ rqk, const Seqs sq, int H, unsigned flags) {
+    extern __shared__ __align__(16) uint8_t ut_smem[];
+    // the sequential kernel that follows may be scheduled now (it waits for this
+    // grid's completion before it reads the tiles)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int gch = blockIdx.x, h = blockIdx.y;
+    const int b = tc::seq_of_chunk(sq, gch);
+    const Span sp = tc::seq_span(sq, b);
+    const int c = gch - sp.chunk0, T = sp.len, t0 = c * C;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const size_t tile = (size_t)gch * H + h;
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_K);
+    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_Q);
+    float *TF = reinterpret_cast<float *>(ut_smem + SM_Q);
+    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_Q);
+    float *AF = reinterpret_cast<float *>(ut_smem + SM_A);
+    __nv_bfloat16 *Tb = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_A);
+    __nv_bfloat16 *Pb = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_P);
+    float *g2s = reinterpret_cast<float *>(ut_smem + SM_G);
+    float *bes = g2s + C, *bgs = g2s + 2 * C, *rks = g2s + 3 * C, *rqs = g2s + 4 * C;
+
+    // q and k rows of the chunk (zero-filled past the end): 32 x 16 B per row
+#pragma unroll 4
+    for (int m = 0; m < C * (DK / 8) / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int r = idx / (DK / 8), piece = idx % (DK / 8);
+        const bool in = t0 + r < T;
+        const size_t row = (size_t)(sp.off + (in ? t0 + r : 0)) * H + h;
+        cp_async16(Ks + r * LDKW + 8 * piece, k + row * DK + 8 * piece, in ? 16u : 0u);
+        cp_async16(Qs + r * LDKW + 8 * piece, q + row * DK + 8 * piece, in ? 16u : 0u);
+    }
+    if (warp == 0) {
+        // running sum of log alpha over rows lane and lane + 32, in log2 units
+        float la[2], be[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            const bool in = t0 + r < T;
+            const size_t gi = (size_t)(sp.off + t0 + r) * H + h;
+            const float2 gp = in ? gate_pair(log_alpha[gi], beta[gi], flags) : make_float2(0.f, 0.f);
+            la[hh] = gp.x;
+            be[hh] = gp.y;
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, la[0], off);
+            const float y1 = __shfl_up_sync(0xffffffffu, la[1], off);
+            if (lane >= off) {
+                la[0] += y0;
+                la[1] += y1;
+            }
+        }
+        la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float g2 = la[hh] * LOG2E;
+            g2s[lane + 32 * hh] = g2;
+            bes[lane + 32 * hh] = be[hh];
+            bgs[lane + 32 * hh] = be[hh] * tc::ex2(g2);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    if constexpr (kNorm) {
+        // 1/|k_r| (threads 0-63) and 1/|q_r| (threads 64-127), one row each
+        const int r = tid & (C - 1);
+        const bool isq = tid >= C;
+        const uint4 *row = reinterpret_cast<const uint4 *>((isq ? Qs : Ks) + r * LDKW);
+        float ss = 0.f;
+#pragma unroll 8
+        for (int m = 0; m < DK / 8; ++m) {
+            const uint4 u = row[m];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                ss += f.x * f.x + f.y * f.y;
+            }
+        }
+        const float rn = rsqrtf(ss + kNormEps);
+        if (isq) {
+            rqs[r] = rn;
+        } else {
+            rks[r] = rn;
+            bgs[r] *= rn;
+        }
+        rqk[tile * 2 * C + (isq ? 0 : C) + r] = rn;
+        __syncthreads();
+    }
+
+    // Gram K K^T and Q K^T on and below the diagonal: warp w takes rows 16 w .. + 15
+    // and the 2 w + 2 column tiles of 8 up to the diagonal (one pass over the keys
+    // for both products), then gates them:
+    //   A_ri = beta_r exp(g_r - g_i) k_r . k_i    (i < r, else 0)
+    //   P_ri = exp(g_r - g_i) q_r . k_i           (i <= r, else 0)
+    {
+        const int RB = warp, ntiles = 2 * RB + 2;
+        float accg[8][4] = {}, accp[8][4] = {};
+        const int mi = lane >> 3, ri = lane & 7;
+        const int arow_off = (16 * RB + ri + 8 * (mi & 1)) * LDKW + 8 * (mi >> 1);
+        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi >> 1)) * LDKW + 8 * (mi & 1);
+#pragma unroll 2
+        for (int ks = 0; ks < DK / 16; ++ks) {
+            const int k0 = 16 * ks;
+            uint32_t ak[4], aq[4];
+            ldmatrix_x4(ak, Ks + arow_off + k0);
+            ldmatrix_x4(aq, Qs + arow_off + k0);
+#pragma unroll
+            for (int jp = 0; jp < 4; ++jp) {
+                if (2 * jp < ntiles) {
+                    uint32_t bq[4];
+                    ldmatrix_x4(bq, brow + 16 * jp * LDKW + k0);
+                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+                    mma_bf16_16x8x16(accg[2 * jp], ak, b0);
+                    mma_bf16_16x8x16(accg[2 * jp + 1], ak, b1);
+                    mma_bf16_16x8x16(accp[2 * jp], aq, b0);
+                    mma_bf16_16x8x16(accp[2 * jp + 1], aq, b1);
+                }
+            }
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = 16 * RB + g + 8 * hr;
+            const float gr = g2s[r];
+            const float br = kNorm ? bes[r] * rks[r] : bes[r];
+            const float pr = kNorm ? rqs[r] : 1.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = 8 * j + 2 * t;
+                float p0 = 0.f, p1 = 0.f;
+                if (j < ntiles) {
+                    // exponents are <= 0 where selected (g is non-increasing)
+                    const float e0 = tc::ex2(gr - g2s[i]), e1 = tc::ex2(gr - g2s[i + 1]);
+                    const float k0 = kNorm ? rks[i] : 1.f, k1 = kNorm ? rks[i + 1] : 1.f;
+                    const float a0 = (i < r) ? br * k0 * e0 * accg[j][2 * hr] : 0.f;
+                    const float a1 = (i + 1 < r) ? br * k1 * e1 * accg[j][2 * hr + 1] : 0.f;
+                    p0 = (i <= r) ? pr * k0 * e0 * accp[j][2 * hr] : 0.f;
+                    p1 = (i + 1 <= r) ? pr * k1 * e1 * accp[j][2 * hr + 1] : 0.f;
+                    *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
+                }
+                *reinterpret_cast<uint32_t *>(Pb + r * LDB + i) = tc::pack_bf16(p0, p1);
+            }
+        }
+    }
+    __syncthreads();  // A and P complete; Q is no longer read (its buffer becomes T)
+    if (tid < C) tc::ut_diag(AF, TF, tid);
+    __syncthreads();
+    tc::ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
+
+    // [P; T''] to the workspace (8 threads per 128-byte row), T'' = T diag(beta)
+    __nv_bfloat16 *dpt = pt + tile * PT_ELEMS;
+#pragma unroll 2
+    for (int m = 0; m < PT_ELEMS / 8 / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int rt = idx >> 3, i0 = 8 * (idx & 7);
+        uint4 val;
+        if (rt < C) {
+            val = *reinterpret_cast<const uint4 *>(Pb + rt * LDB + i0);
+        } else {
+            const int r = rt - C;
+            const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
+            const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
+            const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (i0 + e <= r) ? tv[e] * bes[i0 + e] : 0.f;
+            val = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                             tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+        }
+        *reinterpret_cast<uint4 *>(dpt + rt * C + i0) = val;
+    }
+    // T' = T diag(beta gamma / |k|) (lower triangle) as bf16 over the dead A buffer
+#pragma unroll
+    for (int m = 0; m < C * C / 8 / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int r = idx >> 3, i0 = 8 * (idx & 7);
+        const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
+        const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
+        const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = (i0 + e <= r) ? tv[e] * bgs[i0 + e] : 0.f;
+        *reinterpret_cast<uint4 *>(Tb + r * LDB + i0) =
+            make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                       tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+    }
+    __syncthreads();  // T' complete; T is no longer read (its buffer becomes W)
+
+    // W = T' K: warp w takes rows 16 w .. + 15 (T' is lower triangular, so only
+    // chunk rows 0 .. 16 w + 15 contribute), in two passes of 128 key columns
+    {
+        const int mi = lane >> 3, ri = lane & 7;
+        const __nv_bfloat16 *arow = Tb + (16 * warp + ri + 8 * (mi & 1)) * LDB + 8 * (mi >> 1);
+        // B = K (chunk row i = k index, key = n index), stored with k along the rows
+        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi & 1)) * LDKW + 8 * (mi >> 1);
+#pragma unroll 1
+        for (int nh = 0; nh < 2; ++nh) {
+            float acc[16][4] = {};
+#pragma unroll 1
+            for (int ks = 0; ks <= warp; ++ks) {
+                uint32_t a[4];
+                ldmatrix_x4(a, arow + 16 * ks);
+#pragma unroll
+                for (int np = 0; np < 8; ++np) {
+                    uint32_t bq[4];
+                    ldmatrix_x4_trans(bq, brow + 16 * ks * LDKW + 128 * nh + 16 * np);
+                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+                    mma_bf16_16x8x16(acc[2 * np], a, b0);
+                    mma_bf16_16x8x16(acc[2 * np + 1], a, b1);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int col = 128 * nh + 8 * j + 2 * t;
+                *reinterpret_cast<uint32_t *>(Ws + (16 * warp + g) * LDKW + col) =
+                    tc::pack_bf16(acc[j][0], acc[j][1]);
+                *reinterpret_cast<uint32_t *>(Ws + (16 * warp + g + 8) * LDKW + col) =
+                    tc::pack_bf16(acc[j][2], acc[j][3]);
+            }
+        }
+    }
+    __syncthreads();
+    __nv_bfloat16 *dw = wt + tile * W_ELEMS;
+#pragma unroll 4
+    for (int m = 0; m < W_ELEMS / 8 / UT_THREADS; ++m) {
+        const int idx = tid + UT_THREADS * m;
+        const int r = idx >> 5, piece = idx & 31;
+        *reinterpret_cast<uint4 *>(dw + r * DK + 8 * piece) =
+            *reinterpret_cast<const uint4 *>(Ws + r * LDKW + 8 * piece);
+    }
+}
+
+// ----------------------------------------------------- sequential kernel --
+constexpr int BLK = 8192;                       // one 64 x 64 bf16 tile (64 rows of 128 B)
+constexpr int SM_QW = 0;                        // per key block: Q (8 KiB), then W (8 KiB)
+constexpr int SM_KT = SM_QW + KB * 2 * BLK;     // K: 4 key blocks of 8 KiB
+constexpr int SM_VP = SM_KT + KB * BLK;         // 2 stages: V (8 KiB), [P; T''] (16 KiB)
+constexpr int VP_STAGE = 3 * BLK;
+constexpr int SM_SB = SM_VP + 2 * VP_STAGE;     // S^T bf16: 256 key rows x 128 B (MN-major B)
+constexpr int SM_UN = SM_SB + DK * 128;         // U' bf16 (MN-major B)
+constexpr int SM_UP = SM_UN + BLK;              // diag(exp(g_last - g) / |k|) U' bf16
+constexpr int SM_GV = SM_UP + BLK;              // gate vectors, 2 stages
+constexpr int GV_GAM = 0;                       // gamma_r (/ |q_r| when normalising)
+constexpr int GV_DCY = 64;                      // exp(g_last - g_r) (/ |k_r| when normalising)
+constexpr int GV_GL = 128;                      // gamma_last
+constexpr int GV_STRIDE = 256;
+constexpr int SM_BAR = SM_GV + 2 * GV_STRIDE * 4;
+constexpr int NBAR = 16;
+constexpr int SM_MISC = SM_BAR + NBAR * 8;      // TMEM base, abort flag
+constexpr int SMEM_BYTES = SM_MISC + 16 + 1024; // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(SM_KT % 1024 == 0 && SM_VP % 1024 == 0 && SM_SB % 1024 == 0 &&
+              SM_UN % 1024 == 0 && SM_UP % 1024 == 0 && VP_STAGE % 1024 == 0,
+              "1024-byte aligned swizzled tiles");
+
+// TMEM columns: S^T (keys 0-127 in 0-63, keys 128-255 in 64-127), X, U, Y
+constexpr uint32_t TM_ST = 0, TM_X = 128, TM_U = 192, TM_Y = 256;
+constexpr uint32_t TM_COLS = 512;
+
+enum {
+    B_QW_FULL = 0,      // TMA: [Q; W] (1 + tx)
+    B_QW_EMPTY = 1,     // chain commit after X (1)
+    B_K_FULL = 2,       // TMA: K (1 + tx)
+    B_K_EMPTY = 3,      // chain commit after the state update (1)
+    B_VP_FULL = 4,      // [2] TMA: V, [P; T''] (tx) + gate vectors (1)
+    B_VP_EMPTY = 6,     // [2] chain commit after Y (1)
+    B_U_FULL = 8,       // U-product commit (1)
+    B_U_EMPTY = 9,      // state warps that read U (4)
+    B_X_FULL = 10,      // chain commit after X (1)
+    B_U_READY = 11,     // state warps: U', decayed U' and the Y preload written (8)
+    B_ST_FULL = 12,     // chain commit after the state update (1)
+    B_S_READY = 13,     // state warps: S^T hand-off done (8)
+    B_Y_FULL = 14,      // chain commit after Y (1)
+    B_COUNT = 15
+};
+static_assert(B_COUNT <= NBAR, "barrier slots");
+
+constexpr int W_TMA = 0, W_CHAIN = 1, W_UMMA = 2;
+constexpr int W_STATE0 = 4, NSTATEW = 8;
+constexpr int NTHREADS = 32 * (W_STATE0 + NSTATEW);
+
+struct Params {
+    const float *log_alpha;
+    const float *S0;
+    __nv_bfloat16 *o;
+    float *S_T;
+    const float *rqk;      // 1/|q|, 1/|k| per chunk row from the UT kernel (normalising only)
+    Seqs sq;
+    int H, Dv;
+    unsigned flags;
+};
+
+template <bool kNorm>
+__global__ void __launch_bounds__(NTHREADS, 1)
+gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_pt, const Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx cx;
+    cx.base = base;
+    cx.bar = reinterpret_cast<uint64_t *>(base + SM_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + SM_MISC);
+    cx.abort = reinterpret_cast<volatile uint32_t *>(base + SM_MISC + 4);
+    cx.err = &g_tcw_error;
+    float *gv_all = reinterpret_cast<float *>(base + SM_GV);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int vt = blockIdx.x, h = blockIdx.y;
+    const int b = p.sq.order ? p.sq.order[blockIdx.z] : (int)blockIdx.z;
+    const int v0 = vt * DVT;
+    const int H = p.H;
+    const Span sp = tc::seq_span(p.sq, b);
+    const int T = sp.len, NT = (T + C - 1) / C;
+    const size_t head = (size_t)b * H + h;
+    if (NT == 0) {
+        if (p.S_T)
+            for (int e = threadIdx.x; e < DVT * DK; e += NTHREADS) {
+                const size_t idx = head * p.Dv * DK + (size_t)v0 * DK + e;
+                p.S_T[idx] = p.S0 ? p.S0[idx] : 0.f;
+            }
+        return;
+    }
+
+    if (tid == 0) {
+        int counts[B_COUNT];
+        for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
+        counts[B_U_EMPTY] = NSTATEW / 2;
+        counts[B_U_READY] = counts[B_S_READY] = NSTATEW;
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bar + i, counts[i]);
+        *cx.abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == W_CHAIN) {
+        tmem_alloc(tmem_slot, TM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == W_TMA && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_w);
+        prefetch_tensormap(&tm_pt);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == W_TMA) {
+        // ------------------------------------------------ TMA loads, gate vectors
+        float nla[2], nrq[2] = {1.f, 1.f}, nrk[2] = {1.f, 1.f};  // next chunk's gate values
+        const auto fetch = [&](int cc) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = lane + 32 * hh;
+                const bool in = cc * C + r < T;
+                const size_t gi = (size_t)(sp.off + cc * C + r) * H + h;
+                nla[hh] = in ? p.log_alpha[gi] : 0.f;
+                if (kNorm) {
+                    const size_t tl = (size_t)(sp.chunk0 + cc) * H + h;
+                    nrq[hh] = p.rqk[tl * 2 * C + r];
+                    nrk[hh] = p.rqk[tl * 2 * C + C + r];
+                }
+            }
+        };
+        // the tiles (and the norms) come from the UT kernel launched just before
+        // this one (programmatic dependent launch): wait for its completion
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        fetch(0);
+        int n_vp = 0, n_qw = 0, n_k = 0;  // stages issued
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1, t0 = c * C;
+            const int tile = (sp.chunk0 + c) * H + h;
+            float la[2];
+            const float rq2[2] = {nrq[0], nrq[1]}, rk2[2] = {nrk[0], nrk[1]};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const bool in = t0 + lane + 32 * hh < T;
+                const float x = nla[hh];
+                la[hh] = in ? ((p.flags & kFlagGateLogits) ? neg_softplus(x) : x) : 0.f;
+            }
+            if (c + 1 < NT) fetch(c + 1);
+            // V and [P; T''] of chunk c once the Y product of chunk c - 2 is done
+            if (c >= 2 && !tc::warp_wait(cx, B_VP_EMPTY + s, ((c - 2) >> 1) & 1)) break;
+            uint8_t *vp = base + SM_VP + s * VP_STAGE;
+            if (lane == 0) {
+                mbar_expect_tx(cx.bar + B_VP_FULL + s, VP_STAGE);
+                tma_load_4d(vp, &tm_v, cx.bar + B_VP_FULL + s, v0, h, sp.off + t0, 0);
+                tma_load_3d(vp + BLK, &tm_pt, cx.bar + B_VP_FULL + s, 0, 0, tile);
+            }
+            n_vp = c + 1;
+            // gate vectors of chunk c (running sums in log2 units; rows past the
+            // end carry log alpha = 0)
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y0 = __shfl_up_sync(0xffffffffu, la[0], off);
+                const float y1 = __shfl_up_sync(0xffffffffu, la[1], off);
+                if (lane >= off) {
+                    la[0] += y0;
+                    la[1] += y1;
+                }
+            }
+            la[1] += __shfl_sync(0xffffffffu, la[0], 31);
+            const float g0 = la[0] * LOG2E, g1 = la[1] * LOG2E;
+            const float glast = __shfl_sync(0xffffffffu, g1, 31);
+            float *gv = gv_all + s * GV_STRIDE;
+            gv[GV_GAM + lane] = tc::ex2(g0) * rq2[0];
+            gv[GV_GAM + 32 + lane] = tc::ex2(g1) * rq2[1];
+            gv[GV_DCY + lane] = tc::ex2(glast - g0) * rk2[0];
+            gv[GV_DCY + 32 + lane] = tc::ex2(glast - g1) * rk2[1];
+            if (lane == 0) gv[GV_GL] = tc::ex2(glast);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(cx.bar + B_VP_FULL + s);
+            // [Q; W] of chunk c once the X product of chunk c - 1 is done
+            if (c >= 1 && !tc::warp_wait(cx, B_QW_EMPTY, (c - 1) & 1)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(cx.bar + B_QW_FULL, 2 * KB * BLK);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(base + SM_QW + kb * 2 * BLK, &tm_q, cx.bar + B_QW_FULL, kb * 64, h,
+                                sp.off + t0, 0);
+                    tma_load_3d(base + SM_QW + kb * 2 * BLK + BLK, &tm_w, cx.bar + B_QW_FULL,
+                                kb * 64, 0, tile);
+                }
+            }
+            n_qw = c + 1;
+            // K of chunk c once the state update of chunk c - 1 is done
+            if (c >= 1 && !tc::warp_wait(cx, B_K_EMPTY, (c - 1) & 1)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(cx.bar + B_K_FULL, KB * BLK);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_4d(base + SM_KT + kb * BLK, &tm_k, cx.bar + B_K_FULL, kb * 64, h,
+                                sp.off + t0, 0);
+                // a later chunk's tiles start streaming from DRAM into L2 now
+                const int cq = c + 2;
+                if (cq < NT) {
+                    const int tq = (sp.chunk0 + cq) * H + h;
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_prefetch_l2_4d(&tm_q, kb * 64, h, sp.off + cq * C, 0);
+                        tma_prefetch_l2_4d(&tm_k, kb * 64, h, sp.off + cq * C, 0);
+                        tma_prefetch_l2_3d(&tm_w, kb * 64, 0, tq);
+                    }
+                    tma_prefetch_l2_4d(&tm_v, v0, h, sp.off + cq * C, 0);
+                    tma_prefetch_l2_3d(&tm_pt, 0, 0, tq);
+                }
+            }
+            n_k = c + 1;
+        }
+        // never leave with copies in flight: wait (bounded) for the last phases
+        if (lane == 0) {
+            const auto drain = [&](uint64_t *bar, uint32_t parity) {
+                const uint64_t t0 = tc::now_ns();
+                while (!mbar_try_wait(bar, parity) && tc::now_ns() - t0 < tc::kTimeoutNs) {
+                }
+            };
+            if (n_qw > 0) drain(cx.bar + B_QW_FULL, (n_qw - 1) & 1);
+            if (n_k > 0) drain(cx.bar + B_K_FULL, (n_k - 1) & 1);
+            for (int c = n_vp - 2 < 0 ? 0 : n_vp - 2; c < n_vp; ++c)
+                drain(cx.bar + B_VP_FULL + (c & 1), (c >> 1) & 1);
+        }
+    } else if (warp == W_UMMA) {
+        // ---------------------------------------------- MMA: U = [P; T''] V
+        const uint32_t idesc_u = idesc_bf16(128, DVT, false, true);
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            const uint32_t vp = smem_u32(base + SM_VP + s * VP_STAGE);
+            if (!tc::warp_wait(cx, B_VP_FULL + s, (c >> 1) & 1)) break;
+            if (c >= 1 && !tc::warp_wait(cx, B_U_EMPTY, (c - 1) & 1)) break;
+            tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + TM_U, desc_sw128(vp + BLK + kk * 32, 16, 1024),
+                             desc_sw128(vp + kk * 2048, 16, 1024), idesc_u, kk > 0);
+                mma_commit(cx.bar + B_U_FULL);
+            }
+            __syncwarp();
+        }
+    } else if (warp == W_CHAIN) {
+        // ---------------------------------------------- MMA: sequential chain
+        const uint32_t idesc_x = idesc_bf16(128, DVT, false, true);
+        const uint32_t idesc_s = idesc_bf16(128, DVT, true, true);
+        const uint32_t qw = smem_u32(base + SM_QW), kt = smem_u32(base + SM_KT),
+                       sb = smem_u32(base + SM_SB), un = smem_u32(base + SM_UN),
+                       up = smem_u32(base + SM_UP);
+        for (int c = 0; c < NT; ++c) {
+            const int s = c & 1;
+            const uint32_t vp = smem_u32(base + SM_VP + s * VP_STAGE);
+            if (!tc::warp_wait(cx, B_QW_FULL, c & 1)) break;
+            if (!tc::warp_wait(cx, B_S_READY, c & 1)) break;
+            tc_fence_after();
+            // X = [Q; W] S^T: A K-major (per key block, Q rows then W rows), B = S^T MN-major
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    mma_bf16(tmem + TM_X, desc_sw128(qw + (kk >> 2) * 2 * BLK + (kk & 3) * 32, 16, 1024),
+                             desc_sw128(sb + kk * 2048, 16, 1024), idesc_x, kk > 0);
+                mma_commit(cx.bar + B_X_FULL);
+                mma_commit(cx.bar + B_QW_EMPTY);
+            }
+            __syncwarp();
+            if (!tc::warp_wait(cx, B_U_READY, c & 1)) break;
+            if (!tc::warp_wait(cx, B_K_FULL, c & 1)) break;
+            if (!tc::warp_wait(cx, B_VP_FULL + s, (c >> 1) & 1)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                // S^T_h += K_h^T (decayed U') for the key halves: A = K^T (MN-major,
+                // two 64-key blocks 8 KiB apart), B = decayed U' (MN-major)
+#pragma unroll
+                for (int hk = 0; hk < 2; ++hk)
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tmem + TM_ST + 64 * hk,
+                                 desc_sw128(kt + hk * 2 * BLK + kk * 2048, BLK, 1024),
+                                 desc_sw128(up + kk * 2048, 16, 1024), idesc_s, 1u);
+                mma_commit(cx.bar + B_ST_FULL);
+                mma_commit(cx.bar + B_K_EMPTY);
+                // Y += [P; T''] U'  (Y holds gamma Q S^T; rows 64-127 unused)
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + TM_Y, desc_sw128(vp + BLK + kk * 32, 16, 1024),
+                             desc_sw128(un + kk * 2048, 16, 1024), idesc_x, 1u);
+                mma_commit(cx.bar + B_Y_FULL);
+                mma_commit(cx.bar + B_VP_EMPTY + s);
+            }
+            __syncwarp();
+        }
+    } else if (warp >= W_STATE0) {
+        // ------------------------------------------------------------ STATE
+        // warp w reads TMEM lanes 32 (w % 4) .. + 31; hf selects the key half of
+        // S^T (hand-off) or the 32-column half of X / U / Y (epilogues)
+        const int q = warp & 3, hf = (warp - W_STATE0) >> 2;
+        const int lrow = 32 * q + lane;
+        const int key = 128 * hf + lrow;  // this thread's row of S^T in the hand-off
+        const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+        const uint32_t st_col = TM_ST + 64 * hf;
+        uint8_t *sbuf = base + SM_SB;
+        // initial state: S^T row `key` = S0[v0 .. v0 + 63][key]; TMEM copy pre-scaled by gamma_last
+        {
+            const bool have = tc::warp_wait(cx, B_VP_FULL + 0, 0);
+            const float gl = gv_all[GV_GL];
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+                float sv[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + 16 * pc + j) * DK + key] : 0.f;
+                tc::store16_bf16(sbuf, key, pc, sv);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sv[j] *= gl;
+                if (have) tmem_st16(lane_addr + st_col + 16 * pc, sv);
+            }
+            fence_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
+            tc::warp_arrive(cx, B_S_READY);
+        }
+        for (int c = 0; c < NT; ++c) {
+            if (__any_sync(0xffffffffu, *cx.abort != 0u)) break;
+            const int s = c & 1, t0 = c * C;
+            const float *gv = gv_all + s * GV_STRIDE;
+            if (!tc::warp_wait(cx, B_X_FULL, c & 1)) break;
+            tc_fence_after();
+            if (q >= 2) {
+                // U' = U - W S^T for chunk row r -> U' and its decayed copy (bf16)
+                const int r = lrow - 64;
+                if (!tc::warp_wait(cx, B_U_FULL, c & 1)) break;
+                tc_fence_after();
+                const float dc = gv[GV_DCY + r];
+                float x0[16], x1[16], u0[16], u1[16];
+                tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
+                tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
+                tmem_ld16(lane_addr + TM_U + 32 * hf, u0);
+                tmem_ld16(lane_addr + TM_U + 32 * hf + 16, u1);
+                tmem_wait_ld();
+                tc_fence_before();
+                tc::warp_arrive(cx, B_U_EMPTY);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    u0[j] -= x0[j];
+                    u1[j] -= x1[j];
+                }
+                tc::store16_bf16(base + SM_UN, r, 2 * hf, u0);
+                tc::store16_bf16(base + SM_UN, r, 2 * hf + 1, u1);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    u0[j] *= dc;
+                    u1[j] *= dc;
+                }
+                tc::store16_bf16(base + SM_UP, r, 2 * hf, u0);
+                tc::store16_bf16(base + SM_UP, r, 2 * hf + 1, u1);
+                fence_async_smem();
+                tc_fence_before();
+                tc::warp_arrive(cx, B_U_READY);
+            } else {
+                // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y
+                const float gr = gv[GV_GAM + lrow];
+                float x0[16], x1[16];
+                tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
+                tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    x0[j] *= gr;
+                    x1[j] *= gr;
+                }
+                tmem_st16(lane_addr + TM_Y + 32 * hf, x0);
+                tmem_st16(lane_addr + TM_Y + 32 * hf + 16, x1);
+                tmem_wait_st();
+                tc_fence_before();
+                tc::warp_arrive(cx, B_U_READY);
+            }
+            // state hand-off: S^T (updated) -> bf16 copy; TMEM pre-scaled by the
+            // next chunk's gamma_last
+            if (!tc::warp_wait(cx, B_ST_FULL, c & 1)) break;
+            tc_fence_after();
+            {
+                const bool last = c + 1 >= NT;
+                bool have = false;
+                float gl = 1.f;
+                if (!last) {
+                    have = tc::warp_wait(cx, B_VP_FULL + (s ^ 1), ((c + 1) >> 1) & 1);
+                    gl = gv_all[(s ^ 1) * GV_STRIDE + GV_GL];
+                }
+                float sv[4][16];
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc) tmem_ld16(lane_addr + st_col + 16 * pc, sv[pc]);
+                tmem_wait_ld();
+                if (!last) {
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc) tc::store16_bf16(sbuf, key, pc, sv[pc]);
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sv[pc][j] *= gl;
+                    if (have)
+#pragma unroll
+                        for (int pc = 0; pc < 4; ++pc) tmem_st16(lane_addr + st_col + 16 * pc, sv[pc]);
+                    fence_async_smem();
+                    tmem_wait_st();
+                } else if (p.S_T) {
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            p.S_T[(head * p.Dv + v0 + 16 * pc + j) * DK + key] = sv[pc][j];
+                }
+                tc_fence_before();
+                tc::warp_arrive(cx, B_S_READY);
+                if (!last && !have) break;
+            }
+            // chunk output rows (TMEM lanes 0-63)
+            if (q < 2) {
+                if (!tc::warp_wait(cx, B_Y_FULL, c & 1)) break;
+                tc_fence_after();
+                float y0[16], y1[16];
+                tmem_ld16(lane_addr + TM_Y + 32 * hf, y0);
+                tmem_ld16(lane_addr + TM_Y + 32 * hf + 16, y1);
+                tmem_wait_ld();
+                if (t0 + lrow < T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        p.o + ((size_t)(sp.off + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
+#pragma unroll
+                    for (int kq = 0; kq < 2; ++kq) {
+                        dst[kq] = make_uint4(tc::pack_bf16(y0[8 * kq + 0], y0[8 * kq + 1]),
+                                             tc::pack_bf16(y0[8 * kq + 2], y0[8 * kq + 3]),
+                                             tc::pack_bf16(y0[8 * kq + 4], y0[8 * kq + 5]),
+                                             tc::pack_bf16(y0[8 * kq + 6], y0[8 * kq + 7]));
+                        dst[2 + kq] = make_uint4(tc::pack_bf16(y1[8 * kq + 0], y1[8 * kq + 1]),
+                                                 tc::pack_bf16(y1[8 * kq + 2], y1[8 * kq + 3]),
+                                                 tc::pack_bf16(y1[8 * kq + 4], y1[8 * kq + 5]),
+                                                 tc::pack_bf16(y1[8 * kq + 6], y1[8 * kq + 7]));
+                    }
+                }
+                tc_fence_before();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == W_CHAIN) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// W tiles, [n_tiles, 64, 256] bf16: box of 64 keys x 64 rows of one tile, 128B swizzle.
+bool make_map_w(CUtensorMap *m, const void *ptr, long long n_tiles) {
+    auto enc = tc::encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)C, (cuuint64_t)n_tiles};
+    cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)W_ELEMS * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tcw
+
+// Workspace: [chunk offsets and launch order, variable lengths only][[P; T'']
+// tiles][W tiles][1/|q|, 1/|k| per chunk row, normalising only].
+size_t tcw_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
+                                unsigned flags) {
+    const size_t tiles = (size_t)total_chunks * H;
+    const size_t norm = (flags & kFlagL2Norm) ? tiles * 2 * tc::C * sizeof(float) : 0;
+    return tc_offsets_bytes(n_seq, varlen) +
+           tiles * (tcw::PT_ELEMS + tcw::W_ELEMS) * sizeof(__nv_bfloat16) + norm;
+}
+
+cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
+                                  const int *cu_seqlens, long long total_chunks, int H, int Dv,
+                                  unsigned flags, void *workspace, cudaStream_t st) {
+    const bool varlen = cu_seqlens != nullptr;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
+    const size_t tiles = (size_t)total_chunks * H;
+    auto *pt = reinterpret_cast<__nv_bfloat16 *>(ws + tc_offsets_bytes(n_seq, varlen));
+    __nv_bfloat16 *wt = pt + tiles * tcw::PT_ELEMS;
+    float *rqk = (flags & kFlagL2Norm) ? reinterpret_cast<float *>(wt + tiles * tcw::W_ELEMS)
+                                       : nullptr;
+    const long long n_maps = total_chunks > 0 ? (long long)tiles : 1;
+    CUtensorMap mq, mk, mv, mw, mp;
+    if (!tc::make_map(&mq, q, 1, (int)total_T, H, tcw::DK) ||
+        !tc::make_map(&mk, k, 1, (int)total_T, H, tcw::DK) ||
+        !tc::make_map(&mv, v, 1, (int)total_T, H, Dv) || !tcw::make_map_w(&mw, wt, n_maps) ||
+        !tc::make_map_tt(&mp, pt, n_maps))
+        return cudaErrorInvalidValue;
+    if (varlen) {
+        const cudaError_t e0 = launch_seq_schedule(cu_seqlens, n_seq, cu_chunks,
+                                                   cu_chunks + n_seq + 1, st);
+        if (e0 != cudaSuccess) return e0;
+    }
+    const tc::Seqs sq{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
+                      n_seq};
+    tcw::Params p;
+    p.log_alpha = log_alpha;
+    p.S0 = S0;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.S_T = S_T;
+    p.rqk = rqk;
+    p.sq = sq;
+    p.H = H;
+    p.Dv = Dv;
+    p.flags = flags;
+    const bool norm = (flags & kFlagL2Norm) != 0;
+    auto *ut = norm ? tcw::gdn_utw_kernel<true> : tcw::gdn_utw_kernel<false>;
+    auto *seq = norm ? tcw::gdn_chunk_tcw_kernel<true> : tcw::gdn_chunk_tcw_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tcw::UT_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, tcw::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (total_chunks > 0)
+        ut<<<dim3((unsigned)total_chunks, H, 1), tcw::UT_THREADS, tcw::UT_SMEM, st>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+            log_alpha, beta, pt, wt, rqk, sq, H, flags);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Dv / tcw::DVT, H, n_seq);
+    cfg.blockDim = dim3(tcw::NTHREADS);
+    cfg.dynamicSmemBytes = tcw::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mw, mp, p);
+    if (e != cudaSuccess) return e;
+    return cudaPeekAtLastError();
+}
+
+cudaError_t read_and_clear_device_error_wide(unsigned int *flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_tcw_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_tcw_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace gdn

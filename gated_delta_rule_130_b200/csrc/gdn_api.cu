@@ -81,7 +81,7 @@ size_t gdn_chunk_fwd_workspace_size_ex(int B, int T, int H, int Dk, int Dv, int 
                                        gdn_dtype_t dtype, unsigned flags) {
     const int path = gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype);
     if (flags & ~kKnownFlags) return 0;
-    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H, flags);
+    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H, flags, Dk);
     if (path == GDN_PATH_SIMT) {
         const size_t base = gdn::simt_workspace_bytes(B, T, H, chunk);
         return flags ? align256(base) + gdn::prologue_bytes(B, T, H, Dk, dtype == GDN_BF16, flags)
@@ -178,7 +178,7 @@ size_t gdn_chunk_fwd_varlen_workspace_size(const int *cu_seqlens_host, int N, in
     if (N == 0 || H == 0 || off.total == 0) return 0;
     const bool bf16 = dtype == GDN_BF16;
     if (gdn::tc_supported(N, off.max_len, H, Dk, Dv, chunk, bf16))
-        return gdn::tc_workspace_bytes_seqs(N, off.chunks64, H, true, flags);
+        return gdn::tc_workspace_bytes_seqs(N, off.chunks64, H, true, flags, Dk);
     // CUDA-core path: one sequence at a time (scratch for the longest), prologue once
     const size_t base = gdn::simt_workspace_bytes(1, off.max_len, H, chunk);
     return flags ? align256(base) +
@@ -436,9 +436,11 @@ gdn_status_t gdn_debug_withhold_first_arrival(int enable) {
 
 gdn_status_t gdn_check_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
-    unsigned int flag = 0;
-    if (gdn::read_and_clear_device_error(&flag) != cudaSuccess) return GDN_ERR_CUDA;
-    return flag ? GDN_ERR_CUDA : GDN_OK;
+    unsigned int flag = 0, flag_wide = 0;
+    if (gdn::read_and_clear_device_error(&flag) != cudaSuccess ||
+        gdn::read_and_clear_device_error_wide(&flag_wide) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return (flag | flag_wide) ? GDN_ERR_CUDA : GDN_OK;
 }
 
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,

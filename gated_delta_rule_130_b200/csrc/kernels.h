@@ -67,11 +67,15 @@ cudaError_t launch_decode_cw(const void *q, const void *k, const void *v, const 
                              const float *bg, const float *wg, float *S, void *o, int B, int H,
                              int Dk, int Dv, bool bf16, cudaStream_t st);
 
-// tcgen05 chunkwise forward (bf16, Dk = 128, chunk 64): chunk_tc.cu.  The
-// workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of every head.
-// With the L2-normalisation flag the workspace also holds 1/|k| per token.
+// tcgen05 chunkwise forward (bf16, chunk 64, Dv a multiple of 64; Dk = 128 in
+// chunk_tc.cu, Dk = 256 in chunk_tc_wide.cu, chosen by Dk inside these calls).
+// Dk = 128: the workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of
+// every head (and 1/|k| per token with the L2-normalisation flag).  Dk = 256:
+// one bf16 [P; T''] tile (128 x 64) and one bf16 W tile (64 x 256) per chunk of
+// every head (and 1/|q|, 1/|k| per token with the flag).
+constexpr int tcw_dk = 256;
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
-size_t tc_workspace_bytes(int B, int T, int H, unsigned flags);
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk = 128);
 // S_hist (optional): the state entering every chunk, [B*H][NT][Dv][Dk] float32.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
@@ -82,7 +86,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 // total_chunks = sum of ceil(length / 64).  The workspace then starts with the
 // per-sequence chunk offsets (computed on the device).
 size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                               unsigned flags);
+                               unsigned flags, int Dk = 128);
 cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
@@ -90,9 +94,25 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  int Dv, unsigned flags, void *workspace, cudaStream_t st,
                                  float *S_hist = nullptr);
 
+// Shared by both tcgen05 files (chunk_tc.cu): bytes of the per-sequence chunk
+// offsets and launch order at the start of a packed batch's workspace, and the
+// one-block kernel that computes them on the device.
+size_t tc_offsets_bytes(int n_seq, bool varlen);
+cudaError_t launch_seq_schedule(const int *cu_seqlens, int n_seq, int *cu_chunks, int *order,
+                                cudaStream_t st);
+// The Dk = 256 path (chunk_tc_wide.cu); reached through the tc_* calls above.
+size_t tcw_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
+                                unsigned flags);
+cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
+                                  const int *cu_seqlens, long long total_chunks, int H, int Dv,
+                                  unsigned flags, void *workspace, cudaStream_t st);
+
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).
 cudaError_t read_and_clear_device_error(unsigned int *flag);
+cudaError_t read_and_clear_device_error_wide(unsigned int *flag);  // the Dk = 256 kernel's flag
 // Test hook: the sequential tcgen05 kernel withholds its first stage's arrival
 // (every CTA then times out, about two seconds, and sets that flag).
 cudaError_t set_withhold_first_arrival(bool on);

@@ -236,6 +236,16 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *row_pt
                  : "r"(smem_u32(row_ptr)));
 }
 
+// The same four matrices, each transposed on delivery: lane l gives the address
+// of row l % 8 of matrix l / 8 (a row of the stored matrix) and receives, in
+// r[m], elements (2 (l % 4), l / 4) and (2 (l % 4) + 1, l / 4) of matrix m --
+// the B fragment of mma.sync from a matrix stored with k along its rows.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void *row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_ptr)));
+}
+
 // D (16 x 8, f32) += A (16 x 16, bf16, row-major) B (16 x 8, bf16, column-major).
 // Lane (g = lane / 4, t = lane % 4) holds a = {A[g][2t..], A[g+8][2t..],
 // A[g][2t+8..], A[g+8][2t+8..]} and b = {B[2t..][g], B[2t+8..][g]} as bf16

@@ -5,6 +5,8 @@
 // sequences.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -41,7 +43,7 @@ struct Ctx {
 };
 
 // Bounded wait; false (and the CTA-wide abort flag set) on timeout or abort.
-__device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
+static __device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
     uint64_t *b = cx.bar + idx;
 #ifdef GDN_WAIT_TEST_SLEEP_NS
     {
@@ -81,7 +83,7 @@ __device__ __noinline__ bool wait_bar(const Ctx &cx, int idx, uint32_t parity) {
 
 // Slow path of warp_wait: lane 0 polls (so waiting warps do not compete with
 // working warps for the shared-memory pipe) and the result is broadcast.
-__device__ __noinline__ bool warp_wait_slow(const Ctx &cx, int idx, uint32_t parity) {
+static __device__ __noinline__ bool warp_wait_slow(const Ctx &cx, int idx, uint32_t parity) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = wait_bar(cx, idx, parity);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -262,6 +264,13 @@ __device__ __forceinline__ int seq_of_chunk(const Seqs &q, int g) {
     }
     return lo;
 }
+
+// Host side, defined in chunk_tc.cu: the driver's tensor-map encoder, and the
+// maps of a [B, T, H, D] bf16 tensor (box 64 channels x 1 head x 64 tokens x 1,
+// 128-byte swizzle) and of a [n_tiles, 128, 64] bf16 tile array (box one tile).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int D);
+bool make_map_tt(CUtensorMap *m, const void *ptr, long long n_tiles);
 
 }  // namespace tc
 }  // namespace gdn

@@ -64,10 +64,12 @@ typedef enum {
     GDN_PATH_NONE = 0,     /* empty problem: nothing (or only a state copy) runs */
     GDN_PATH_SIMT = 1,     /* two CUDA-core kernels: chunk preparation, then the
                               sequential state/output pass; needs a workspace */
-    GDN_PATH_TCGEN05 = 2   /* bf16, Dk = 128, chunk 64, Dv a multiple of 64: the
-                              per-chunk UT transform for all chunks in parallel
-                              (into the workspace), then one tcgen05 tensor-core
-                              kernel for the sequential pass; needs a workspace */
+    GDN_PATH_TCGEN05 = 2   /* bf16, Dk = 128 or 256, chunk 64, Dv a multiple of
+                              64: the per-chunk UT transform for all chunks in
+                              parallel (into the workspace; at Dk = 256 also the
+                              gated Q K^T and W = T diag(beta gamma) K), then one
+                              tcgen05 tensor-core kernel for the sequential pass;
+                              needs a workspace */
 } gdn_path_t;
 
 /* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0

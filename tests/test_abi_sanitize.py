@@ -45,13 +45,13 @@ cudaError_t launch_chunk_simt(const void *, const void *, const void *, const fl
                               const float *, void *, float *, int, int, int, int, int, int, bool,
                               void *, cudaStream_t) { return ok(); }
 bool tc_supported(int, int, int, int, int, int, bool) { return false; }
-size_t tc_workspace_bytes(int B, int T, int H, unsigned) {
-    return (size_t)B * H * (((size_t)T + 63) / 64) * 16384; }
+size_t tc_workspace_bytes(int B, int T, int H, unsigned, int Dk) {
+    return (size_t)B * H * (((size_t)T + 63) / 64) * (Dk == 256 ? 49152 : 16384); }
 cudaError_t launch_chunk_tc(const void *, const void *, const void *, const float *, const float *,
                             const float *, void *, float *, int, int, int, int, int, unsigned,
                             void *, cudaStream_t, float *) { return ok(); }
-size_t tc_workspace_bytes_seqs(int n, long long chunks, int H, bool, unsigned) {
-    return ((size_t)n + 1) * 8 + (size_t)chunks * H * 16384; }
+size_t tc_workspace_bytes_seqs(int n, long long chunks, int H, bool, unsigned, int Dk) {
+    return ((size_t)n + 1) * 8 + (size_t)chunks * H * (Dk == 256 ? 49152 : 16384); }
 cudaError_t launch_chunk_tc_seqs(const void *, const void *, const void *, const float *,
                                  const float *, const float *, void *, float *, int, int, long long,
                                  const int *, long long, int, int, int, unsigned, void *,
@@ -76,6 +76,8 @@ cudaError_t launch_decode_cw(const void *, const void *, const void *, const flo
                              const float *, float *, void *, int, int, int, int, bool,
                              cudaStream_t) { return ok(); }
 cudaError_t read_and_clear_device_error(unsigned int *flag) { *flag = 0; return ok(); }
+cudaError_t read_and_clear_device_error_wide(unsigned int *flag) { *flag = 0; return ok(); }
+cudaError_t set_withhold_first_arrival(bool) { return ok(); }
 }  // namespace gdn
 """
 
