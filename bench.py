@@ -281,7 +281,7 @@ def run_ours(args):
     from gated_delta_rule_130_b200 import binding as G
 
     pk, pk_kind = peaks()
-    w = I.workload(I.HEADLINE)
+    w = parse_workload(args.workload) if args.chunk_only else I.workload(I.HEADLINE)
     inp_cpu = I.chunk_inputs(w, seed=w.seed + rank)
     inp = {n: (t.to(device) if t is not None else None) for n, t in inp_cpu.items()}
     path = G.chunk_fwd_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
@@ -632,6 +632,17 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def parse_workload(spec: str):
+    """'name' or 'name:B=2,T=1024' -- a workload of the table with its sizes overridden
+    (for profiling a smaller case of the same kernel)."""
+    name, _, rest = spec.partition(":")
+    over = {}
+    for item in filter(None, rest.split(",")):
+        key, _, val = item.partition("=")
+        over[key.strip()] = int(val)
+    return I.workload(name, **over)
+
+
 def run_decode_only(args):
     """--decode-only: the decode step alone (batch 256, H 16, d 128, state in place),
     for counter captures of its kernel; prints one short JSON line."""
@@ -671,6 +682,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-only", action="store_true",
                     help="time the chunkwise forward only (no decode, end-to-end or CPU legs)")
+    ap.add_argument("--workload", default=I.HEADLINE,
+                    help="with --chunk-only: the workload to time, 'name' or 'name:B=2,T=1024'")
     ap.add_argument("--decode-only", action="store_true",
                     help="time the decode step alone (one GPU, for counter captures)")
     args = ap.parse_args()

@@ -15,8 +15,9 @@
 //
 // Two kernels on one stream:
 //  1. gdn_ut_kernel, one CTA per (batch, head, chunk), all chunks in parallel:
-//     the Gram matrix (bf16 mma.sync, float32 accumulation), its gating, the
-//     UT solve in float32 and the bf16 tile [T'; T''] = [T diag(beta gamma);
+//     the Gram matrix (one tcgen05 product of the TMA-loaded K chunk, float32
+//     in tensor memory), its gating, the UT solve in float32 and the bf16 tile
+//     [T'; T''] = [T diag(beta gamma);
 //     T diag(beta)] (128 x 64) into a workspace.  None of it depends on S, and
 //     the solve is a chain of small dependent steps: run wide, it is hidden by
 //     parallelism instead of sitting in front of the sequential pass.
@@ -287,27 +288,33 @@ seq_schedule(const int *__restrict__ cu, int n, int *__restrict__ cu_chunks,
 // ------------------------------------------------------------- UT kernel --
 // One CTA of 4 warps per (global chunk g, head h): [T'; T''] of that chunk,
 // bf16, 128 rows x 64 columns, row-major, at tt + (g H + h) 128 x 64.
-// Six CTAs fit on an SM (shared memory and registers), so six chunks are in
-// flight per SM and the solve's dependent steps overlap across chunks.
+// The chunk's K rows arrive by TMA (128-byte swizzle) and the Gram matrix K K^T
+// is one tcgen05 product (M = N = 64, K = 128) into tensor memory, from where
+// each warp reads 16 rows (an M = 64 product puts row m in TMEM lane
+// 32 (m / 16) + m % 16).  Five CTAs fit on an SM (39 KiB of shared memory, 64
+// TMEM columns each), so five chunks are in flight per SM and the solve's
+// dependent steps overlap across chunks.
 constexpr int UT_THREADS = 128;
-constexpr int LDK = DK + 8;                        // bf16 row stride of the staged K chunk
-constexpr int UT_SM_KT = 0;                        // K chunk (64 x LDK bf16), then T (64 x LDA f32)
+constexpr int UT_SM_KT = 0;                        // K chunk (KB blocks of 64 x 128 B), then T
 constexpr int UT_SM_AF = C * LDA * 4;              // A (64 x LDA f32); N_IJ overwrite A_IJ
 constexpr int UT_SM_GT = UT_SM_AF + C * LDA * 4;   // g log2(e), beta, beta gamma |k|^-1, |k|^-1
-// shared memory of the plain / the normalising instantiation (the latter keeps 1/|k|)
-constexpr int ut_smem_bytes(bool norm) { return UT_SM_GT + (norm ? 4 : 3) * C * 4; }
+constexpr int UT_SM_BAR = UT_SM_GT + 4 * C * 4;    // 2 mbarriers, TMEM base, abort flag
+constexpr int UT_SMEM = UT_SM_BAR + 32 + 1024;     // + alignment slack (1024-byte tiles)
+constexpr uint32_t UT_TM_COLS = 64;
 constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
-static_assert(C * LDK * 2 <= UT_SM_AF, "K chunk fits in the T buffer");
-static_assert(UT_SM_AF % 16 == 0 && UT_SM_GT % 16 == 0, "16-byte aligned UT buffers");
+static_assert(KB * 8192 <= UT_SM_AF, "K chunk fits in the T buffer");
+static_assert(UT_SM_AF % 1024 == 0 && UT_SM_GT % 16 == 0 && UT_SM_BAR % 8 == 0,
+              "aligned UT buffers");
 
 // kNorm: q and k are L2-normalised inside the kernels (1/|k| folded into the
 // Gram rows and T', and written to rk_out); without it the kernel is unchanged.
 template <bool kNorm>
-__global__ void __launch_bounds__(UT_THREADS, 6)
-gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
+__global__ void __launch_bounds__(UT_THREADS, 5)
+gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ log_alpha,
               const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt,
               float *__restrict__ rk_out, const Seqs sq, int H, unsigned flags) {
-    extern __shared__ __align__(16) uint8_t ut_smem[];
+    extern __shared__ __align__(1024) uint8_t ut_raw[];
+    uint8_t *ut_smem = ut_raw + ((1024u - (smem_u32(ut_raw) & 1023u)) & 1023u);
     // the sequential kernel that follows on the stream may be scheduled now (it
     // waits for this grid's completion before it reads the tiles)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -317,22 +324,41 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
     const Span sp = seq_span(sq, b);
     const int c = gch - sp.chunk0, T = sp.len;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
     const int t0 = c * C;
-    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ut_smem + UT_SM_KT);
     float *TF = reinterpret_cast<float *>(ut_smem + UT_SM_KT);
     float *AF = reinterpret_cast<float *>(ut_smem + UT_SM_AF);
     float *g2s = reinterpret_cast<float *>(ut_smem + UT_SM_GT);
     float *bes = g2s + C, *bgs = g2s + 2 * C, *rks = g2s + 3 * C;
+    Ctx cx;
+    cx.base = ut_smem;
+    cx.bar = reinterpret_cast<uint64_t *>(ut_smem + UT_SM_BAR);  // [0] K landed, [1] Gram done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ut_smem + UT_SM_BAR + 16);
+    cx.abort = reinterpret_cast<volatile uint32_t *>(ut_smem + UT_SM_BAR + 20);
+    cx.err = &g_tc_error;
 
-    // K rows of the chunk (zero-filled past the end of the sequence): 16 x 16 B per row
+    if (tid == 0) {
+        mbar_init(cx.bar + 0, 1);
+        mbar_init(cx.bar + 1, 1);
+        *cx.abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, UT_TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // K rows of the chunk.  Rows past the end of the sequence (the next
+    // sequence's, or TMA's zero fill past the last token) get beta = 0 and
+    // log alpha = 0 below, which zeroes their rows of A and their columns of
+    // T' and T'' (T restricted to them is the identity).
+    if (tid == 0) {
+        mbar_arrive_expect_tx(cx.bar + 0, KB * 8192);
 #pragma unroll
-    for (int m = 0; m < C * (DK / 8) / UT_THREADS; ++m) {
-        const int idx = tid + UT_THREADS * m;
-        const int r = idx / (DK / 8), piece = idx % (DK / 8);
-        const bool in = t0 + r < T;
-        const __nv_bfloat16 *src = k + ((size_t)(sp.off + (in ? t0 + r : 0)) * H + h) * DK + 8 * piece;
-        cp_async16(Ks + r * LDK + 8 * piece, src, in ? 16u : 0u);
+        for (int kb = 0; kb < KB; ++kb)
+            tma_load_4d(ut_smem + UT_SM_KT + kb * 8192, &tm_k, cx.bar + 0, kb * 64, h, sp.off + t0, 0);
     }
     if (warp == 0) {
         // running sum of log alpha over rows lane and lane + 32, in log2 units
@@ -364,80 +390,81 @@ gdn_ut_kernel(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log
             bes[lane + 32 * hh] = be[hh];
             bgs[lane + 32 * hh] = be[hh] * ex2(g2);
         }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    // 1/|k_r| per row (two threads a row), folded into the Gram rows and the
-    // columns of T'; kept in the workspace for the sequential kernel
-    if constexpr (kNorm) {
-        const int r = tid >> 1, half = tid & 1;
-        const uint4 *row = reinterpret_cast<const uint4 *>(Ks + r * LDK + 64 * half);
-        float ss = 0.f;
+    } else if (warp == 1) {
+        // Gram G = K K^T: A = K (K-major, per key block), B = K (K-major: N rows = tokens)
+        const bool landed = warp_wait(cx, 0, 0);
+        tc_fence_after();
+        if (landed && lane == 0) {
+            const uint32_t kt = smem_u32(ut_smem + UT_SM_KT);
+            const uint32_t idesc = idesc_bf16(64, 64, false, false);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const uint4 u = row[m];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                ss += f.x * f.x + f.y * f.y;
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_bf16(tmem, desc_sw128(kt + koff, 16, 1024), desc_sw128(kt + koff, 16, 1024),
+                         idesc, kk > 0);
             }
+            mma_commit(cx.bar + 1);
         }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        if (half == 0) {
-            const float rkv = rsqrtf(ss + kNormEps);
+        __syncwarp();
+    }
+    __syncthreads();  // the gate vectors are written
+    // row r = 16 w + l of G (lanes l < 16 of warp w; lanes 16-31 read unused TMEM)
+    const int r = 16 * warp + lane;
+    const bool row_lane = lane < 16;
+    float gr_row[C];
+    {
+        const bool done = warp_wait(cx, 1, 0);
+        tc_fence_after();
+        if (done) {
+            const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+            for (int pc = 0; pc < C / 16; ++pc) {
+                float v[16];
+                tmem_ld16(lane_addr + 16 * pc, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) gr_row[16 * pc + j] = v[j];
+            }
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int j = 0; j < C; ++j) gr_row[j] = 0.f;
+        }
+    }
+    tc_fence_before();
+    if constexpr (kNorm) {
+        // |k_r|^2 is the diagonal of K K^T; 1/|k| folds into the Gram rows and T',
+        // and is kept in the workspace for the sequential kernel
+        if (row_lane) {
+            float d = 0.f;
+#pragma unroll
+            for (int j = 0; j < C; ++j) d = (j == r) ? gr_row[j] : d;
+            const float rkv = rsqrtf(fmaxf(d, 0.f) + kNormEps);
             rks[r] = rkv;
             bgs[r] *= rkv;
             rk_out[((size_t)gch * H + h) * C + r] = rkv;
         }
         __syncthreads();
     }
-
-    // Gram K K^T on and below the diagonal: warp w takes rows 16 w .. + 15 and the
-    // 2 w + 2 column tiles of 8 up to the diagonal, then gates it into A:
-    //   A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0
-    {
-        const int RB = warp, ntiles = 2 * RB + 2;
-        float acc[8][4] = {};
-        // ldmatrix row addresses: A (rows 16 RB.., matrices [rows 0-7 | 8-15] x
-        // [cols 0-7 | 8-15]) and B (a pair of 8-row tiles x [cols 0-7 | 8-15])
-        const int mi = lane >> 3, ri = lane & 7;
-        const __nv_bfloat16 *arow = Ks + (16 * RB + ri + 8 * (mi & 1)) * LDK + 8 * (mi >> 1);
-        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi >> 1)) * LDK + 8 * (mi & 1);
+    // A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0 (row r, all columns)
+    if (row_lane) {
+        const float grl = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
 #pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-            const int k0 = 16 * ks;
-            uint32_t a[4];
-            ldmatrix_x4(a, arow + k0);
+        for (int i4 = 0; i4 < C / 4; ++i4) {
+            float a[4];
 #pragma unroll
-            for (int jp = 0; jp < 4; ++jp) {
-                if (2 * jp < ntiles) {
-                    uint32_t bq[4];
-                    ldmatrix_x4(bq, brow + 16 * jp * LDK + k0);
-                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
-                    mma_bf16_16x8x16(acc[2 * jp], a, b0);
-                    mma_bf16_16x8x16(acc[2 * jp + 1], a, b1);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * i4 + e;
+                const float s = kNorm ? br * rks[i] : br;
+                a[e] = (i < r) ? s * ex2(grl - g2s[i]) * gr_row[i] : 0.f;
             }
-        }
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int r = 16 * RB + g + 8 * hr;
-            const float gr = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j < ntiles) {
-                    const int i = 8 * j + 2 * t;
-                    const float s0 = kNorm ? br * rks[i] : br, s1 = kNorm ? br * rks[i + 1] : br;
-                    const float a0 = (i < r) ? s0 * ex2(gr - g2s[i]) * acc[j][2 * hr] : 0.f;
-                    const float a1 =
-                        (i + 1 < r) ? s1 * ex2(gr - g2s[i + 1]) * acc[j][2 * hr + 1] : 0.f;
-                    *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
-                }
-            }
+            *reinterpret_cast<float4 *>(AF + r * LDA + 4 * i4) = make_float4(a[0], a[1], a[2], a[3]);
         }
     }
-    __syncthreads();  // A complete; K no longer read, its buffer becomes T
+    __syncthreads();  // A complete; TMEM and K no longer read (K's buffer becomes T)
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, UT_TM_COLS);
+    }
     if (tid < C) ut_diag(AF, TF, tid);
     __syncthreads();
     ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
@@ -1153,14 +1180,14 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
     const bool norm = (flags & kFlagL2Norm) != 0;
     auto *ut = norm ? tc::gdn_ut_kernel<true> : tc::gdn_ut_kernel<false>;
     auto *seq = norm ? tc::gdn_chunk_tc_kernel<true> : tc::gdn_chunk_tc_kernel<false>;
-    const int ut_smem = tc::ut_smem_bytes(norm);
+    const int ut_smem = tc::UT_SMEM;
     cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize, ut_smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (total_chunks > 0)
         ut<<<dim3((unsigned)total_chunks, H, 1), tc::UT_THREADS, ut_smem, st>>>(
-            static_cast<const __nv_bfloat16 *>(k), log_alpha, beta, tt, rk, p.sq, H, flags);
+            mk, log_alpha, beta, tt, rk, p.sq, H, flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the CTAs may start (TMEM, barriers, the initial

@@ -17,11 +17,12 @@
 // and WY products next to a two-stage ring, so the key-side work moves to the
 // parallel kernel:
 //  1. gdn_utw_kernel, one CTA per (chunk, head), all chunks in parallel: the
-//     Gram matrix and Q K^T (bf16 mma.sync, float32 accumulation), the gating,
-//     the blocked UT solve, and W = T diag(beta gamma) K; it writes the bf16
-//     tiles [P; T''] (128 x 64, T'' = T diag(beta)) and W (64 x 256) of each
-//     chunk to the workspace.  None of it depends on the state, and it is
-//     formed once per head instead of once per value slice.
+//     Gram matrix and Q K^T (one tcgen05 product from TMA-loaded tiles), the
+//     gating, the blocked UT solve, and W = T diag(beta gamma) K (a second
+//     tcgen05 product); it writes the bf16 tiles [P; T''] (128 x 64, T'' =
+//     T diag(beta)) and W (64 x 256) of each chunk to the workspace.  None of
+//     it depends on the state, and it is formed once per head instead of once
+//     per value slice.
 //  2. gdn_chunk_tcw_kernel, one CTA per (sequence, head, 64 value channels),
 //     walking the chunks in order with S^T (256 x 64, float32, as two 128-lane
 //     halves) resident in tensor memory.  Products (tcgen05.mma, M = 128, bf16
@@ -71,29 +72,38 @@ constexpr float LOG2E = 1.4426950408889634f;
 // One CTA of 4 warps per (global chunk g, head h).  Outputs at tile index
 // g H + h: [P; T''] (128 x 64 bf16, row-major), W (64 x 256 bf16, row-major) and,
 // when normalising, 1/|q| and 1/|k| of the chunk's rows (2 x 64 float32).
+// The chunk's K and Q rows arrive by TMA (128-byte swizzle), interleaved per
+// 64-key block as K | Q so that [K; Q] is one 128-row operand, and both
+// products are tcgen05.mma into tensor memory:
+//   G = [K; Q] K^T   (M = 128, N = 64; N = 128 with [K; Q]^T when normalising,
+//                     whose diagonals give |k|^2 and |q|^2): lanes 0-63 the Gram
+//                     matrix, lanes 64-127 Q K^T
+//   W = T' K         (M = 64, two products of N = 128 key columns; A = T' from
+//                     shared memory, B = K MN-major), after the UT solve
+// An M = 64 product puts row m in TMEM lane 32 (m / 16) + m % 16.  Two CTAs
+// fit on an SM (105 KiB of shared memory, 256 TMEM columns each).
 constexpr int UT_THREADS = 128;
-constexpr int LDKW = DK + 8;                       // bf16 row stride of staged K, Q and W
-constexpr int LDB = C + 8;                         // bf16 row stride of P and T'
-constexpr int SM_K = 0;                            // K chunk (64 x LDKW bf16)
-constexpr int SM_Q = SM_K + C * LDKW * 2;          // Q chunk; then T (f32); then W staging
-constexpr int SM_A = SM_Q + C * LDKW * 2;          // A (f32, 64 x LDA); then T' (bf16)
-constexpr int SM_P = SM_A + C * LDA * 4;           // P (bf16, 64 x LDB)
-constexpr int SM_G = SM_P + C * LDB * 2;           // 5 x 64 floats of per-row gates and norms
-constexpr int UT_SMEM = SM_G + 5 * C * 4;
+constexpr int SM_KQ = 0;                           // per key block: K (8 KiB), then Q (8 KiB)
+constexpr int KQ_BLK = 16384;
+constexpr int SM_AF = SM_KQ + KB * KQ_BLK;         // A (f32, 64 x LDA); then T' (bf16, swizzled)
+constexpr int SM_TF = SM_AF + C * LDA * 4;         // T (f32, 64 x LDA)
+constexpr int SM_G = SM_TF + C * LDA * 4;          // 5 x 64 floats of per-row gates and norms
+constexpr int SM_UBAR = SM_G + 5 * C * 4;          // 3 mbarriers, TMEM base, abort flag
+constexpr int UT_SMEM = SM_UBAR + 48 + 1024;       // + alignment slack (1024-byte tiles)
+constexpr uint32_t UT_TM_COLS = 256;
 constexpr int PT_ELEMS = 2 * C * C;
 constexpr int W_ELEMS = C * DK;
-static_assert(C * LDA * 4 <= C * LDKW * 2, "T fits in the Q buffer");
-static_assert(C * LDB * 2 <= C * LDA * 4, "T' fits in the A buffer");
-static_assert(SM_Q % 16 == 0 && SM_A % 16 == 0 && SM_P % 16 == 0 && SM_G % 16 == 0,
-              "16-byte aligned buffers");
+static_assert(SM_AF % 1024 == 0 && SM_TF % 16 == 0 && SM_G % 16 == 0 && SM_UBAR % 8 == 0,
+              "aligned UT buffers");
 
 template <bool kNorm>
 __global__ void __launch_bounds__(UT_THREADS, 2)
-gdn_utw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                __nv_bfloat16 *__restrict__ pt, __nv_bfloat16 *__restrict__ wt,
                float *__restrict__ rqk, const Seqs sq, int H, unsigned flags) {
-    extern __shared__ __align__(16) uint8_t ut_smem[];
+    extern __shared__ __align__(1024) uint8_t ut_raw[];
+    uint8_t *sm = ut_raw + ((1024u - (smem_u32(ut_raw) & 1023u)) & 1023u);
     // the sequential kernel that follows may be scheduled now (it waits for this
     // grid's completion before it reads the tiles)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -102,27 +112,44 @@ gdn_utw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
     const Span sp = tc::seq_span(sq, b);
     const int c = gch - sp.chunk0, T = sp.len, t0 = c * C;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
     const size_t tile = (size_t)gch * H + h;
-    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_K);
-    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_Q);
-    float *TF = reinterpret_cast<float *>(ut_smem + SM_Q);
-    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_Q);
-    float *AF = reinterpret_cast<float *>(ut_smem + SM_A);
-    __nv_bfloat16 *Tb = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_A);
-    __nv_bfloat16 *Pb = reinterpret_cast<__nv_bfloat16 *>(ut_smem + SM_P);
-    float *g2s = reinterpret_cast<float *>(ut_smem + SM_G);
+    float *AF = reinterpret_cast<float *>(sm + SM_AF);
+    float *TF = reinterpret_cast<float *>(sm + SM_TF);
+    float *g2s = reinterpret_cast<float *>(sm + SM_G);
     float *bes = g2s + C, *bgs = g2s + 2 * C, *rks = g2s + 3 * C, *rqs = g2s + 4 * C;
+    Ctx cx;
+    cx.base = sm;
+    cx.bar = reinterpret_cast<uint64_t *>(sm + SM_UBAR);  // [0] K, Q landed [1] G done [2] W done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SM_UBAR + 24);
+    cx.abort = reinterpret_cast<volatile uint32_t *>(sm + SM_UBAR + 28);
+    cx.err = &g_tcw_error;
 
-    // q and k rows of the chunk (zero-filled past the end): 32 x 16 B per row
-#pragma unroll 4
-    for (int m = 0; m < C * (DK / 8) / UT_THREADS; ++m) {
-        const int idx = tid + UT_THREADS * m;
-        const int r = idx / (DK / 8), piece = idx % (DK / 8);
-        const bool in = t0 + r < T;
-        const size_t row = (size_t)(sp.off + (in ? t0 + r : 0)) * H + h;
-        cp_async16(Ks + r * LDKW + 8 * piece, k + row * DK + 8 * piece, in ? 16u : 0u);
-        cp_async16(Qs + r * LDKW + 8 * piece, q + row * DK + 8 * piece, in ? 16u : 0u);
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(cx.bar + i, 1);
+        *cx.abort = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, UT_TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    // K and Q rows of the chunk.  Rows past the end of the sequence (the next
+    // sequence's, or TMA's zero fill) get beta = 0 and log alpha = 0: their rows
+    // of A and their columns of T', T'' and P vanish, and their rows of P are
+    // outputs of tokens that are never stored.
+    if (tid == 0) {
+        mbar_arrive_expect_tx(cx.bar + 0, 2 * KB * 8192);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+            tma_load_4d(sm + SM_KQ + kb * KQ_BLK, &tm_k, cx.bar + 0, kb * 64, h, sp.off + t0, 0);
+            tma_load_4d(sm + SM_KQ + kb * KQ_BLK + 8192, &tm_q, cx.bar + 0, kb * 64, h,
+                        sp.off + t0, 0);
+        }
     }
     if (warp == 0) {
         // running sum of log alpha over rows lane and lane + 32, in log2 units
@@ -153,175 +180,183 @@ gdn_utw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
             bes[lane + 32 * hh] = be[hh];
             bgs[lane + 32 * hh] = be[hh] * tc::ex2(g2);
         }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    if constexpr (kNorm) {
-        // 1/|k_r| (threads 0-63) and 1/|q_r| (threads 64-127), one row each
-        const int r = tid & (C - 1);
-        const bool isq = tid >= C;
-        const uint4 *row = reinterpret_cast<const uint4 *>((isq ? Qs : Ks) + r * LDKW);
-        float ss = 0.f;
-#pragma unroll 8
-        for (int m = 0; m < DK / 8; ++m) {
-            const uint4 u = row[m];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    } else if (warp == 1) {
+        const bool landed = tc::warp_wait(cx, 0, 0);
+        tc_fence_after();
+        if (landed && lane == 0) {
+            const uint32_t kq = smem_u32(sm + SM_KQ);
+            const uint32_t idesc = idesc_bf16(128, kNorm ? 128 : 64, false, false);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                ss += f.x * f.x + f.y * f.y;
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * KQ_BLK + (kk & 3) * 32;
+                mma_bf16(tmem, desc_sw128(kq + off, 16, 1024), desc_sw128(kq + off, 16, 1024),
+                         idesc, kk > 0);
             }
+            mma_commit(cx.bar + 1);
         }
-        const float rn = rsqrtf(ss + kNormEps);
-        if (isq) {
+        __syncwarp();
+    }
+    __syncthreads();  // the gate vectors are written
+    // warps 0, 1: Gram row r = 32 w + lane; warps 2, 3: Q K^T row r = 32 (w - 2) + lane
+    const bool is_p = warp >= 2;
+    const int r = 32 * (warp & 1) + lane;
+    float row[C];
+    float dg = 0.f;  // |k_r|^2 or |q_r|^2 from the diagonals
+    {
+        const bool done = tc::warp_wait(cx, 1, 0);
+        tc_fence_after();
+        if (done) {
+#pragma unroll
+            for (int pc = 0; pc < C / 16; ++pc) {
+                float v[16];
+                tmem_ld16(lane_addr + 16 * pc, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) row[16 * pc + j] = v[j];
+            }
+            if constexpr (kNorm) {
+                // Q Q^T (lanes 64-127, columns 64-127) for |q_r|^2
+                float v[16];
+#pragma unroll
+                for (int pc = 0; pc < C / 16; ++pc) {
+                    tmem_ld16(lane_addr + 64 + 16 * pc, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dg = (16 * pc + j == r) ? v[j] : dg;
+                }
+                if (!is_p) {
+#pragma unroll
+                    for (int j = 0; j < C; ++j) dg = (j == r) ? row[j] : dg;
+                }
+            }
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int j = 0; j < C; ++j) row[j] = 0.f;
+        }
+    }
+    tc_fence_before();
+    if constexpr (kNorm) {
+        const float rn = rsqrtf(fmaxf(dg, 0.f) + kNormEps);
+        if (is_p) {
             rqs[r] = rn;
         } else {
             rks[r] = rn;
             bgs[r] *= rn;
         }
-        rqk[tile * 2 * C + (isq ? 0 : C) + r] = rn;
+        rqk[tile * 2 * C + (is_p ? 0 : C) + r] = rn;
         __syncthreads();
     }
-
-    // Gram K K^T and Q K^T on and below the diagonal: warp w takes rows 16 w .. + 15
-    // and the 2 w + 2 column tiles of 8 up to the diagonal (one pass over the keys
-    // for both products), then gates them:
-    //   A_ri = beta_r exp(g_r - g_i) k_r . k_i    (i < r, else 0)
-    //   P_ri = exp(g_r - g_i) q_r . k_i           (i <= r, else 0)
     {
-        const int RB = warp, ntiles = 2 * RB + 2;
-        float accg[8][4] = {}, accp[8][4] = {};
-        const int mi = lane >> 3, ri = lane & 7;
-        const int arow_off = (16 * RB + ri + 8 * (mi & 1)) * LDKW + 8 * (mi >> 1);
-        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi >> 1)) * LDKW + 8 * (mi & 1);
-#pragma unroll 2
-        for (int ks = 0; ks < DK / 16; ++ks) {
-            const int k0 = 16 * ks;
-            uint32_t ak[4], aq[4];
-            ldmatrix_x4(ak, Ks + arow_off + k0);
-            ldmatrix_x4(aq, Qs + arow_off + k0);
+        // A_ri = beta_r exp(g_r - g_i) k_r . k_i  (i < r)      -> A (float32)
+        // P_ri = exp(g_r - g_i) q_r . k_i         (i <= r)     -> [P; T''] rows 0-63
+        const float grl = g2s[r];
+        const float sr = is_p ? (kNorm ? rqs[r] : 1.f) : (kNorm ? bes[r] * rks[r] : bes[r]);
+        __nv_bfloat16 *dp = pt + tile * PT_ELEMS + r * C;
 #pragma unroll
-            for (int jp = 0; jp < 4; ++jp) {
-                if (2 * jp < ntiles) {
-                    uint32_t bq[4];
-                    ldmatrix_x4(bq, brow + 16 * jp * LDKW + k0);
-                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
-                    mma_bf16_16x8x16(accg[2 * jp], ak, b0);
-                    mma_bf16_16x8x16(accg[2 * jp + 1], ak, b1);
-                    mma_bf16_16x8x16(accp[2 * jp], aq, b0);
-                    mma_bf16_16x8x16(accp[2 * jp + 1], aq, b1);
-                }
+        for (int i8 = 0; i8 < C / 8; ++i8) {
+            float a[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i = 8 * i8 + e;
+                const float s = kNorm ? sr * rks[i] : sr;
+                const bool keep = is_p ? (i <= r) : (i < r);
+                // exponents are <= 0 where kept (g is non-increasing)
+                a[e] = keep ? s * tc::ex2(grl - g2s[i]) * row[i] : 0.f;
             }
-        }
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int r = 16 * RB + g + 8 * hr;
-            const float gr = g2s[r];
-            const float br = kNorm ? bes[r] * rks[r] : bes[r];
-            const float pr = kNorm ? rqs[r] : 1.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = 8 * j + 2 * t;
-                float p0 = 0.f, p1 = 0.f;
-                if (j < ntiles) {
-                    // exponents are <= 0 where selected (g is non-increasing)
-                    const float e0 = tc::ex2(gr - g2s[i]), e1 = tc::ex2(gr - g2s[i + 1]);
-                    const float k0 = kNorm ? rks[i] : 1.f, k1 = kNorm ? rks[i + 1] : 1.f;
-                    const float a0 = (i < r) ? br * k0 * e0 * accg[j][2 * hr] : 0.f;
-                    const float a1 = (i + 1 < r) ? br * k1 * e1 * accg[j][2 * hr + 1] : 0.f;
-                    p0 = (i <= r) ? pr * k0 * e0 * accp[j][2 * hr] : 0.f;
-                    p1 = (i + 1 <= r) ? pr * k1 * e1 * accp[j][2 * hr + 1] : 0.f;
-                    *reinterpret_cast<float2 *>(AF + r * LDA + i) = make_float2(a0, a1);
-                }
-                *reinterpret_cast<uint32_t *>(Pb + r * LDB + i) = tc::pack_bf16(p0, p1);
+            if (is_p) {
+                *reinterpret_cast<uint4 *>(dp + 8 * i8) =
+                    make_uint4(tc::pack_bf16(a[0], a[1]), tc::pack_bf16(a[2], a[3]),
+                               tc::pack_bf16(a[4], a[5]), tc::pack_bf16(a[6], a[7]));
+            } else {
+                *reinterpret_cast<float4 *>(AF + r * LDA + 8 * i8) = make_float4(a[0], a[1], a[2], a[3]);
+                *reinterpret_cast<float4 *>(AF + r * LDA + 8 * i8 + 4) = make_float4(a[4], a[5], a[6], a[7]);
             }
         }
     }
-    __syncthreads();  // A and P complete; Q is no longer read (its buffer becomes T)
+    __syncthreads();  // A complete, G no longer read
     if (tid < C) tc::ut_diag(AF, TF, tid);
     __syncthreads();
     tc::ut_offdiag4(AF, TF, tid);  // ends with a CTA-wide barrier
 
-    // [P; T''] to the workspace (8 threads per 128-byte row), T'' = T diag(beta)
-    __nv_bfloat16 *dpt = pt + tile * PT_ELEMS;
-#pragma unroll 2
-    for (int m = 0; m < PT_ELEMS / 8 / UT_THREADS; ++m) {
-        const int idx = tid + UT_THREADS * m;
-        const int rt = idx >> 3, i0 = 8 * (idx & 7);
-        uint4 val;
-        if (rt < C) {
-            val = *reinterpret_cast<const uint4 *>(Pb + rt * LDB + i0);
-        } else {
-            const int r = rt - C;
-            const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
-            const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
-            const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = (i0 + e <= r) ? tv[e] * bes[i0 + e] : 0.f;
-            val = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
-                             tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
-        }
-        *reinterpret_cast<uint4 *>(dpt + rt * C + i0) = val;
-    }
-    // T' = T diag(beta gamma / |k|) (lower triangle) as bf16 over the dead A buffer
-#pragma unroll
-    for (int m = 0; m < C * C / 8 / UT_THREADS; ++m) {
-        const int idx = tid + UT_THREADS * m;
-        const int r = idx >> 3, i0 = 8 * (idx & 7);
-        const float4 ta = *reinterpret_cast<const float4 *>(TF + r * LDA + i0);
-        const float4 tb = *reinterpret_cast<const float4 *>(TF + r * LDA + i0 + 4);
-        const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = (i0 + e <= r) ? tv[e] * bgs[i0 + e] : 0.f;
-        *reinterpret_cast<uint4 *>(Tb + r * LDB + i0) =
-            make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
-                       tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
-    }
-    __syncthreads();  // T' complete; T is no longer read (its buffer becomes W)
-
-    // W = T' K: warp w takes rows 16 w .. + 15 (T' is lower triangular, so only
-    // chunk rows 0 .. 16 w + 15 contribute), in two passes of 128 key columns
+    // T'' = T diag(beta) -> [P; T''] rows 64-127 (8 threads per 128-byte row), and
+    // T' = T diag(beta gamma / |k|) as the swizzled bf16 A operand of W = T' K
+    // (over the dead A buffer); both lower triangular
     {
-        const int mi = lane >> 3, ri = lane & 7;
-        const __nv_bfloat16 *arow = Tb + (16 * warp + ri + 8 * (mi & 1)) * LDB + 8 * (mi >> 1);
-        // B = K (chunk row i = k index, key = n index), stored with k along the rows
-        const __nv_bfloat16 *brow = Ks + (ri + 8 * (mi & 1)) * LDKW + 8 * (mi >> 1);
-#pragma unroll 1
-        for (int nh = 0; nh < 2; ++nh) {
-            float acc[16][4] = {};
-#pragma unroll 1
-            for (int ks = 0; ks <= warp; ++ks) {
-                uint32_t a[4];
-                ldmatrix_x4(a, arow + 16 * ks);
+        __nv_bfloat16 *dpt = pt + tile * PT_ELEMS + C * C;
+        uint8_t *tp = sm + SM_AF;
 #pragma unroll
-                for (int np = 0; np < 8; ++np) {
-                    uint32_t bq[4];
-                    ldmatrix_x4_trans(bq, brow + 16 * ks * LDKW + 128 * nh + 16 * np);
-                    const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
-                    mma_bf16_16x8x16(acc[2 * np], a, b0);
-                    mma_bf16_16x8x16(acc[2 * np + 1], a, b1);
-                }
+        for (int m = 0; m < C * C / 8 / UT_THREADS; ++m) {
+            const int idx = tid + UT_THREADS * m;
+            const int rr = idx >> 3, i0 = 8 * (idx & 7);
+            const float4 ta = *reinterpret_cast<const float4 *>(TF + rr * LDA + i0);
+            const float4 tb = *reinterpret_cast<const float4 *>(TF + rr * LDA + i0 + 4);
+            const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+            float x[8], y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const bool low = i0 + e <= rr;
+                x[e] = low ? tv[e] * bes[i0 + e] : 0.f;
+                y[e] = low ? tv[e] * bgs[i0 + e] : 0.f;
             }
+            *reinterpret_cast<uint4 *>(dpt + rr * C + i0) =
+                make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                           tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+            *reinterpret_cast<uint4 *>(tp + sw128_offset(rr, 2 * i0)) =
+                make_uint4(tc::pack_bf16(y[0], y[1]), tc::pack_bf16(y[2], y[3]),
+                           tc::pack_bf16(y[4], y[5]), tc::pack_bf16(y[6], y[7]));
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // T' is in shared memory for the tensor cores
+    if (warp == 1) {
+        tc_fence_after();
+        if (lane == 0) {
+            // W = T' K: A = T' (K-major, 64 rows), B = K (MN-major: 64-key blocks
+            // KQ_BLK apart, 16 chunk rows per step)
+            const uint32_t tp = smem_u32(sm + SM_AF), kq = smem_u32(sm + SM_KQ);
+            const uint32_t idesc = idesc_bf16(64, 128, false, true);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int col = 128 * nh + 8 * j + 2 * t;
-                *reinterpret_cast<uint32_t *>(Ws + (16 * warp + g) * LDKW + col) =
-                    tc::pack_bf16(acc[j][0], acc[j][1]);
-                *reinterpret_cast<uint32_t *>(Ws + (16 * warp + g + 8) * LDKW + col) =
-                    tc::pack_bf16(acc[j][2], acc[j][3]);
+            for (int nh = 0; nh < 2; ++nh)
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + 128 * nh, desc_sw128(tp + kk * 32, 16, 1024),
+                             desc_sw128(kq + nh * 2 * KQ_BLK + kk * 2048, KQ_BLK, 1024), idesc,
+                             kk > 0);
+            mma_commit(cx.bar + 2);
+        }
+        __syncwarp();
+    }
+    {
+        // W rows: row 16 w + l in TMEM lane 32 w + l (l < 16), 256 columns -> 512 B
+        const bool done = tc::warp_wait(cx, 2, 0);
+        tc_fence_after();
+        const int wr = 16 * warp + lane;
+        __nv_bfloat16 *dw = wt + tile * W_ELEMS + (size_t)wr * DK;
+#pragma unroll 1
+        for (int pc = 0; pc < DK / 16; pc += 2) {
+            float v0[16], v1[16];
+            tmem_ld16(lane_addr + 16 * pc, v0);
+            tmem_ld16(lane_addr + 16 * pc + 16, v1);
+            tmem_wait_ld();
+            if (done && lane < 16) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dw + 16 * pc);
+                d4[0] = make_uint4(tc::pack_bf16(v0[0], v0[1]), tc::pack_bf16(v0[2], v0[3]),
+                                   tc::pack_bf16(v0[4], v0[5]), tc::pack_bf16(v0[6], v0[7]));
+                d4[1] = make_uint4(tc::pack_bf16(v0[8], v0[9]), tc::pack_bf16(v0[10], v0[11]),
+                                   tc::pack_bf16(v0[12], v0[13]), tc::pack_bf16(v0[14], v0[15]));
+                d4[2] = make_uint4(tc::pack_bf16(v1[0], v1[1]), tc::pack_bf16(v1[2], v1[3]),
+                                   tc::pack_bf16(v1[4], v1[5]), tc::pack_bf16(v1[6], v1[7]));
+                d4[3] = make_uint4(tc::pack_bf16(v1[8], v1[9]), tc::pack_bf16(v1[10], v1[11]),
+                                   tc::pack_bf16(v1[12], v1[13]), tc::pack_bf16(v1[14], v1[15]));
             }
         }
     }
+    tc_fence_before();
     __syncthreads();
-    __nv_bfloat16 *dw = wt + tile * W_ELEMS;
-#pragma unroll 4
-    for (int m = 0; m < W_ELEMS / 8 / UT_THREADS; ++m) {
-        const int idx = tid + UT_THREADS * m;
-        const int r = idx >> 5, piece = idx & 31;
-        *reinterpret_cast<uint4 *>(dw + r * DK + 8 * piece) =
-            *reinterpret_cast<const uint4 *>(Ws + r * LDKW + 8 * piece);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, UT_TM_COLS);
     }
 }
 
@@ -857,8 +892,7 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
     if (e != cudaSuccess) return e;
     if (total_chunks > 0)
         ut<<<dim3((unsigned)total_chunks, H, 1), tcw::UT_THREADS, tcw::UT_SMEM, st>>>(
-            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-            log_alpha, beta, pt, wt, rqk, sq, H, flags);
+            mq, mk, log_alpha, beta, pt, wt, rqk, sq, H, flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
