@@ -41,6 +41,8 @@ def _load():
     lib.gdn_chunk_fwd_workspace_size.restype = Z
     lib.gdn_chunk_fwd_path.argtypes = [I, I, I, I, I, I, I]
     lib.gdn_chunk_fwd_path.restype = I
+    lib.gdn_chunk_fwd_variant.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_fwd_variant.restype = I
     lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, vp]
     lib.gdn_decode_step.restype = I
     U = ctypes.c_uint
@@ -136,6 +138,16 @@ def chunk_fwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
     if p < 0:
         raise GdnError("invalid or unsupported sizes")
     return PATH_NAMES[p]
+
+
+VARIANT_NAMES = {0: None, 1: "fused", 2: "precomputed"}
+
+
+def chunk_fwd_variant(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16):
+    """Which tcgen05 variant a chunk_fwd call with these sizes runs: "fused",
+    "precomputed", or None off the tcgen05 path."""
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    return VARIANT_NAMES[int(LIB.gdn_chunk_fwd_variant(B, T, H, Dk, Dv, chunk, code))]
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, chunk: int = 64, out=None, S_T=None,

@@ -533,7 +533,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
     if (tc_recompute(B, Tlen, H, Dk, Dv, C, bf16)) {
         // T, P, g on the CUDA cores; the chunk states from the tensor-core forward
         uint8_t *tail = reinterpret_cast<uint8_t *>(ws_prep + base_floats(B, Tlen, H, Dk, Dv, C));
-        void *o_scratch = tail + ((tc_workspace_bytes(B, Tlen, H, 0) + 255) & ~size_t(255));
+        void *o_scratch = tail + ((tc_workspace_bytes_fused(B, Tlen, H, 0) + 255) & ~size_t(255));
         e = launch_bwd_recompute(q, k, v, la, beta, S0, B, Tlen, H, Dk, Dv, C, bf16, ws_prep,
                                  nullptr, st);
         if (e != cudaSuccess) return e;
@@ -569,7 +569,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
 size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
     size_t n = base_floats(B, T, H, Dk, Dv, chunk) * sizeof(float);
     if (tc_recompute(B, T, H, Dk, Dv, chunk, bf16))
-        n += ((tc_workspace_bytes(B, T, H, 0) + 255) & ~size_t(255)) +
+        n += ((tc_workspace_bytes_fused(B, T, H, 0) + 255) & ~size_t(255)) +
              (size_t)B * T * H * Dv * sizeof(__nv_bfloat16);
     return n;
 }

@@ -1111,21 +1111,41 @@ size_t tc_offsets_bytes(int n_seq, bool varlen) {
     return varlen ? ((2 * (size_t)n_seq + 1) * sizeof(int) + 255) & ~size_t(255) : 0;
 }
 
-size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                               unsigned flags, int Dk) {
-    if (Dk == tcw_dk) return tcw_workspace_bytes_seqs(n_seq, total_chunks, H, varlen, flags);
+// The fused variant's sequential grid has Dv / 64 x H x (sequences) CTAs of one
+// SM each; below this many the GPU is mostly idle, HBM bandwidth is to spare,
+// and the precomputed variant's shorter per-chunk chain wins.
+constexpr int kFewSeqCtas = 74;
+
+bool tc_precomputed(int n_seq, int H, int Dk, int Dv) {
+    return Dk == 256 || (long long)(Dv / tc::DVT) * H * n_seq < kFewSeqCtas;
+}
+
+static size_t fused_workspace_bytes(int n_seq, long long total_chunks, int H, bool varlen,
+                                    unsigned flags) {
     const size_t tiles = (size_t)total_chunks * H * tc::TT_ELEMS * sizeof(__nv_bfloat16);
     const size_t rk = (flags & kFlagL2Norm) ? (size_t)total_chunks * H * tc::C * sizeof(float) : 0;
     return tc_offsets_bytes(n_seq, varlen) + tiles + rk;
 }
 
-size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk) {
+size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
+                               unsigned flags, int Dk, int Dv) {
+    if (tc_precomputed(n_seq, H, Dk, Dv))
+        return tcw_workspace_bytes_seqs(n_seq, total_chunks, H, varlen, flags, Dk);
+    return fused_workspace_bytes(n_seq, total_chunks, H, varlen, flags);
+}
+
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk, int Dv) {
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
-    return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags, Dk);
+    return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags, Dk, Dv);
+}
+
+size_t tc_workspace_bytes_fused(int B, int T, int H, unsigned flags) {
+    const long long NT = ((long long)T + tc::C - 1) / tc::C;
+    return fused_workspace_bytes(B, (long long)B * NT, H, false, flags);
 }
 
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
-    return bf16 && chunk == tc::C && (Dk == tc::DK || Dk == tcw_dk) && Dv % tc::DVT == 0 &&
+    return bf16 && chunk == tc::C && (Dk == tc::DK || Dk == 256) && Dv % tc::DVT == 0 &&
            B >= 1 && T >= 1 && H >= 1 && tc::encode_fn() != nullptr;
 }
 
@@ -1141,11 +1161,11 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
                                  int Dv, unsigned flags, void *workspace, cudaStream_t st,
                                  float *S_hist) {
-    if (Dk == tcw_dk) {
-        if (S_hist) return cudaErrorInvalidValue;  // the state history is a Dk = 128 feature
+    // the state history (for the backward) is a feature of the fused variant
+    if (S_hist && Dk != tc::DK) return cudaErrorInvalidValue;
+    if (!S_hist && tc_precomputed(n_seq, H, Dk, Dv))
         return launch_chunk_tcw_seqs(q, k, v, log_alpha, beta, S0, o, S_T, n_seq, T_fixed, total_T,
-                                     cu_seqlens, total_chunks, H, Dv, flags, workspace, st);
-    }
+                                     cu_seqlens, total_chunks, H, Dk, Dv, flags, workspace, st);
     const bool varlen = cu_seqlens != nullptr;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;

@@ -63,8 +63,6 @@ using tc::LDA;
 using tc::Seqs;
 using tc::Span;
 
-constexpr int DK = 256;
-constexpr int KB = DK / 64;        // 64-key blocks
 constexpr int DVT = 64;            // value channels per CTA of the sequential kernel
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -80,28 +78,37 @@ constexpr float LOG2E = 1.4426950408889634f;
 //                     matrix, lanes 64-127 Q K^T
 //   W = T' K         (M = 64, two products of N = 128 key columns; A = T' from
 //                     shared memory, B = K MN-major), after the UT solve
-// An M = 64 product puts row m in TMEM lane 32 (m / 16) + m % 16.  Two CTAs
-// fit on an SM (105 KiB of shared memory, 256 TMEM columns each).
+// An M = 64 product puts row m in TMEM lane 32 (m / 16) + m % 16.  At Dk = 256
+// two CTAs fit on an SM (105 KiB of shared memory, 256 TMEM columns each), at
+// Dk = 128 three (73 KiB, 128 columns).
 constexpr int UT_THREADS = 128;
 constexpr int SM_KQ = 0;                           // per key block: K (8 KiB), then Q (8 KiB)
 constexpr int KQ_BLK = 16384;
-constexpr int SM_AF = SM_KQ + KB * KQ_BLK;         // A (f32, 64 x LDA); then T' (bf16, swizzled)
-constexpr int SM_TF = SM_AF + C * LDA * 4;         // T (f32, 64 x LDA)
-constexpr int SM_G = SM_TF + C * LDA * 4;          // 5 x 64 floats of per-row gates and norms
-constexpr int SM_UBAR = SM_G + 5 * C * 4;          // 3 mbarriers, TMEM base, abort flag
-constexpr int UT_SMEM = SM_UBAR + 48 + 1024;       // + alignment slack (1024-byte tiles)
-constexpr uint32_t UT_TM_COLS = 256;
 constexpr int PT_ELEMS = 2 * C * C;
-constexpr int W_ELEMS = C * DK;
-static_assert(SM_AF % 1024 == 0 && SM_TF % 16 == 0 && SM_G % 16 == 0 && SM_UBAR % 8 == 0,
-              "aligned UT buffers");
+template <int DK>
+struct UtDims {
+    static constexpr int KB = DK / 64;                        // 64-key blocks
+    static constexpr int SM_AF = SM_KQ + KB * KQ_BLK;         // A (f32, 64 x LDA); then T' (bf16, swizzled)
+    static constexpr int SM_TF = SM_AF + C * LDA * 4;         // T (f32, 64 x LDA)
+    static constexpr int SM_G = SM_TF + C * LDA * 4;          // 5 x 64 floats of per-row gates and norms
+    static constexpr int SM_UBAR = SM_G + 5 * C * 4;          // 3 mbarriers, TMEM base, abort flag
+    static constexpr int UT_SMEM = SM_UBAR + 48 + 1024;       // + alignment slack (1024-byte tiles)
+    static constexpr uint32_t UT_TM_COLS = DK;                // G (<= 128 columns), then W
+    static constexpr int W_ELEMS = C * DK;
+    static_assert(SM_AF % 1024 == 0 && SM_TF % 16 == 0 && SM_G % 16 == 0 && SM_UBAR % 8 == 0,
+                  "aligned UT buffers");
+};
 
-template <bool kNorm>
-__global__ void __launch_bounds__(UT_THREADS, 2)
+template <int DK, bool kNorm>
+__global__ void __launch_bounds__(UT_THREADS, DK == 256 ? 2 : 3)
 gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                __nv_bfloat16 *__restrict__ pt, __nv_bfloat16 *__restrict__ wt,
                float *__restrict__ rqk, const Seqs sq, int H, unsigned flags) {
+    using L = UtDims<DK>;
+    constexpr int KB = L::KB, SM_AF = L::SM_AF, SM_TF = L::SM_TF, SM_G = L::SM_G,
+                  SM_UBAR = L::SM_UBAR, W_ELEMS = L::W_ELEMS;
+    constexpr uint32_t UT_TM_COLS = L::UT_TM_COLS;
     extern __shared__ __align__(1024) uint8_t ut_raw[];
     uint8_t *sm = ut_raw + ((1024u - (smem_u32(ut_raw) & 1023u)) & 1023u);
     // the sequential kernel that follows may be scheduled now (it waits for this
@@ -313,11 +320,11 @@ gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
         if (lane == 0) {
             // W = T' K: A = T' (K-major, 64 rows), B = K (MN-major: 64-key blocks
-            // KQ_BLK apart, 16 chunk rows per step)
+            // KQ_BLK apart, 16 chunk rows per step), 128 key columns per product
             const uint32_t tp = smem_u32(sm + SM_AF), kq = smem_u32(sm + SM_KQ);
             const uint32_t idesc = idesc_bf16(64, 128, false, true);
 #pragma unroll
-            for (int nh = 0; nh < 2; ++nh)
+            for (int nh = 0; nh < DK / 128; ++nh)
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     mma_bf16(tmem + 128 * nh, desc_sw128(tp + kk * 32, 16, 1024),
@@ -362,46 +369,56 @@ gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 // ----------------------------------------------------- sequential kernel --
 constexpr int BLK = 8192;                       // one 64 x 64 bf16 tile (64 rows of 128 B)
-constexpr int SM_QW = 0;                        // per key block: Q (8 KiB), then W (8 KiB)
-constexpr int SM_KT = SM_QW + KB * 2 * BLK;     // K: 4 key blocks of 8 KiB
-constexpr int SM_VP = SM_KT + KB * BLK;         // 2 stages: V (8 KiB), [P; T''] (16 KiB)
-constexpr int VP_STAGE = 3 * BLK;
-constexpr int SM_SB = SM_VP + 2 * VP_STAGE;     // S^T bf16: 256 key rows x 128 B (MN-major B)
-constexpr int SM_UN = SM_SB + DK * 128;         // U' bf16 (MN-major B)
-constexpr int SM_UP = SM_UN + BLK;              // diag(exp(g_last - g) / |k|) U' bf16
-constexpr int SM_GV = SM_UP + BLK;              // gate vectors, 2 stages
+constexpr int VP_STAGE = 3 * BLK;               // V (8 KiB), [P; T''] (16 KiB)
 constexpr int GV_GAM = 0;                       // gamma_r (/ |q_r| when normalising)
 constexpr int GV_DCY = 64;                      // exp(g_last - g_r) (/ |k_r| when normalising)
 constexpr int GV_GL = 128;                      // gamma_last
 constexpr int GV_STRIDE = 256;
-constexpr int SM_BAR = SM_GV + 2 * GV_STRIDE * 4;
-constexpr int NBAR = 16;
-constexpr int SM_MISC = SM_BAR + NBAR * 8;      // TMEM base, abort flag
-constexpr int SMEM_BYTES = SM_MISC + 16 + 1024; // + alignment slack
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(SM_KT % 1024 == 0 && SM_VP % 1024 == 0 && SM_SB % 1024 == 0 &&
-              SM_UN % 1024 == 0 && SM_UP % 1024 == 0 && VP_STAGE % 1024 == 0,
-              "1024-byte aligned swizzled tiles");
+constexpr int NBAR = 20;
 
-// TMEM columns: S^T (keys 0-127 in 0-63, keys 128-255 in 64-127), X, U, Y
-constexpr uint32_t TM_ST = 0, TM_X = 128, TM_U = 192, TM_Y = 256;
-constexpr uint32_t TM_COLS = 512;
+// Shared memory and TMEM of the sequential kernel for Dk = 128 or 256.  The
+// [Q; W] and K tiles have NQ stages: two at Dk = 128, one at Dk = 256 (where
+// two would not fit beside the 256-row state copy).
+template <int DK>
+struct SeqDims {
+    static constexpr int KB = DK / 64;          // 64-key blocks
+    static constexpr int NH = DK / 128;         // 128-lane halves of S^T
+    static constexpr int NQ = DK == 128 ? 2 : 1;
+    static constexpr int QW_BYTES = KB * 2 * BLK, K_BYTES = KB * BLK;
+    static constexpr int SM_QW = 0;                         // per key block: Q, then W
+    static constexpr int SM_KT = SM_QW + NQ * QW_BYTES;     // K, key blocks of 8 KiB
+    static constexpr int SM_VP = SM_KT + NQ * K_BYTES;      // 2 stages of V, [P; T'']
+    static constexpr int SM_SB = SM_VP + 2 * VP_STAGE;      // S^T bf16: DK rows x 128 B (MN-major B)
+    static constexpr int SM_UN = SM_SB + DK * 128;          // U' bf16 (MN-major B)
+    static constexpr int SM_UP = SM_UN + BLK;               // diag(exp(g_last - g) / |k|) U' bf16
+    static constexpr int SM_GV = SM_UP + BLK;               // gate vectors, 2 stages
+    static constexpr int SM_BAR = SM_GV + 2 * GV_STRIDE * 4;
+    static constexpr int SM_MISC = SM_BAR + NBAR * 8;       // TMEM base, abort flag
+    static constexpr int SMEM_BYTES = SM_MISC + 16 + 1024;  // + alignment slack
+    // TMEM columns: S^T (keys 128 h .. in columns 64 h ..), X, U, Y
+    static constexpr uint32_t TM_ST = 0, TM_X = 64 * NH, TM_U = TM_X + 64, TM_Y = TM_U + 64;
+    static constexpr uint32_t TM_COLS = TM_Y + 64 <= 256 ? 256 : 512;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    static_assert(SM_KT % 1024 == 0 && SM_VP % 1024 == 0 && SM_SB % 1024 == 0 &&
+                      SM_UN % 1024 == 0 && SM_UP % 1024 == 0 && VP_STAGE % 1024 == 0,
+                  "1024-byte aligned swizzled tiles");
+};
 
 enum {
-    B_QW_FULL = 0,      // TMA: [Q; W] (1 + tx)
-    B_QW_EMPTY = 1,     // chain commit after X (1)
-    B_K_FULL = 2,       // TMA: K (1 + tx)
-    B_K_EMPTY = 3,      // chain commit after the state update (1)
-    B_VP_FULL = 4,      // [2] TMA: V, [P; T''] (tx) + gate vectors (1)
-    B_VP_EMPTY = 6,     // [2] chain commit after Y (1)
-    B_U_FULL = 8,       // U-product commit (1)
-    B_U_EMPTY = 9,      // state warps that read U (4)
-    B_X_FULL = 10,      // chain commit after X (1)
-    B_U_READY = 11,     // state warps: U', decayed U' and the Y preload written (8)
-    B_ST_FULL = 12,     // chain commit after the state update (1)
-    B_S_READY = 13,     // state warps: S^T hand-off done (8)
-    B_Y_FULL = 14,      // chain commit after Y (1)
-    B_COUNT = 15
+    B_QW_FULL = 0,      // [2] TMA: [Q; W] (1 + tx)
+    B_QW_EMPTY = 2,     // [2] chain commit after X (1)
+    B_K_FULL = 4,       // [2] TMA: K (1 + tx)
+    B_K_EMPTY = 6,      // [2] chain commit after the state update (1)
+    B_VP_FULL = 8,      // [2] TMA: V, [P; T''] (tx) + gate vectors (1)
+    B_VP_EMPTY = 10,    // [2] chain commit after Y (1)
+    B_U_FULL = 12,      // U-product commit (1)
+    B_U_EMPTY = 13,     // state warps that read U (4)
+    B_X_FULL = 14,      // chain commit after X (1)
+    B_U_READY = 15,     // state warps: U', decayed U' and the Y preload written (8)
+    B_ST_FULL = 16,     // chain commit after the state update (1)
+    B_S_READY = 17,     // state warps: S^T hand-off done (8)
+    B_Y_FULL = 18,      // chain commit after Y (1)
+    B_COUNT = 19
 };
 static_assert(B_COUNT <= NBAR, "barrier slots");
 
@@ -420,11 +437,18 @@ struct Params {
     unsigned flags;
 };
 
-template <bool kNorm>
+template <int DK, bool kNorm>
 __global__ void __launch_bounds__(NTHREADS, 1)
 gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_pt, const Params p) {
+    using L = SeqDims<DK>;
+    constexpr int KB = L::KB, NH = L::NH, NQ = L::NQ;
+    constexpr int SM_QW = L::SM_QW, SM_KT = L::SM_KT, SM_VP = L::SM_VP, SM_SB = L::SM_SB,
+                  SM_UN = L::SM_UN, SM_UP = L::SM_UP, SM_GV = L::SM_GV, SM_BAR = L::SM_BAR,
+                  SM_MISC = L::SM_MISC;
+    constexpr uint32_t TM_ST = L::TM_ST, TM_X = L::TM_X, TM_U = L::TM_U, TM_Y = L::TM_Y,
+                       TM_COLS = L::TM_COLS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
@@ -542,26 +566,29 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (lane == 0) gv[GV_GL] = tc::ex2(glast);
             __syncwarp();
             if (lane == 0) mbar_arrive(cx.bar + B_VP_FULL + s);
-            // [Q; W] of chunk c once the X product of chunk c - 1 is done
-            if (c >= 1 && !tc::warp_wait(cx, B_QW_EMPTY, (c - 1) & 1)) break;
+            // [Q; W] of chunk c once the X product of chunk c - NQ is done
+            const int sq = c % NQ, pq = (c / NQ) & 1;
+            if (c >= NQ && !tc::warp_wait(cx, B_QW_EMPTY + sq, pq ^ 1)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(cx.bar + B_QW_FULL, 2 * KB * BLK);
+                uint8_t *qwb = base + SM_QW + sq * L::QW_BYTES;
+                mbar_arrive_expect_tx(cx.bar + B_QW_FULL + sq, L::QW_BYTES);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(base + SM_QW + kb * 2 * BLK, &tm_q, cx.bar + B_QW_FULL, kb * 64, h,
+                    tma_load_4d(qwb + kb * 2 * BLK, &tm_q, cx.bar + B_QW_FULL + sq, kb * 64, h,
                                 sp.off + t0, 0);
-                    tma_load_3d(base + SM_QW + kb * 2 * BLK + BLK, &tm_w, cx.bar + B_QW_FULL,
+                    tma_load_3d(qwb + kb * 2 * BLK + BLK, &tm_w, cx.bar + B_QW_FULL + sq,
                                 kb * 64, 0, tile);
                 }
             }
             n_qw = c + 1;
-            // K of chunk c once the state update of chunk c - 1 is done
-            if (c >= 1 && !tc::warp_wait(cx, B_K_EMPTY, (c - 1) & 1)) break;
+            // K of chunk c once the state update of chunk c - NQ is done
+            if (c >= NQ && !tc::warp_wait(cx, B_K_EMPTY + sq, pq ^ 1)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(cx.bar + B_K_FULL, KB * BLK);
+                uint8_t *ktb = base + SM_KT + sq * L::K_BYTES;
+                mbar_arrive_expect_tx(cx.bar + B_K_FULL + sq, L::K_BYTES);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
-                    tma_load_4d(base + SM_KT + kb * BLK, &tm_k, cx.bar + B_K_FULL, kb * 64, h,
+                    tma_load_4d(ktb + kb * BLK, &tm_k, cx.bar + B_K_FULL + sq, kb * 64, h,
                                 sp.off + t0, 0);
                 // a later chunk's tiles start streaming from DRAM into L2 now
                 const int cq = c + 2;
@@ -586,8 +613,10 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 while (!mbar_try_wait(bar, parity) && tc::now_ns() - t0 < tc::kTimeoutNs) {
                 }
             };
-            if (n_qw > 0) drain(cx.bar + B_QW_FULL, (n_qw - 1) & 1);
-            if (n_k > 0) drain(cx.bar + B_K_FULL, (n_k - 1) & 1);
+            for (int c = n_qw - NQ < 0 ? 0 : n_qw - NQ; c < n_qw; ++c)
+                drain(cx.bar + B_QW_FULL + c % NQ, (c / NQ) & 1);
+            for (int c = n_k - NQ < 0 ? 0 : n_k - NQ; c < n_k; ++c)
+                drain(cx.bar + B_K_FULL + c % NQ, (c / NQ) & 1);
             for (int c = n_vp - 2 < 0 ? 0 : n_vp - 2; c < n_vp; ++c)
                 drain(cx.bar + B_VP_FULL + (c & 1), (c >> 1) & 1);
         }
@@ -613,13 +642,14 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ---------------------------------------------- MMA: sequential chain
         const uint32_t idesc_x = idesc_bf16(128, DVT, false, true);
         const uint32_t idesc_s = idesc_bf16(128, DVT, true, true);
-        const uint32_t qw = smem_u32(base + SM_QW), kt = smem_u32(base + SM_KT),
-                       sb = smem_u32(base + SM_SB), un = smem_u32(base + SM_UN),
+        const uint32_t sb = smem_u32(base + SM_SB), un = smem_u32(base + SM_UN),
                        up = smem_u32(base + SM_UP);
         for (int c = 0; c < NT; ++c) {
-            const int s = c & 1;
+            const int s = c & 1, sq = c % NQ, pq = (c / NQ) & 1;
             const uint32_t vp = smem_u32(base + SM_VP + s * VP_STAGE);
-            if (!tc::warp_wait(cx, B_QW_FULL, c & 1)) break;
+            const uint32_t qw = smem_u32(base + SM_QW + sq * L::QW_BYTES);
+            const uint32_t kt = smem_u32(base + SM_KT + sq * L::K_BYTES);
+            if (!tc::warp_wait(cx, B_QW_FULL + sq, pq)) break;
             if (!tc::warp_wait(cx, B_S_READY, c & 1)) break;
             tc_fence_after();
             // X = [Q; W] S^T: A K-major (per key block, Q rows then W rows), B = S^T MN-major
@@ -629,25 +659,25 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     mma_bf16(tmem + TM_X, desc_sw128(qw + (kk >> 2) * 2 * BLK + (kk & 3) * 32, 16, 1024),
                              desc_sw128(sb + kk * 2048, 16, 1024), idesc_x, kk > 0);
                 mma_commit(cx.bar + B_X_FULL);
-                mma_commit(cx.bar + B_QW_EMPTY);
+                mma_commit(cx.bar + B_QW_EMPTY + sq);
             }
             __syncwarp();
             if (!tc::warp_wait(cx, B_U_READY, c & 1)) break;
-            if (!tc::warp_wait(cx, B_K_FULL, c & 1)) break;
+            if (!tc::warp_wait(cx, B_K_FULL + sq, pq)) break;
             if (!tc::warp_wait(cx, B_VP_FULL + s, (c >> 1) & 1)) break;
             tc_fence_after();
             if (lane == 0) {
                 // S^T_h += K_h^T (decayed U') for the key halves: A = K^T (MN-major,
                 // two 64-key blocks 8 KiB apart), B = decayed U' (MN-major)
 #pragma unroll
-                for (int hk = 0; hk < 2; ++hk)
+                for (int hk = 0; hk < NH; ++hk)
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
                         mma_bf16(tmem + TM_ST + 64 * hk,
                                  desc_sw128(kt + hk * 2 * BLK + kk * 2048, BLK, 1024),
                                  desc_sw128(up + kk * 2048, 16, 1024), idesc_s, 1u);
                 mma_commit(cx.bar + B_ST_FULL);
-                mma_commit(cx.bar + B_K_EMPTY);
+                mma_commit(cx.bar + B_K_EMPTY + sq);
                 // Y += [P; T''] U'  (Y holds gamma Q S^T; rows 64-127 unused)
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
@@ -660,25 +690,29 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
     } else if (warp >= W_STATE0) {
         // ------------------------------------------------------------ STATE
-        // warp w reads TMEM lanes 32 (w % 4) .. + 31; hf selects the key half of
-        // S^T (hand-off) or the 32-column half of X / U / Y (epilogues)
+        // warp w reads TMEM lanes 32 (w % 4) .. + 31; hf selects the 32-column
+        // half of X / U / Y (epilogues) and, in the hand-off, the key half of S^T
+        // (Dk = 256: 64 value columns of keys 128 hf + lane) or the 32 value
+        // columns (Dk = 128)
+        constexpr int NPC = 2 * NH;  // 16-column pieces of S^T per thread
         const int q = warp & 3, hf = (warp - W_STATE0) >> 2;
         const int lrow = 32 * q + lane;
-        const int key = 128 * hf + lrow;  // this thread's row of S^T in the hand-off
+        const int key = (NH == 2 ? 128 * hf : 0) + lrow;  // this thread's row of S^T
+        const int col0 = NH == 2 ? 0 : 32 * hf;           // its first value column
         const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t st_col = TM_ST + 64 * hf;
+        const uint32_t st_col = TM_ST + (NH == 2 ? 64 * hf : 0) + col0;
         uint8_t *sbuf = base + SM_SB;
         // initial state: S^T row `key` = S0[v0 .. v0 + 63][key]; TMEM copy pre-scaled by gamma_last
         {
             const bool have = tc::warp_wait(cx, B_VP_FULL + 0, 0);
             const float gl = gv_all[GV_GL];
 #pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 0; pc < NPC; ++pc) {
                 float sv[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + 16 * pc + j) * DK + key] : 0.f;
-                tc::store16_bf16(sbuf, key, pc, sv);
+                    sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + col0 + 16 * pc + j) * DK + key] : 0.f;
+                tc::store16_bf16(sbuf, key, col0 / 16 + pc, sv);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) sv[j] *= gl;
                 if (have) tmem_st16(lane_addr + st_col + 16 * pc, sv);
@@ -755,28 +789,28 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     have = tc::warp_wait(cx, B_VP_FULL + (s ^ 1), ((c + 1) >> 1) & 1);
                     gl = gv_all[(s ^ 1) * GV_STRIDE + GV_GL];
                 }
-                float sv[4][16];
+                float sv[NPC][16];
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc) tmem_ld16(lane_addr + st_col + 16 * pc, sv[pc]);
+                for (int pc = 0; pc < NPC; ++pc) tmem_ld16(lane_addr + st_col + 16 * pc, sv[pc]);
                 tmem_wait_ld();
                 if (!last) {
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc) tc::store16_bf16(sbuf, key, pc, sv[pc]);
+                    for (int pc = 0; pc < NPC; ++pc) tc::store16_bf16(sbuf, key, col0 / 16 + pc, sv[pc]);
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
+                    for (int pc = 0; pc < NPC; ++pc)
 #pragma unroll
                         for (int j = 0; j < 16; ++j) sv[pc][j] *= gl;
                     if (have)
 #pragma unroll
-                        for (int pc = 0; pc < 4; ++pc) tmem_st16(lane_addr + st_col + 16 * pc, sv[pc]);
+                        for (int pc = 0; pc < NPC; ++pc) tmem_st16(lane_addr + st_col + 16 * pc, sv[pc]);
                     fence_async_smem();
                     tmem_wait_st();
                 } else if (p.S_T) {
 #pragma unroll
-                    for (int pc = 0; pc < 4; ++pc)
+                    for (int pc = 0; pc < NPC; ++pc)
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            p.S_T[(head * p.Dv + v0 + 16 * pc + j) * DK + key] = sv[pc][j];
+                            p.S_T[(head * p.Dv + v0 + col0 + 16 * pc + j) * DK + key] = sv[pc][j];
                 }
                 tc_fence_before();
                 tc::warp_arrive(cx, B_S_READY);
@@ -819,12 +853,12 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
 }
 
-// W tiles, [n_tiles, 64, 256] bf16: box of 64 keys x 64 rows of one tile, 128B swizzle.
-bool make_map_w(CUtensorMap *m, const void *ptr, long long n_tiles) {
+// W tiles, [n_tiles, 64, DK] bf16: box of 64 keys x 64 rows of one tile, 128B swizzle.
+bool make_map_w(CUtensorMap *m, const void *ptr, long long n_tiles, int DK) {
     auto enc = tc::encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)C, (cuuint64_t)n_tiles};
-    cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)W_ELEMS * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)C * DK * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)C, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
@@ -838,67 +872,39 @@ bool make_map_w(CUtensorMap *m, const void *ptr, long long n_tiles) {
 // Workspace: [chunk offsets and launch order, variable lengths only][[P; T'']
 // tiles][W tiles][1/|q|, 1/|k| per chunk row, normalising only].
 size_t tcw_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                                unsigned flags) {
+                                unsigned flags, int Dk) {
     const size_t tiles = (size_t)total_chunks * H;
     const size_t norm = (flags & kFlagL2Norm) ? tiles * 2 * tc::C * sizeof(float) : 0;
     return tc_offsets_bytes(n_seq, varlen) +
-           tiles * (tcw::PT_ELEMS + tcw::W_ELEMS) * sizeof(__nv_bfloat16) + norm;
+           tiles * (tcw::PT_ELEMS + (size_t)tc::C * Dk) * sizeof(__nv_bfloat16) + norm;
 }
 
-cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
-                                  const float *log_alpha, const float *beta, const float *S0,
-                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
-                                  const int *cu_seqlens, long long total_chunks, int H, int Dv,
-                                  unsigned flags, void *workspace, cudaStream_t st) {
-    const bool varlen = cu_seqlens != nullptr;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
-    const size_t tiles = (size_t)total_chunks * H;
-    auto *pt = reinterpret_cast<__nv_bfloat16 *>(ws + tc_offsets_bytes(n_seq, varlen));
-    __nv_bfloat16 *wt = pt + tiles * tcw::PT_ELEMS;
-    float *rqk = (flags & kFlagL2Norm) ? reinterpret_cast<float *>(wt + tiles * tcw::W_ELEMS)
-                                       : nullptr;
-    const long long n_maps = total_chunks > 0 ? (long long)tiles : 1;
-    CUtensorMap mq, mk, mv, mw, mp;
-    if (!tc::make_map(&mq, q, 1, (int)total_T, H, tcw::DK) ||
-        !tc::make_map(&mk, k, 1, (int)total_T, H, tcw::DK) ||
-        !tc::make_map(&mv, v, 1, (int)total_T, H, Dv) || !tcw::make_map_w(&mw, wt, n_maps) ||
-        !tc::make_map_tt(&mp, pt, n_maps))
-        return cudaErrorInvalidValue;
-    if (varlen) {
-        const cudaError_t e0 = launch_seq_schedule(cu_seqlens, n_seq, cu_chunks,
-                                                   cu_chunks + n_seq + 1, st);
-        if (e0 != cudaSuccess) return e0;
-    }
-    const tc::Seqs sq{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
-                      n_seq};
-    tcw::Params p;
-    p.log_alpha = log_alpha;
-    p.S0 = S0;
-    p.o = static_cast<__nv_bfloat16 *>(o);
-    p.S_T = S_T;
-    p.rqk = rqk;
-    p.sq = sq;
-    p.H = H;
-    p.Dv = Dv;
-    p.flags = flags;
-    const bool norm = (flags & kFlagL2Norm) != 0;
-    auto *ut = norm ? tcw::gdn_utw_kernel<true> : tcw::gdn_utw_kernel<false>;
-    auto *seq = norm ? tcw::gdn_chunk_tcw_kernel<true> : tcw::gdn_chunk_tcw_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tcw::UT_SMEM);
+namespace tcw {
+
+template <int DK, bool kNorm>
+cudaError_t launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                   const CUtensorMap &mw, const CUtensorMap &mp, const Params &p,
+                   const float *log_alpha, const float *beta, __nv_bfloat16 *pt,
+                   __nv_bfloat16 *wt, float *rqk, long long total_chunks, int n_seq,
+                   cudaStream_t st) {
+    auto *ut = gdn_utw_kernel<DK, kNorm>;
+    auto *seq = gdn_chunk_tcw_kernel<DK, kNorm>;
+    constexpr int ut_smem = UtDims<DK>::UT_SMEM, seq_smem = SeqDims<DK>::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize, ut_smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, tcw::SMEM_BYTES);
+    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
     if (e != cudaSuccess) return e;
     if (total_chunks > 0)
-        ut<<<dim3((unsigned)total_chunks, H, 1), tcw::UT_THREADS, tcw::UT_SMEM, st>>>(
-            mq, mk, log_alpha, beta, pt, wt, rqk, sq, H, flags);
+        ut<<<dim3((unsigned)total_chunks, p.H, 1), UT_THREADS, ut_smem, st>>>(
+            mq, mk, log_alpha, beta, pt, wt, rqk, p.sq, p.H, p.flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
+    // programmatic dependent launch: the CTAs may set up while the UT kernel
+    // drains; the TMA warp waits for its completion before the first load
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(Dv / tcw::DVT, H, n_seq);
-    cfg.blockDim = dim3(tcw::NTHREADS);
-    cfg.dynamicSmemBytes = tcw::SMEM_BYTES;
+    cfg.gridDim = dim3(p.Dv / DVT, p.H, n_seq);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = seq_smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -908,6 +914,57 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
     e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mw, mp, p);
     if (e != cudaSuccess) return e;
     return cudaPeekAtLastError();
+}
+
+}  // namespace tcw
+
+cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
+                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
+                                  int Dv, unsigned flags, void *workspace, cudaStream_t st) {
+    if (Dk != 128 && Dk != 256) return cudaErrorInvalidValue;
+    const bool varlen = cu_seqlens != nullptr;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
+    const size_t tiles = (size_t)total_chunks * H;
+    auto *pt = reinterpret_cast<__nv_bfloat16 *>(ws + tc_offsets_bytes(n_seq, varlen));
+    __nv_bfloat16 *wt = pt + tiles * tcw::PT_ELEMS;
+    float *rqk = (flags & kFlagL2Norm) ? reinterpret_cast<float *>(wt + tiles * tc::C * Dk)
+                                       : nullptr;
+    const long long n_maps = total_chunks > 0 ? (long long)tiles : 1;
+    CUtensorMap mq, mk, mv, mw, mp;
+    if (!tc::make_map(&mq, q, 1, (int)total_T, H, Dk) ||
+        !tc::make_map(&mk, k, 1, (int)total_T, H, Dk) ||
+        !tc::make_map(&mv, v, 1, (int)total_T, H, Dv) || !tcw::make_map_w(&mw, wt, n_maps, Dk) ||
+        !tc::make_map_tt(&mp, pt, n_maps))
+        return cudaErrorInvalidValue;
+    if (varlen) {
+        const cudaError_t e0 = launch_seq_schedule(cu_seqlens, n_seq, cu_chunks,
+                                                   cu_chunks + n_seq + 1, st);
+        if (e0 != cudaSuccess) return e0;
+    }
+    tcw::Params p;
+    p.log_alpha = log_alpha;
+    p.S0 = S0;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.S_T = S_T;
+    p.rqk = rqk;
+    p.sq = tc::Seqs{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
+                    n_seq};
+    p.H = H;
+    p.Dv = Dv;
+    p.flags = flags;
+    const bool norm = (flags & kFlagL2Norm) != 0;
+    if (Dk == 256)
+        return norm ? tcw::launch<256, true>(mq, mk, mv, mw, mp, p, log_alpha, beta, pt, wt, rqk,
+                                             total_chunks, n_seq, st)
+                    : tcw::launch<256, false>(mq, mk, mv, mw, mp, p, log_alpha, beta, pt, wt, rqk,
+                                              total_chunks, n_seq, st);
+    return norm ? tcw::launch<128, true>(mq, mk, mv, mw, mp, p, log_alpha, beta, pt, wt, rqk,
+                                         total_chunks, n_seq, st)
+                : tcw::launch<128, false>(mq, mk, mv, mw, mp, p, log_alpha, beta, pt, wt, rqk,
+                                          total_chunks, n_seq, st);
 }
 
 cudaError_t read_and_clear_device_error_wide(unsigned int *flag) {

@@ -77,11 +77,16 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype
     return GDN_PATH_SIMT;
 }
 
+int gdn_chunk_fwd_variant(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
+    if (gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype) != GDN_PATH_TCGEN05) return 0;
+    return gdn::tc_precomputed(B, H, Dk, Dv) ? 2 : 1;
+}
+
 size_t gdn_chunk_fwd_workspace_size_ex(int B, int T, int H, int Dk, int Dv, int chunk,
                                        gdn_dtype_t dtype, unsigned flags) {
     const int path = gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype);
     if (flags & ~kKnownFlags) return 0;
-    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H, flags, Dk);
+    if (path == GDN_PATH_TCGEN05) return gdn::tc_workspace_bytes(B, T, H, flags, Dk, Dv);
     if (path == GDN_PATH_SIMT) {
         const size_t base = gdn::simt_workspace_bytes(B, T, H, chunk);
         return flags ? align256(base) + gdn::prologue_bytes(B, T, H, Dk, dtype == GDN_BF16, flags)
@@ -178,7 +183,7 @@ size_t gdn_chunk_fwd_varlen_workspace_size(const int *cu_seqlens_host, int N, in
     if (N == 0 || H == 0 || off.total == 0) return 0;
     const bool bf16 = dtype == GDN_BF16;
     if (gdn::tc_supported(N, off.max_len, H, Dk, Dv, chunk, bf16))
-        return gdn::tc_workspace_bytes_seqs(N, off.chunks64, H, true, flags, Dk);
+        return gdn::tc_workspace_bytes_seqs(N, off.chunks64, H, true, flags, Dk, Dv);
     // CUDA-core path: one sequence at a time (scratch for the longest), prologue once
     const size_t base = gdn::simt_workspace_bytes(1, off.max_len, H, chunk);
     return flags ? align256(base) +

@@ -67,15 +67,23 @@ cudaError_t launch_decode_cw(const void *q, const void *k, const void *v, const 
                              const float *bg, const float *wg, float *S, void *o, int B, int H,
                              int Dk, int Dv, bool bf16, cudaStream_t st);
 
-// tcgen05 chunkwise forward (bf16, chunk 64, Dv a multiple of 64; Dk = 128 in
-// chunk_tc.cu, Dk = 256 in chunk_tc_wide.cu, chosen by Dk inside these calls).
-// Dk = 128: the workspace holds one bf16 [T'; T''] tile (128 x 64) per chunk of
-// every head (and 1/|k| per token with the L2-normalisation flag).  Dk = 256:
-// one bf16 [P; T''] tile (128 x 64) and one bf16 W tile (64 x 256) per chunk of
-// every head (and 1/|q|, 1/|k| per token with the flag).
-constexpr int tcw_dk = 256;
+// tcgen05 chunkwise forward (bf16, chunk 64, Dk = 128 or 256, Dv a multiple of
+// 64), in one of two variants chosen inside these calls from the sizes:
+//  - fused (chunk_tc.cu, Dk = 128): the parallel kernel writes one bf16
+//    [T'; T''] tile (128 x 64) per chunk of every head (and 1/|k| per token
+//    with the L2-normalisation flag); the sequential kernel forms Q K^T and the
+//    WY factors itself.  Chosen when the sequential grid fills most of the GPU.
+//  - precomputed (chunk_tc_wide.cu, Dk = 256 always, Dk = 128 when the
+//    sequential grid would leave most SMs idle): the parallel kernel also forms
+//    the gated Q K^T and W, writing one bf16 [P; T''] tile (128 x 64) and one
+//    bf16 W tile (64 x Dk) per chunk of every head (and 1/|q|, 1/|k| per token
+//    with the flag); the sequential kernel keeps only the state-dependent
+//    products, a shorter chain per chunk.
 bool tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
-size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk = 128);
+bool tc_precomputed(int n_seq, int H, int Dk, int Dv);
+size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk, int Dv);
+// The fused variant's workspace (the backward's state recompute uses it).
+size_t tc_workspace_bytes_fused(int B, int T, int H, unsigned flags);
 // S_hist (optional): the state entering every chunk, [B*H][NT][Dv][Dk] float32.
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                             const float *beta, const float *S0, void *o, float *S_T, int B, int T,
@@ -86,7 +94,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 // total_chunks = sum of ceil(length / 64).  The workspace then starts with the
 // per-sequence chunk offsets (computed on the device).
 size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                               unsigned flags, int Dk = 128);
+                               unsigned flags, int Dk, int Dv);
 cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
@@ -100,14 +108,14 @@ cudaError_t launch_chunk_tc_seqs(const void *q, const void *k, const void *v,
 size_t tc_offsets_bytes(int n_seq, bool varlen);
 cudaError_t launch_seq_schedule(const int *cu_seqlens, int n_seq, int *cu_chunks, int *order,
                                 cudaStream_t st);
-// The Dk = 256 path (chunk_tc_wide.cu); reached through the tc_* calls above.
+// The precomputed variant (chunk_tc_wide.cu); reached through the tc_* calls above.
 size_t tcw_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool varlen,
-                                unsigned flags);
+                                unsigned flags, int Dk);
 cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                                   const float *log_alpha, const float *beta, const float *S0,
                                   void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
-                                  const int *cu_seqlens, long long total_chunks, int H, int Dv,
-                                  unsigned flags, void *workspace, cudaStream_t st);
+                                  const int *cu_seqlens, long long total_chunks, int H, int Dk,
+                                  int Dv, unsigned flags, void *workspace, cudaStream_t st);
 
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).

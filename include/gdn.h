@@ -72,6 +72,15 @@ typedef enum {
                               needs a workspace */
 } gdn_path_t;
 
+/* Which of the two tcgen05 variants a gdn_chunk_fwd call with these sizes runs
+ * (the pages have no counterpart; both compute the same result):
+ * 0 = not the tcgen05 path (or invalid sizes), 1 = fused (the sequential kernel
+ * forms Q K^T and the WY factors itself; Dk = 128 when the sequential grid of
+ * Dv / 64 x H x B CTAs fills most of the GPU), 2 = precomputed (the parallel
+ * kernel also forms the gated Q K^T and W per chunk; Dk = 256, and Dk = 128 with
+ * fewer than 74 sequential CTAs).  The workspace size depends on it. */
+int gdn_chunk_fwd_variant(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype);
+
 /* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0
  * (a zero size is an empty problem and is not an error); B, H <= 65535 and
  * B * H * (T + 64) <= 2^40 (so that no byte count derived from the sizes can

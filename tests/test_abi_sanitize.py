@@ -45,12 +45,15 @@ cudaError_t launch_chunk_simt(const void *, const void *, const void *, const fl
                               const float *, void *, float *, int, int, int, int, int, int, bool,
                               void *, cudaStream_t) { return ok(); }
 bool tc_supported(int, int, int, int, int, int, bool) { return false; }
-size_t tc_workspace_bytes(int B, int T, int H, unsigned, int Dk) {
+bool tc_precomputed(int, int, int Dk, int) { return Dk == 256; }
+size_t tc_workspace_bytes(int B, int T, int H, unsigned, int Dk, int) {
     return (size_t)B * H * (((size_t)T + 63) / 64) * (Dk == 256 ? 49152 : 16384); }
+size_t tc_workspace_bytes_fused(int B, int T, int H, unsigned) {
+    return (size_t)B * H * (((size_t)T + 63) / 64) * 16384; }
 cudaError_t launch_chunk_tc(const void *, const void *, const void *, const float *, const float *,
                             const float *, void *, float *, int, int, int, int, int, unsigned,
                             void *, cudaStream_t, float *) { return ok(); }
-size_t tc_workspace_bytes_seqs(int n, long long chunks, int H, bool, unsigned, int Dk) {
+size_t tc_workspace_bytes_seqs(int n, long long chunks, int H, bool, unsigned, int Dk, int) {
     return ((size_t)n + 1) * 8 + (size_t)chunks * H * (Dk == 256 ? 49152 : 16384); }
 cudaError_t launch_chunk_tc_seqs(const void *, const void *, const void *, const float *,
                                  const float *, const float *, void *, float *, int, int, long long,

@@ -68,11 +68,14 @@ def test_gate_laws_bf16_small(gdn, gate_law):
 
 
 def test_tc_path_workspace(gdn):
-    # one bf16 [T'; T''] tile (128 x 64) per chunk of every (batch, head)
-    B, T, H = 2, 130, 3
-    assert gdn.chunk_fwd_path(B, T, H, 128, 128, 64, torch.bfloat16) == "tcgen05"
-    assert gdn.chunk_fwd_workspace_size(B, T, H, 128, 128, 64, torch.bfloat16) == \
-        B * H * 3 * 128 * 64 * 2
+    # fused variant: one bf16 [T'; T''] tile (128 x 64) per chunk of every (batch,
+    # head); precomputed variant: one [P; T''] tile (128 x 64) and one W tile (64 x 128)
+    B, T = 2, 130
+    for H, variant, per_chunk in ((40, "fused", 128 * 64), (3, "precomputed", 2 * 128 * 64)):
+        assert gdn.chunk_fwd_path(B, T, H, 128, 128, 64, torch.bfloat16) == "tcgen05"
+        assert gdn.chunk_fwd_variant(B, T, H, 128, 128, 64, torch.bfloat16) == variant
+        assert gdn.chunk_fwd_workspace_size(B, T, H, 128, 128, 64, torch.bfloat16) == \
+            B * H * 3 * per_chunk * 2
 
 
 def test_tc_path_ignores_workspace_contents(gdn):

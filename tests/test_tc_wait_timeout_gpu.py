@@ -1,6 +1,6 @@
 """Failure detection of the tcgen05 chunkwise forward, made to happen without a
-GPU fault: the test hook gdn_debug_withhold_first_arrival makes the sequential
-kernel's TMA warp withhold the arrival that publishes its first stage, so every
+GPU fault: the test hook gdn_debug_withhold_first_arrival makes the fused
+variant's sequential kernel's TMA warp withhold the arrival that publishes its first stage, so every
 warp's first bounded wait (about two seconds) runs out.  The CTAs record the
 error flag, stop, drain their copies and release their tensor memory;
 gdn_check_device_status must report it, and the next call (hook off) must run
@@ -25,8 +25,11 @@ def gdn():
 
 
 def test_bounded_wait_runs_out_and_context_survives(gdn):
-    w = I.workload("bf16_T2k", B=1, H=2, T=128, Dv=64, s0_law="normal002", seed=91)
+    # the hook is in the fused variant's sequential kernel: 80 CTAs (heads x one
+    # value slice) select it
+    w = I.workload("bf16_T2k", B=1, H=80, T=128, Dv=64, s0_law="normal002", seed=91)
     assert gdn.chunk_fwd_path(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16) == "tcgen05"
+    assert gdn.chunk_fwd_variant(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16) == "fused"
     inp = I.chunk_inputs(w)
     d = {n: (t.cuda() if t is not None else None) for n, t in inp.items()}
     gdn.check_device_status()  # a clean flag to start from

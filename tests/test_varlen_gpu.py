@@ -117,16 +117,23 @@ def test_varlen_serving_mix_sampled_heads(gdn):
     _check(o, S, inp, TOL_BF16, heads=[0, 5, c["H"] - 1])
 
 
-def test_varlen_tcgen05_workspace_size(gdn):
-    """One bf16 [T'; T''] tile (128 x 64) per chunk of 64 and head, after the
-    per-sequence chunk offsets: the size follows the chunks, not the tokens."""
-    f = lambda cu: gdn.chunk_fwd_varlen_workspace_size(cu, 4, 128, 128, 64, torch.bfloat16)
-    tile = 4 * 128 * 64 * 2
+@pytest.mark.parametrize("H,variant", [(4, "precomputed"), (20, "fused")])
+def test_varlen_tcgen05_workspace_size(gdn, H, variant):
+    """Per chunk of 64 and head, after the per-sequence chunk offsets: one bf16
+    [T'; T''] tile (128 x 64) in the fused variant, one [P; T''] tile and one W
+    tile (64 x 128) in the precomputed one (chosen with few sequential CTAs, two
+    sequences x H heads x 2 value slices here): the size follows the chunks, not
+    the tokens."""
+    f = lambda cu, **kw: gdn.chunk_fwd_varlen_workspace_size(cu, H, 128, 128, 64,
+                                                             torch.bfloat16, **kw)
+    assert gdn.chunk_fwd_variant(2, 66, H, 128, 128, 64, torch.bfloat16) == variant
+    tile = H * 128 * 64 * 2 * (2 if variant == "precomputed" else 1)
     assert f([0, 64, 128]) == f([0, 1, 2]) == 256 + 2 * tile
     assert f([0, 1, 66]) == 256 + 3 * tile
-    # with L2 normalisation the per-row key scales (float32) follow the tiles
-    assert gdn.chunk_fwd_varlen_workspace_size([0, 1, 66], 4, 128, 128, 64, torch.bfloat16,
-                                               l2norm_qk=True) == 256 + 3 * tile + 3 * 4 * 64 * 4
+    # with L2 normalisation the per-row scales (float32) follow the tiles: 1/|k|
+    # in the fused variant, 1/|q| and 1/|k| in the precomputed one
+    rows = 64 * 4 * (2 if variant == "precomputed" else 1)
+    assert f([0, 1, 66], l2norm_qk=True) == 256 + 3 * tile + 3 * H * rows
 
 
 def test_varlen_device_offsets_give_the_same_bits(gdn):

@@ -74,15 +74,18 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(gdn):
     assert _noalloc(gdn, d, None, None, w, 64) == 2  # GDN_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("B,H,T", [(1, 2, 512), (1, 16, 2048)], ids=["256KiB", "8MiB"])
-def test_noalloc_tcgen05_path_matches_oracle(gdn, B, H, T):
+@pytest.mark.parametrize("B,H,T,variant,size", [(1, 2, 256, "precomputed", 256 << 10),
+                                                 (2, 64, 256, "fused", 8 << 20)],
+                         ids=["precomputed-256KiB", "fused-8MiB"])
+def test_noalloc_tcgen05_path_matches_oracle(gdn, B, H, T, variant, size):
     # bf16, Dk = 128, chunk 64: the tcgen05 path, its tiles in the fixed array;
-    # B1 H16 T2048 needs the whole 8 MiB
+    # B2 H64 T256 (fused) needs the whole 8 MiB
     from parity import head_slices, oracle_chunk
     w = I.workload("bf16_T2k", B=B, H=H, T=T, s0_law="normal002")
     assert gdn.chunk_fwd_path(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16) == "tcgen05"
+    assert gdn.chunk_fwd_variant(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16) == variant
     need = gdn.chunk_fwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, 64, torch.bfloat16)
-    assert 0 < need <= SCRATCH
+    assert need == size <= SCRATCH
     units = I.sample_units(w, min(4, B * H))
     for seed in (31, 32):
         inp = I.chunk_inputs(w, seed=seed)
