@@ -1,0 +1,364 @@
+// Channel-wise gates (the Gated DeltaNet-2 reading, "Gated DeltaNet-2:
+// Decoupling Erase and Write in Linear Attention", abstract: a decay per key
+// channel, an erase gate on the key side and a write gate on the value side,
+// "channel-wise decay absorbed into asymmetric erase factors"),
+//   S_t = S_{t-1} Diag(alpha_t) (I - (b_t o k_t) k_t^T) + (w_t o v_t) k_t^T,  o_t = S_t q_t,
+// on the tensor cores: bf16 q/k/v/o, Dk = 128, chunk 64, Dv a multiple of 64.
+//
+// Per chunk (rows r, i; Lam_r the running sum of log alpha over the chunk, per
+// key channel; S the incoming state):
+//   A_ri = sum_j b_rj k_rj k_ij exp(Lam_rj - Lam_ij)   (i < r),   T = (I + A)^-1
+//   P_ri = sum_j q_rj k_ij exp(Lam_rj - Lam_ij)        (i <= r)
+//   W    = T (b o K o exp(Lam)),   U = T (w o V),   U' = U - W S^T
+//   O    = (Q o exp(Lam)) S^T + P U'
+//   S   <- S Diag(exp(Lam_last)) + U'^T (K o exp(Lam_last - Lam))
+// which is the shape of the scalar precomputed variant (chunk_tc_wide.cu) with
+// Q, K and V replaced by Q o exp(Lam), K o exp(Lam_last - Lam) and w o V and the
+// state's decay a vector over the key channels.  Two kernels:
+//  1. gdn_ut_cw_kernel, one CTA of 8 warps per (chunk, head, batch), all chunks
+//     in parallel.  The decays between rows are channel-wise, so they cannot be
+//     taken out of the key products as row and column scales; split the chunk
+//     into 16-row blocks:
+//       - a block I against an earlier block J factors through the reference
+//         row m = 16 I - 1 between them: exp(Lam_r - Lam_i) =
+//         exp(Lam_r - Lam_m) exp(Lam_m - Lam_i), both factors <= 1 (no overflow
+//         for any decay), so A_IJ = L_I R_I,J^T and P_IJ = M_I R_I,J^T with
+//         L_I = b o K_I o 2^(Lam_I - Lam_m), M_I = Q_I o 2^(Lam_I - Lam_m),
+//         R = K_J o 2^(Lam_m - Lam_J): bf16 mma.sync products of 16-row blocks
+//         (the factorisation is per block pair; 16 rows is below the M = 64 of
+//         a tcgen05 product);
+//       - the four diagonal blocks are summed directly over the channels in
+//         float32 (exp2 of the exact differences), one warp pair per block;
+//     then the blocked UT solve, W = T (b o K o 2^Lam) (mma.sync), and the
+//     operands of the sequential kernel: [P; T''] (T'' = T with the columns of
+//     rows past the end zeroed), W, Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
+//     and 2^Lam_last per key channel, into the workspace.
+//  2. the precomputed variant's sequential tcgen05 kernel in its channel-wise
+//     mode (launch_chunk_tcw_seq_cw in chunk_tc_wide.cu).
+// Lam is kept in log2 units (exp2 of the hardware approximation).  Rows past a
+// ragged end are zero tokens (k = q = b = w = 0, log alpha = 0).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace cwt {
+
+using namespace sm100;
+using tc::C;
+using tc::LDA;
+
+constexpr int DK = 128;
+constexpr int THREADS = 256;                  // 8 warps
+constexpr int LDF = DK + 1;                   // float32 row stride of the per-channel arrays
+constexpr int LDT = C + 8;                    // bf16 row stride of T for the W product
+constexpr int SM_K = 0;                       // k (f32, 64 x LDF)
+constexpr int SM_Q = SM_K + C * LDF * 4;      // q
+constexpr int SM_BK = SM_Q + C * LDF * 4;     // b o k
+constexpr int SM_LM = SM_BK + C * LDF * 4;    // Lam log2(e) (running sums per channel)
+constexpr int SM_AF = SM_LM + C * LDF * 4;    // A (f32, 64 x LDA); then T as bf16
+constexpr int SM_TF = SM_AF + C * LDA * 4;    // T (f32)
+constexpr int SM_PF = SM_TF + C * LDA * 4;    // P (f32)
+constexpr int NPAIR = 136;                    // (r, i), i <= r, of a 16 x 16 block
+constexpr int SM_DS = SM_PF + C * LDA * 4;    // diagonal blocks: the second channel half's sums
+constexpr int SMEM = SM_DS + 4 * NPAIR * 2 * 4;
+constexpr int PT_ELEMS = 2 * C * C, W_ELEMS = C * DK;
+constexpr float LOG2E = 1.4426950408889634f;
+static_assert(SM_AF % 16 == 0 && SM_TF % 16 == 0 && SM_PF % 16 == 0 && SM_DS % 16 == 0,
+              "16-byte aligned buffers");
+static_assert(SMEM <= 227 * 1024, "shared memory budget");
+
+__global__ void __launch_bounds__(THREADS, 1)
+gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                 const __nv_bfloat16 *__restrict__ v, const float *__restrict__ la,
+                 const float *__restrict__ bg, const float *__restrict__ wg,
+                 __nv_bfloat16 *__restrict__ qe, __nv_bfloat16 *__restrict__ kd,
+                 __nv_bfloat16 *__restrict__ vw, __nv_bfloat16 *__restrict__ pt,
+                 __nv_bfloat16 *__restrict__ wt, float *__restrict__ glk, int T, int H, int Dv) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    // the sequential kernel that follows may be scheduled now (it waits for this
+    // grid's completion before it reads what this kernel writes)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int NT = (T + C - 1) / C;
+    const int t0 = c * C, n = min(C, T - t0);
+    const size_t tok0 = (size_t)b * T + t0;
+    const size_t tile = ((size_t)b * NT + c) * H + h;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    float *KF = reinterpret_cast<float *>(sm + SM_K);
+    float *QF = reinterpret_cast<float *>(sm + SM_Q);
+    float *BK = reinterpret_cast<float *>(sm + SM_BK);
+    float *LM = reinterpret_cast<float *>(sm + SM_LM);
+    float *AF = reinterpret_cast<float *>(sm + SM_AF);
+    float *TF = reinterpret_cast<float *>(sm + SM_TF);
+    float *PF = reinterpret_cast<float *>(sm + SM_PF);
+    float *DS = reinterpret_cast<float *>(sm + SM_DS);
+    __nv_bfloat16 *TB = reinterpret_cast<__nv_bfloat16 *>(sm + SM_AF);
+
+    // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread
+    // -> (channel, half of the rows), so each row is read as 128 consecutive values
+    const int jc = tid & (DK - 1), half = tid >> 7;
+    for (int rr = 0; rr < C / 2; ++rr) {
+        const int r = half * (C / 2) + rr;
+        float kv = 0.f, qv = 0.f, bv = 0.f, lv = 0.f;
+        if (r < n) {
+            const size_t off = ((tok0 + r) * H + h) * DK + jc;
+            kv = __bfloat162float(k[off]);
+            qv = __bfloat162float(q[off]);
+            bv = bg[off];
+            lv = la[off];
+        }
+        KF[r * LDF + jc] = kv;
+        QF[r * LDF + jc] = qv;
+        BK[r * LDF + jc] = bv * kv;
+        LM[r * LDF + jc] = lv * LOG2E;
+    }
+    __syncthreads();
+    {   // running sums over the rows, per channel: each half locally, then the
+        // second half adds the first half's total
+        float acc = 0.f;
+        for (int rr = 0; rr < C / 2; ++rr) {
+            const int r = half * (C / 2) + rr;
+            acc += LM[r * LDF + jc];
+            LM[r * LDF + jc] = acc;
+        }
+    }
+    __syncthreads();
+    if (half == 1) {
+        const float base = LM[(C / 2 - 1) * LDF + jc];
+        for (int r = C / 2; r < C; ++r) LM[r * LDF + jc] += base;
+    }
+    __syncthreads();
+
+    // diagonal 16-blocks, summed directly: warps 2I and 2I+1 take block I, each
+    // half of the channels; lane -> pairs p = lane + 32 m of the block's lower
+    // triangle (p = r (r + 1) / 2 + i)
+    {
+        const int I = warp >> 1, ch = warp & 1;
+        int pr[5], pi[5];
+        float accA[5], accP[5];
+#pragma unroll
+        for (int m = 0; m < 5; ++m) {
+            const int p = lane + 32 * m;
+            int r = 0;
+            while ((r + 1) * (r + 2) / 2 <= p) ++r;
+            pr[m] = 16 * I + r;
+            pi[m] = 16 * I + (p - r * (r + 1) / 2);
+            accA[m] = accP[m] = 0.f;
+        }
+#pragma unroll 2
+        for (int jj = 0; jj < DK / 2; ++jj) {
+            const int j = (DK / 2) * ch + jj;
+#pragma unroll
+            for (int m = 0; m < 5; ++m) {
+                if (lane + 32 * m < NPAIR) {
+                    const int R = pr[m], Ii = pi[m];
+                    const float e = tc::ex2(LM[R * LDF + j] - LM[Ii * LDF + j]) * KF[Ii * LDF + j];
+                    accA[m] = fmaf(BK[R * LDF + j], e, accA[m]);
+                    accP[m] = fmaf(QF[R * LDF + j], e, accP[m]);
+                }
+            }
+        }
+        float *ds = DS + I * NPAIR * 2;
+        if (ch == 1) {
+#pragma unroll
+            for (int m = 0; m < 5; ++m)
+                if (lane + 32 * m < NPAIR) {
+                    ds[2 * (lane + 32 * m)] = accA[m];
+                    ds[2 * (lane + 32 * m) + 1] = accP[m];
+                }
+        }
+        __syncthreads();
+        if (ch == 0) {
+#pragma unroll
+            for (int m = 0; m < 5; ++m)
+                if (lane + 32 * m < NPAIR) {
+                    const float a = accA[m] + ds[2 * (lane + 32 * m)];
+                    const float pp = accP[m] + ds[2 * (lane + 32 * m) + 1];
+                    AF[pr[m] * LDA + pi[m]] = pr[m] > pi[m] ? a : 0.f;
+                    PF[pr[m] * LDA + pi[m]] = pp;
+                }
+        }
+    }
+    // blocks I > J through the reference row m = 16 I - 1 (warps 0-5, one pair each)
+    if (warp < 6) {
+        const int I = warp == 0 ? 1 : (warp < 3 ? 2 : 3);
+        const int J = warp == 0 ? 0 : (warp < 3 ? warp - 1 : warp - 3);
+        const int mref = 16 * I - 1;
+        float accA[2][4] = {}, accP[2][4] = {};
+#pragma unroll 2
+        for (int ks = 0; ks < DK / 16; ++ks) {
+            const int j0 = 16 * ks;
+            uint32_t aL[4], aM[4];
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl) {  // a0 (g, 2t) a1 (g+8, 2t) a2 (g, 2t+8) a3 (g+8, 2t+8)
+                const int r = 16 * I + g + 8 * (sl & 1), j = j0 + 2 * t + 8 * (sl >> 1);
+                const float e0 = tc::ex2(LM[r * LDF + j] - LM[mref * LDF + j]);
+                const float e1 = tc::ex2(LM[r * LDF + j + 1] - LM[mref * LDF + j + 1]);
+                aL[sl] = tc::pack_bf16(BK[r * LDF + j] * e0, BK[r * LDF + j + 1] * e1);
+                aM[sl] = tc::pack_bf16(QF[r * LDF + j] * e0, QF[r * LDF + j + 1] * e1);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                // B[kk][n] = K_i o 2^(Lam_m - Lam_i) at row i = 16 J + 8 nt + n, channel j0 + kk
+                const int i = 16 * J + 8 * nt + g;
+                uint32_t bb[2];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int j = j0 + 2 * t + 8 * hb;
+                    const float e0 = tc::ex2(LM[mref * LDF + j] - LM[i * LDF + j]);
+                    const float e1 = tc::ex2(LM[mref * LDF + j + 1] - LM[i * LDF + j + 1]);
+                    bb[hb] = tc::pack_bf16(KF[i * LDF + j] * e0, KF[i * LDF + j + 1] * e1);
+                }
+                mma_bf16_16x8x16(accA[nt], aL, bb);
+                mma_bf16_16x8x16(accP[nt], aM, bb);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = 16 * J + 8 * nt + 2 * t;
+            const int r0 = 16 * I + g, r1 = r0 + 8;
+            *reinterpret_cast<float2 *>(AF + r0 * LDA + col) = make_float2(accA[nt][0], accA[nt][1]);
+            *reinterpret_cast<float2 *>(AF + r1 * LDA + col) = make_float2(accA[nt][2], accA[nt][3]);
+            *reinterpret_cast<float2 *>(PF + r0 * LDA + col) = make_float2(accP[nt][0], accP[nt][1]);
+            *reinterpret_cast<float2 *>(PF + r1 * LDA + col) = make_float2(accP[nt][2], accP[nt][3]);
+        }
+    }
+    __syncthreads();  // A and P complete
+
+    // T = (I + A)^-1: diagonal blocks by substitution, the rest by block products
+    // on warps 0-3 (named barrier 1)
+    if (tid < C) tc::ut_diag(AF, TF, tid);
+    __syncthreads();
+    if (tid < 128) tc::ut_offdiag4<1>(AF, TF, tid);
+    __syncthreads();
+
+    // [P; T''] (T'' = T with zero columns for rows past the end), and T as bf16
+    // over the dead A buffer; 8 threads per 128-byte row
+    {
+        __nv_bfloat16 *dpt = pt + tile * PT_ELEMS;
+#pragma unroll
+        for (int m = 0; m < PT_ELEMS / 8 / THREADS; ++m) {
+            const int idx = tid + THREADS * m;
+            const int rt = idx >> 3, i0 = 8 * (idx & 7), r = rt & (C - 1);
+            const float *src = (rt < C ? PF : TF) + r * LDA + i0;
+            const float4 sa = *reinterpret_cast<const float4 *>(src);
+            const float4 sb = *reinterpret_cast<const float4 *>(src + 4);
+            const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (i0 + e <= r && (rt < C || i0 + e < n)) ? sv[e] : 0.f;
+            *reinterpret_cast<uint4 *>(dpt + rt * C + i0) =
+                make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                           tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+            if (rt >= C) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = (i0 + e <= r) ? sv[e] : 0.f;
+                *reinterpret_cast<uint4 *>(TB + r * LDT + i0) =
+                    make_uint4(tc::pack_bf16(y[0], y[1]), tc::pack_bf16(y[2], y[3]),
+                               tc::pack_bf16(y[4], y[5]), tc::pack_bf16(y[6], y[7]));
+            }
+        }
+        if (tid < DK) glk[tile * DK + tid] = tc::ex2(LM[(C - 1) * LDF + tid]);
+    }
+    __syncthreads();
+
+    // W = T (b o K o 2^Lam): warp w -> rows 16 (w % 4) .. + 15 (T is lower
+    // triangular: chunk rows up to 16 (w % 4) + 15 contribute), channels
+    // 64 (w / 4) .. + 63
+    {
+        const int RB = warp & 3, nh = warp >> 2;
+        const int mi = lane >> 3, ri = lane & 7;
+        const __nv_bfloat16 *arow = TB + (16 * RB + ri + 8 * (mi & 1)) * LDT + 8 * (mi >> 1);
+        float acc[8][4] = {};
+        for (int ks = 0; ks <= RB; ++ks) {
+            uint32_t a[4];
+            ldmatrix_x4(a, arow + 16 * ks);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int j = 64 * nh + 8 * nt + g;  // B[kk][n] at chunk row 16 ks + kk, channel j
+                uint32_t bb[2];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int i = 16 * ks + 2 * t + 8 * hb;
+                    bb[hb] = tc::pack_bf16(BK[i * LDF + j] * tc::ex2(LM[i * LDF + j]),
+                                           BK[(i + 1) * LDF + j] * tc::ex2(LM[(i + 1) * LDF + j]));
+                }
+                mma_bf16_16x8x16(acc[nt], a, bb);
+            }
+        }
+        __nv_bfloat16 *dw = wt + tile * W_ELEMS;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int col = 64 * nh + 8 * nt + 2 * t;
+            const int r0 = 16 * RB + g;
+            *reinterpret_cast<uint32_t *>(dw + r0 * DK + col) = tc::pack_bf16(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<uint32_t *>(dw + (r0 + 8) * DK + col) =
+                tc::pack_bf16(acc[nt][2], acc[nt][3]);
+        }
+    }
+
+    // the sequential kernel's token operands: Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
+    for (int rr = 0; rr < C / 2; ++rr) {
+        const int r = half * (C / 2) + rr;
+        if (r < n) {
+            const size_t off = ((tok0 + r) * H + h) * DK + jc;
+            const float lr = LM[r * LDF + jc];
+            qe[off] = __float2bfloat16_rn(QF[r * LDF + jc] * tc::ex2(lr));
+            kd[off] = __float2bfloat16_rn(KF[r * LDF + jc] * tc::ex2(LM[(C - 1) * LDF + jc] - lr));
+        }
+    }
+    for (int idx = tid; idx < n * Dv; idx += THREADS) {
+        const int r = idx / Dv, jv = idx - r * Dv;
+        const size_t off = ((tok0 + r) * H + h) * Dv + jv;
+        vw[off] = __float2bfloat16_rn(__bfloat162float(v[off]) * wg[off]);
+    }
+}
+
+}  // namespace cwt
+
+bool cw_tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
+    return bf16 && chunk == cwt::C && Dk == cwt::DK && Dv % 64 == 0 && B >= 1 && T >= 1 &&
+           H >= 1 && tc::encode_fn() != nullptr;
+}
+
+// Workspace: [Q o 2^Lam, K o 2^(Lam_last - Lam): [B*T, H, 128] bf16 each][w o V:
+// [B*T, H, Dv] bf16][[P; T''] tiles][W tiles][2^Lam_last per key channel].
+size_t cw_tc_workspace_bytes(int B, int T, int H, int Dv) {
+    const size_t tok = (size_t)B * T * H;
+    const size_t tiles = (size_t)B * ((T + cwt::C - 1) / cwt::C) * H;
+    return tok * (2 * cwt::DK + Dv) * sizeof(__nv_bfloat16) +
+           tiles * (cwt::PT_ELEMS + cwt::W_ELEMS) * sizeof(__nv_bfloat16) +
+           tiles * cwt::DK * sizeof(float);
+}
+
+cudaError_t launch_chunk_cw_tc(const void *q, const void *k, const void *v, const float *la,
+                               const float *bg, const float *wg, const float *S0, void *o,
+                               float *S_T, int B, int T, int H, int Dv, void *workspace,
+                               cudaStream_t st) {
+    const size_t tok = (size_t)B * T * H;
+    const int NT = (T + cwt::C - 1) / cwt::C;
+    const size_t tiles = (size_t)B * NT * H;
+    auto *qe = static_cast<__nv_bfloat16 *>(workspace);
+    __nv_bfloat16 *kd = qe + tok * cwt::DK;
+    __nv_bfloat16 *vw = kd + tok * cwt::DK;
+    __nv_bfloat16 *pt = vw + tok * Dv;
+    __nv_bfloat16 *wt = pt + tiles * cwt::PT_ELEMS;
+    float *glk = reinterpret_cast<float *>(wt + tiles * cwt::W_ELEMS);
+    cudaError_t e = cudaFuncSetAttribute(cwt::gdn_ut_cw_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, cwt::SMEM);
+    if (e != cudaSuccess) return e;
+    cwt::gdn_ut_cw_kernel<<<dim3(NT, H, B), cwt::THREADS, cwt::SMEM, st>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), la, bg, wg, qe, kd, vw, pt, wt, glk, T, H, Dv);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    return launch_chunk_tcw_seq_cw(qe, kd, vw, pt, wt, glk, S0, o, S_T, B, T, H, Dv, st);
+}
+
+}  // namespace gdn

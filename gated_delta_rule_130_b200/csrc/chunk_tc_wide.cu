@@ -54,6 +54,24 @@ namespace gdn {
 // Set by a CTA of gdn_chunk_tcw_kernel that gave up waiting.
 __device__ unsigned int g_tcw_error = 0;
 
+// Optional per-role timeline of the sequential kernel's CTA (0,0,0), chunks
+// 0-63, for performance work: build with -DGDN_TRACE; that build alone exports
+// gdn_tracew_wide_read() (end of this file).  Compiled out otherwise.
+#ifdef GDN_TRACE
+__device__ unsigned long long g_trace_wide[64 * 16];
+#define TW(c, ev)                                                                       \
+    do {                                                                                \
+        if ((threadIdx.x & 31) == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&            \
+            blockIdx.z == 0 && (c) < 64)                                                \
+            g_trace_wide[(c) * 16 + (ev)] = clock64();                                  \
+        __syncwarp();                                                                   \
+    } while (0)
+#else
+#define TW(c, ev) \
+    do {          \
+    } while (0)
+#endif
+
 namespace tcw {
 
 using namespace sm100;
@@ -373,7 +391,8 @@ constexpr int VP_STAGE = 3 * BLK;               // V (8 KiB), [P; T''] (16 KiB)
 constexpr int GV_GAM = 0;                       // gamma_r (/ |q_r| when normalising)
 constexpr int GV_DCY = 64;                      // exp(g_last - g_r) (/ |k_r| when normalising)
 constexpr int GV_GL = 128;                      // gamma_last
-constexpr int GV_STRIDE = 256;
+constexpr int GV_GLK = 256;                     // channel-wise gates: exp(Lam_last) per key channel
+constexpr int GV_STRIDE = 512;
 constexpr int NBAR = 20;
 
 // Shared memory and TMEM of the sequential kernel for Dk = 128 or 256.  The
@@ -432,6 +451,12 @@ struct Params {
     __nv_bfloat16 *o;
     float *S_T;
     const float *rqk;      // 1/|q|, 1/|k| per chunk row from the UT kernel (normalising only)
+    // Channel-wise gates (chunk_cw_tc.cu): the per-chunk decay per key channel,
+    // exp(Lam_last), [tiles][DK] float32.  When set, the Q, K and V operands are
+    // already Q o exp(Lam), K o exp(Lam_last - Lam) and w o V, so gamma_r and
+    // exp(g_last - g_r) are 1 and the state's decay is this per-key vector
+    // (log_alpha is not read).
+    const float *glk;
     Seqs sq;
     int H, Dv;
     unsigned flags;
@@ -504,7 +529,16 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp == W_TMA) {
         // ------------------------------------------------ TMA loads, gate vectors
         float nla[2], nrq[2] = {1.f, 1.f}, nrk[2] = {1.f, 1.f};  // next chunk's gate values
+        constexpr int NGL = DK / 32;                               // per-key decays per lane
+        float ngl[NGL];
+        const bool cw = p.glk != nullptr;
         const auto fetch = [&](int cc) {
+            if (cw) {
+                const size_t tl = (size_t)(sp.chunk0 + cc) * H + h;
+#pragma unroll
+                for (int m = 0; m < NGL; ++m) ngl[m] = p.glk[tl * DK + lane + 32 * m];
+                return;
+            }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = lane + 32 * hh;
@@ -526,13 +560,17 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int c = 0; c < NT; ++c) {
             const int s = c & 1, t0 = c * C;
             const int tile = (sp.chunk0 + c) * H + h;
-            float la[2];
+            float la[2] = {0.f, 0.f}, gl2[NGL];
             const float rq2[2] = {nrq[0], nrq[1]}, rk2[2] = {nrk[0], nrk[1]};
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const bool in = t0 + lane + 32 * hh < T;
-                const float x = nla[hh];
-                la[hh] = in ? ((p.flags & kFlagGateLogits) ? neg_softplus(x) : x) : 0.f;
+            for (int m = 0; m < NGL; ++m) gl2[m] = cw ? ngl[m] : 1.f;
+            if (!cw) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const bool in = t0 + lane + 32 * hh < T;
+                    const float x = nla[hh];
+                    la[hh] = in ? ((p.flags & kFlagGateLogits) ? neg_softplus(x) : x) : 0.f;
+                }
             }
             if (c + 1 < NT) fetch(c + 1);
             // V and [P; T''] of chunk c once the Y product of chunk c - 2 is done
@@ -543,6 +581,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tma_load_4d(vp, &tm_v, cx.bar + B_VP_FULL + s, v0, h, sp.off + t0, 0);
                 tma_load_3d(vp + BLK, &tm_pt, cx.bar + B_VP_FULL + s, 0, 0, tile);
             }
+            TW(c, 0);
             n_vp = c + 1;
             // gate vectors of chunk c (running sums in log2 units; rows past the
             // end carry log alpha = 0)
@@ -559,11 +598,14 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const float g0 = la[0] * LOG2E, g1 = la[1] * LOG2E;
             const float glast = __shfl_sync(0xffffffffu, g1, 31);
             float *gv = gv_all + s * GV_STRIDE;
+            // (channel-wise gates: la = 0, so gamma and the row decays are 1)
             gv[GV_GAM + lane] = tc::ex2(g0) * rq2[0];
             gv[GV_GAM + 32 + lane] = tc::ex2(g1) * rq2[1];
             gv[GV_DCY + lane] = tc::ex2(glast - g0) * rk2[0];
             gv[GV_DCY + 32 + lane] = tc::ex2(glast - g1) * rk2[1];
             if (lane == 0) gv[GV_GL] = tc::ex2(glast);
+#pragma unroll
+            for (int m = 0; m < NGL; ++m) gv[GV_GLK + lane + 32 * m] = gl2[m];
             __syncwarp();
             if (lane == 0) mbar_arrive(cx.bar + B_VP_FULL + s);
             // [Q; W] of chunk c once the X product of chunk c - NQ is done
@@ -580,6 +622,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                                 kb * 64, 0, tile);
                 }
             }
+            TW(c, 1);
             n_qw = c + 1;
             // K of chunk c once the state update of chunk c - NQ is done
             if (c >= NQ && !tc::warp_wait(cx, B_K_EMPTY + sq, pq ^ 1)) break;
@@ -604,6 +647,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     tma_prefetch_l2_3d(&tm_pt, 0, 0, tq);
                 }
             }
+            TW(c, 2);
             n_k = c + 1;
         }
         // never leave with copies in flight: wait (bounded) for the last phases
@@ -637,6 +681,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mma_commit(cx.bar + B_U_FULL);
             }
             __syncwarp();
+            TW(c, 3);
         }
     } else if (warp == W_CHAIN) {
         // ---------------------------------------------- MMA: sequential chain
@@ -651,6 +696,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const uint32_t kt = smem_u32(base + SM_KT + sq * L::K_BYTES);
             if (!tc::warp_wait(cx, B_QW_FULL + sq, pq)) break;
             if (!tc::warp_wait(cx, B_S_READY, c & 1)) break;
+            TW(c, 4);
             tc_fence_after();
             // X = [Q; W] S^T: A K-major (per key block, Q rows then W rows), B = S^T MN-major
             if (lane == 0) {
@@ -662,9 +708,11 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mma_commit(cx.bar + B_QW_EMPTY + sq);
             }
             __syncwarp();
+            TW(c, 5);
             if (!tc::warp_wait(cx, B_U_READY, c & 1)) break;
             if (!tc::warp_wait(cx, B_K_FULL + sq, pq)) break;
             if (!tc::warp_wait(cx, B_VP_FULL + s, (c >> 1) & 1)) break;
+            TW(c, 6);
             tc_fence_after();
             if (lane == 0) {
                 // S^T_h += K_h^T (decayed U') for the key halves: A = K^T (MN-major,
@@ -687,6 +735,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mma_commit(cx.bar + B_VP_EMPTY + s);
             }
             __syncwarp();
+            TW(c, 7);
         }
     } else if (warp >= W_STATE0) {
         // ------------------------------------------------------------ STATE
@@ -703,9 +752,10 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t st_col = TM_ST + (NH == 2 ? 64 * hf : 0) + col0;
         uint8_t *sbuf = base + SM_SB;
         // initial state: S^T row `key` = S0[v0 .. v0 + 63][key]; TMEM copy pre-scaled by gamma_last
+        const bool cw = p.glk != nullptr;
         {
             const bool have = tc::warp_wait(cx, B_VP_FULL + 0, 0);
-            const float gl = gv_all[GV_GL];
+            const float gl = cw ? gv_all[GV_GLK + key] : gv_all[GV_GL];
 #pragma unroll
             for (int pc = 0; pc < NPC; ++pc) {
                 float sv[16];
@@ -727,6 +777,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int s = c & 1, t0 = c * C;
             const float *gv = gv_all + s * GV_STRIDE;
             if (!tc::warp_wait(cx, B_X_FULL, c & 1)) break;
+            if (warp == W_STATE0 + 2) TW(c, 8);
             tc_fence_after();
             if (q >= 2) {
                 // U' = U - W S^T for chunk row r -> U' and its decayed copy (bf16)
@@ -759,6 +810,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 fence_async_smem();
                 tc_fence_before();
                 tc::warp_arrive(cx, B_U_READY);
+                if (warp == W_STATE0 + 2) TW(c, 9);
             } else {
                 // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y
                 const float gr = gv[GV_GAM + lrow];
@@ -776,10 +828,12 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tmem_wait_st();
                 tc_fence_before();
                 tc::warp_arrive(cx, B_U_READY);
+                if (warp == W_STATE0) TW(c, 13);
             }
             // state hand-off: S^T (updated) -> bf16 copy; TMEM pre-scaled by the
             // next chunk's gamma_last
             if (!tc::warp_wait(cx, B_ST_FULL, c & 1)) break;
+            if (warp == W_STATE0) TW(c, 10);
             tc_fence_after();
             {
                 const bool last = c + 1 >= NT;
@@ -787,7 +841,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 float gl = 1.f;
                 if (!last) {
                     have = tc::warp_wait(cx, B_VP_FULL + (s ^ 1), ((c + 1) >> 1) & 1);
-                    gl = gv_all[(s ^ 1) * GV_STRIDE + GV_GL];
+                    gl = gv_all[(s ^ 1) * GV_STRIDE + (cw ? GV_GLK + key : GV_GL)];
                 }
                 float sv[NPC][16];
 #pragma unroll
@@ -814,6 +868,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 tc_fence_before();
                 tc::warp_arrive(cx, B_S_READY);
+                if (warp == W_STATE0) TW(c, 11);
                 if (!last && !have) break;
             }
             // chunk output rows (TMEM lanes 0-63)
@@ -840,6 +895,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                 }
                 tc_fence_before();
+                if (warp == W_STATE0) TW(c, 12);
             }
         }
     }
@@ -950,6 +1006,7 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.S_T = S_T;
     p.rqk = rqk;
+    p.glk = nullptr;
     p.sq = tc::Seqs{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
                     n_seq};
     p.H = H;
@@ -966,6 +1023,54 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                 : tcw::launch<128, false>(mq, mk, mv, mw, mp, p, log_alpha, beta, pt, wt, rqk,
                                           total_chunks, n_seq, st);
 }
+
+cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *vw,
+                                    const void *pt, const void *wt, const float *glk,
+                                    const float *S0, void *o, float *S_T, int B, int T, int H,
+                                    int Dv, cudaStream_t st) {
+    constexpr int DK = 128;
+    const long long NT = ((long long)T + tc::C - 1) / tc::C;
+    const long long n_tiles = (long long)B * NT * H;
+    CUtensorMap mq, mk, mv, mw, mp;
+    if (!tc::make_map(&mq, qe, 1, B * T, H, DK) || !tc::make_map(&mk, kd, 1, B * T, H, DK) ||
+        !tc::make_map(&mv, vw, 1, B * T, H, Dv) || !tcw::make_map_w(&mw, wt, n_tiles, DK) ||
+        !tc::make_map_tt(&mp, pt, n_tiles))
+        return cudaErrorInvalidValue;
+    tcw::Params p;
+    p.log_alpha = nullptr;
+    p.S0 = S0;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.S_T = S_T;
+    p.rqk = nullptr;
+    p.glk = glk;
+    p.sq = tc::Seqs{nullptr, nullptr, nullptr, T, B};
+    p.H = H;
+    p.Dv = Dv;
+    p.flags = 0u;
+    auto *seq = tcw::gdn_chunk_tcw_kernel<DK, false>;
+    constexpr int seq_smem = tcw::SeqDims<DK>::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Dv / tcw::DVT, H, B);
+    cfg.blockDim = dim3(tcw::NTHREADS);
+    cfg.dynamicSmemBytes = seq_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mw, mp, p);
+    if (e != cudaSuccess) return e;
+    return cudaPeekAtLastError();
+}
+
+#ifdef GDN_TRACE
+extern "C" int gdn_tracew_wide_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_trace_wide, sizeof(g_trace_wide));
+}
+#endif
 
 cudaError_t read_and_clear_device_error_wide(unsigned int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_tcw_error, sizeof(unsigned int));

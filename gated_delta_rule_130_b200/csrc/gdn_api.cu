@@ -346,12 +346,20 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+int gdn_chunk_fwd_cw_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
+    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::cw_supported(Dk, chunk))
+        return -1;
+    if (empty_problem(B, T, H)) return GDN_PATH_NONE;
+    if (gdn::cw_tc_supported(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16)) return GDN_PATH_TCGEN05;
+    return GDN_PATH_SIMT;
+}
+
 size_t gdn_chunk_fwd_cw_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
                                        gdn_dtype_t dtype) {
-    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::cw_supported(Dk, chunk))
-        return 0;
-    if (empty_problem(B, T, H)) return 0;
-    return gdn::cw_workspace_bytes(B, T, H, Dk, chunk);
+    const int path = gdn_chunk_fwd_cw_path(B, T, H, Dk, Dv, chunk, dtype);
+    if (path == GDN_PATH_TCGEN05) return gdn::cw_tc_workspace_bytes(B, T, H, Dv);
+    if (path == GDN_PATH_SIMT) return gdn::cw_workspace_bytes(B, T, H, Dk, chunk);
+    return 0;
 }
 
 gdn_status_t gdn_chunk_fwd_cw(const void *q, const void *k, const void *v,
@@ -396,15 +404,19 @@ gdn_status_t gdn_chunk_fwd_cw(const void *q, const void *k, const void *v,
     if (S_T && S0 && S_T != S0 && overlaps(S_T, state_bytes, S0, state_bytes))
         return GDN_ERR_INVALID_ARG;
     if (S_T && overlaps(S_T, state_bytes, o, o_bytes)) return GDN_ERR_INVALID_ARG;
-    const size_t need = gdn::cw_workspace_bytes(B, T, H, Dk, chunk);
+    const size_t need = gdn_chunk_fwd_cw_workspace_size(B, T, H, Dk, Dv, chunk, dtype);
     if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
     for (const auto &a : in)
         if (overlaps(workspace, need, a.p, a.n)) return GDN_ERR_INVALID_ARG;
     if (overlaps(workspace, need, o, o_bytes) ||
         (S_T && overlaps(workspace, need, S_T, state_bytes)))
         return GDN_ERR_INVALID_ARG;
-    const cudaError_t e = gdn::launch_chunk_cw(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, Dk,
-                                               Dv, chunk, dtype == GDN_BF16, workspace, st);
+    const bool tc = gdn::cw_tc_supported(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16);
+    const cudaError_t e =
+        tc ? gdn::launch_chunk_cw_tc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, Dv, workspace,
+                                     st)
+           : gdn::launch_chunk_cw(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, Dk, Dv, chunk,
+                                  dtype == GDN_BF16, workspace, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -117,6 +117,24 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                                   const int *cu_seqlens, long long total_chunks, int H, int Dk,
                                   int Dv, unsigned flags, void *workspace, cudaStream_t st);
 
+// The precomputed variant's sequential kernel (Dk = 128) in its channel-wise
+// mode: operands Q o exp(Lam), K o exp(Lam_last - Lam), w o V ([B*T, H, D] bf16),
+// the [P; T''] and W tiles and exp(Lam_last) per key channel ([tiles][128]
+// float32), all from chunk_cw_tc.cu's parallel kernel.
+cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *vw,
+                                    const void *pt, const void *wt, const float *glk,
+                                    const float *S0, void *o, float *S_T, int B, int T, int H,
+                                    int Dv, cudaStream_t st);
+
+// Channel-wise gates on the tensor cores (bf16, Dk = 128, chunk 64, Dv a
+// multiple of 64): chunk_cw_tc.cu.
+bool cw_tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
+size_t cw_tc_workspace_bytes(int B, int T, int H, int Dv);
+cudaError_t launch_chunk_cw_tc(const void *q, const void *k, const void *v, const float *la,
+                               const float *bg, const float *wg, const float *S0, void *o,
+                               float *S_T, int B, int T, int H, int Dv, void *workspace,
+                               cudaStream_t st);
+
 // Read and clear the flag a fused-kernel CTA sets when one of its bounded waits
 // times out (synchronous).
 cudaError_t read_and_clear_device_error(unsigned int *flag);

@@ -199,6 +199,10 @@ __device__ __forceinline__ void store16x16(const float (&acc)[2][4], float *__re
 //   phase 2  T_{J+1,J} = -N_{J+1,J} T_JJ                              (3 warps)
 //   phase 3  T_{J+2,J} = -(N_{J+2,J} T_JJ + N_{J+2,J+1} T_{J+1,J})    (2 warps)
 //   phase 4  T_30 = -(N_30 T_00 + N_31 T_10 + N_32 T_20)              (1 warp)
+// kBar = 0: the CTA has exactly these 4 warps and synchronises with
+// __syncthreads; kBar > 0: only warps 0-3 of a larger CTA call it and they
+// synchronise on named barrier kBar (128 threads).
+template <int kBar = 0>
 __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__restrict__ TF,
                                             int p) {
     const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
@@ -214,7 +218,10 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
             store16x16(acc, blk(AF, I, J), LDA, 1.f, g, t);
         }
     }
-    __syncthreads();
+    if constexpr (kBar > 0)
+        named_barrier(kBar, 128);
+    else
+        __syncthreads();
     // block column J of T needs only its own earlier blocks and the N blocks:
     // warp J walks down it, T_IJ = -sum_{K=J}^{I-1} N_IK T_KJ, with no CTA barrier
     if (w < 3) {
@@ -227,7 +234,10 @@ __device__ __forceinline__ void ut_offdiag4(float *__restrict__ AF, float *__res
             __syncwarp();
         }
     }
-    __syncthreads();
+    if constexpr (kBar > 0)
+        named_barrier(kBar, 128);
+    else
+        __syncthreads();
 }
 
 // ------------------------------------------------------------- sequences --

@@ -297,6 +297,13 @@ gdn_status_t gdn_chunk_fwd_cw(const void *q, const void *k, const void *v,
                               int B, int T, int H, int Dk, int Dv, int chunk,
                               gdn_dtype_t dtype, void *workspace, size_t workspace_bytes,
                               void *stream);
+/* Which kernels gdn_chunk_fwd_cw runs for these sizes (gdn_path_t; -1 for
+ * invalid sizes): GDN_PATH_TCGEN05 for bf16, Dk = 128, chunk 64 and Dv a
+ * multiple of 64 -- a parallel per-chunk kernel (the channel-wise decays taken
+ * through 16-row blocks, the UT transform, W and the decayed operands) and the
+ * sequential tcgen05 kernel with a per-key-channel state decay -- else
+ * GDN_PATH_SIMT (CUDA cores).  The workspace size depends on it. */
+int gdn_chunk_fwd_cw_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype);
 size_t gdn_chunk_fwd_cw_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
                                        gdn_dtype_t dtype);
 

@@ -69,6 +69,11 @@ cudaError_t launch_chunk_bwd(const void *, const void *, const void *, const flo
                              const float *, const void *, const float *, void *, void *, void *,
                              float *, float *, float *, int, int, int, int, int, int, bool, void *,
                              cudaStream_t) { return ok(); }
+bool cw_tc_supported(int, int, int, int, int, int, bool) { return false; }
+size_t cw_tc_workspace_bytes(int, int, int, int) { return 0; }
+cudaError_t launch_chunk_cw_tc(const void *, const void *, const void *, const float *,
+                               const float *, const float *, const float *, void *, float *, int,
+                               int, int, int, void *, cudaStream_t) { return ok(); }
 bool cw_supported(int Dk, int chunk) { return Dk <= 128 && (chunk == 16 || chunk == 32 || chunk == 64); }
 size_t cw_workspace_bytes(int B, int T, int H, int Dk, int C) {
     return (size_t)B * H * (((size_t)T + C - 1) / C) * (2 * (size_t)C * C + (size_t)C * Dk) * 4; }
