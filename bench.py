@@ -643,6 +643,35 @@ def parse_workload(spec: str):
     return I.workload(name, **over)
 
 
+def run_cw_only(args):
+    """--cw-only: the channel-wise-gate forward alone on --workload (one GPU, for
+    counter captures); prints one short JSON line."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from gated_delta_rule_130_b200 import binding as G
+    w = parse_workload(args.workload)
+    cin = I.cw_inputs(w, device=device)
+    o = torch.empty((w.B, w.T, w.H, w.Dv), dtype=w.torch_dtype, device=device)
+    S = torch.empty((w.B, w.H, w.Dv, w.Dk), dtype=torch.float32, device=device)
+    ws = torch.empty(max(G.chunk_fwd_cw_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                       w.torch_dtype), 1),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        G.chunk_fwd_cw(cin["q"], cin["k"], cin["v"], cin["log_alpha"], cin["b"], cin["w"],
+                       cin["S0"], chunk=w.chunk, out=o, S_T=S, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    steps = args.steps or 20
+    ms = time_loop(step, steps, torch.cuda.current_stream(device), 1) / steps
+    print(json.dumps({"leg": "channel_wise", "workload": args.workload,
+                      "path": G.chunk_fwd_cw_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                  w.torch_dtype),
+                      "ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+                      "steps": steps}), flush=True)
+
+
 def run_decode_only(args):
     """--decode-only: the decode step alone (batch 256, H 16, d 128, state in place),
     for counter captures of its kernel; prints one short JSON line."""
@@ -686,9 +715,13 @@ def main():
                     help="with --chunk-only: the workload to time, 'name' or 'name:B=2,T=1024'")
     ap.add_argument("--decode-only", action="store_true",
                     help="time the decode step alone (one GPU, for counter captures)")
+    ap.add_argument("--cw-only", action="store_true",
+                    help="time the channel-wise-gate forward alone on --workload (one GPU)")
     args = ap.parse_args()
     if args.decode_only:
         run_decode_only(args)
+    elif args.cw_only:
+        run_cw_only(args)
     elif args.impl == "reference":
         if args.steps is None:
             args.steps = 10

@@ -15,7 +15,7 @@
 // which is the shape of the scalar precomputed variant (chunk_tc_wide.cu) with
 // Q, K and V replaced by Q o exp(Lam), K o exp(Lam_last - Lam) and w o V and the
 // state's decay a vector over the key channels.  Two kernels:
-//  1. gdn_ut_cw_kernel, one CTA of 8 warps per (chunk, head, batch), all chunks
+//  1. gdn_ut_cw_kernel, one CTA of 16 warps per (chunk, head, batch), all chunks
 //     in parallel.  The decays between rows are channel-wise, so they cannot be
 //     taken out of the key products as row and column scales; split the chunk
 //     into 16-row blocks:
@@ -27,8 +27,10 @@
 //         R = K_J o 2^(Lam_m - Lam_J): bf16 mma.sync products of 16-row blocks
 //         (the factorisation is per block pair; 16 rows is below the M = 64 of
 //         a tcgen05 product);
-//       - the four diagonal blocks are summed directly over the channels in
-//         float32 (exp2 of the exact differences), one warp pair per block;
+//       - inside a diagonal block, rows 8-15 against rows 0-7 factor the same
+//         way through the block's row 7 (mma.sync); the two 8 x 8 diagonal
+//         sub-blocks are summed directly over the channels in float32 (exp2 of
+//         the exact differences), four warps per block;
 //     then the blocked UT solve, W = T (b o K o 2^Lam) (mma.sync), and the
 //     operands of the sequential kernel: [P; T''] (T'' = T with the columns of
 //     rows past the end zeroed), W, Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
@@ -52,7 +54,7 @@ using tc::C;
 using tc::LDA;
 
 constexpr int DK = 128;
-constexpr int THREADS = 256;                  // 8 warps
+constexpr int THREADS = 512;                  // 16 warps
 constexpr int LDF = DK + 1;                   // float32 row stride of the per-channel arrays
 constexpr int LDT = C + 8;                    // bf16 row stride of T for the W product
 constexpr int SM_K = 0;                       // k (f32, 64 x LDF)
@@ -62,9 +64,9 @@ constexpr int SM_LM = SM_BK + C * LDF * 4;    // Lam log2(e) (running sums per c
 constexpr int SM_AF = SM_LM + C * LDF * 4;    // A (f32, 64 x LDA); then T as bf16
 constexpr int SM_TF = SM_AF + C * LDA * 4;    // T (f32)
 constexpr int SM_PF = SM_TF + C * LDA * 4;    // P (f32)
-constexpr int NPAIR = 136;                    // (r, i), i <= r, of a 16 x 16 block
-constexpr int SM_DS = SM_PF + C * LDA * 4;    // diagonal blocks: the second channel half's sums
-constexpr int SMEM = SM_DS + 4 * NPAIR * 2 * 4;
+constexpr int NPAIR = 72;                     // (r, i), i <= r, of the two 8 x 8 diagonal sub-blocks
+constexpr int SM_DS = SM_PF + C * LDA * 4;    // diagonal blocks: channel quarters 1-3 partial sums
+constexpr int SMEM = SM_DS + 4 * 3 * NPAIR * 2 * 4;
 constexpr int PT_ELEMS = 2 * C * C, W_ELEMS = C * DK;
 constexpr float LOG2E = 1.4426950408889634f;
 static_assert(SM_AF % 16 == 0 && SM_TF % 16 == 0 && SM_PF % 16 == 0 && SM_DS % 16 == 0,
@@ -100,61 +102,73 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     __nv_bfloat16 *TB = reinterpret_cast<__nv_bfloat16 *>(sm + SM_AF);
 
     // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread
-    // -> (channel, half of the rows), so each row is read as 128 consecutive values
-    const int jc = tid & (DK - 1), half = tid >> 7;
-    for (int rr = 0; rr < C / 2; ++rr) {
-        const int r = half * (C / 2) + rr;
-        float kv = 0.f, qv = 0.f, bv = 0.f, lv = 0.f;
-        if (r < n) {
-            const size_t off = ((tok0 + r) * H + h) * DK + jc;
-            kv = __bfloat162float(k[off]);
-            qv = __bfloat162float(q[off]);
-            bv = bg[off];
-            lv = la[off];
+    // -> (channel, quarter of the rows), so each row is read as 128 consecutive
+    // values; eight rows' loads are issued before any is used (one CTA per SM:
+    // the loads in flight are what hides the memory latency)
+    constexpr int RQ = C / 4;                      // rows per quarter
+    const int jc = tid & (DK - 1), rq = tid >> 7;
+    constexpr int RB8 = 8;
+    for (int r8 = 0; r8 < RQ; r8 += RB8) {
+        float kv[RB8], qv[RB8], bv[RB8], lv[RB8];
+#pragma unroll
+        for (int u = 0; u < RB8; ++u) {
+            const int r = rq * RQ + r8 + u;
+            const size_t off = ((tok0 + (r < n ? r : 0)) * H + h) * DK + jc;
+            const bool in = r < n;
+            kv[u] = in ? __bfloat162float(k[off]) : 0.f;
+            qv[u] = in ? __bfloat162float(q[off]) : 0.f;
+            bv[u] = in ? bg[off] : 0.f;
+            lv[u] = in ? la[off] : 0.f;
         }
-        KF[r * LDF + jc] = kv;
-        QF[r * LDF + jc] = qv;
-        BK[r * LDF + jc] = bv * kv;
-        LM[r * LDF + jc] = lv * LOG2E;
+#pragma unroll
+        for (int u = 0; u < RB8; ++u) {
+            const int r = rq * RQ + r8 + u;
+            KF[r * LDF + jc] = kv[u];
+            QF[r * LDF + jc] = qv[u];
+            BK[r * LDF + jc] = bv[u] * kv[u];
+            LM[r * LDF + jc] = lv[u] * LOG2E;
+        }
     }
     __syncthreads();
-    {   // running sums over the rows, per channel: each half locally, then the
-        // second half adds the first half's total
+    {   // running sums over the rows, per channel: each quarter locally, then the
+        // totals of the earlier quarters are added
         float acc = 0.f;
-        for (int rr = 0; rr < C / 2; ++rr) {
-            const int r = half * (C / 2) + rr;
+        for (int rr = 0; rr < RQ; ++rr) {
+            const int r = rq * RQ + rr;
             acc += LM[r * LDF + jc];
             LM[r * LDF + jc] = acc;
         }
     }
     __syncthreads();
-    if (half == 1) {
-        const float base = LM[(C / 2 - 1) * LDF + jc];
-        for (int r = C / 2; r < C; ++r) LM[r * LDF + jc] += base;
+    {
+        float base = 0.f;
+        for (int qq = 0; qq < rq; ++qq) base += LM[(qq * RQ + RQ - 1) * LDF + jc];
+        __syncthreads();
+        for (int rr = 0; rr < RQ; ++rr) LM[(rq * RQ + rr) * LDF + jc] += base;
     }
     __syncthreads();
 
-    // diagonal 16-blocks, summed directly: warps 2I and 2I+1 take block I, each
-    // half of the channels; lane -> pairs p = lane + 32 m of the block's lower
-    // triangle (p = r (r + 1) / 2 + i)
+    // the two 8 x 8 diagonal sub-blocks of each diagonal 16-block, summed
+    // directly: warps 4I .. 4I+3 take block I, each a quarter of the channels;
+    // lane -> pairs P = lane + 32 m: sub-block s = P / 36, p = P % 36 = r (r + 1) / 2 + i
     {
-        const int I = warp >> 1, ch = warp & 1;
-        int pr[5], pi[5];
-        float accA[5], accP[5];
+        const int I = warp >> 2, ch = warp & 3;
+        int pr[3], pi[3];
+        float accA[3], accP[3];
 #pragma unroll
-        for (int m = 0; m < 5; ++m) {
-            const int p = lane + 32 * m;
+        for (int m = 0; m < 3; ++m) {
+            const int P = lane + 32 * m, sb = P / 36, p = P % 36;
             int r = 0;
             while ((r + 1) * (r + 2) / 2 <= p) ++r;
-            pr[m] = 16 * I + r;
-            pi[m] = 16 * I + (p - r * (r + 1) / 2);
+            pr[m] = 16 * I + 8 * sb + r;
+            pi[m] = 16 * I + 8 * sb + (p - r * (r + 1) / 2);
             accA[m] = accP[m] = 0.f;
         }
 #pragma unroll 2
-        for (int jj = 0; jj < DK / 2; ++jj) {
-            const int j = (DK / 2) * ch + jj;
+        for (int jj = 0; jj < DK / 4; ++jj) {
+            const int j = (DK / 4) * ch + jj;
 #pragma unroll
-            for (int m = 0; m < 5; ++m) {
+            for (int m = 0; m < 3; ++m) {
                 if (lane + 32 * m < NPAIR) {
                     const int R = pr[m], Ii = pi[m];
                     const float e = tc::ex2(LM[R * LDF + j] - LM[Ii * LDF + j]) * KF[Ii * LDF + j];
@@ -163,22 +177,26 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 }
             }
         }
-        float *ds = DS + I * NPAIR * 2;
-        if (ch == 1) {
+        float *ds = DS + I * 3 * NPAIR * 2;   // partial sums of channel quarters 1-3
+        if (ch > 0) {
 #pragma unroll
-            for (int m = 0; m < 5; ++m)
+            for (int m = 0; m < 3; ++m)
                 if (lane + 32 * m < NPAIR) {
-                    ds[2 * (lane + 32 * m)] = accA[m];
-                    ds[2 * (lane + 32 * m) + 1] = accP[m];
+                    ds[((ch - 1) * NPAIR + lane + 32 * m) * 2] = accA[m];
+                    ds[((ch - 1) * NPAIR + lane + 32 * m) * 2 + 1] = accP[m];
                 }
         }
         __syncthreads();
         if (ch == 0) {
 #pragma unroll
-            for (int m = 0; m < 5; ++m)
+            for (int m = 0; m < 3; ++m)
                 if (lane + 32 * m < NPAIR) {
-                    const float a = accA[m] + ds[2 * (lane + 32 * m)];
-                    const float pp = accP[m] + ds[2 * (lane + 32 * m) + 1];
+                    float a = accA[m], pp = accP[m];
+#pragma unroll
+                    for (int cq = 0; cq < 3; ++cq) {
+                        a += ds[(cq * NPAIR + lane + 32 * m) * 2];
+                        pp += ds[(cq * NPAIR + lane + 32 * m) * 2 + 1];
+                    }
                     AF[pr[m] * LDA + pi[m]] = pr[m] > pi[m] ? a : 0.f;
                     PF[pr[m] * LDA + pi[m]] = pp;
                 }
@@ -228,6 +246,39 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             *reinterpret_cast<float2 *>(PF + r1 * LDA + col) = make_float2(accP[nt][2], accP[nt][3]);
         }
     }
+    // rows 8-15 against rows 0-7 of each diagonal block through its row 7 (warps
+    // 6-9, one block each): a 16 x 8 product whose rows 0-7 are left zero
+    if (warp >= 6 && warp < 10) {
+        const int I = warp - 6, mref = 16 * I + 7;
+        float accA[4] = {}, accP[4] = {};
+#pragma unroll 2
+        for (int ks = 0; ks < DK / 16; ++ks) {
+            const int j0 = 16 * ks;
+            uint32_t aL[4] = {0u, 0u, 0u, 0u}, aM[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int sl = 1; sl < 4; sl += 2) {  // a1 (g+8, 2t), a3 (g+8, 2t+8)
+                const int r = 16 * I + 8 + g, j = j0 + 2 * t + 8 * (sl >> 1);
+                const float e0 = tc::ex2(LM[r * LDF + j] - LM[mref * LDF + j]);
+                const float e1 = tc::ex2(LM[r * LDF + j + 1] - LM[mref * LDF + j + 1]);
+                aL[sl] = tc::pack_bf16(BK[r * LDF + j] * e0, BK[r * LDF + j + 1] * e1);
+                aM[sl] = tc::pack_bf16(QF[r * LDF + j] * e0, QF[r * LDF + j + 1] * e1);
+            }
+            const int i = 16 * I + g;  // B[kk][n] = K_i o 2^(Lam_m - Lam_i), n = g
+            uint32_t bb[2];
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const int j = j0 + 2 * t + 8 * hb;
+                const float e0 = tc::ex2(LM[mref * LDF + j] - LM[i * LDF + j]);
+                const float e1 = tc::ex2(LM[mref * LDF + j + 1] - LM[i * LDF + j + 1]);
+                bb[hb] = tc::pack_bf16(KF[i * LDF + j] * e0, KF[i * LDF + j + 1] * e1);
+            }
+            mma_bf16_16x8x16(accA, aL, bb);
+            mma_bf16_16x8x16(accP, aM, bb);
+        }
+        const int r1 = 16 * I + 8 + g, col = 16 * I + 2 * t;
+        *reinterpret_cast<float2 *>(AF + r1 * LDA + col) = make_float2(accA[2], accA[3]);
+        *reinterpret_cast<float2 *>(PF + r1 * LDA + col) = make_float2(accP[2], accP[3]);
+    }
     __syncthreads();  // A and P complete
 
     // T = (I + A)^-1: diagonal blocks by substitution, the rest by block products
@@ -270,18 +321,18 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 
     // W = T (b o K o 2^Lam): warp w -> rows 16 (w % 4) .. + 15 (T is lower
     // triangular: chunk rows up to 16 (w % 4) + 15 contribute), channels
-    // 64 (w / 4) .. + 63
+    // 32 (w / 4) .. + 31
     {
         const int RB = warp & 3, nh = warp >> 2;
         const int mi = lane >> 3, ri = lane & 7;
         const __nv_bfloat16 *arow = TB + (16 * RB + ri + 8 * (mi & 1)) * LDT + 8 * (mi >> 1);
-        float acc[8][4] = {};
+        float acc[4][4] = {};
         for (int ks = 0; ks <= RB; ++ks) {
             uint32_t a[4];
             ldmatrix_x4(a, arow + 16 * ks);
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int j = 64 * nh + 8 * nt + g;  // B[kk][n] at chunk row 16 ks + kk, channel j
+            for (int nt = 0; nt < 4; ++nt) {
+                const int j = 32 * nh + 8 * nt + g;  // B[kk][n] at chunk row 16 ks + kk, channel j
                 uint32_t bb[2];
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
@@ -294,8 +345,8 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
         __nv_bfloat16 *dw = wt + tile * W_ELEMS;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int col = 64 * nh + 8 * nt + 2 * t;
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = 32 * nh + 8 * nt + 2 * t;
             const int r0 = 16 * RB + g;
             *reinterpret_cast<uint32_t *>(dw + r0 * DK + col) = tc::pack_bf16(acc[nt][0], acc[nt][1]);
             *reinterpret_cast<uint32_t *>(dw + (r0 + 8) * DK + col) =
@@ -304,8 +355,8 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     }
 
     // the sequential kernel's token operands: Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
-    for (int rr = 0; rr < C / 2; ++rr) {
-        const int r = half * (C / 2) + rr;
+    for (int rr = 0; rr < RQ; ++rr) {
+        const int r = rq * RQ + rr;
         if (r < n) {
             const size_t off = ((tok0 + r) * H + h) * DK + jc;
             const float lr = LM[r * LDF + jc];
@@ -313,10 +364,26 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             kd[off] = __float2bfloat16_rn(KF[r * LDF + jc] * tc::ex2(LM[(C - 1) * LDF + jc] - lr));
         }
     }
-    for (int idx = tid; idx < n * Dv; idx += THREADS) {
-        const int r = idx / Dv, jv = idx - r * Dv;
-        const size_t off = ((tok0 + r) * H + h) * Dv + jv;
-        vw[off] = __float2bfloat16_rn(__bfloat162float(v[off]) * wg[off]);
+    // w o V, eight loads of each in flight per thread
+    for (int base = 0; base < n * Dv; base += RB8 * THREADS) {
+        float vv[RB8], ww[RB8];
+#pragma unroll
+        for (int u = 0; u < RB8; ++u) {
+            const int idx = base + u * THREADS + tid;
+            const int r = idx / Dv, jv = idx - r * Dv;
+            const bool in = idx < n * Dv;
+            const size_t off = ((tok0 + (in ? r : 0)) * H + h) * Dv + (in ? jv : 0);
+            vv[u] = in ? __bfloat162float(v[off]) : 0.f;
+            ww[u] = in ? wg[off] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < RB8; ++u) {
+            const int idx = base + u * THREADS + tid;
+            if (idx < n * Dv) {
+                const int r = idx / Dv, jv = idx - r * Dv;
+                vw[((tok0 + r) * H + h) * Dv + jv] = __float2bfloat16_rn(vv[u] * ww[u]);
+            }
+        }
     }
 }
 
