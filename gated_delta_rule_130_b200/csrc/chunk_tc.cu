@@ -291,9 +291,9 @@ seq_schedule(const int *__restrict__ cu, int n, int *__restrict__ cu_chunks,
 // The chunk's K rows arrive by TMA (128-byte swizzle) and the Gram matrix K K^T
 // is one tcgen05 product (M = N = 64, K = 128) into tensor memory, from where
 // each warp reads 16 rows (an M = 64 product puts row m in TMEM lane
-// 32 (m / 16) + m % 16).  Five CTAs fit on an SM (39 KiB of shared memory, 64
-// TMEM columns each), so five chunks are in flight per SM and the solve's
-// dependent steps overlap across chunks.
+// 32 (m / 16) + m % 16).  Six CTAs fit on an SM (37 KiB of shared memory, 64
+// TMEM columns, 80 registers a thread), so six chunks are in flight per SM and
+// the solve's dependent steps overlap across chunks.
 constexpr int UT_THREADS = 128;
 constexpr int UT_SM_KT = 0;                        // K chunk (KB blocks of 64 x 128 B), then T
 constexpr int UT_SM_AF = C * LDA * 4;              // A (64 x LDA f32); N_IJ overwrite A_IJ
@@ -303,13 +303,13 @@ constexpr int UT_SMEM = UT_SM_BAR + 32 + 1024;     // + alignment slack (1024-by
 constexpr uint32_t UT_TM_COLS = 64;
 constexpr int TT_ELEMS = 2 * C * C;                // one [T'; T''] tile
 static_assert(KB * 8192 <= UT_SM_AF, "K chunk fits in the T buffer");
-static_assert(UT_SM_AF % 1024 == 0 && UT_SM_GT % 16 == 0 && UT_SM_BAR % 8 == 0,
-              "aligned UT buffers");
+static_assert(UT_SM_GT % 16 == 0 && UT_SM_BAR % 8 == 0, "aligned UT buffers");
+static_assert(6 * (UT_SMEM + 1024) <= 228 * 1024, "six CTAs per SM");
 
 // kNorm: q and k are L2-normalised inside the kernels (1/|k| folded into the
 // Gram rows and T', and written to rk_out); without it the kernel is unchanged.
 template <bool kNorm>
-__global__ void __launch_bounds__(UT_THREADS, 5)
+__global__ void __launch_bounds__(UT_THREADS, 6)
 gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ log_alpha,
               const float *__restrict__ beta, __nv_bfloat16 *__restrict__ tt,
               float *__restrict__ rk_out, const Seqs sq, int H, unsigned flags) {
@@ -408,36 +408,41 @@ gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict_
         __syncwarp();
     }
     __syncthreads();  // the gate vectors are written
-    // row r = 16 w + l of G (lanes l < 16 of warp w; lanes 16-31 read unused TMEM)
+    // row r = 16 w + l of G (lanes l < 16 of warp w; lanes 16-31 read unused TMEM),
+    // in two halves of 32 columns (fewer live registers)
     const int r = 16 * warp + lane;
     const bool row_lane = lane < 16;
-    float gr_row[C];
-    {
-        const bool done = warp_wait(cx, 1, 0);
-        tc_fence_after();
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const bool done = warp_wait(cx, 1, 0);
+    tc_fence_after();
+    const auto load_half = [&](int hc, float (&v)[32]) {
         if (done) {
-            const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-            for (int pc = 0; pc < C / 16; ++pc) {
-                float v[16];
-                tmem_ld16(lane_addr + 16 * pc, v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) gr_row[16 * pc + j] = v[j];
-            }
+            float a[16], b2[16];
+            tmem_ld16(lane_addr + 32 * hc, a);
+            tmem_ld16(lane_addr + 32 * hc + 16, b2);
             tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                v[j] = a[j];
+                v[16 + j] = b2[j];
+            }
         } else {
 #pragma unroll
-            for (int j = 0; j < C; ++j) gr_row[j] = 0.f;
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
         }
-    }
-    tc_fence_before();
+    };
     if constexpr (kNorm) {
         // |k_r|^2 is the diagonal of K K^T; 1/|k| folds into the Gram rows and T',
         // and is kept in the workspace for the sequential kernel
+        // row r = 16 w + l has its diagonal in columns 16 w .. + 15 (warp-uniform)
+        float v[16];
+        tmem_ld16(lane_addr + 16 * warp, v);
+        tmem_wait_ld();
         if (row_lane) {
             float d = 0.f;
 #pragma unroll
-            for (int j = 0; j < C; ++j) d = (j == r) ? gr_row[j] : d;
+            for (int j = 0; j < 16; ++j) d = (j == lane) ? v[j] : d;
+            if (!done) d = 0.f;
             const float rkv = rsqrtf(fmaxf(d, 0.f) + kNormEps);
             rks[r] = rkv;
             bgs[r] *= rkv;
@@ -446,20 +451,27 @@ gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict_
         __syncthreads();
     }
     // A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0 (row r, all columns)
-    if (row_lane) {
-        const float grl = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
+#pragma unroll 1
+    for (int hc = 0; hc < 2; ++hc) {
+        float v[32];
+        load_half(hc, v);
+        if (row_lane) {
+            const float grl = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
 #pragma unroll
-        for (int i4 = 0; i4 < C / 4; ++i4) {
-            float a[4];
+            for (int i4 = 0; i4 < 8; ++i4) {
+                float a[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = 4 * i4 + e;
-                const float s = kNorm ? br * rks[i] : br;
-                a[e] = (i < r) ? s * ex2(grl - g2s[i]) * gr_row[i] : 0.f;
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 32 * hc + 4 * i4 + e;
+                    const float sc = kNorm ? br * rks[i] : br;
+                    a[e] = (i < r) ? sc * ex2(grl - g2s[i]) * v[4 * i4 + e] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(AF + r * LDA + 32 * hc + 4 * i4) =
+                    make_float4(a[0], a[1], a[2], a[3]);
             }
-            *reinterpret_cast<float4 *>(AF + r * LDA + 4 * i4) = make_float4(a[0], a[1], a[2], a[3]);
         }
     }
+    tc_fence_before();
     __syncthreads();  // A complete; TMEM and K no longer read (K's buffer becomes T)
     if (warp == 0) {
         tc_fence_after();

@@ -18,7 +18,7 @@ namespace tc {
 using namespace sm100;
 
 constexpr int C = 64;          // chunk length (tokens)
-constexpr int LDA = 72;        // padded float32 row stride of A and T (16-B rows)
+constexpr int LDA = 68;        // padded float32 row stride of A and T (16-B rows)
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
