@@ -561,10 +561,13 @@ def run_ours(args):
                                       device) / n_d
         cd_bytes = wd.B * wd.H * (8 * wd.Dv * wd.Dk + esz * (2 * wd.Dk + 2 * wd.Dv) +
                                   4 * (2 * wd.Dk + wd.Dv))
+        cw_path = G.chunk_fwd_cw_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
         channel_wise = {
             "workload": "headline_T4k shape with a decay and an erase gate per key channel and "
                         "a write gate per value channel (float32 gates)",
-            "path": "CUDA cores, float32 arithmetic (2 launches per call)",
+            "path": ("tcgen05: per-chunk kernel (16-row blocks of the channel-wise decays, "
+                     "mma.sync) + sequential tcgen05 kernel, 2 launches per call"
+                     if cw_path == "tcgen05" else "CUDA cores, float32 arithmetic (2 launches)"),
             "ms_per_step": c_ms, "tokens_per_s": world * tokens / (c_ms * 1e-3),
             "achieved": c_bytes / (c_ms * 1e-3) / 1e9, "unit": "GB/s",
             "frac": c_bytes / (c_ms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes": c_bytes,
@@ -579,7 +582,7 @@ def run_ours(args):
     configs = None
     if not args.chunk_only:
         configs = []
-        for name, n_steps in (("bf16_T2k", 50), ("long_T32k", 20), ("wide_dk256_dv512", 3)):
+        for name, n_steps in (("bf16_T2k", 50), ("long_T32k", 20), ("wide_dk256_dv512", 20)):
             wc = I.workload(name)
             cin = I.chunk_inputs(wc, seed=wc.seed + rank, device=device)
             co = torch.empty((wc.B, wc.T, wc.H, wc.Dv), dtype=wc.torch_dtype, device=device)
@@ -601,9 +604,13 @@ def run_ours(args):
                 "workload": f"{name}: B={wc.B} H={wc.H} T={wc.T} Dk={wc.Dk} Dv={wc.Dv} "
                             f"chunk={wc.chunk} bf16, gates {wc.gate_law}, S0 {wc.s0_law}",
                 "path": G.chunk_fwd_path(wc.B, wc.T, wc.H, wc.Dk, wc.Dv, wc.chunk, wc.torch_dtype),
+                "variant": G.chunk_fwd_variant(wc.B, wc.T, wc.H, wc.Dk, wc.Dv, wc.chunk,
+                                               wc.torch_dtype),
                 "ms_per_step": c_ms, "tokens_per_s": world * wc.B * wc.T / (c_ms * 1e-3),
                 "hbm_frac": cb / (c_ms * 1e-3) / 1e9 / hbm_peak,
-                "tc_frac": cf / (c_ms * 1e-3) / 1e12 / tc_peak, "steps": n_steps})
+                "tc_frac": cf / (c_ms * 1e-3) / 1e12 / tc_peak, "tc_target": 0.5,
+                "bound": "tensor" if cf / cb > tc_peak * 1e12 / (hbm_peak * 1e9) else "hbm",
+                "steps": n_steps})
             del cin, co, cS, cw_
 
     cpu = None
