@@ -67,6 +67,7 @@ def _check(gdn, inp, tol=TOL_BF16, variant=None):
     og, sg = o.float().cpu().numpy(), S.cpu().numpy()
     assert np.isfinite(og).all() and np.isfinite(sg).all()
     eo, es = rel_l2(og, o_ref), rel_l2(sg, S_ref)
+    print(f"rel-L2 o={eo:.2e} S_T={es:.2e} shape={tuple(inp['q'].shape)} Dv={inp['v'].shape[3]}")
     assert eo <= tol and es <= tol, f"rel-L2 o={eo:.3e} S_T={es:.3e} (tol {tol})"
     return eo, es
 
