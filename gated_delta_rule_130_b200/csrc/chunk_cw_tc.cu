@@ -47,6 +47,22 @@
 #include "tc_common.cuh"
 
 namespace gdn {
+
+// Optional phase timeline of CTA (0,0,0) of the parallel kernel for performance
+// work: build with -DGDN_TRACE; that build alone exports gdn_trace_cw_read().
+#ifdef GDN_TRACE
+__device__ unsigned long long g_trace_cw[16];
+#define TCW(ev)                                                                           \
+    do {                                                                                  \
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)   \
+            g_trace_cw[ev] = clock64();                                                   \
+    } while (0)
+#else
+#define TCW(ev) \
+    do {        \
+    } while (0)
+#endif
+
 namespace cwt {
 
 using namespace sm100;
@@ -100,6 +116,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     float *PF = reinterpret_cast<float *>(sm + SM_PF);
     float *DS = reinterpret_cast<float *>(sm + SM_DS);
     __nv_bfloat16 *TB = reinterpret_cast<__nv_bfloat16 *>(sm + SM_AF);
+    TCW(0);
 
     // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread
     // -> (channel, quarter of the rows), so each row is read as 128 consecutive
@@ -130,6 +147,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
     }
     __syncthreads();
+    TCW(1);
     {   // running sums over the rows, per channel: each quarter locally, then the
         // totals of the earlier quarters are added
         float acc = 0.f;
@@ -147,6 +165,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         for (int rr = 0; rr < RQ; ++rr) LM[(rq * RQ + rr) * LDF + jc] += base;
     }
     __syncthreads();
+    TCW(2);
 
     // the two 8 x 8 diagonal sub-blocks of each diagonal 16-block, summed
     // directly: warps 4I .. 4I+3 take block I, each a quarter of the channels;
@@ -202,6 +221,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 }
         }
     }
+    TCW(3);
     // blocks I > J through the reference row m = 16 I - 1 (warps 0-5, one pair each)
     if (warp < 6) {
         const int I = warp == 0 ? 1 : (warp < 3 ? 2 : 3);
@@ -280,6 +300,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         *reinterpret_cast<float2 *>(PF + r1 * LDA + col) = make_float2(accP[2], accP[3]);
     }
     __syncthreads();  // A and P complete
+    TCW(4);
 
     // T = (I + A)^-1: diagonal blocks by substitution, the rest by block products
     // on warps 0-3 (named barrier 1)
@@ -287,6 +308,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     __syncthreads();
     if (tid < 128) tc::ut_offdiag4<1>(AF, TF, tid);
     __syncthreads();
+    TCW(5);
 
     // [P; T''] (T'' = T with zero columns for rows past the end), and T as bf16
     // over the dead A buffer; 8 threads per 128-byte row
@@ -318,6 +340,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         if (tid < DK) glk[tile * DK + tid] = tc::ex2(LM[(C - 1) * LDF + tid]);
     }
     __syncthreads();
+    TCW(6);
 
     // W = T (b o K o 2^Lam): warp w -> rows 16 (w % 4) .. + 15 (T is lower
     // triangular: chunk rows up to 16 (w % 4) + 15 contribute), channels
@@ -354,6 +377,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
     }
 
+    TCW(7);
     // the sequential kernel's token operands: Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
     for (int rr = 0; rr < RQ; ++rr) {
         const int r = rq * RQ + rr;
@@ -364,6 +388,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             kd[off] = __float2bfloat16_rn(KF[r * LDF + jc] * tc::ex2(LM[(C - 1) * LDF + jc] - lr));
         }
     }
+    TCW(8);
     // w o V, eight loads of each in flight per thread
     for (int base = 0; base < n * Dv; base += RB8 * THREADS) {
         float vv[RB8], ww[RB8];
@@ -385,9 +410,16 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             }
         }
     }
+    TCW(9);
 }
 
 }  // namespace cwt
+
+#ifdef GDN_TRACE
+extern "C" int gdn_trace_cw_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_trace_cw, sizeof(g_trace_cw));
+}
+#endif
 
 bool cw_tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
     return bf16 && chunk == cwt::C && Dk == cwt::DK && Dv % 64 == 0 && B >= 1 && T >= 1 &&
