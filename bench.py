@@ -516,13 +516,15 @@ def run_ours(args):
         b_ms = _max_over_ranks(time_loop(bwd_step, n_b, stream, world), world, device) / n_b
         bb = bwd_bytes(w, inp["S0"] is not None)
         b_gbs = bb / (b_ms * 1e-3) / 1e9
+        b_path = G.chunk_bwd_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
         backward = {"workload": "headline_T4k backward: dq, dk, dv, dlog_alpha, dbeta, dS0 "
                                 "from d_o and dS_T",
-                    "path": "CUDA cores, float32 arithmetic (4 launches per call)",
+                    "path": b_path,
+                    "kernels": BWD_KERNELS[b_path],
                     "ms_per_step": b_ms, "tokens_per_s": world * tokens / (b_ms * 1e-3),
                     "achieved": b_gbs, "unit": "GB/s", "peak": hbm_peak,
                     "frac": b_gbs / hbm_peak, "algorithmic_bytes": bb, "steps": n_b,
-                    "gpu_launches": 4 * n_b}
+                    "gpu_launches": len(BWD_KERNELS[b_path]) * n_b}
 
     # channel-wise gates (decay per key channel, erase and write gates) on the
     # headline shape, and their decode step at batch 256
@@ -650,6 +652,45 @@ def parse_workload(spec: str):
     return I.workload(name, **over)
 
 
+# the kernels one chunkwise backward launches, per path
+BWD_KERNELS = {
+    "tcgen05": ["gdn_utw_kernel (P, T'', W and T tiles)", "gdn_ut_kernel (the chunk states)",
+                "gdn_chunk_tc_kernel (the chunk states)", "gdn_bwd_chain_kernel (dS', dS0)",
+                "gdn_bwd_grads_kernel (dq, dk, dv, dlog_alpha, dbeta)"],
+    "simt": ["chunk_prep (T, P, g)", "gdn_ut_kernel (the chunk states)",
+             "gdn_chunk_tc_kernel (the chunk states)", "bwd_state", "bwd_grads"],
+}
+
+
+def run_bwd_only(args):
+    """--bwd-only: the chunkwise backward alone on --workload (one GPU, for counter
+    captures); prints one short JSON line."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from gated_delta_rule_130_b200 import binding as G
+    w = parse_workload(args.workload)
+    inp = {n: (t.to(device) if t is not None else None) for n, t in I.chunk_inputs(w).items()}
+    gen = torch.Generator().manual_seed(w.seed + 99)
+    bdo = torch.randn((w.B, w.T, w.H, w.Dv), generator=gen).to(w.torch_dtype).to(device)
+    bdS = torch.randn((w.B, w.H, w.Dv, w.Dk), generator=gen).to(device)
+    ws = torch.empty(max(G.chunk_bwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk,
+                                                    w.torch_dtype), 1),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        G.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                    bdo, bdS, chunk=w.chunk, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    steps = args.steps or 20
+    ms = time_loop(step, steps, torch.cuda.current_stream(device), 1) / steps
+    print(json.dumps({"leg": "backward", "workload": args.workload,
+                      "path": G.chunk_bwd_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype),
+                      "ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+                      "steps": steps}), flush=True)
+
+
 def run_cw_only(args):
     """--cw-only: the channel-wise-gate forward alone on --workload (one GPU, for
     counter captures); prints one short JSON line."""
@@ -724,8 +765,12 @@ def main():
                     help="time the decode step alone (one GPU, for counter captures)")
     ap.add_argument("--cw-only", action="store_true",
                     help="time the channel-wise-gate forward alone on --workload (one GPU)")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="time the chunkwise backward alone on --workload (one GPU)")
     args = ap.parse_args()
-    if args.decode_only:
+    if args.bwd_only:
+        run_bwd_only(args)
+    elif args.decode_only:
         run_decode_only(args)
     elif args.cw_only:
         run_cw_only(args)

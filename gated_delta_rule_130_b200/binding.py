@@ -63,6 +63,8 @@ def _load():
     lib.gdn_chunk_bwd.restype = I
     lib.gdn_chunk_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.gdn_chunk_bwd_workspace_size.restype = Z
+    lib.gdn_chunk_bwd_path.argtypes = [I, I, I, I, I, I, I]
+    lib.gdn_chunk_bwd_path.restype = I
     lib.gdn_chunk_fwd_cw.argtypes = [vp, vp, vp, fp, fp, fp, fp, vp, fp, I, I, I, I, I, I, I, vp,
                                      Z, vp]
     lib.gdn_chunk_fwd_cw.restype = I
@@ -254,6 +256,15 @@ def chunk_bwd(q, k, v, log_alpha, beta, S0, d_o, dS_T=None, chunk: int = 64, wor
                            _stream_ptr(dev))
     _check(st, "gdn_chunk_bwd")
     return dq, dk, dv, dla, dbe, dS0
+
+
+def chunk_bwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
+    """Which kernels chunk_bwd runs for these sizes: "tcgen05", "simt" or "none"."""
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    st = int(LIB.gdn_chunk_bwd_path(B, T, H, Dk, Dv, chunk, code))
+    if st < 0:
+        raise GdnError("gdn_chunk_bwd_path: invalid sizes")
+    return PATH_NAMES[st]
 
 
 def chunk_fwd_cw_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:

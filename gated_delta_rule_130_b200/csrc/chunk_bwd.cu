@@ -567,6 +567,7 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
 }  // namespace
 
 size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16) {
+    if (bwd_tc_supported(B, T, H, Dk, Dv, chunk, bf16)) return bwd_tc_workspace_bytes(B, T, H, Dv);
     size_t n = base_floats(B, T, H, Dk, Dv, chunk) * sizeof(float);
     if (tc_recompute(B, T, H, Dk, Dv, chunk, bf16))
         n += ((tc_workspace_bytes_fused(B, T, H, 0) + 255) & ~size_t(255)) +
@@ -584,6 +585,9 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              const float *dS_T, void *dq, void *dk, void *dv, float *dla,
                              float *dbeta, float *dS0, int B, int T, int H, int Dk, int Dv,
                              int chunk, bool bf16, void *workspace, cudaStream_t st) {
+    if (bwd_tc_supported(B, T, H, Dk, Dv, chunk, bf16))
+        return launch_chunk_bwd_tc(q, k, v, la, beta, S0, d_o, dS_T, dq, dk, dv, dla, dbeta, dS0, B,
+                                   T, H, Dv, workspace, st);
     return bf16 ? launch_bwd_t<__nv_bfloat16>(q, k, v, la, beta, S0, d_o, dS_T, dq, dk, dv, dla,
                                               dbeta, dS0, B, T, H, Dk, Dv, chunk, workspace, st)
                 : launch_bwd_t<float>(q, k, v, la, beta, S0, d_o, dS_T, dq, dk, dv, dla, dbeta,

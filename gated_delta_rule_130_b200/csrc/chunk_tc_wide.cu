@@ -86,8 +86,9 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 // ------------------------------------------------------------- UT kernel --
 // One CTA of 4 warps per (global chunk g, head h).  Outputs at tile index
-// g H + h: [P; T''] (128 x 64 bf16, row-major), W (64 x 256 bf16, row-major) and,
-// when normalising, 1/|q| and 1/|k| of the chunk's rows (2 x 64 float32).
+// g H + h: [P; T''] (128 x 64 bf16, row-major), W (64 x DK bf16, row-major),
+// optionally T itself (64 x 64 bf16, row-major, for the backward) and, when
+// normalising, 1/|q| and 1/|k| of the chunk's rows (2 x 64 float32).
 // The chunk's K and Q rows arrive by TMA (128-byte swizzle), interleaved per
 // 64-key block as K | Q so that [K; Q] is one 128-row operand, and both
 // products are tcgen05.mma into tensor memory:
@@ -122,7 +123,8 @@ __global__ void __launch_bounds__(UT_THREADS, DK == 256 ? 2 : 3)
 gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                __nv_bfloat16 *__restrict__ pt, __nv_bfloat16 *__restrict__ wt,
-               float *__restrict__ rqk, const Seqs sq, int H, unsigned flags) {
+               __nv_bfloat16 *__restrict__ tr, float *__restrict__ rqk, const Seqs sq, int H,
+               unsigned flags) {
     using L = UtDims<DK>;
     constexpr int KB = L::KB, SM_AF = L::SM_AF, SM_TF = L::SM_TF, SM_G = L::SM_G,
                   SM_UBAR = L::SM_UBAR, W_ELEMS = L::W_ELEMS;
@@ -329,6 +331,13 @@ gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             *reinterpret_cast<uint4 *>(tp + sw128_offset(rr, 2 * i0)) =
                 make_uint4(tc::pack_bf16(y[0], y[1]), tc::pack_bf16(y[2], y[3]),
                            tc::pack_bf16(y[4], y[5]), tc::pack_bf16(y[6], y[7]));
+            if (tr) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = i0 + e <= rr ? tv[e] : 0.f;
+                *reinterpret_cast<uint4 *>(tr + tile * C * C + rr * C + i0) =
+                    make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                               tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+            }
         }
     }
     fence_async_smem();
@@ -952,7 +961,7 @@ cudaError_t launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorM
     if (e != cudaSuccess) return e;
     if (total_chunks > 0)
         ut<<<dim3((unsigned)total_chunks, p.H, 1), UT_THREADS, ut_smem, st>>>(
-            mq, mk, log_alpha, beta, pt, wt, rqk, p.sq, p.H, p.flags);
+            mq, mk, log_alpha, beta, pt, wt, nullptr, rqk, p.sq, p.H, p.flags);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the CTAs may set up while the UT kernel
@@ -1063,6 +1072,29 @@ cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mw, mp, p);
     if (e != cudaSuccess) return e;
+    return cudaPeekAtLastError();
+}
+
+// The parallel kernel alone for the backward (Dk = 128, gates as given, B
+// sequences of T tokens): per chunk and head the [P; T''] tile, the W tile and
+// T itself, at tile index (b NT + c) H + h.
+cudaError_t launch_ut_tiles_bwd(const void *q, const void *k, const float *log_alpha,
+                                const float *beta, int B, int T, int H, void *pt, void *wt,
+                                void *tr, cudaStream_t st) {
+    constexpr int DK = 128;
+    const long long NT = ((long long)T + tc::C - 1) / tc::C;
+    if (B < 1 || NT < 1) return cudaSuccess;
+    CUtensorMap mq, mk;
+    if (!tc::make_map(&mq, q, 1, B * T, H, DK) || !tc::make_map(&mk, k, 1, B * T, H, DK))
+        return cudaErrorInvalidValue;
+    auto *ut = tcw::gdn_utw_kernel<DK, false>;
+    constexpr int ut_smem = tcw::UtDims<DK>::UT_SMEM;
+    cudaError_t e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize, ut_smem);
+    if (e != cudaSuccess) return e;
+    const tc::Seqs sq{nullptr, nullptr, nullptr, T, B};
+    ut<<<dim3((unsigned)(B * NT), H, 1), tcw::UT_THREADS, ut_smem, st>>>(
+        mq, mk, log_alpha, beta, static_cast<__nv_bfloat16 *>(pt),
+        static_cast<__nv_bfloat16 *>(wt), static_cast<__nv_bfloat16 *>(tr), nullptr, sq, H, 0u);
     return cudaPeekAtLastError();
 }
 

@@ -346,6 +346,14 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+int gdn_chunk_bwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
+    if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::bwd_supported(Dk, chunk))
+        return -1;
+    if (empty_problem(B, T, H)) return GDN_PATH_NONE;
+    if (gdn::bwd_tc_supported(B, T, H, Dk, Dv, chunk, dtype == GDN_BF16)) return GDN_PATH_TCGEN05;
+    return GDN_PATH_SIMT;
+}
+
 int gdn_chunk_fwd_cw_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
     if (check_sizes(B, T, H, Dk, Dv, chunk, dtype) != GDN_OK || !gdn::cw_supported(Dk, chunk))
         return -1;
@@ -453,11 +461,12 @@ gdn_status_t gdn_debug_withhold_first_arrival(int enable) {
 
 gdn_status_t gdn_check_device_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return GDN_ERR_CUDA;
-    unsigned int flag = 0, flag_wide = 0;
+    unsigned int flag = 0, flag_wide = 0, flag_bwd = 0;
     if (gdn::read_and_clear_device_error(&flag) != cudaSuccess ||
-        gdn::read_and_clear_device_error_wide(&flag_wide) != cudaSuccess)
+        gdn::read_and_clear_device_error_wide(&flag_wide) != cudaSuccess ||
+        gdn::read_and_clear_device_error_bwd(&flag_bwd) != cudaSuccess)
         return GDN_ERR_CUDA;
-    return (flag | flag_wide) ? GDN_ERR_CUDA : GDN_OK;
+    return (flag | flag_wide | flag_bwd) ? GDN_ERR_CUDA : GDN_OK;
 }
 
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -54,6 +54,21 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              float *dbeta, float *dS0, int B, int T, int H, int Dk, int Dv,
                              int chunk, bool bf16, void *workspace, cudaStream_t st);
 
+// Tensor-core chunkwise backward (bf16, Dk = 128, chunk 64, Dv 64 or 128):
+// chunk_bwd_tc.cu, reached through launch_chunk_bwd.  Its recompute uses the
+// precomputed variant's parallel kernel for the [P; T''], W and T tiles of every
+// chunk (chunk_tc_wide.cu, launch_ut_tiles_bwd) and the fused forward for S_hist.
+bool bwd_tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
+size_t bwd_tc_workspace_bytes(int B, int T, int H, int Dv);
+cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, const float *la,
+                                const float *beta, const float *S0, const void *d_o,
+                                const float *dS_T, void *dq, void *dk, void *dv, float *dla,
+                                float *dbeta, float *dS0, int B, int T, int H, int Dv,
+                                void *workspace, cudaStream_t st);
+cudaError_t launch_ut_tiles_bwd(const void *q, const void *k, const float *log_alpha,
+                                const float *beta, int B, int T, int H, void *pt, void *wt,
+                                void *tr, cudaStream_t st);
+
 // Channel-wise gates (decay per key channel, erase gate b on the key side,
 // write gate w on the value side; CUDA cores, Dk <= 128): chunk_cw.cu.
 // log alpha and b are [B,T,H,Dk] float32, w is [B,T,H,Dv] float32.
@@ -139,6 +154,7 @@ cudaError_t launch_chunk_cw_tc(const void *q, const void *k, const void *v, cons
 // times out (synchronous).
 cudaError_t read_and_clear_device_error(unsigned int *flag);
 cudaError_t read_and_clear_device_error_wide(unsigned int *flag);  // the Dk = 256 kernel's flag
+cudaError_t read_and_clear_device_error_bwd(unsigned int *flag);   // the backward's tcgen05 kernels
 // Test hook: the sequential tcgen05 kernel withholds its first stage's arrival
 // (every CTA then times out, about two seconds, and sets that flag).
 cudaError_t set_withhold_first_arrival(bool on);

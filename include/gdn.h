@@ -249,15 +249,20 @@ gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v,
  *   outputs dq, dk [B,T,H,Dk] and dv [B,T,H,Dv] in `dtype`; dlog_alpha, dbeta
  *           [B,T,H] float32; dS0 [B,H,Dv,Dk] float32 or NULL (not written).
  *
- * Arithmetic is float32 on the CUDA cores (bf16 inputs are widened; bf16
- * gradients are rounded once at the end).  Three launches: the forward's
- * per-chunk T, P, g and chunk states are recomputed into the workspace
- * (gdn_chunk_bwd_workspace_size bytes: (2 C^2 + C + 2 Dv Dk) floats per chunk
- * and head), the state gradient is walked back over the chunks, and the
- * per-chunk gradients are formed in parallel.  Limits as for the forward plus
- * Dk <= 128 (GDN_ERR_UNSUPPORTED otherwise).  Outputs must not overlap any
- * input or each other; the workspace must not overlap anything.  T = 0 only
- * sets dS0 = dS_T.  Enqueued on `stream`.
+ * Two paths (gdn_chunk_bwd_path).  GDN_PATH_TCGEN05 (bf16, Dk = 128, chunk 64,
+ * Dv 64 or 128): the forward's chunk tiles (P, T'', W, T) and the state
+ * entering every chunk are recomputed on the tensor cores, the state gradient
+ * is walked back over the chunks with dS^T in tensor memory, and the per-chunk
+ * gradients are tcgen05 products in parallel over the chunks; bf16 operands,
+ * float32 accumulation.  GDN_PATH_SIMT otherwise: float32 on the CUDA cores
+ * (bf16 inputs widened), the same three steps.  bf16 gradients are rounded
+ * once at the end.  The workspace (gdn_chunk_bwd_workspace_size bytes) holds
+ * the recomputed tiles and chunk states and the state gradients.  Limits as
+ * for the forward plus Dk <= 128 (GDN_ERR_UNSUPPORTED otherwise).  Outputs
+ * must not overlap any input or each other; the workspace must not overlap
+ * anything.  T = 0 only sets dS0 = dS_T.  Enqueued on `stream`; a bounded
+ * wait of the tensor-core kernels that ran out is reported by
+ * gdn_check_device_status.
  */
 gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta, const float *S0,
@@ -268,6 +273,10 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v,
                            void *stream);
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int Dk, int Dv, int chunk,
                                     gdn_dtype_t dtype);
+/* Which kernels gdn_chunk_bwd runs for these sizes (gdn_path_t; -1 for invalid
+ * or unsupported sizes): GDN_PATH_TCGEN05 for bf16, Dk = 128, chunk 64, Dv 64
+ * or 128, else GDN_PATH_SIMT.  The workspace size depends on it. */
+int gdn_chunk_bwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype);
 
 /*
  * Channel-wise gates.  "Gated DeltaNet-2: Decoupling Erase and Write in Linear

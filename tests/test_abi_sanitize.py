@@ -85,6 +85,8 @@ cudaError_t launch_decode_cw(const void *, const void *, const void *, const flo
                              cudaStream_t) { return ok(); }
 cudaError_t read_and_clear_device_error(unsigned int *flag) { *flag = 0; return ok(); }
 cudaError_t read_and_clear_device_error_wide(unsigned int *flag) { *flag = 0; return ok(); }
+cudaError_t read_and_clear_device_error_bwd(unsigned int *flag) { *flag = 0; return ok(); }
+bool bwd_tc_supported(int, int, int, int, int, int, bool) { return false; }
 cudaError_t set_withhold_first_arrival(bool) { return ok(); }
 }  // namespace gdn
 """
