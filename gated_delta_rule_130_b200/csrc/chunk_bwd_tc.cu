@@ -36,8 +36,8 @@
 // gamma is tiny, and with it the term beta_r Z_r . X_r.
 //
 // Launches (one stream): the precomputed forward's parallel kernel for the
-// [P; T''], W and T tiles (chunk_tc_wide.cu), the fused tensor-core forward for
-// the state entering every chunk (chunk_tc.cu, S_hist), then
+// [P; T''], W and T tiles and its sequential kernel, fed those tiles, for the
+// state entering every chunk in bf16 (chunk_tc_wide.cu), then
 //  1. gdn_bwd_chain_kernel: one CTA per (sequence, head, 64 value channels)
 //     walking the chunks backwards with dS^T (128 keys x 64 values, float32) in
 //     tensor memory; per chunk R = K dS'^T (M = 64), dU' = P^T dO + D o R in an
@@ -64,6 +64,23 @@ namespace gdn {
 
 // Set by a CTA of the backward's tensor-core kernels that gave up waiting.
 __device__ unsigned int g_bwd_error = 0;
+
+// Optional phase timeline of two CTAs of the gradient kernel (chunk 0 and chunk
+// 63 of head 8, batch 0) for performance work: build with -DGDN_TRACE; that
+// build alone exports gdn_trace_bwd_read().  Compiled out otherwise.
+#ifdef GDN_TRACE
+__device__ unsigned long long g_trace_bwd[2 * 16];
+#define TG(ev)                                                                          \
+    do {                                                                                \
+        if (threadIdx.x == 0 && blockIdx.z == 0 &&                                      \
+            ((blockIdx.x == 0 && blockIdx.y == 0) || (blockIdx.x == 63 && blockIdx.y == 8))) \
+            g_trace_bwd[(blockIdx.x == 0 ? 0 : 16) + (ev)] = clock64();                 \
+    } while (0)
+#else
+#define TG(ev) \
+    do {       \
+    } while (0)
+#endif
 
 namespace btc {
 
@@ -476,9 +493,13 @@ struct L {
     static constexpr int SM_DP = SM_V;          // dP o Gamma over V
     static constexpr int SM_EE = SM_DU;         // E + E^T over U'
     static constexpr int SM_ES = SM_ZB;         // E (row-major scratch) over -beta gamma o Z
-    // per-row float arrays in SM_MISC
-    enum { F_G2 = 0, F_BE, F_GAM, F_DCY, F_UR, F_ZN, F_ZX, F_XR, F_XC, F_DG, F_QS, NF };
-    static constexpr int SM_SCAL = SM_MISC + NF * 64 * 4;   // [0] <dS', S>, [1] gamma_last, [2..3] sums
+    // per-row float arrays in SM_MISC: the gate vectors, then partial sums written
+    // with plain stores (no shared-memory atomics): two column halves per row for
+    // the row sums, four row quarters per column for the column sums
+    enum { F_G2 = 0, F_BE, F_GAM, F_DCY, F_UR = 4, F_ZN = 6, F_ZX = 8, F_XR = 10, F_DG = 12,
+           F_QS = 14, F_XC = 16, NF = 20 };
+    // [1] gamma_last, [2] [4] the final scans' warp totals, [8 + w] warp w's part of <dS', S>
+    static constexpr int SM_SCAL = SM_MISC + NF * 64 * 4;
     static constexpr int SM_BAR = SM_SCAL + 64;
     static constexpr int SMEM_BYTES = SM_BAR + 5 * 8 + 16 + 1024;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -489,13 +510,14 @@ struct L {
 // dQ 128..255, dK 256..383.
 constexpr uint32_t TM_KK = 448, TM_DP = 0, TM_DA = 64, TM_Q2 = 128, TM_K2 = 256, TM_COLS = 512;
 
+// The state entering each chunk and the gradient of the state leaving it come by
+// TMA from [B*H][NT][Dv][Dk] bf16 arrays (tm_sh, tm_dsh: boxes of 64 keys x DV rows).
 struct Params {
     const float *log_alpha, *beta;
-    const float *S_hist;                // [B*H][NT][Dv][Dk] float32 (the state entering each chunk)
-    const __nv_bfloat16 *dS_hist;       // [B*H][NT][Dv][Dk] bf16 (the gradient of the state leaving it)
     __nv_bfloat16 *dq, *dk, *dv;
     float *dla, *dbeta;
     int T, H, NT;
+    int pf_stride;  // the SM count: each CTA prefetches into L2 the inputs of CTA + pf_stride
 };
 
 template <int DV>
@@ -503,6 +525,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_pt, const __grid_constant__ CUtensorMap tm_t,
+                     const __grid_constant__ CUtensorMap tm_sh, const __grid_constant__ CUtensorMap tm_dsh,
                      const Params p) {
     using Ly = L<DV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -518,17 +541,16 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           *dcys = fv + Ly::F_DCY * 64;
     float *rs_ur = fv + Ly::F_UR * 64, *rs_zn = fv + Ly::F_ZN * 64, *rs_zx = fv + Ly::F_ZX * 64,
           *rs_x = fv + Ly::F_XR * 64, *cs_x = fv + Ly::F_XC * 64, *rs_dg = fv + Ly::F_DG * 64,
-          *rs_qs = fv + Ly::F_QS * 64;
+          *rs_qs = fv + Ly::F_QS * 64;  // [hf][64] (cs_x: [quarter][64])
     float *scal = reinterpret_cast<float *>(base + Ly::SM_SCAL);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = p.T, H = p.H, NT = p.NT, t0 = c * C;
     const int tile = (b * NT + c) * H + h;
-    const size_t hist = (((size_t)b * H + h) * NT + c) * (size_t)DV * DK;
+    const int hist = (b * H + h) * NT + c;
+    TG(0);
 
-    for (int i = tid; i < (Ly::NF - Ly::F_UR) * 64; i += NTHREADS) fv[Ly::F_UR * 64 + i] = 0.f;
-    if (tid < 16) scal[tid] = 0.f;
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(cx.bar + i, 1);
         *cx.abort = 0u;
@@ -542,10 +564,11 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    TG(1);
 
     if (tid == 0) {
         uint64_t *fb = cx.bar + 0;
-        mbar_arrive_expect_tx(fb, 4 * PANEL + 2 * Ly::VB + 3 * PANEL);
+        mbar_arrive_expect_tx(fb, 4 * PANEL + 2 * Ly::VB + 3 * PANEL + 4 * DV * 128);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
             tma_load_4d(base + Ly::SM_K + kb * PANEL, &tm_k, fb, kb * 64, h, t0, b);
@@ -558,6 +581,34 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         tma_load_3d(base + Ly::SM_P, &tm_pt, fb, 0, 0, tile);
         tma_load_3d(base + Ly::SM_T, &tm_t, fb, 0, 0, tile);
+        // [S; dS'] per 64-key panel: S rows 0 .. DV - 1, dS' rows DV .. 2 DV - 1
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL, &tm_sh, fb, kb * 64, 0, hist);
+            tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL + DV * 128, &tm_dsh, fb, kb * 64, 0, hist);
+        }
+        // one CTA per SM: the CTA one wave later (linear index + SM count) finds its
+        // inputs in L2, their DRAM reads overlapping this CTA's products
+        const long long lin = blockIdx.x + (long long)NT * (blockIdx.y + (long long)H * blockIdx.z);
+        const long long nxt = lin + p.pf_stride;
+        if (p.pf_stride > 0 && nxt < (long long)NT * H * gridDim.z) {
+            const int c2 = (int)(nxt % NT), h2 = (int)((nxt / NT) % H), b2 = (int)(nxt / ((long long)NT * H));
+            const int t2 = c2 * C, tile2 = (b2 * NT + c2) * H + h2, hist2 = (b2 * H + h2) * NT + c2;
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+                tma_prefetch_l2_4d(&tm_k, kb * 64, h2, t2, b2);
+                tma_prefetch_l2_4d(&tm_q, kb * 64, h2, t2, b2);
+                tma_prefetch_l2_3d(&tm_sh, kb * 64, 0, hist2);
+                tma_prefetch_l2_3d(&tm_dsh, kb * 64, 0, hist2);
+            }
+#pragma unroll
+            for (int vb = 0; vb < DV / 64; ++vb) {
+                tma_prefetch_l2_4d(&tm_v, vb * 64, h2, t2, b2);
+                tma_prefetch_l2_4d(&tm_do, vb * 64, h2, t2, b2);
+            }
+            tma_prefetch_l2_3d(&tm_pt, 0, 0, tile2);
+            tma_prefetch_l2_3d(&tm_t, 0, 0, tile2);
+        }
     }
     if (warp == 0) {
         // gates of the chunk's rows lane, lane + 32 (rows past the end: 0)
@@ -592,33 +643,8 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         if (lane == 0) scal[1] = tc::ex2(glast);
     }
-    {   // S (float32) and dS' (bf16) -> [S; dS'] per key panel, and <dS', S>
-        float dot = 0.f;
-        for (int idx = tid; idx < DV * 16; idx += NTHREADS) {
-            const int i = idx >> 4, ch = idx & 15, kp = ch >> 3, cb = (ch & 7) * 16;
-            const float4 *sp = reinterpret_cast<const float4 *>(p.S_hist + hist + (size_t)i * DK + ch * 8);
-            const float4 a = sp[0], a2 = sp[1];
-            const uint4 d = *reinterpret_cast<const uint4 *>(p.dS_hist + hist + (size_t)i * DK + ch * 8);
-            uint8_t *pan = base + Ly::SM_SD + kp * Ly::SD_PANEL;
-            *reinterpret_cast<uint4 *>(pan + sw128_offset(i, cb)) =
-                make_uint4(tc::pack_bf16(a.x, a.y), tc::pack_bf16(a.z, a.w),
-                           tc::pack_bf16(a2.x, a2.y), tc::pack_bf16(a2.z, a2.w));
-            *reinterpret_cast<uint4 *>(pan + sw128_offset(DV + i, cb)) = d;
-            const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
-            const float sv[8] = {a.x, a.y, a.z, a.w, a2.x, a2.y, a2.z, a2.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
-                dot = fmaf(f.x, sv[2 * e], fmaf(f.y, sv[2 * e + 1], dot));
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        if (lane == 0) atomicAdd(&scal[0], dot);
-    }
-    fence_async_smem();
-    tc_fence_before();
     __syncthreads();
+    TG(2);
 
     // epilogue threads: warp w -> TMEM lanes 32 (w % 4) + l, chunk row r = 16 (w % 4) + l
     // for l < 16 (M = 64 layout), column half hf = w / 4
@@ -642,6 +668,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (tid == 0) {
         const bool landed = tc::wait_bar(cx, 0, 0);
         tc_fence_after();
+        TG(3);
         if (landed) {
 #pragma unroll
             for (int j = 0; j < DK / 16; ++j)
@@ -660,6 +687,28 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     bool ok = tc::warp_wait(cx, 1, 0);
     tc_fence_after();
+    TG(4);
+    {   // <dS', S> from the two bf16 tiles (same swizzle: element for element at a
+        // fixed distance of DV rows), after this thread has seen the copies land
+        ok = tc::warp_wait(cx, 0, 0) && ok;
+        float dot = 0.f;
+        for (int idx = tid; idx < 2 * DV * 8; idx += NTHREADS) {
+            const int kb = idx / (DV * 8), o = (idx % (DV * 8)) * 16;
+            const uint8_t *pan = base + Ly::SM_SD + kb * Ly::SD_PANEL;
+            const uint4 a = *reinterpret_cast<const uint4 *>(pan + o);
+            const uint4 d = *reinterpret_cast<const uint4 *>(pan + DV * 128 + o);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[e]));
+                const float2 fd = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
+                dot = fmaf(fa.x, fd.x, fmaf(fa.y, fd.y, dot));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        if (lane == 0) scal[8 + warp] = dot;
+    }
     constexpr int NPC = DV / 32;  // 16-value pieces per thread
     // epilogue A: X = -gamma o (K S^T), dU' = P^T dO + D o (K dS'^T)
 #pragma unroll 1
@@ -685,6 +734,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_before();
     __syncthreads();
 
+    TG(5);
     // ---------------- phase B: U' = T'' V + T'' X, Z = T^T dU'
     if (tid == 0) {
         tc_fence_after();
@@ -707,6 +757,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     ok = tc::warp_wait(cx, 2, 0) && ok;
     tc_fence_after();
+    TG(6);
     // epilogue B: U', D o U', Z, -beta gamma o Z, dV = beta o Z, gamma o dO (over X,
     // after the thread's own X piece is read), row dots
     {
@@ -752,15 +803,16 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
         if (act) {
-            atomicAdd(&rs_ur[r], ur);
-            atomicAdd(&rs_zn[r], zv + zx);
-            atomicAdd(&rs_zx[r], zx);
+            rs_ur[64 * hf + r] = ur;
+            rs_zn[64 * hf + r] = zv + zx;
+            rs_zx[64 * hf + r] = zx;
         }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
+    TG(7);
     // ---------------- phase C: dP = dO U'^T, dA' = Z U'^T, dQ = (gamma o dO) S,
     //                  dK = (D o U') dS' + (-beta gamma o Z) S
     if (tid == 0) {
@@ -785,12 +837,14 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     ok = tc::warp_wait(cx, 3, 0) && ok;
     tc_fence_after();
+    TG(8);
     // epilogue C (row r, columns 32 hf .. + 31 of the 64 x 64 matrices):
     // dP o Gamma (bf16 tile), E (row-major scratch), dbeta's and dg's sums, and
     // gamma_r (dO S)_r . q_r from the dQ accumulator before (dP o Gamma) K joins it
     {
         const float br = act ? bes[r] : 0.f, g2r = act ? g2s[r] : 0.f;
-        __nv_bfloat16 *es = reinterpret_cast<__nv_bfloat16 *>(base + Ly::SM_ES);
+        // E^T (row-major scratch): entry (i, r) holds E_ri
+        __nv_bfloat16 *est = reinterpret_cast<__nv_bfloat16 *>(base + Ly::SM_ES);
         float xr = 0.f, dgr = 0.f, qs = 0.f;
 #pragma unroll 1
         for (int pc = 0; pc < 4; ++pc) {
@@ -804,7 +858,9 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int j = 0; j < 16; ++j) qs = fmaf(x[j], qv[j], qs);
             }
         }
-#pragma unroll 1
+        TG(13);
+        float ev[2][16];
+#pragma unroll
         for (int pc = 0; pc < 2; ++pc) {
             const int i0 = 32 * hf + 16 * pc;
             float dp[16], da[16], kk[16];
@@ -814,7 +870,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tmem_wait_ld();
             float pv[16];
             if (act) load16_bf16(base + Ly::SM_P, r, i0 >> 4, pv);
-            float col[16], ev[16];
+            float col[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = i0 + e;
@@ -826,14 +882,16 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const float x = (slow ? dp[e] * pv[e] : 0.f) + dA * br * Gk;
                 xr += x;
                 dgr = fmaf(dA, Gk, dgr);
-                ev[e] = br * dA * G;
+                ev[pc][e] = br * dA * G;
                 col[e] = x;
                 dp[e] = dpg;
             }
             if (act) {
                 tc::store16_bf16(base + Ly::SM_DP, r, i0 >> 4, dp);
-                store16_global_bf16(es + r * C + i0, ev);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) est[(i0 + e) * C + r] = __float2bfloat16_rn(ev[pc][e]);
             }
+            // column sums over this warp's 16 rows (lanes 16-31 hold zeros)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 float v = col[e];
@@ -841,25 +899,40 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 v += __shfl_xor_sync(0xffffffffu, v, 4);
                 v += __shfl_xor_sync(0xffffffffu, v, 2);
                 v += __shfl_xor_sync(0xffffffffu, v, 1);
-                if (lane == 0) atomicAdd(&cs_x[i0 + e], v);
+                col[e] = v;
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) cs_x[64 * q + i0 + e] = col[e];
             }
         }
         if (act) {
-            atomicAdd(&rs_x[r], xr);
-            atomicAdd(&rs_dg[r], dgr);
-            atomicAdd(&rs_qs[r], qs);
+            rs_x[64 * hf + r] = xr;
+            rs_dg[64 * hf + r] = dgr;
+            rs_qs[64 * hf + r] = qs;
         }
-        __syncthreads();  // E complete
+        TG(14);
+        __syncthreads();  // E^T complete
+        TG(15);
         if (act) {
 #pragma unroll
             for (int pc = 0; pc < 2; ++pc) {
                 const int i0 = 32 * hf + 16 * pc;
-                float ee[16];
+                float et[16], ee[16];
+                // row r of E^T is column r of E: E_ir for the rows i > r
+                const uint4 *src = reinterpret_cast<const uint4 *>(est + r * C + i0);
+                const uint4 u0 = src[0], u1 = src[1];
+                const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                    et[2 * e] = f.x;
+                    et[2 * e + 1] = f.y;
+                }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int i = i0 + e;
-                    ee[e] = i < r ? __bfloat162float(es[r * C + i])
-                                  : (i > r ? __bfloat162float(es[i * C + r]) : 0.f);
+                    ee[e] = i < r ? ev[pc][e] : (i > r ? et[e] : 0.f);
                 }
                 tc::store16_bf16(base + Ly::SM_EE, r, i0 >> 4, ee);
             }
@@ -869,6 +942,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_before();
     __syncthreads();
 
+    TG(9);
     // ---------------- phase D: dQ += (dP o Gamma) K, dK += (dP o Gamma)^T Q + (E + E^T) K
     if (tid == 0) {
         tc_fence_after();
@@ -888,6 +962,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     ok = tc::warp_wait(cx, 4, 0) && ok;
     tc_fence_after();
+    TG(10);
     // final epilogue: dq, dk (row r, keys 64 hf .. + 63)
     {
         const bool in = act && t0 + r < T;
@@ -907,15 +982,23 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
+    TG(11);
     if (tid < C) {
         // dlog alpha_r = (the sum of dg over rows >= r) + (the sum of the state
         // update's decay terms over rows < r); warp 0 holds rows 0-31, warp 1 rows 32-63
         const int rr = tid;
-        float dg = rs_qs[rr] + rs_x[rr] - cs_x[rr] + bes[rr] * rs_zx[rr];
-        if (rr == C - 1) dg += scal[1] * scal[0];
+        const float xc = cs_x[rr] + cs_x[64 + rr] + cs_x[128 + rr] + cs_x[192 + rr];
+        float dg = rs_qs[rr] + rs_qs[64 + rr] + rs_x[rr] + rs_x[64 + rr] - xc +
+                   bes[rr] * (rs_zx[rr] + rs_zx[64 + rr]);
+        if (rr == C - 1) {
+            float dot = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) dot += scal[8 + w];
+            dg += scal[1] * dot;
+        }
         // the prefix is an exclusive scan of the shifted terms, never an inclusive
         // sum minus the row's own term (D = 1 on the last row makes that term large)
-        const float hterm = dcys[rr] * rs_ur[rr];
+        const float hterm = dcys[rr] * (rs_ur[rr] + rs_ur[64 + rr]);
         float hp = __shfl_up_sync(0xffffffffu, hterm, 1);
         if (lane == 0) hp = 0.f;
 #pragma unroll
@@ -934,9 +1017,10 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (ok && t0 + rr < T) {
             const size_t gi = ((size_t)b * T + t0 + rr) * H + h;
             p.dla[gi] = dlog;
-            p.dbeta[gi] = rs_zn[rr] + rs_dg[rr];
+            p.dbeta[gi] = rs_zn[rr] + rs_zn[64 + rr] + rs_dg[rr] + rs_dg[64 + rr];
         }
     }
+    TG(12);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -975,25 +1059,22 @@ bool make_map_wt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 }
 
 struct Ws {
-    __nv_bfloat16 *pt, *wt, *tr, *dS_hist, *o_scratch;
-    float *S_hist;
-    void *fused;
+    __nv_bfloat16 *pt, *wt, *tr, *S_hist, *dS_hist, *o_scratch;
     size_t bytes;
 };
 
 inline size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace: [P; T''] tiles | W tiles | T tiles | S_hist (float32) | dS_hist (bf16) |
-// the fused forward's workspace | its scratch output.
+// Workspace: [P; T''] tiles | W tiles | T tiles | S_hist | dS_hist (both bf16) |
+// the recompute's scratch output.
 Ws carve(void *base, int B, int T, int H, int Dv) {
     const size_t NT = ((size_t)T + C - 1) / C, tiles = (size_t)B * NT * H;
     const size_t states = (size_t)B * H * NT * Dv * DK;
-    const size_t sz[7] = {tiles * 2 * C * C * 2, tiles * C * DK * 2, tiles * C * C * 2, states * 4,
-                          states * 2, tc_workspace_bytes_fused(B, T, H, 0u),
-                          (size_t)B * T * H * Dv * 2};
+    const size_t sz[6] = {tiles * 2 * C * C * 2, tiles * C * DK * 2, tiles * C * C * 2, states * 2,
+                          states * 2, (size_t)B * T * H * Dv * 2};
     uint8_t *p = static_cast<uint8_t *>(base);
-    size_t off[7], o = 0;
-    for (int i = 0; i < 7; ++i) {
+    size_t off[6], o = 0;
+    for (int i = 0; i < 6; ++i) {
         off[i] = o;
         o += up256(sz[i]);
     }
@@ -1001,23 +1082,40 @@ Ws carve(void *base, int B, int T, int H, int Dv) {
     w.pt = reinterpret_cast<__nv_bfloat16 *>(p + off[0]);
     w.wt = reinterpret_cast<__nv_bfloat16 *>(p + off[1]);
     w.tr = reinterpret_cast<__nv_bfloat16 *>(p + off[2]);
-    w.S_hist = reinterpret_cast<float *>(p + off[3]);
+    w.S_hist = reinterpret_cast<__nv_bfloat16 *>(p + off[3]);
     w.dS_hist = reinterpret_cast<__nv_bfloat16 *>(p + off[4]);
-    w.fused = p + off[5];
-    w.o_scratch = reinterpret_cast<__nv_bfloat16 *>(p + off[6]);
+    w.o_scratch = reinterpret_cast<__nv_bfloat16 *>(p + off[5]);
     w.bytes = o;
     return w;
+}
+
+// [n, Dv, 128] bf16 state arrays: box of 64 keys x `rows` value rows of one state.
+bool make_map_states(CUtensorMap *m, const void *ptr, int Dv, int rows, long long n) {
+    auto enc = tc::encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)Dv, (cuuint64_t)n};
+    cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)Dv * DK * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int DV>
 cudaError_t launch_grads(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                          const CUtensorMap &mdo, const CUtensorMap &mpt, const CUtensorMap &mt,
-                         const grads::Params &gp, int B, cudaStream_t st) {
+                         const grads::Params &gp, const Ws &w, int B, cudaStream_t st) {
+    const long long n_hist = (long long)B * gp.H * gp.NT;
+    CUtensorMap msh, mdsh;
+    if (!make_map_states(&msh, w.S_hist, DV, DV, n_hist) ||
+        !make_map_states(&mdsh, w.dS_hist, DV, DV, n_hist))
+        return cudaErrorInvalidValue;
     auto *kern = grads::gdn_bwd_grads_kernel<DV>;
     constexpr int smem = grads::L<DV>::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(gp.NT, gp.H, B), grads::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mpt, mt, gp);
+    kern<<<dim3(gp.NT, gp.H, B), grads::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mpt, mt, msh, mdsh, gp);
     return cudaPeekAtLastError();
 }
 
@@ -1042,10 +1140,8 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
     const long long n_tiles = (long long)B * NT * H;
     Ws w = carve(workspace, B, T, H, Dv);
     // recompute: the chunk tiles, then the state entering every chunk
-    cudaError_t e = launch_ut_tiles_bwd(q, k, la, beta, B, T, H, w.pt, w.wt, w.tr, st);
-    if (e != cudaSuccess) return e;
-    e = launch_chunk_tc(q, k, v, la, beta, S0, w.o_scratch, nullptr, B, T, H, DK, Dv, 0u, w.fused,
-                        st, w.S_hist);
+    cudaError_t e = launch_recompute_bwd(q, k, v, la, beta, S0, B, T, H, Dv, w.pt, w.wt, w.tr,
+                                         w.S_hist, w.o_scratch, st);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mdo, mw, mp, mpt, mt;
     if (!tc::make_map(&mq, q, B, T, H, DK) || !tc::make_map(&mk, k, B, T, H, DK) ||
@@ -1073,8 +1169,6 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
     grads::Params gp;
     gp.log_alpha = la;
     gp.beta = beta;
-    gp.S_hist = w.S_hist;
-    gp.dS_hist = w.dS_hist;
     gp.dq = static_cast<__nv_bfloat16 *>(dq);
     gp.dk = static_cast<__nv_bfloat16 *>(dk);
     gp.dv = static_cast<__nv_bfloat16 *>(dv);
@@ -1083,9 +1177,22 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
     gp.T = T;
     gp.H = H;
     gp.NT = NT;
-    return Dv == 128 ? launch_grads<128>(mq, mk, mv, mdo, mpt, mt, gp, B, st)
-                     : launch_grads<64>(mq, mk, mv, mdo, mpt, mt, gp, B, st);
+    {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaErrorUnknown;
+        gp.pf_stride = sms;
+    }
+    return Dv == 128 ? launch_grads<128>(mq, mk, mv, mdo, mpt, mt, gp, w, B, st)
+                     : launch_grads<64>(mq, mk, mv, mdo, mpt, mt, gp, w, B, st);
 }
+
+#ifdef GDN_TRACE
+extern "C" int gdn_trace_bwd_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_trace_bwd, sizeof(g_trace_bwd));
+}
+#endif
 
 cudaError_t read_and_clear_device_error_bwd(unsigned int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_bwd_error, sizeof(unsigned int));

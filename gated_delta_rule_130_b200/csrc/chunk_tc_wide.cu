@@ -466,6 +466,9 @@ struct Params {
     // exp(g_last - g_r) are 1 and the state's decay is this per-key vector
     // (log_alpha is not read).
     const float *glk;
+    // optional (fixed-length batches, the backward's recompute): the state entering
+    // every chunk, [B*H][NT][Dv][DK] bf16
+    __nv_bfloat16 *S_hist;
     Seqs sq;
     int H, Dv;
     unsigned flags;
@@ -772,6 +775,11 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int j = 0; j < 16; ++j)
                     sv[j] = p.S0 ? p.S0[(head * p.Dv + v0 + col0 + 16 * pc + j) * DK + key] : 0.f;
                 tc::store16_bf16(sbuf, key, col0 / 16 + pc, sv);
+                if (p.S_hist)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        p.S_hist[((size_t)head * NT * p.Dv + v0 + col0 + 16 * pc + j) * DK + key] =
+                            __float2bfloat16_rn(sv[j]);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) sv[j] *= gl;
                 if (have) tmem_st16(lane_addr + st_col + 16 * pc, sv);
@@ -859,6 +867,13 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (!last) {
 #pragma unroll
                     for (int pc = 0; pc < NPC; ++pc) tc::store16_bf16(sbuf, key, col0 / 16 + pc, sv[pc]);
+                    if (p.S_hist)  // the state entering chunk c + 1
+#pragma unroll
+                        for (int pc = 0; pc < NPC; ++pc)
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                p.S_hist[(((size_t)head * NT + c + 1) * p.Dv + v0 + col0 + 16 * pc + j) * DK +
+                                         key] = __float2bfloat16_rn(sv[pc][j]);
 #pragma unroll
                     for (int pc = 0; pc < NPC; ++pc)
 #pragma unroll
@@ -1016,6 +1031,7 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
     p.S_T = S_T;
     p.rqk = rqk;
     p.glk = nullptr;
+    p.S_hist = nullptr;
     p.sq = tc::Seqs{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
                     n_seq};
     p.H = H;
@@ -1052,6 +1068,7 @@ cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *
     p.S_T = S_T;
     p.rqk = nullptr;
     p.glk = glk;
+    p.S_hist = nullptr;
     p.sq = tc::Seqs{nullptr, nullptr, nullptr, T, B};
     p.H = H;
     p.Dv = Dv;
@@ -1075,12 +1092,15 @@ cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *
     return cudaPeekAtLastError();
 }
 
-// The parallel kernel alone for the backward (Dk = 128, gates as given, B
-// sequences of T tokens): per chunk and head the [P; T''] tile, the W tile and
-// T itself, at tile index (b NT + c) H + h.
-cudaError_t launch_ut_tiles_bwd(const void *q, const void *k, const float *log_alpha,
-                                const float *beta, int B, int T, int H, void *pt, void *wt,
-                                void *tr, cudaStream_t st) {
+// The backward's recompute (Dk = 128, gates as given, B sequences of T tokens):
+// the parallel kernel writes per chunk and head the [P; T''] tile, the W tile and
+// T itself (tile index (b NT + c) H + h); the sequential kernel, fed those tiles,
+// records the state entering every chunk in bf16 ([B*H][NT][Dv][128]) and writes
+// its output to o_scratch.
+cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 int B, int T, int H, int Dv, void *pt, void *wt, void *tr,
+                                 void *S_hist, void *o_scratch, cudaStream_t st) {
     constexpr int DK = 128;
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
     if (B < 1 || NT < 1) return cudaSuccess;
@@ -1095,6 +1115,41 @@ cudaError_t launch_ut_tiles_bwd(const void *q, const void *k, const float *log_a
     ut<<<dim3((unsigned)(B * NT), H, 1), tcw::UT_THREADS, ut_smem, st>>>(
         mq, mk, log_alpha, beta, static_cast<__nv_bfloat16 *>(pt),
         static_cast<__nv_bfloat16 *>(wt), static_cast<__nv_bfloat16 *>(tr), nullptr, sq, H, 0u);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    const long long n_tiles = (long long)B * NT * H;
+    CUtensorMap mv, mw, mp;
+    if (!tc::make_map(&mv, v, 1, B * T, H, Dv) || !tcw::make_map_w(&mw, wt, n_tiles, DK) ||
+        !tc::make_map_tt(&mp, pt, n_tiles))
+        return cudaErrorInvalidValue;
+    tcw::Params p;
+    p.log_alpha = log_alpha;
+    p.S0 = S0;
+    p.o = static_cast<__nv_bfloat16 *>(o_scratch);
+    p.S_T = nullptr;
+    p.rqk = nullptr;
+    p.glk = nullptr;
+    p.S_hist = static_cast<__nv_bfloat16 *>(S_hist);
+    p.sq = sq;
+    p.H = H;
+    p.Dv = Dv;
+    p.flags = 0u;
+    auto *seq = tcw::gdn_chunk_tcw_kernel<DK, false>;
+    constexpr int seq_smem = tcw::SeqDims<DK>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Dv / tcw::DVT, H, B);
+    cfg.blockDim = dim3(tcw::NTHREADS);
+    cfg.dynamicSmemBytes = seq_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, seq, mq, mk, mv, mw, mp, p);
+    if (e != cudaSuccess) return e;
     return cudaPeekAtLastError();
 }
 

@@ -55,9 +55,9 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              int chunk, bool bf16, void *workspace, cudaStream_t st);
 
 // Tensor-core chunkwise backward (bf16, Dk = 128, chunk 64, Dv 64 or 128):
-// chunk_bwd_tc.cu, reached through launch_chunk_bwd.  Its recompute uses the
-// precomputed variant's parallel kernel for the [P; T''], W and T tiles of every
-// chunk (chunk_tc_wide.cu, launch_ut_tiles_bwd) and the fused forward for S_hist.
+// chunk_bwd_tc.cu, reached through launch_chunk_bwd.  Its recompute is the
+// precomputed variant (chunk_tc_wide.cu, launch_recompute_bwd): the [P; T''], W
+// and T tiles of every chunk, then the state entering every chunk (bf16).
 bool bwd_tc_supported(int B, int T, int H, int Dk, int Dv, int chunk, bool bf16);
 size_t bwd_tc_workspace_bytes(int B, int T, int H, int Dv);
 cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, const float *la,
@@ -65,9 +65,10 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
                                 const float *dS_T, void *dq, void *dk, void *dv, float *dla,
                                 float *dbeta, float *dS0, int B, int T, int H, int Dv,
                                 void *workspace, cudaStream_t st);
-cudaError_t launch_ut_tiles_bwd(const void *q, const void *k, const float *log_alpha,
-                                const float *beta, int B, int T, int H, void *pt, void *wt,
-                                void *tr, cudaStream_t st);
+cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 int B, int T, int H, int Dv, void *pt, void *wt, void *tr,
+                                 void *S_hist, void *o_scratch, cudaStream_t st);
 
 // Channel-wise gates (decay per key channel, erase gate b on the key side,
 // write gate w on the value side; CUDA cores, Dk <= 128): chunk_cw.cu.
