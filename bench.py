@@ -654,8 +654,8 @@ def parse_workload(spec: str):
 
 # the kernels one chunkwise backward launches, per path
 BWD_KERNELS = {
-    "tcgen05": ["gdn_utw_kernel (P, T'', W and T tiles)", "gdn_ut_kernel (the chunk states)",
-                "gdn_chunk_tc_kernel (the chunk states)", "gdn_bwd_chain_kernel (dS', dS0)",
+    "tcgen05": ["gdn_utw_kernel (P, T'', W and T tiles)",
+                "gdn_chunk_tcw_kernel (the chunk states, bf16)", "gdn_bwd_chain_kernel (dS', dS0)",
                 "gdn_bwd_grads_kernel (dq, dk, dv, dlog_alpha, dbeta)"],
     "simt": ["chunk_prep (T, P, g)", "gdn_ut_kernel (the chunk states)",
              "gdn_chunk_tc_kernel (the chunk states)", "bwd_state", "bwd_grads"],
