@@ -144,7 +144,7 @@ def chunk_fwd_path(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16) -> str:
     return PATH_NAMES[p]
 
 
-VARIANT_NAMES = {0: None, 1: "fused", 2: "precomputed"}
+VARIANT_NAMES = {0: None, 1: "fused", 2: "precomputed", 3: "split"}
 
 
 def chunk_fwd_variant(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16):

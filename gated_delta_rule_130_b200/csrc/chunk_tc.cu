@@ -1147,6 +1147,8 @@ size_t tc_workspace_bytes_seqs(int n_seq, long long total_chunks, int H, bool va
 }
 
 size_t tc_workspace_bytes(int B, int T, int H, unsigned flags, int Dk, int Dv) {
+    if (tc_precomputed(B, H, Dk, Dv) && tcw_split_segments(B, T, H, Dk, Dv) > 1)
+        return tcw_split_workspace_bytes(B, T, H, Dv, flags);
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
     return tc_workspace_bytes_seqs(B, (long long)B * NT, H, false, flags, Dk, Dv);
 }

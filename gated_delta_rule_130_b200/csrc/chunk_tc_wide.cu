@@ -457,7 +457,7 @@ constexpr int NTHREADS = 32 * (W_STATE0 + NSTATEW);
 struct Params {
     const float *log_alpha;
     const float *S0;
-    __nv_bfloat16 *o;
+    __nv_bfloat16 *o;      // null: the output is not stored (the segment maps of a split sequence)
     float *S_T;
     const float *rqk;      // 1/|q|, 1/|k| per chunk row from the UT kernel (normalising only)
     // Channel-wise gates (chunk_cw_tc.cu): the per-chunk decay per key channel,
@@ -469,6 +469,9 @@ struct Params {
     // optional (fixed-length batches, the backward's recompute): the state entering
     // every chunk, [B*H][NT][Dv][DK] bf16
     __nv_bfloat16 *S_hist;
+    // tm_v maps a 64-token zero tensor (V = 0; every later token is out of bounds
+    // and loads as zeros): its L2 prefetches are skipped
+    bool v_zero;
     Seqs sq;
     int H, Dv;
     unsigned flags;
@@ -655,7 +658,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         tma_prefetch_l2_4d(&tm_k, kb * 64, h, sp.off + cq * C, 0);
                         tma_prefetch_l2_3d(&tm_w, kb * 64, 0, tq);
                     }
-                    tma_prefetch_l2_4d(&tm_v, v0, h, sp.off + cq * C, 0);
+                    if (!p.v_zero) tma_prefetch_l2_4d(&tm_v, v0, h, sp.off + cq * C, 0);
                     tma_prefetch_l2_3d(&tm_pt, 0, 0, tq);
                 }
             }
@@ -903,7 +906,7 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tmem_ld16(lane_addr + TM_Y + 32 * hf, y0);
                 tmem_ld16(lane_addr + TM_Y + 32 * hf + 16, y1);
                 tmem_wait_ld();
-                if (t0 + lrow < T) {
+                if (p.o && t0 + lrow < T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
                         p.o + ((size_t)(sp.off + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
 #pragma unroll
@@ -998,6 +1001,187 @@ cudaError_t launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorM
 
 }  // namespace tcw
 
+// ------------------------------------------------------------ split sequences
+// Where the sequential grid covers less than a quarter of the GPU, each sequence of
+// a fixed-length batch (Dk = 128, T a multiple of the segment length) is cut into
+// G segments of whole chunks and the chain runs on all segments at once.  The
+// chunk recurrence is affine in the state, so a segment maps its start state to
+// its end state as S_end = S_start M + N (M = the product over its chunks of
+// gamma_last I - W^T diag(exp(g_last - g)) K, Dk x Dk; N its end state from a zero
+// start): pass 1 forms N (the chain from S = 0) and M (the chain with V = 0 from
+// S = I, Dk rows of "values") for every segment but the last of each sequence, a
+// scan (chunk_split.cu) chains the segments' start states, and pass 2 runs the
+// chain on every segment from its true start state for the outputs and the final
+// state.  About three chain passes over the sequence instead of one, on G times as
+// many CTAs.
+int tcw_split_segments(int B, int T, int H, int Dk, int Dv) {
+    static const int sms = [] {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        return n;
+    }();
+    if (Dk != 128 || B < 1 || T < 1 || T % tc::C != 0 || Dv % tcw::DVT != 0) return 1;
+    const long long ctas = (long long)(Dv / tcw::DVT) * H * B;
+    if (ctas * 4 > sms) return 1;
+    const int NT = T / tc::C;
+    for (int G = 8; G >= 2; --G)
+        if (NT % G == 0 && NT / G >= 16 && ctas * G <= sms) return G;
+    return 1;
+}
+
+namespace tcw {
+
+// Regions of a split call's workspace after the tiles ([P; T''], W, 1/|q| and 1/|k|):
+// N and S_T of every segment ([B G][H][Dv][128] float32), M ([B G][H][128][128]),
+// the segments' start states ([B G][H][Dv][128]), 64 zero token rows ([64][H][128]
+// bf16) and pass 1's launch order (the segments but the last of each sequence).
+struct SplitWs {
+    __nv_bfloat16 *pt, *wt, *zrow;
+    float *rqk, *N, *M, *Ss, *STs;
+    int *order;
+    size_t bytes;
+};
+
+inline size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
+
+SplitWs split_carve(void *base, int B, int T, int H, int Dv, unsigned flags) {
+    constexpr int DK = 128;
+    const int G = tcw_split_segments(B, T, H, DK, Dv);
+    const long long NT = T / tc::C, total_chunks = (long long)B * NT;
+    const size_t tiles = (size_t)total_chunks * H;
+    const size_t nseg = (size_t)B * G * H;
+    const size_t sz[9] = {tiles * PT_ELEMS * 2, tiles * tc::C * DK * 2,
+                          (flags & kFlagL2Norm) ? tiles * 2 * tc::C * 4 : 0,
+                          nseg * Dv * DK * 4, nseg * DK * DK * 4, nseg * Dv * DK * 4,
+                          nseg * Dv * DK * 4, (size_t)tc::C * H * DK * 2,
+                          (size_t)B * G * sizeof(int)};
+    uint8_t *p = static_cast<uint8_t *>(base);
+    size_t off[9], o = 0;
+    for (int i = 0; i < 9; ++i) {
+        off[i] = o;
+        o += up256(sz[i]);
+    }
+    SplitWs w;
+    w.pt = reinterpret_cast<__nv_bfloat16 *>(p + off[0]);
+    w.wt = reinterpret_cast<__nv_bfloat16 *>(p + off[1]);
+    w.rqk = sz[2] ? reinterpret_cast<float *>(p + off[2]) : nullptr;
+    w.N = reinterpret_cast<float *>(p + off[3]);
+    w.M = reinterpret_cast<float *>(p + off[4]);
+    w.Ss = reinterpret_cast<float *>(p + off[5]);
+    w.STs = reinterpret_cast<float *>(p + off[6]);
+    w.zrow = reinterpret_cast<__nv_bfloat16 *>(p + off[7]);
+    w.order = reinterpret_cast<int *>(p + off[8]);
+    w.bytes = o;
+    return w;
+}
+
+template <bool kNorm>
+cudaError_t launch_split_t(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *S0, void *o, float *S_T, int B, int T,
+                           int H, int Dv, unsigned flags, void *workspace, cudaStream_t st) {
+    constexpr int DK = 128;
+    const int G = tcw_split_segments(B, T, H, DK, Dv);
+    const int NT = T / tc::C, nseg = B * G;
+    const long long total_chunks = (long long)B * NT, n_tiles = total_chunks * H;
+    SplitWs w = split_carve(workspace, B, T, H, Dv, flags);
+    CUtensorMap mq, mk, mv, mz, mw, mp;
+    if (!tc::make_map(&mq, q, 1, B * T, H, DK) || !tc::make_map(&mk, k, 1, B * T, H, DK) ||
+        !tc::make_map(&mv, v, 1, B * T, H, Dv) || !tc::make_map(&mz, w.zrow, 1, tc::C, H, DK) ||
+        !make_map_w(&mw, w.wt, n_tiles, DK) || !tc::make_map_tt(&mp, w.pt, n_tiles))
+        return cudaErrorInvalidValue;
+    // M = I for every segment, the zero token rows, pass 1's order
+    cudaError_t e = launch_split_init(w.M, (long long)nseg * H, w.zrow, tc::C * H, w.order, B, G, st);
+    if (e != cudaSuccess) return e;
+    // the tiles of every chunk, once (the sequences as given)
+    auto *ut = gdn_utw_kernel<DK, kNorm>;
+    auto *seq = gdn_chunk_tcw_kernel<DK, kNorm>;
+    constexpr int ut_smem = UtDims<DK>::UT_SMEM, seq_smem = SeqDims<DK>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(ut, cudaFuncAttributeMaxDynamicSharedMemorySize, ut_smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(seq, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+    if (e != cudaSuccess) return e;
+    ut<<<dim3((unsigned)total_chunks, H, 1), UT_THREADS, ut_smem, st>>>(
+        mq, mk, log_alpha, beta, w.pt, w.wt, nullptr, w.rqk, tc::Seqs{nullptr, nullptr, nullptr, T, B},
+        H, flags);
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    // the segments as sequences of T / G tokens: global chunk b NT + c keeps its tile
+    Params p;
+    p.log_alpha = log_alpha;
+    p.rqk = w.rqk;
+    p.glk = nullptr;
+    p.S_hist = nullptr;
+    p.sq = tc::Seqs{nullptr, nullptr, nullptr, T / G, nseg};
+    p.H = H;
+    p.flags = flags;
+    // pdl: programmatic dependent launch after the previous kernel (the state warps
+    // read S0 before the TMA warp's wait, so only where S0 was written earlier)
+    const auto run = [&](const CUtensorMap &vmap, int dv, bool pdl, int n_ctas_z) -> cudaError_t {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(dv / DVT, H, n_ctas_z);
+        cfg.blockDim = dim3(NTHREADS);
+        cfg.dynamicSmemBytes = seq_smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        p.Dv = dv;
+        const cudaError_t e1 = cudaLaunchKernelEx(&cfg, seq, mq, mk, vmap, mw, mp, p);
+        return e1 != cudaSuccess ? e1 : cudaPeekAtLastError();
+    };
+    // pass 1, every segment but the last of each sequence (blockIdx.z through the
+    // order array): N from a zero start; M with V = 0 from S = I (in place)
+    p.sq.order = w.order;
+    p.S0 = nullptr;
+    p.S_T = w.N;
+    p.o = nullptr;
+    p.v_zero = false;
+    if ((e = run(mv, Dv, true, B * (G - 1))) != cudaSuccess) return e;
+    p.S0 = w.M;
+    p.S_T = w.M;
+    p.v_zero = true;
+    if ((e = run(mz, DK, true, B * (G - 1))) != cudaSuccess) return e;
+    p.sq.order = nullptr;
+    // the segments' start states
+    if ((e = launch_split_scan(S0, w.N, w.M, w.Ss, B, G, H, Dv, st)) != cudaSuccess) return e;
+    // pass 2: every segment from its start state
+    p.S0 = w.Ss;
+    p.S_T = w.STs;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.v_zero = false;
+    if ((e = run(mv, Dv, false, nseg)) != cudaSuccess) return e;
+    if (S_T) {
+        const size_t per = (size_t)H * Dv * DK;
+        for (int b = 0; b < B; ++b) {
+            e = cudaMemcpyAsync(S_T + b * per, w.STs + ((size_t)b * G + G - 1) * per,
+                                per * sizeof(float), cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
+}  // namespace tcw
+
+size_t tcw_split_workspace_bytes(int B, int T, int H, int Dv, unsigned flags) {
+    return tcw::split_carve(nullptr, B, T, H, Dv, flags).bytes;
+}
+
+cudaError_t launch_chunk_tcw_split(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta, const float *S0,
+                                   void *o, float *S_T, int B, int T, int H, int Dv,
+                                   unsigned flags, void *workspace, cudaStream_t st) {
+    return (flags & kFlagL2Norm)
+               ? tcw::launch_split_t<true>(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dv,
+                                           flags, workspace, st)
+               : tcw::launch_split_t<false>(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, Dv,
+                                            flags, workspace, st);
+}
+
 cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                                   const float *log_alpha, const float *beta, const float *S0,
                                   void *o, float *S_T, int n_seq, int T_fixed, long long total_T,
@@ -1005,6 +1189,9 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                                   int Dv, unsigned flags, void *workspace, cudaStream_t st) {
     if (Dk != 128 && Dk != 256) return cudaErrorInvalidValue;
     const bool varlen = cu_seqlens != nullptr;
+    if (!varlen && n_seq > 0 && tcw_split_segments(n_seq, T_fixed, H, Dk, Dv) > 1)
+        return launch_chunk_tcw_split(q, k, v, log_alpha, beta, S0, o, S_T, n_seq, T_fixed, H, Dv,
+                                      flags, workspace, st);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *cu_chunks = varlen ? reinterpret_cast<int *>(ws) : nullptr;
     const size_t tiles = (size_t)total_chunks * H;
@@ -1032,6 +1219,7 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
     p.rqk = rqk;
     p.glk = nullptr;
     p.S_hist = nullptr;
+    p.v_zero = false;
     p.sq = tc::Seqs{cu_seqlens, cu_chunks, varlen ? cu_chunks + n_seq + 1 : nullptr, T_fixed,
                     n_seq};
     p.H = H;
@@ -1069,6 +1257,7 @@ cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *
     p.rqk = nullptr;
     p.glk = glk;
     p.S_hist = nullptr;
+    p.v_zero = false;
     p.sq = tc::Seqs{nullptr, nullptr, nullptr, T, B};
     p.H = H;
     p.Dv = Dv;
@@ -1130,6 +1319,7 @@ cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
     p.rqk = nullptr;
     p.glk = nullptr;
     p.S_hist = static_cast<__nv_bfloat16 *>(S_hist);
+    p.v_zero = false;
     p.sq = sq;
     p.H = H;
     p.Dv = Dv;

@@ -79,7 +79,8 @@ int gdn_chunk_fwd_path(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype
 
 int gdn_chunk_fwd_variant(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype) {
     if (gdn_chunk_fwd_path(B, T, H, Dk, Dv, chunk, dtype) != GDN_PATH_TCGEN05) return 0;
-    return gdn::tc_precomputed(B, H, Dk, Dv) ? 2 : 1;
+    if (!gdn::tc_precomputed(B, H, Dk, Dv)) return 1;
+    return gdn::tcw_split_segments(B, T, H, Dk, Dv) > 1 ? 3 : 2;
 }
 
 size_t gdn_chunk_fwd_workspace_size_ex(int B, int T, int H, int Dk, int Dv, int chunk,

@@ -133,6 +133,24 @@ cudaError_t launch_chunk_tcw_seqs(const void *q, const void *k, const void *v,
                                   const int *cu_seqlens, long long total_chunks, int H, int Dk,
                                   int Dv, unsigned flags, void *workspace, cudaStream_t st);
 
+// A fixed-length batch whose sequential grid covers under a quarter of the GPU
+// (Dk = 128, T a multiple of 64 G) runs split into G segments per sequence
+// (chunk_tc_wide.cu; the precomputed variant's kernels, reached through
+// launch_chunk_tcw_seqs): tcw_split_segments gives G (1: not split).
+int tcw_split_segments(int B, int T, int H, int Dk, int Dv);
+size_t tcw_split_workspace_bytes(int B, int T, int H, int Dv, unsigned flags);
+cudaError_t launch_chunk_tcw_split(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta, const float *S0,
+                                   void *o, float *S_T, int B, int T, int H, int Dv,
+                                   unsigned flags, void *workspace, cudaStream_t st);
+// Its small kernels (chunk_split.cu): M[i] = I (128 x 128) for i < n_maps, `rows`
+// zero rows of 128 bf16 and the order of pass 1 (every segment but the last of
+// each of the B sequences); the scan of the segments' start states.
+cudaError_t launch_split_init(float *M, long long n_maps, void *zrow, int rows, int *order, int B,
+                              int G, cudaStream_t st);
+cudaError_t launch_split_scan(const float *S0, const float *N, const float *M, float *Ss, int B,
+                              int G, int H, int Dv, cudaStream_t st);
+
 // The precomputed variant's sequential kernel (Dk = 128) in its channel-wise
 // mode: operands Q o exp(Lam), K o exp(Lam_last - Lam), w o V ([B*T, H, D] bf16),
 // the [P; T''] and W tiles and exp(Lam_last) per key channel ([tiles][128]

@@ -72,13 +72,18 @@ typedef enum {
                               needs a workspace */
 } gdn_path_t;
 
-/* Which of the two tcgen05 variants a gdn_chunk_fwd call with these sizes runs
- * (the pages have no counterpart; both compute the same result):
+/* Which tcgen05 variant a gdn_chunk_fwd call with these sizes runs (the pages
+ * have no counterpart; all compute the same result up to rounding):
  * 0 = not the tcgen05 path (or invalid sizes), 1 = fused (the sequential kernel
  * forms Q K^T and the WY factors itself; Dk = 128 when the sequential grid of
  * Dv / 64 x H x B CTAs fills most of the GPU), 2 = precomputed (the parallel
  * kernel also forms the gated Q K^T and W per chunk; Dk = 256, and Dk = 128 with
- * fewer than 74 sequential CTAs).  The workspace size depends on it. */
+ * fewer than 74 sequential CTAs), 3 = split (precomputed, with each sequence cut
+ * into G segments of whole chunks when the sequential grid covers under a quarter
+ * of the GPU, Dk = 128 and T a multiple of 64 G: the chunk recurrence is affine in
+ * the state, so each segment's map S_end = S_start M + N is formed in parallel, a
+ * scan gives every segment's start state, and the segments then run at once).
+ * The workspace size depends on it. */
 int gdn_chunk_fwd_variant(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype_t dtype);
 
 /* Limits: 1 <= Dk <= 256, 1 <= Dv <= 512, chunk in {16, 32, 64}; B, T, H >= 0

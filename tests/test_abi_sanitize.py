@@ -87,6 +87,7 @@ cudaError_t read_and_clear_device_error(unsigned int *flag) { *flag = 0; return 
 cudaError_t read_and_clear_device_error_wide(unsigned int *flag) { *flag = 0; return ok(); }
 cudaError_t read_and_clear_device_error_bwd(unsigned int *flag) { *flag = 0; return ok(); }
 bool bwd_tc_supported(int, int, int, int, int, int, bool) { return false; }
+int tcw_split_segments(int, int, int, int, int) { return 1; }
 cudaError_t set_withhold_first_arrival(bool) { return ok(); }
 }  // namespace gdn
 """
