@@ -566,7 +566,8 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     TG(1);
 
-    if (tid == 0) {
+    // warp 1 issues the copies and warp 2 the prefetches while warp 0 loads the gates
+    if (tid == 32) {
         uint64_t *fb = cx.bar + 0;
         mbar_arrive_expect_tx(fb, 4 * PANEL + 2 * Ly::VB + 3 * PANEL + 4 * DV * 128);
 #pragma unroll
@@ -587,6 +588,8 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL, &tm_sh, fb, kb * 64, 0, hist);
             tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL + DV * 128, &tm_dsh, fb, kb * 64, 0, hist);
         }
+    }
+    if (tid == 64) {
         // one CTA per SM: the CTA one wave later (linear index + SM count) finds its
         // inputs in L2, their DRAM reads overlapping this CTA's products
         const long long lin = blockIdx.x + (long long)NT * (blockIdx.y + (long long)H * blockIdx.z);
