@@ -168,8 +168,9 @@ gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // K and Q rows of the chunk.  Rows past the end of the sequence (the next
     // sequence's, or TMA's zero fill) get beta = 0 and log alpha = 0: their rows
     // of A and their columns of T', T'' and P vanish, and their rows of P are
-    // outputs of tokens that are never stored.
-    if (tid == 0) {
+    // outputs of tokens that are never stored.  Warp 1 (the MMA issuer, which waits
+    // for them) starts the copies, so that warp 0's gate loads start at once.
+    if (tid == 32) {
         mbar_arrive_expect_tx(cx.bar + 0, 2 * KB * 8192);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb) {
