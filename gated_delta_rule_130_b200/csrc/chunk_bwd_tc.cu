@@ -44,7 +44,7 @@
 //     epilogue, and dS^T = gamma_last dS'^T + Q^T (gamma o dO) - W^T dU'
 //     (M = 128).  It records dS' (bf16) for every chunk and writes dS0.
 //  2. gdn_bwd_grads_kernel: one CTA per (chunk, head), all chunks in parallel;
-//     ten tcgen05 products in four dependent phases with epilogues between
+//     twelve groups of tcgen05 products in four dependent phases, epilogues between
 //     them (every operand a 128-byte-swizzled bf16 tile in shared memory, every
 //     accumulator in TMEM), then dq, dk, dv, dlog alpha and dbeta.
 // Rows past the end of a sequence are loaded as zeros (four-dimensional tensor
@@ -492,7 +492,7 @@ struct L {
     static constexpr int SM_ZT = SM_P + PANEL;  // Z over T'' and T
     static constexpr int SM_DP = SM_V;          // dP o Gamma over V
     static constexpr int SM_EE = SM_DU;         // E + E^T over U'
-    static constexpr int SM_ES = SM_ZB;         // E (row-major scratch) over -beta gamma o Z
+    static constexpr int SM_ES = SM_ZB;         // E^T (row-major scratch) over -beta gamma o Z
     // per-row float arrays in SM_MISC: the gate vectors, then partial sums written
     // with plain stores (no shared-memory atomics): two column halves per row for
     // the row sums, four row quarters per column for the column sums
@@ -842,7 +842,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     tc_fence_after();
     TG(8);
     // epilogue C (row r, columns 32 hf .. + 31 of the 64 x 64 matrices):
-    // dP o Gamma (bf16 tile), E (row-major scratch), dbeta's and dg's sums, and
+    // dP o Gamma (bf16 tile), E^T (row-major scratch), dbeta's and dg's sums, and
     // gamma_r (dO S)_r . q_r from the dQ accumulator before (dP o Gamma) K joins it
     {
         const float br = act ? bes[r] : 0.f, g2r = act ? g2s[r] : 0.f;
