@@ -289,38 +289,56 @@ decode_cw_vec(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             qq[m + u] = qv[u];
         }
     }
+    // o_i = (alpha o S_i + c_i k) . q = (alpha o S_i) . q + c_i (k . q): both of a
+    // row's sums come from the row as read, and the rows' reductions interleave
+    float kq = 0.f;
+#pragma unroll
+    for (int m = 0; m < NPL; ++m) kq += kk[m] * qq[m];
+    float4 sv[ROWS][NPL / 4];
+#pragma unroll
+    for (int rr = 0; rr < ROWS; ++rr) {
+        const float *s = S + (row0 + rr) * Dk + j0;
+#pragma unroll
+        for (int m = 0; m < NPL; m += 4) sv[rr][m / 4] = *reinterpret_cast<const float4 *>(s + m);
+    }
+    float e[ROWS], sq[ROWS];
+#pragma unroll
+    for (int rr = 0; rr < ROWS; ++rr) {
+        e[rr] = 0.f;
+        sq[rr] = 0.f;
+#pragma unroll
+        for (int m = 0; m < NPL; m += 4) {
+            const float a[4] = {al[m] * sv[rr][m / 4].x, al[m + 1] * sv[rr][m / 4].y,
+                                al[m + 2] * sv[rr][m / 4].z, al[m + 3] * sv[rr][m / 4].w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                e[rr] += a[u] * bk[m + u];
+                sq[rr] += a[u] * qq[m + u];
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+#pragma unroll
+        for (int rr = 0; rr < ROWS; ++rr) {
+            e[rr] += __shfl_xor_sync(0xffffffffu, e[rr], off);
+            sq[rr] += __shfl_xor_sync(0xffffffffu, sq[rr], off);
+        }
+    }
 #pragma unroll
     for (int rr = 0; rr < ROWS; ++rr) {
         const long long row = row0 + rr;
         const int i = (int)(row - head * Dv);
+        const float c = wg[head * Dv + i] * to_f32(v[head * Dv + i]) - e[rr];
         float *s = S + row * Dk + j0;
-        float d[NPL];
-        float e = 0.f;
-#pragma unroll
-        for (int m = 0; m < NPL; m += 4) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(s + m);
-            d[m] = al[m] * s4.x;
-            d[m + 1] = al[m + 1] * s4.y;
-            d[m + 2] = al[m + 2] * s4.z;
-            d[m + 3] = al[m + 3] * s4.w;
-        }
-#pragma unroll
-        for (int m = 0; m < NPL; ++m) e += d[m] * bk[m];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
-        const float c = wg[head * Dv + i] * to_f32(v[head * Dv + i]) - e;
-        float acc = 0.f;
-#pragma unroll
-        for (int m = 0; m < NPL; ++m) {
-            d[m] += c * kk[m];
-            acc += d[m] * qq[m];
-        }
 #pragma unroll
         for (int m = 0; m < NPL; m += 4)
-            *reinterpret_cast<float4 *>(s + m) = make_float4(d[m], d[m + 1], d[m + 2], d[m + 3]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) o[row] = from_f32<T>(acc);
+            *reinterpret_cast<float4 *>(s + m) =
+                make_float4(al[m] * sv[rr][m / 4].x + c * kk[m], al[m + 1] * sv[rr][m / 4].y + c * kk[m + 1],
+                            al[m + 2] * sv[rr][m / 4].z + c * kk[m + 2],
+                            al[m + 3] * sv[rr][m / 4].w + c * kk[m + 3]);
+        if (lane == 0) o[row] = from_f32<T>(sq[rr] + c * kq);
     }
 }
 
