@@ -168,56 +168,93 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     TCW(2);
 
     // the two 8 x 8 diagonal sub-blocks of each diagonal 16-block, summed
-    // directly: warps 4I .. 4I+3 take block I, each a quarter of the channels;
-    // lane -> pairs P = lane + 32 m: sub-block s = P / 36, p = P % 36 = r (r + 1) / 2 + i
+    // directly: warps 4I .. 4I+3 take block I, each a quarter of the channels.
+    // Lane -> sub-block s, the rows rp and 7 - rp of it (rp + 1 and 8 - rp pairs
+    // (r, i), i <= r: nine in all) and 8 of the warp's 32 channels (cs), so each
+    // row's values are loaded once per channel and the columns' values are shared
+    // by the two rows; the four lanes of a row pair then add their channel parts.
     {
         const int I = warp >> 2, ch = warp & 3;
-        int pr[3], pi[3];
-        float accA[3], accP[3];
-#pragma unroll
-        for (int m = 0; m < 3; ++m) {
-            const int P = lane + 32 * m, sb = P / 36, p = P % 36;
-            int r = 0;
-            while ((r + 1) * (r + 2) / 2 <= p) ++r;
-            pr[m] = 16 * I + 8 * sb + r;
-            pi[m] = 16 * I + 8 * sb + (p - r * (r + 1) / 2);
-            accA[m] = accP[m] = 0.f;
-        }
+        const int sb = lane >> 4, rp = (lane >> 2) & 3, cs = lane & 3;
+        const int i0 = 16 * I + 8 * sb;
+        const int rA = i0 + rp, rB = i0 + 7 - rp;
+        float aA[4] = {}, pA[4] = {}, aB[8] = {}, pB[8] = {};
 #pragma unroll 2
-        for (int jj = 0; jj < DK / 4; ++jj) {
-            const int j = (DK / 4) * ch + jj;
+        for (int jj = 0; jj < 8; ++jj) {
+            const int j = 32 * ch + 8 * cs + jj;
+            const float lA = LM[rA * LDF + j], lB = LM[rB * LDF + j];
+            const float bA = BK[rA * LDF + j], bB = BK[rB * LDF + j];
+            const float qA = QF[rA * LDF + j], qB = QF[rB * LDF + j];
 #pragma unroll
-            for (int m = 0; m < 3; ++m) {
-                if (lane + 32 * m < NPAIR) {
-                    const int R = pr[m], Ii = pi[m];
-                    const float e = tc::ex2(LM[R * LDF + j] - LM[Ii * LDF + j]) * KF[Ii * LDF + j];
-                    accA[m] = fmaf(BK[R * LDF + j], e, accA[m]);
-                    accP[m] = fmaf(QF[R * LDF + j], e, accP[m]);
+            for (int ii = 0; ii < 8; ++ii) {
+                const float lI = LM[(i0 + ii) * LDF + j], kI = KF[(i0 + ii) * LDF + j];
+                // exponents are <= 0 where kept (Lam is non-increasing down the rows)
+                const float eB = ii <= 7 - rp ? tc::ex2(fminf(lB - lI, 0.f)) * kI : 0.f;
+                aB[ii] = fmaf(bB, eB, aB[ii]);
+                pB[ii] = fmaf(qB, eB, pB[ii]);
+                if (ii < 4) {
+                    const float eA = ii <= rp ? tc::ex2(fminf(lA - lI, 0.f)) * kI : 0.f;
+                    aA[ii] = fmaf(bA, eA, aA[ii]);
+                    pA[ii] = fmaf(qA, eA, pA[ii]);
                 }
             }
         }
-        float *ds = DS + I * 3 * NPAIR * 2;   // partial sums of channel quarters 1-3
-        if (ch > 0) {
 #pragma unroll
-            for (int m = 0; m < 3; ++m)
-                if (lane + 32 * m < NPAIR) {
-                    ds[((ch - 1) * NPAIR + lane + 32 * m) * 2] = accA[m];
-                    ds[((ch - 1) * NPAIR + lane + 32 * m) * 2 + 1] = accP[m];
+        for (int ii = 0; ii < 8; ++ii) {
+            aB[ii] += __shfl_xor_sync(0xffffffffu, aB[ii], 1);
+            aB[ii] += __shfl_xor_sync(0xffffffffu, aB[ii], 2);
+            pB[ii] += __shfl_xor_sync(0xffffffffu, pB[ii], 1);
+            pB[ii] += __shfl_xor_sync(0xffffffffu, pB[ii], 2);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            aA[ii] += __shfl_xor_sync(0xffffffffu, aA[ii], 1);
+            aA[ii] += __shfl_xor_sync(0xffffffffu, aA[ii], 2);
+            pA[ii] += __shfl_xor_sync(0xffffffffu, pA[ii], 1);
+            pA[ii] += __shfl_xor_sync(0xffffffffu, pA[ii], 2);
+        }
+        // pair slots of this row pair: k < 8 - rp -> (rB, i0 + k), else (rA, i0 + k - (8 - rp))
+        float *ds = DS + I * 3 * NPAIR * 2;   // partial sums of channel quarters 1-3
+        const int slot0 = (sb * 4 + rp) * 9;
+        if (ch > 0 && cs == 0) {
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii)
+                if (ii <= 7 - rp) {
+                    ds[((ch - 1) * NPAIR + slot0 + ii) * 2] = aB[ii];
+                    ds[((ch - 1) * NPAIR + slot0 + ii) * 2 + 1] = pB[ii];
+                }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+                if (ii <= rp) {
+                    ds[((ch - 1) * NPAIR + slot0 + 8 - rp + ii) * 2] = aA[ii];
+                    ds[((ch - 1) * NPAIR + slot0 + 8 - rp + ii) * 2 + 1] = pA[ii];
                 }
         }
         __syncthreads();
-        if (ch == 0) {
+        if (ch == 0 && cs == 0) {
 #pragma unroll
-            for (int m = 0; m < 3; ++m)
-                if (lane + 32 * m < NPAIR) {
-                    float a = accA[m], pp = accP[m];
+            for (int ii = 0; ii < 8; ++ii)
+                if (ii <= 7 - rp) {
+                    float a = aB[ii], pp = pB[ii];
 #pragma unroll
                     for (int cq = 0; cq < 3; ++cq) {
-                        a += ds[(cq * NPAIR + lane + 32 * m) * 2];
-                        pp += ds[(cq * NPAIR + lane + 32 * m) * 2 + 1];
+                        a += ds[(cq * NPAIR + slot0 + ii) * 2];
+                        pp += ds[(cq * NPAIR + slot0 + ii) * 2 + 1];
                     }
-                    AF[pr[m] * LDA + pi[m]] = pr[m] > pi[m] ? a : 0.f;
-                    PF[pr[m] * LDA + pi[m]] = pp;
+                    AF[rB * LDA + i0 + ii] = rB > i0 + ii ? a : 0.f;
+                    PF[rB * LDA + i0 + ii] = pp;
+                }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+                if (ii <= rp) {
+                    float a = aA[ii], pp = pA[ii];
+#pragma unroll
+                    for (int cq = 0; cq < 3; ++cq) {
+                        a += ds[(cq * NPAIR + slot0 + 8 - rp + ii) * 2];
+                        pp += ds[(cq * NPAIR + slot0 + 8 - rp + ii) * 2 + 1];
+                    }
+                    AF[rA * LDA + i0 + ii] = rA > i0 + ii ? a : 0.f;
+                    PF[rA * LDA + i0 + ii] = pp;
                 }
         }
     }
