@@ -118,34 +118,49 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     __nv_bfloat16 *TB = reinterpret_cast<__nv_bfloat16 *>(sm + SM_AF);
     TCW(0);
 
-    // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread
-    // -> (channel, quarter of the rows), so each row is read as 128 consecutive
-    // values; eight rows' loads are issued before any is used (one CTA per SM:
-    // the loads in flight are what hides the memory latency)
-    constexpr int RQ = C / 4;                      // rows per quarter
-    const int jc = tid & (DK - 1), rq = tid >> 7;
-    constexpr int RB8 = 8;
-    for (int r8 = 0; r8 < RQ; r8 += RB8) {
-        float kv[RB8], qv[RB8], bv[RB8], lv[RB8];
+    // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread ->
+    // (row, 16 consecutive channels): 16-byte loads, all twelve in flight before any
+    // is used (one CTA per SM: the loads in flight are what hides the memory latency)
+    {
+        const int r = tid >> 3, jc0 = 16 * (tid & 7);
+        const bool in = r < n;
+        const size_t off = ((tok0 + (in ? r : 0)) * H + h) * DK + jc0;
+        uint4 k8[2], q8[2];
+        float4 b4[4], l4[4];
 #pragma unroll
-        for (int u = 0; u < RB8; ++u) {
-            const int r = rq * RQ + r8 + u;
-            const size_t off = ((tok0 + (r < n ? r : 0)) * H + h) * DK + jc;
-            const bool in = r < n;
-            kv[u] = in ? __bfloat162float(k[off]) : 0.f;
-            qv[u] = in ? __bfloat162float(q[off]) : 0.f;
-            bv[u] = in ? bg[off] : 0.f;
-            lv[u] = in ? la[off] : 0.f;
+        for (int u = 0; u < 2; ++u) {
+            k8[u] = in ? *reinterpret_cast<const uint4 *>(k + off + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+            q8[u] = in ? *reinterpret_cast<const uint4 *>(q + off + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < RB8; ++u) {
-            const int r = rq * RQ + r8 + u;
-            KF[r * LDF + jc] = kv[u];
-            QF[r * LDF + jc] = qv[u];
-            BK[r * LDF + jc] = bv[u] * kv[u];
-            LM[r * LDF + jc] = lv[u] * LOG2E;
+        for (int u = 0; u < 4; ++u) {
+            b4[u] = in ? *reinterpret_cast<const float4 *>(bg + off + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            l4[u] = in ? *reinterpret_cast<const float4 *>(la + off + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        const uint32_t kw[8] = {k8[0].x, k8[0].y, k8[0].z, k8[0].w, k8[1].x, k8[1].y, k8[1].z, k8[1].w};
+        const uint32_t qw[8] = {q8[0].x, q8[0].y, q8[0].z, q8[0].w, q8[1].x, q8[1].y, q8[1].z, q8[1].w};
+        const float bv[16] = {b4[0].x, b4[0].y, b4[0].z, b4[0].w, b4[1].x, b4[1].y, b4[1].z, b4[1].w,
+                              b4[2].x, b4[2].y, b4[2].z, b4[2].w, b4[3].x, b4[3].y, b4[3].z, b4[3].w};
+        const float lv[16] = {l4[0].x, l4[0].y, l4[0].z, l4[0].w, l4[1].x, l4[1].y, l4[1].z, l4[1].w,
+                              l4[2].x, l4[2].y, l4[2].z, l4[2].w, l4[3].x, l4[3].y, l4[3].z, l4[3].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kw[e]));
+            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qw[e]));
+            const int j = jc0 + 2 * e;
+            KF[r * LDF + j] = kf.x;
+            KF[r * LDF + j + 1] = kf.y;
+            QF[r * LDF + j] = qf.x;
+            QF[r * LDF + j + 1] = qf.y;
+            BK[r * LDF + j] = bv[2 * e] * kf.x;
+            BK[r * LDF + j + 1] = bv[2 * e + 1] * kf.y;
+            LM[r * LDF + j] = lv[2 * e] * LOG2E;
+            LM[r * LDF + j + 1] = lv[2 * e + 1] * LOG2E;
         }
     }
+    // per-channel passes below: thread -> (channel jc, quarter rq of the rows)
+    constexpr int RQ = C / 4;                      // rows per quarter
+    const int jc = tid & (DK - 1), rq = tid >> 7;
     __syncthreads();
     TCW(1);
     {   // running sums over the rows, per channel: each quarter locally, then the
@@ -426,26 +441,28 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
     }
     TCW(8);
-    // w o V, eight loads of each in flight per thread
-    for (int base = 0; base < n * Dv; base += RB8 * THREADS) {
-        float vv[RB8], ww[RB8];
+    // w o V: thread -> (row, 16 consecutive value channels), 16-byte loads
+    for (int item = tid; item < C * (Dv / 16); item += THREADS) {
+        const int r = item / (Dv / 16), jv0 = 16 * (item % (Dv / 16));
+        if (r >= n) continue;
+        const size_t off = ((tok0 + r) * H + h) * Dv + jv0;
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(v + off);
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(v + off + 8);
+        float4 w4[4];
 #pragma unroll
-        for (int u = 0; u < RB8; ++u) {
-            const int idx = base + u * THREADS + tid;
-            const int r = idx / Dv, jv = idx - r * Dv;
-            const bool in = idx < n * Dv;
-            const size_t off = ((tok0 + (in ? r : 0)) * H + h) * Dv + (in ? jv : 0);
-            vv[u] = in ? __bfloat162float(v[off]) : 0.f;
-            ww[u] = in ? wg[off] : 0.f;
-        }
+        for (int u = 0; u < 4; ++u) w4[u] = *reinterpret_cast<const float4 *>(wg + off + 4 * u);
+        const uint32_t vw_[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const float wv[16] = {w4[0].x, w4[0].y, w4[0].z, w4[0].w, w4[1].x, w4[1].y, w4[1].z, w4[1].w,
+                              w4[2].x, w4[2].y, w4[2].z, w4[2].w, w4[3].x, w4[3].y, w4[3].z, w4[3].w};
+        uint32_t out[8];
 #pragma unroll
-        for (int u = 0; u < RB8; ++u) {
-            const int idx = base + u * THREADS + tid;
-            if (idx < n * Dv) {
-                const int r = idx / Dv, jv = idx - r * Dv;
-                vw[((tok0 + r) * H + h) * Dv + jv] = __float2bfloat16_rn(vv[u] * ww[u]);
-            }
+        for (int e = 0; e < 8; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vw_[e]));
+            out[e] = tc::pack_bf16(f.x * wv[2 * e], f.y * wv[2 * e + 1]);
         }
+        uint4 *dst = reinterpret_cast<uint4 *>(vw + off);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
     }
     TCW(9);
 }
