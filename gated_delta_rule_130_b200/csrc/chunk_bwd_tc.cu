@@ -416,22 +416,17 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 break;
             }
             tc_fence_after();
-            float r0[16], r1[16], d0[16], d1[16];
-            tmem_ld16(lane_addr + TM_R + 32 * hf, r0);
-            tmem_ld16(lane_addr + TM_R + 32 * hf + 16, r1);
-            tmem_ld16(lane_addr + TM_PD + 64 * s + 32 * hf, d0);
-            tmem_ld16(lane_addr + TM_PD + 64 * s + 32 * hf + 16, d1);
+            // chunk row 16 q + l % 16, values 32 hf + 16 (l / 16) .. + 15 (16-lane loads)
+            float r0[16], d0[16];
+            tmem_ld16x2<16>(lane_addr + TM_R + 32 * hf, r0);
+            tmem_ld16x2<16>(lane_addr + TM_PD + 64 * s + 32 * hf, d0);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = 16 * q + lane;
+            {
+                const int r = 16 * q + (lane & 15);
                 const float dc = gv[GV_DCY + r];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    d0[j] = -fmaf(dc, r0[j], d0[j]);
-                    d1[j] = -fmaf(dc, r1[j], d1[j]);
-                }
-                tc::store16_bf16(base + SM_DU, r, 2 * hf, d0);
-                tc::store16_bf16(base + SM_DU, r, 2 * hf + 1, d1);
+                for (int j = 0; j < 16; ++j) d0[j] = -fmaf(dc, r0[j], d0[j]);
+                tc::store16_bf16(base + SM_DU, r, 2 * hf + (lane >> 4), d0);
             }
             fence_async_smem();
             tc_fence_before();
@@ -649,11 +644,11 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     TG(2);
 
-    // epilogue threads: warp w -> TMEM lanes 32 (w % 4) + l, chunk row r = 16 (w % 4) + l
-    // for l < 16 (M = 64 layout), column half hf = w / 4
-    const int q = warp & 3, hf = warp >> 2;
+    // epilogue threads: warp w -> chunk row r = 16 (w % 4) + (l % 16), in TMEM lane
+    // 32 (w % 4) + l % 16 (M = 64 layout), column half hf = w / 4; the 16-lane loads
+    // give lanes 16-31 the second quarter of the warp's columns (sub = 1)
+    const int q = warp & 3, hf = warp >> 2, sub = lane >> 4;
     const int r = 16 * q + (lane & 15);
-    const bool act = lane < 16;
     const uint32_t la_ = tmem + ((uint32_t)(32 * q) << 16);
     const uint32_t sK = smem_u32(base + Ly::SM_K), sQ = smem_u32(base + Ly::SM_Q),
                    sDO = smem_u32(base + Ly::SM_DO), sSD = smem_u32(base + Ly::SM_SD),
@@ -712,26 +707,28 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
         if (lane == 0) scal[8 + warp] = dot;
     }
-    constexpr int NPC = DV / 32;  // 16-value pieces per thread
+    // 16-value pieces per thread: columns c0 = hf DV / 2 + 16 pc (lanes 0-15) and
+    // c0 + DV / 4 (lanes 16-31)
+    constexpr int NPC = DV / 64;
+    constexpr int QV = DV / 4;
     // epilogue A: X = -gamma o (K S^T), dU' = P^T dO + D o (K dS'^T)
 #pragma unroll 1
     for (int pc = 0; pc < NPC; ++pc) {
-        const int i0 = hf * (DV / 2) + 16 * pc, vp = i0 >> 6, piece = (i0 & 63) >> 4;
+        const int c0 = hf * (DV / 2) + 16 * pc;
+        const int i0 = c0 + sub * QV, vp = i0 >> 6, piece = (i0 & 63) >> 4;
         float ks[16], rr[16], pd[16];
-        tmem_ld16(la_ + i0, ks);
-        tmem_ld16(la_ + DV + i0, rr);
-        tmem_ld16(la_ + 2 * DV + i0, pd);
+        tmem_ld16x2<QV>(la_ + c0, ks);
+        tmem_ld16x2<QV>(la_ + DV + c0, rr);
+        tmem_ld16x2<QV>(la_ + 2 * DV + c0, pd);
         tmem_wait_ld();
-        if (act) {
-            const float gr = gams[r], dr = dcys[r];
+        const float gr = gams[r], dr = dcys[r];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                ks[j] *= -gr;
-                pd[j] = fmaf(dr, rr[j], pd[j]);
-            }
-            tc::store16_bf16(base + Ly::SM_N + vp * PANEL, r, piece, ks);
-            tc::store16_bf16(base + Ly::SM_DU + vp * PANEL, r, piece, pd);
+        for (int j = 0; j < 16; ++j) {
+            ks[j] *= -gr;
+            pd[j] = fmaf(dr, rr[j], pd[j]);
         }
+        tc::store16_bf16(base + Ly::SM_N + vp * PANEL, r, piece, ks);
+        tc::store16_bf16(base + Ly::SM_DU + vp * PANEL, r, piece, pd);
     }
     fence_async_smem();
     tc_fence_before();
@@ -764,48 +761,51 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // epilogue B: U', D o U', Z, -beta gamma o Z, dV = beta o Z, gamma o dO (over X,
     // after the thread's own X piece is read), row dots
     {
-        const float br = act ? bes[r] : 0.f, gr = act ? gams[r] : 0.f, dr = act ? dcys[r] : 0.f;
-        const bool in = act && t0 + r < T;
+        const float br = bes[r], gr = gams[r], dr = dcys[r];
+        const bool in = t0 + r < T;
         float ur = 0.f, zv = 0.f, zx = 0.f;
 #pragma unroll 1
         for (int pc = 0; pc < NPC; ++pc) {
-            const int i0 = hf * (DV / 2) + 16 * pc, vp = i0 >> 6, piece = (i0 & 63) >> 4;
+            const int c0 = hf * (DV / 2) + 16 * pc;
+            const int i0 = c0 + sub * QV, vp = i0 >> 6, piece = (i0 & 63) >> 4;
             float up[16], rr[16], z[16];
-            tmem_ld16(la_ + 2 * DV + i0, up);
-            tmem_ld16(la_ + DV + i0, rr);
-            tmem_ld16(la_ + i0, z);
+            tmem_ld16x2<QV>(la_ + 2 * DV + c0, up);
+            tmem_ld16x2<QV>(la_ + DV + c0, rr);
+            tmem_ld16x2<QV>(la_ + c0, z);
             tmem_wait_ld();
-            if (act) {
-                float t[16];
-                tc::store16_bf16(base + Ly::SM_UT + vp * PANEL, r, piece, up);
+            float t[16];
+            tc::store16_bf16(base + Ly::SM_UT + vp * PANEL, r, piece, up);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    ur = fmaf(up[j], rr[j], ur);
-                    t[j] = dr * up[j];
-                }
-                tc::store16_bf16(base + Ly::SM_UD + vp * PANEL, r, piece, t);
-                tc::store16_bf16(base + Ly::SM_ZT + vp * PANEL, r, piece, z);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) t[j] = -br * gr * z[j];
-                tc::store16_bf16(base + Ly::SM_ZB + vp * PANEL, r, piece, t);
-                if (in) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) t[j] = br * z[j];
-                    store16_global_bf16(p.dv + (((size_t)b * T + t0 + r) * H + h) * DV + i0, t);
-                }
-                load16_bf16(base + Ly::SM_N + vp * PANEL, r, piece, t);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) zx = fmaf(z[j], t[j], zx);
-                load16_bf16(base + Ly::SM_V + vp * PANEL, r, piece, t);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) zv = fmaf(z[j], t[j], zv);
-                load16_bf16(base + Ly::SM_DO + vp * PANEL, r, piece, t);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) t[j] *= gr;
-                tc::store16_bf16(base + Ly::SM_OG + vp * PANEL, r, piece, t);
+            for (int j = 0; j < 16; ++j) {
+                ur = fmaf(up[j], rr[j], ur);
+                t[j] = dr * up[j];
             }
+            tc::store16_bf16(base + Ly::SM_UD + vp * PANEL, r, piece, t);
+            tc::store16_bf16(base + Ly::SM_ZT + vp * PANEL, r, piece, z);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t[j] = -br * gr * z[j];
+            tc::store16_bf16(base + Ly::SM_ZB + vp * PANEL, r, piece, t);
+            if (in) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) t[j] = br * z[j];
+                store16_global_bf16(p.dv + (((size_t)b * T + t0 + r) * H + h) * DV + i0, t);
+            }
+            load16_bf16(base + Ly::SM_N + vp * PANEL, r, piece, t);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) zx = fmaf(z[j], t[j], zx);
+            load16_bf16(base + Ly::SM_V + vp * PANEL, r, piece, t);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) zv = fmaf(z[j], t[j], zv);
+            load16_bf16(base + Ly::SM_DO + vp * PANEL, r, piece, t);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t[j] *= gr;
+            tc::store16_bf16(base + Ly::SM_OG + vp * PANEL, r, piece, t);
         }
-        if (act) {
+        // the two column quarters of a row (lanes l and l + 16) add up
+        ur += __shfl_xor_sync(0xffffffffu, ur, 16);
+        zv += __shfl_xor_sync(0xffffffffu, zv, 16);
+        zx += __shfl_xor_sync(0xffffffffu, zx, 16);
+        if (sub == 0) {
             rs_ur[64 * hf + r] = ur;
             rs_zn[64 * hf + r] = zv + zx;
             rs_zx[64 * hf + r] = zx;
@@ -841,43 +841,40 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     ok = tc::warp_wait(cx, 3, 0) && ok;
     tc_fence_after();
     TG(8);
-    // epilogue C (row r, columns 32 hf .. + 31 of the 64 x 64 matrices):
+    // epilogue C (row r, columns i0 = 32 hf + 16 sub .. + 15 of the 64 x 64 matrices):
     // dP o Gamma (bf16 tile), E^T (row-major scratch), dbeta's and dg's sums, and
     // gamma_r (dO S)_r . q_r from the dQ accumulator before (dP o Gamma) K joins it
     {
-        const float br = act ? bes[r] : 0.f, g2r = act ? g2s[r] : 0.f;
+        const float br = bes[r], g2r = g2s[r];
         // E^T (row-major scratch): entry (i, r) holds E_ri
         __nv_bfloat16 *est = reinterpret_cast<__nv_bfloat16 *>(base + Ly::SM_ES);
         float xr = 0.f, dgr = 0.f, qs = 0.f;
+        // keys 64 hf + 16 pc (lanes 0-15), + 32 (lanes 16-31)
 #pragma unroll 1
-        for (int pc = 0; pc < 4; ++pc) {
-            float x[16];
-            tmem_ld16(la_ + TM_Q2 + 64 * hf + 16 * pc, x);
+        for (int pc = 0; pc < 2; ++pc) {
+            float x[16], qv[16];
+            tmem_ld16x2<32>(la_ + TM_Q2 + 64 * hf + 16 * pc, x);
             tmem_wait_ld();
-            if (act) {
-                float qv[16];
-                load16_bf16(base + Ly::SM_Q + hf * PANEL, r, pc, qv);
+            load16_bf16(base + Ly::SM_Q + hf * PANEL, r, pc + 2 * sub, qv);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) qs = fmaf(x[j], qv[j], qs);
-            }
+            for (int j = 0; j < 16; ++j) qs = fmaf(x[j], qv[j], qs);
         }
         TG(13);
-        float ev[2][16];
-#pragma unroll
-        for (int pc = 0; pc < 2; ++pc) {
-            const int i0 = 32 * hf + 16 * pc;
+        const int i0 = 32 * hf + 16 * sub;
+        float ev[16];
+        {
             float dp[16], da[16], kk[16];
-            tmem_ld16(la_ + TM_DP + i0, dp);
-            tmem_ld16(la_ + TM_DA + i0, da);
-            tmem_ld16(la_ + TM_KK + i0, kk);
+            tmem_ld16x2<16>(la_ + TM_DP + 32 * hf, dp);
+            tmem_ld16x2<16>(la_ + TM_DA + 32 * hf, da);
+            tmem_ld16x2<16>(la_ + TM_KK + 32 * hf, kk);
             tmem_wait_ld();
             float pv[16];
-            if (act) load16_bf16(base + Ly::SM_P, r, i0 >> 4, pv);
+            load16_bf16(base + Ly::SM_P, r, i0 >> 4, pv);
             float col[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = i0 + e;
-                const bool low = act && i <= r, slow = act && i < r;
+                const bool low = i <= r, slow = i < r;
                 const float G = low ? tc::ex2(g2r - g2s[i]) : 0.f;
                 const float dpg = low ? dp[e] * G : 0.f;
                 const float dA = slow ? -da[e] : 0.f;
@@ -885,16 +882,14 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const float x = (slow ? dp[e] * pv[e] : 0.f) + dA * br * Gk;
                 xr += x;
                 dgr = fmaf(dA, Gk, dgr);
-                ev[pc][e] = br * dA * G;
+                ev[e] = br * dA * G;
                 col[e] = x;
                 dp[e] = dpg;
             }
-            if (act) {
-                tc::store16_bf16(base + Ly::SM_DP, r, i0 >> 4, dp);
+            tc::store16_bf16(base + Ly::SM_DP, r, i0 >> 4, dp);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) est[(i0 + e) * C + r] = __float2bfloat16_rn(ev[pc][e]);
-            }
-            // column sums over this warp's 16 rows (lanes 16-31 hold zeros)
+            for (int e = 0; e < 16; ++e) est[(i0 + e) * C + r] = __float2bfloat16_rn(ev[e]);
+            // column sums over the 16 rows of each half-warp
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 float v = col[e];
@@ -904,12 +899,15 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                 col[e] = v;
             }
-            if (lane == 0) {
+            if ((lane & 15) == 0) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) cs_x[64 * q + i0 + e] = col[e];
             }
         }
-        if (act) {
+        xr += __shfl_xor_sync(0xffffffffu, xr, 16);
+        dgr += __shfl_xor_sync(0xffffffffu, dgr, 16);
+        qs += __shfl_xor_sync(0xffffffffu, qs, 16);
+        if (sub == 0) {
             rs_x[64 * hf + r] = xr;
             rs_dg[64 * hf + r] = dgr;
             rs_qs[64 * hf + r] = qs;
@@ -917,28 +915,24 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         TG(14);
         __syncthreads();  // E^T complete
         TG(15);
-        if (act) {
+        {
+            float et[16], ee[16];
+            // row r of E^T is column r of E: E_ir for the rows i > r
+            const uint4 *src = reinterpret_cast<const uint4 *>(est + r * C + i0);
+            const uint4 u0 = src[0], u1 = src[1];
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
-                const int i0 = 32 * hf + 16 * pc;
-                float et[16], ee[16];
-                // row r of E^T is column r of E: E_ir for the rows i > r
-                const uint4 *src = reinterpret_cast<const uint4 *>(est + r * C + i0);
-                const uint4 u0 = src[0], u1 = src[1];
-                const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                    et[2 * e] = f.x;
-                    et[2 * e + 1] = f.y;
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int i = i0 + e;
-                    ee[e] = i < r ? ev[pc][e] : (i > r ? et[e] : 0.f);
-                }
-                tc::store16_bf16(base + Ly::SM_EE, r, i0 >> 4, ee);
+            for (int e = 0; e < 8; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                et[2 * e] = f.x;
+                et[2 * e + 1] = f.y;
             }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int i = i0 + e;
+                ee[e] = i < r ? ev[e] : (i > r ? et[e] : 0.f);
+            }
+            tc::store16_bf16(base + Ly::SM_EE, r, i0 >> 4, ee);
         }
     }
     fence_async_smem();
@@ -966,15 +960,15 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     ok = tc::warp_wait(cx, 4, 0) && ok;
     tc_fence_after();
     TG(10);
-    // final epilogue: dq, dk (row r, keys 64 hf .. + 63)
+    // final epilogue: dq, dk (row r, keys 64 hf + 32 sub .. + 31)
     {
-        const bool in = act && t0 + r < T;
+        const bool in = t0 + r < T;
 #pragma unroll 1
-        for (int pc = 0; pc < 4; ++pc) {
-            const int k0 = 64 * hf + 16 * pc;
+        for (int pc = 0; pc < 2; ++pc) {
+            const int c0 = 64 * hf + 16 * pc, k0 = c0 + 32 * sub;
             float dq[16], dk[16];
-            tmem_ld16(la_ + TM_Q2 + k0, dq);
-            tmem_ld16(la_ + TM_K2 + k0, dk);
+            tmem_ld16x2<32>(la_ + TM_Q2 + c0, dq);
+            tmem_ld16x2<32>(la_ + TM_K2 + c0, dk);
             tmem_wait_ld();
             if (in) {
                 const size_t row = (((size_t)b * T + t0 + r) * H + h) * DK + k0;

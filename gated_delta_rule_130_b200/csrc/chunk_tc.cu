@@ -408,18 +408,19 @@ gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict_
         __syncwarp();
     }
     __syncthreads();  // the gate vectors are written
-    // row r = 16 w + l of G (lanes l < 16 of warp w; lanes 16-31 read unused TMEM),
-    // in two halves of 32 columns (fewer live registers)
-    const int r = 16 * warp + lane;
+    // row r = 16 w + l % 16 of G (TMEM lane 32 w + l % 16 of warp w), columns
+    // 32 hc .. + 31 with hc = l / 16: the 16-lane loads give lanes 16-31 the second
+    // half of the row
+    const int r = 16 * warp + (lane & 15), hc = lane >> 4;
     const bool row_lane = lane < 16;
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const bool done = warp_wait(cx, 1, 0);
     tc_fence_after();
-    const auto load_half = [&](int hc, float (&v)[32]) {
+    const auto load_half = [&](float (&v)[32]) {
         if (done) {
             float a[16], b2[16];
-            tmem_ld16(lane_addr + 32 * hc, a);
-            tmem_ld16(lane_addr + 32 * hc + 16, b2);
+            tmem_ld16x2<32>(lane_addr, a);
+            tmem_ld16x2<32>(lane_addr + 16, b2);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -450,12 +451,11 @@ gdn_ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float *__restrict_
         }
         __syncthreads();
     }
-    // A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0 (row r, all columns)
-#pragma unroll 1
-    for (int hc = 0; hc < 2; ++hc) {
+    // A_ri = beta_r exp(g_r - g_i) (k_r . k_i) for i < r, else 0 (row r, columns 32 hc .. + 31)
+    {
         float v[32];
-        load_half(hc, v);
-        if (row_lane) {
+        load_half(v);
+        {
             const float grl = g2s[r], br = kNorm ? bes[r] * rks[r] : bes[r];
 #pragma unroll
             for (int i4 = 0; i4 < 8; ++i4) {

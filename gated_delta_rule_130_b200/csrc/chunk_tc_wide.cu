@@ -363,27 +363,23 @@ gdn_utw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     }
     {
-        // W rows: row 16 w + l in TMEM lane 32 w + l (l < 16), 256 columns -> 512 B
+        // W rows: row 16 w + l % 16 in TMEM lane 32 w + l % 16; the 16-lane loads give
+        // lanes 0-15 columns 16 pc .. + 15 and lanes 16-31 the next 16
         const bool done = tc::warp_wait(cx, 2, 0);
         tc_fence_after();
-        const int wr = 16 * warp + lane;
-        __nv_bfloat16 *dw = wt + tile * W_ELEMS + (size_t)wr * DK;
+        const int wr = 16 * warp + (lane & 15);
+        __nv_bfloat16 *dw = wt + tile * W_ELEMS + (size_t)wr * DK + 16 * (lane >> 4);
 #pragma unroll 1
         for (int pc = 0; pc < DK / 16; pc += 2) {
-            float v0[16], v1[16];
-            tmem_ld16(lane_addr + 16 * pc, v0);
-            tmem_ld16(lane_addr + 16 * pc + 16, v1);
+            float v0[16];
+            tmem_ld16x2<16>(lane_addr + 16 * pc, v0);
             tmem_wait_ld();
-            if (done && lane < 16) {
+            if (done) {
                 uint4 *d4 = reinterpret_cast<uint4 *>(dw + 16 * pc);
                 d4[0] = make_uint4(tc::pack_bf16(v0[0], v0[1]), tc::pack_bf16(v0[2], v0[3]),
                                    tc::pack_bf16(v0[4], v0[5]), tc::pack_bf16(v0[6], v0[7]));
                 d4[1] = make_uint4(tc::pack_bf16(v0[8], v0[9]), tc::pack_bf16(v0[10], v0[11]),
                                    tc::pack_bf16(v0[12], v0[13]), tc::pack_bf16(v0[14], v0[15]));
-                d4[2] = make_uint4(tc::pack_bf16(v1[0], v1[1]), tc::pack_bf16(v1[2], v1[3]),
-                                   tc::pack_bf16(v1[4], v1[5]), tc::pack_bf16(v1[6], v1[7]));
-                d4[3] = make_uint4(tc::pack_bf16(v1[8], v1[9]), tc::pack_bf16(v1[10], v1[11]),
-                                   tc::pack_bf16(v1[12], v1[13]), tc::pack_bf16(v1[14], v1[15]));
             }
         }
     }
