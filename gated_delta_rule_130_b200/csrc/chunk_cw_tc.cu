@@ -48,14 +48,16 @@
 
 namespace gdn {
 
-// Optional phase timeline of CTA (0,0,0) of the parallel kernel for performance
-// work: build with -DGDN_TRACE; that build alone exports gdn_trace_cw_read().
+// Optional phase timeline of two CTAs of the parallel kernel (chunk 0 and chunk
+// 63 of head 8, batch 0) for performance work: build with -DGDN_TRACE; that build
+// alone exports gdn_trace_cw_read().
 #ifdef GDN_TRACE
-__device__ unsigned long long g_trace_cw[16];
+__device__ unsigned long long g_trace_cw[2 * 16];
 #define TCW(ev)                                                                           \
     do {                                                                                  \
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)   \
-            g_trace_cw[ev] = clock64();                                                   \
+        if (threadIdx.x == 0 && blockIdx.z == 0 &&                                        \
+            ((blockIdx.x == 0 && blockIdx.y == 0) || (blockIdx.x == 63 && blockIdx.y == 8))) \
+            g_trace_cw[(blockIdx.x == 0 ? 0 : 16) + (ev)] = clock64();                    \
     } while (0)
 #else
 #define TCW(ev) \
@@ -71,7 +73,8 @@ using tc::LDA;
 
 constexpr int DK = 128;
 constexpr int THREADS = 512;                  // 16 warps
-constexpr int LDF = DK + 1;                   // float32 row stride of the per-channel arrays
+constexpr int LDF = DK + 8;                   // float32 row stride of the per-channel arrays:
+                                              // 16-byte rows, conflict-free float2 fragments
 constexpr int LDT = C + 8;                    // bf16 row stride of T for the W product
 constexpr int SM_K = 0;                       // k (f32, 64 x LDF)
 constexpr int SM_Q = SM_K + C * LDF * 4;      // q
@@ -88,6 +91,12 @@ constexpr float LOG2E = 1.4426950408889634f;
 static_assert(SM_AF % 16 == 0 && SM_TF % 16 == 0 && SM_PF % 16 == 0 && SM_DS % 16 == 0,
               "16-byte aligned buffers");
 static_assert(SMEM <= 227 * 1024, "shared memory budget");
+static_assert(LDF % 4 == 0 && (C * LDF * 4) % 16 == 0, "16-byte rows of the per-channel arrays");
+
+// channels j, j + 1 (j even) of row r of a per-channel array
+__device__ __forceinline__ float2 ld2(const float *a, int r, int j) {
+    return *reinterpret_cast<const float2 *>(a + r * LDF + j);
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
 gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -119,43 +128,36 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     TCW(0);
 
     // q, k, b o k and log alpha of the chunk's rows (zero past the end); thread ->
-    // (row, 16 consecutive channels): 16-byte loads, all twelve in flight before any
-    // is used (one CTA per SM: the loads in flight are what hides the memory latency)
+    // (row r, four groups of 4 channels 4 g8 + 32 u), so that the eight threads of a
+    // row store 16-byte groups into eight different bank quads; all sixteen loads
+    // are in flight before any is used (one CTA per SM: the loads in flight are
+    // what hides the memory latency)
     {
-        const int r = tid >> 3, jc0 = 16 * (tid & 7);
+        const int r = tid >> 3, g8 = tid & 7;
         const bool in = r < n;
-        const size_t off = ((tok0 + (in ? r : 0)) * H + h) * DK + jc0;
-        uint4 k8[2], q8[2];
+        const size_t off = ((tok0 + (in ? r : 0)) * H + h) * DK + 4 * g8;
+        uint2 k4[4], q4[4];
         float4 b4[4], l4[4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            k8[u] = in ? *reinterpret_cast<const uint4 *>(k + off + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
-            q8[u] = in ? *reinterpret_cast<const uint4 *>(q + off + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < 4; ++u) {
+            k4[u] = in ? *reinterpret_cast<const uint2 *>(k + off + 32 * u) : make_uint2(0u, 0u);
+            q4[u] = in ? *reinterpret_cast<const uint2 *>(q + off + 32 * u) : make_uint2(0u, 0u);
+            b4[u] = in ? *reinterpret_cast<const float4 *>(bg + off + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            l4[u] = in ? *reinterpret_cast<const float4 *>(la + off + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            b4[u] = in ? *reinterpret_cast<const float4 *>(bg + off + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
-            l4[u] = in ? *reinterpret_cast<const float4 *>(la + off + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        const uint32_t kw[8] = {k8[0].x, k8[0].y, k8[0].z, k8[0].w, k8[1].x, k8[1].y, k8[1].z, k8[1].w};
-        const uint32_t qw[8] = {q8[0].x, q8[0].y, q8[0].z, q8[0].w, q8[1].x, q8[1].y, q8[1].z, q8[1].w};
-        const float bv[16] = {b4[0].x, b4[0].y, b4[0].z, b4[0].w, b4[1].x, b4[1].y, b4[1].z, b4[1].w,
-                              b4[2].x, b4[2].y, b4[2].z, b4[2].w, b4[3].x, b4[3].y, b4[3].z, b4[3].w};
-        const float lv[16] = {l4[0].x, l4[0].y, l4[0].z, l4[0].w, l4[1].x, l4[1].y, l4[1].z, l4[1].w,
-                              l4[2].x, l4[2].y, l4[2].z, l4[2].w, l4[3].x, l4[3].y, l4[3].z, l4[3].w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kw[e]));
-            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qw[e]));
-            const int j = jc0 + 2 * e;
-            KF[r * LDF + j] = kf.x;
-            KF[r * LDF + j + 1] = kf.y;
-            QF[r * LDF + j] = qf.x;
-            QF[r * LDF + j + 1] = qf.y;
-            BK[r * LDF + j] = bv[2 * e] * kf.x;
-            BK[r * LDF + j + 1] = bv[2 * e + 1] * kf.y;
-            LM[r * LDF + j] = lv[2 * e] * LOG2E;
-            LM[r * LDF + j + 1] = lv[2 * e + 1] * LOG2E;
+            const int j = 4 * g8 + 32 * u;
+            const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&k4[u].x));
+            const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&k4[u].y));
+            const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q4[u].x));
+            const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&q4[u].y));
+            *reinterpret_cast<float4 *>(KF + r * LDF + j) = make_float4(k01.x, k01.y, k23.x, k23.y);
+            *reinterpret_cast<float4 *>(QF + r * LDF + j) = make_float4(q01.x, q01.y, q23.x, q23.y);
+            *reinterpret_cast<float4 *>(BK + r * LDF + j) =
+                make_float4(b4[u].x * k01.x, b4[u].y * k01.y, b4[u].z * k23.x, b4[u].w * k23.y);
+            *reinterpret_cast<float4 *>(LM + r * LDF + j) =
+                make_float4(l4[u].x * LOG2E, l4[u].y * LOG2E, l4[u].z * LOG2E, l4[u].w * LOG2E);
         }
     }
     // per-channel passes below: thread -> (channel jc, quarter rq of the rows)
@@ -185,9 +187,11 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     // the two 8 x 8 diagonal sub-blocks of each diagonal 16-block, summed
     // directly: warps 4I .. 4I+3 take block I, each a quarter of the channels.
     // Lane -> sub-block s, the rows rp and 7 - rp of it (rp + 1 and 8 - rp pairs
-    // (r, i), i <= r: nine in all) and 8 of the warp's 32 channels (cs), so each
-    // row's values are loaded once per channel and the columns' values are shared
-    // by the two rows; the four lanes of a row pair then add their channel parts.
+    // (r, i), i <= r: nine in all) and 8 of the warp's 32 channels (the pairs
+    // 8 jb + 2 cs, + 1 for jb < 4: float2 loads whose 8-byte banks differ across a
+    // half-warp), so each row's values are loaded once per channel and the
+    // columns' values are shared by the two rows; the four lanes of a row pair
+    // then add their channel parts.
     {
         const int I = warp >> 2, ch = warp & 3;
         const int sb = lane >> 4, rp = (lane >> 2) & 3, cs = lane & 3;
@@ -195,22 +199,26 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         const int rA = i0 + rp, rB = i0 + 7 - rp;
         float aA[4] = {}, pA[4] = {}, aB[8] = {}, pB[8] = {};
 #pragma unroll 2
-        for (int jj = 0; jj < 8; ++jj) {
-            const int j = 32 * ch + 8 * cs + jj;
-            const float lA = LM[rA * LDF + j], lB = LM[rB * LDF + j];
-            const float bA = BK[rA * LDF + j], bB = BK[rB * LDF + j];
-            const float qA = QF[rA * LDF + j], qB = QF[rB * LDF + j];
+        for (int jb = 0; jb < 4; ++jb) {
+            const int j = 32 * ch + 8 * jb + 2 * cs;
+            const float2 lA = ld2(LM, rA, j), lB = ld2(LM, rB, j);
+            const float2 bA = ld2(BK, rA, j), bB = ld2(BK, rB, j);
+            const float2 qA = ld2(QF, rA, j), qB = ld2(QF, rB, j);
 #pragma unroll
             for (int ii = 0; ii < 8; ++ii) {
-                const float lI = LM[(i0 + ii) * LDF + j], kI = KF[(i0 + ii) * LDF + j];
+                const float2 lI = ld2(LM, i0 + ii, j), kI = ld2(KF, i0 + ii, j);
                 // exponents are <= 0 where kept (Lam is non-increasing down the rows)
-                const float eB = ii <= 7 - rp ? tc::ex2(fminf(lB - lI, 0.f)) * kI : 0.f;
-                aB[ii] = fmaf(bB, eB, aB[ii]);
-                pB[ii] = fmaf(qB, eB, pB[ii]);
+                const bool kB = ii <= 7 - rp;
+                const float eB0 = kB ? tc::ex2(fminf(lB.x - lI.x, 0.f)) * kI.x : 0.f;
+                const float eB1 = kB ? tc::ex2(fminf(lB.y - lI.y, 0.f)) * kI.y : 0.f;
+                aB[ii] = fmaf(bB.y, eB1, fmaf(bB.x, eB0, aB[ii]));
+                pB[ii] = fmaf(qB.y, eB1, fmaf(qB.x, eB0, pB[ii]));
                 if (ii < 4) {
-                    const float eA = ii <= rp ? tc::ex2(fminf(lA - lI, 0.f)) * kI : 0.f;
-                    aA[ii] = fmaf(bA, eA, aA[ii]);
-                    pA[ii] = fmaf(qA, eA, pA[ii]);
+                    const bool kA = ii <= rp;
+                    const float eA0 = kA ? tc::ex2(fminf(lA.x - lI.x, 0.f)) * kI.x : 0.f;
+                    const float eA1 = kA ? tc::ex2(fminf(lA.y - lI.y, 0.f)) * kI.y : 0.f;
+                    aA[ii] = fmaf(bA.y, eA1, fmaf(bA.x, eA0, aA[ii]));
+                    pA[ii] = fmaf(qA.y, eA1, fmaf(qA.x, eA0, pA[ii]));
                 }
             }
         }
@@ -283,14 +291,16 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 #pragma unroll 2
         for (int ks = 0; ks < DK / 16; ++ks) {
             const int j0 = 16 * ks;
+            // Lam of the reference row at the fragments' two channel pairs
+            const float2 lm[2] = {ld2(LM, mref, j0 + 2 * t), ld2(LM, mref, j0 + 2 * t + 8)};
             uint32_t aL[4], aM[4];
 #pragma unroll
             for (int sl = 0; sl < 4; ++sl) {  // a0 (g, 2t) a1 (g+8, 2t) a2 (g, 2t+8) a3 (g+8, 2t+8)
                 const int r = 16 * I + g + 8 * (sl & 1), j = j0 + 2 * t + 8 * (sl >> 1);
-                const float e0 = tc::ex2(LM[r * LDF + j] - LM[mref * LDF + j]);
-                const float e1 = tc::ex2(LM[r * LDF + j + 1] - LM[mref * LDF + j + 1]);
-                aL[sl] = tc::pack_bf16(BK[r * LDF + j] * e0, BK[r * LDF + j + 1] * e1);
-                aM[sl] = tc::pack_bf16(QF[r * LDF + j] * e0, QF[r * LDF + j + 1] * e1);
+                const float2 lr = ld2(LM, r, j), bk = ld2(BK, r, j), qf = ld2(QF, r, j);
+                const float e0 = tc::ex2(lr.x - lm[sl >> 1].x), e1 = tc::ex2(lr.y - lm[sl >> 1].y);
+                aL[sl] = tc::pack_bf16(bk.x * e0, bk.y * e1);
+                aM[sl] = tc::pack_bf16(qf.x * e0, qf.y * e1);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -299,10 +309,8 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 uint32_t bb[2];
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
-                    const int j = j0 + 2 * t + 8 * hb;
-                    const float e0 = tc::ex2(LM[mref * LDF + j] - LM[i * LDF + j]);
-                    const float e1 = tc::ex2(LM[mref * LDF + j + 1] - LM[i * LDF + j + 1]);
-                    bb[hb] = tc::pack_bf16(KF[i * LDF + j] * e0, KF[i * LDF + j + 1] * e1);
+                    const float2 li = ld2(LM, i, j0 + 2 * t + 8 * hb), kf = ld2(KF, i, j0 + 2 * t + 8 * hb);
+                    bb[hb] = tc::pack_bf16(kf.x * tc::ex2(lm[hb].x - li.x), kf.y * tc::ex2(lm[hb].y - li.y));
                 }
                 mma_bf16_16x8x16(accA[nt], aL, bb);
                 mma_bf16_16x8x16(accP[nt], aM, bb);
@@ -326,23 +334,22 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 #pragma unroll 2
         for (int ks = 0; ks < DK / 16; ++ks) {
             const int j0 = 16 * ks;
+            const float2 lm[2] = {ld2(LM, mref, j0 + 2 * t), ld2(LM, mref, j0 + 2 * t + 8)};
             uint32_t aL[4] = {0u, 0u, 0u, 0u}, aM[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
             for (int sl = 1; sl < 4; sl += 2) {  // a1 (g+8, 2t), a3 (g+8, 2t+8)
                 const int r = 16 * I + 8 + g, j = j0 + 2 * t + 8 * (sl >> 1);
-                const float e0 = tc::ex2(LM[r * LDF + j] - LM[mref * LDF + j]);
-                const float e1 = tc::ex2(LM[r * LDF + j + 1] - LM[mref * LDF + j + 1]);
-                aL[sl] = tc::pack_bf16(BK[r * LDF + j] * e0, BK[r * LDF + j + 1] * e1);
-                aM[sl] = tc::pack_bf16(QF[r * LDF + j] * e0, QF[r * LDF + j + 1] * e1);
+                const float2 lr = ld2(LM, r, j), bk = ld2(BK, r, j), qf = ld2(QF, r, j);
+                const float e0 = tc::ex2(lr.x - lm[sl >> 1].x), e1 = tc::ex2(lr.y - lm[sl >> 1].y);
+                aL[sl] = tc::pack_bf16(bk.x * e0, bk.y * e1);
+                aM[sl] = tc::pack_bf16(qf.x * e0, qf.y * e1);
             }
             const int i = 16 * I + g;  // B[kk][n] = K_i o 2^(Lam_m - Lam_i), n = g
             uint32_t bb[2];
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
-                const int j = j0 + 2 * t + 8 * hb;
-                const float e0 = tc::ex2(LM[mref * LDF + j] - LM[i * LDF + j]);
-                const float e1 = tc::ex2(LM[mref * LDF + j + 1] - LM[i * LDF + j + 1]);
-                bb[hb] = tc::pack_bf16(KF[i * LDF + j] * e0, KF[i * LDF + j + 1] * e1);
+                const float2 li = ld2(LM, i, j0 + 2 * t + 8 * hb), kf = ld2(KF, i, j0 + 2 * t + 8 * hb);
+                bb[hb] = tc::pack_bf16(kf.x * tc::ex2(lm[hb].x - li.x), kf.y * tc::ex2(lm[hb].y - li.y));
             }
             mma_bf16_16x8x16(accA, aL, bb);
             mma_bf16_16x8x16(accP, aM, bb);
