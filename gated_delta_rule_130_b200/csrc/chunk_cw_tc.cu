@@ -97,6 +97,10 @@ static_assert(LDF % 4 == 0 && (C * LDF * 4) % 16 == 0, "16-byte rows of the per-
 __device__ __forceinline__ float2 ld2(const float *a, int r, int j) {
     return *reinterpret_cast<const float2 *>(a + r * LDF + j);
 }
+// channels j .. j + 3 (j a multiple of 4)
+__device__ __forceinline__ float4 ld4(const float *a, int r, int j) {
+    return *reinterpret_cast<const float4 *>(a + r * LDF + j);
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
 gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -207,16 +211,17 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 #pragma unroll
             for (int ii = 0; ii < 8; ++ii) {
                 const float2 lI = ld2(LM, i0 + ii, j), kI = ld2(KF, i0 + ii, j);
-                // exponents are <= 0 where kept (Lam is non-increasing down the rows)
+                // exponents are <= 0 where kept (Lam is non-increasing down the rows;
+                // the pairs left out are selected away, whatever their exponent)
                 const bool kB = ii <= 7 - rp;
-                const float eB0 = kB ? tc::ex2(fminf(lB.x - lI.x, 0.f)) * kI.x : 0.f;
-                const float eB1 = kB ? tc::ex2(fminf(lB.y - lI.y, 0.f)) * kI.y : 0.f;
+                const float eB0 = kB ? tc::ex2(lB.x - lI.x) * kI.x : 0.f;
+                const float eB1 = kB ? tc::ex2(lB.y - lI.y) * kI.y : 0.f;
                 aB[ii] = fmaf(bB.y, eB1, fmaf(bB.x, eB0, aB[ii]));
                 pB[ii] = fmaf(qB.y, eB1, fmaf(qB.x, eB0, pB[ii]));
                 if (ii < 4) {
                     const bool kA = ii <= rp;
-                    const float eA0 = kA ? tc::ex2(fminf(lA.x - lI.x, 0.f)) * kI.x : 0.f;
-                    const float eA1 = kA ? tc::ex2(fminf(lA.y - lI.y, 0.f)) * kI.y : 0.f;
+                    const float eA0 = kA ? tc::ex2(lA.x - lI.x) * kI.x : 0.f;
+                    const float eA1 = kA ? tc::ex2(lA.y - lI.y) * kI.y : 0.f;
                     aA[ii] = fmaf(bA.y, eA1, fmaf(bA.x, eA0, aA[ii]));
                     pA[ii] = fmaf(qA.y, eA1, fmaf(qA.x, eA0, pA[ii]));
                 }
@@ -328,7 +333,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     }
     // rows 8-15 against rows 0-7 of each diagonal block through its row 7 (warps
     // 6-9, one block each): a 16 x 8 product whose rows 0-7 are left zero
-    if (warp >= 6 && warp < 10) {
+    else if (warp < 10) {
         const int I = warp - 6, mref = 16 * I + 7;
         float accA[4] = {}, accP[4] = {};
 #pragma unroll 2
@@ -358,14 +363,60 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         *reinterpret_cast<float2 *>(AF + r1 * LDA + col) = make_float2(accA[2], accA[3]);
         *reinterpret_cast<float2 *>(PF + r1 * LDA + col) = make_float2(accP[2], accP[3]);
     }
+    else {
+        // w o V (it needs neither A nor P) on the six warps the block products leave
+        // idle: item -> (row, 16 consecutive value channels), 16-byte loads
+        for (int item = tid - 320; item < C * (Dv / 16); item += THREADS - 320) {
+            const int r = item / (Dv / 16), jv0 = 16 * (item % (Dv / 16));
+            if (r >= n) break;
+            const size_t off = ((tok0 + r) * H + h) * Dv + jv0;
+            const uint4 v0 = *reinterpret_cast<const uint4 *>(v + off);
+            const uint4 v1 = *reinterpret_cast<const uint4 *>(v + off + 8);
+            float4 w4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w4[u] = *reinterpret_cast<const float4 *>(wg + off + 4 * u);
+            const uint32_t vw_[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const float wv[16] = {w4[0].x, w4[0].y, w4[0].z, w4[0].w, w4[1].x, w4[1].y, w4[1].z, w4[1].w,
+                                  w4[2].x, w4[2].y, w4[2].z, w4[2].w, w4[3].x, w4[3].y, w4[3].z, w4[3].w};
+            uint32_t out[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vw_[e]));
+                out[e] = tc::pack_bf16(f.x * wv[2 * e], f.y * wv[2 * e + 1]);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(vw + off);
+            dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+            dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
+    }
     __syncthreads();  // A and P complete
     TCW(4);
 
     // T = (I + A)^-1: diagonal blocks by substitution, the rest by block products
-    // on warps 0-3 (named barrier 1)
-    if (tid < C) tc::ut_diag(AF, TF, tid);
-    __syncthreads();
-    if (tid < 128) tc::ut_offdiag4<1>(AF, TF, tid);
+    // on warps 0-3 (named barrier 1); meanwhile warps 4-15 write the sequential
+    // kernel's token operands Q o 2^Lam and K o 2^(Lam_last - Lam): item -> (row r,
+    // 4 channels 4 g8 + 32 u) as in the input phase (16-byte shared-memory reads
+    // whose bank quads differ across eight threads, 8-byte stores)
+    if (warp < 4) {
+        if (tid < C) tc::ut_diag(AF, TF, tid);
+        named_barrier(1, 128);
+        tc::ut_offdiag4<1>(AF, TF, tid);
+    } else {
+        for (int item = tid - 128; item < C * 32; item += THREADS - 128) {
+            const int r = item >> 5, g8 = item & 7, u = (item >> 3) & 3;
+            if (r >= n) break;
+            const int j = 4 * g8 + 32 * u;
+            const float4 lr = ld4(LM, r, j), ll = ld4(LM, C - 1, j);
+            const float4 qf = ld4(QF, r, j), kf = ld4(KF, r, j);
+            const size_t off = ((tok0 + r) * H + h) * DK + j;
+            *reinterpret_cast<uint2 *>(qe + off) =
+                make_uint2(tc::pack_bf16(qf.x * tc::ex2(lr.x), qf.y * tc::ex2(lr.y)),
+                           tc::pack_bf16(qf.z * tc::ex2(lr.z), qf.w * tc::ex2(lr.w)));
+            *reinterpret_cast<uint2 *>(kd + off) =
+                make_uint2(tc::pack_bf16(kf.x * tc::ex2(ll.x - lr.x), kf.y * tc::ex2(ll.y - lr.y)),
+                           tc::pack_bf16(kf.z * tc::ex2(ll.z - lr.z), kf.w * tc::ex2(ll.w - lr.w)));
+        }
+    }
     __syncthreads();
     TCW(5);
 
@@ -437,40 +488,7 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     }
 
     TCW(7);
-    // the sequential kernel's token operands: Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
-    for (int rr = 0; rr < RQ; ++rr) {
-        const int r = rq * RQ + rr;
-        if (r < n) {
-            const size_t off = ((tok0 + r) * H + h) * DK + jc;
-            const float lr = LM[r * LDF + jc];
-            qe[off] = __float2bfloat16_rn(QF[r * LDF + jc] * tc::ex2(lr));
-            kd[off] = __float2bfloat16_rn(KF[r * LDF + jc] * tc::ex2(LM[(C - 1) * LDF + jc] - lr));
-        }
-    }
     TCW(8);
-    // w o V: thread -> (row, 16 consecutive value channels), 16-byte loads
-    for (int item = tid; item < C * (Dv / 16); item += THREADS) {
-        const int r = item / (Dv / 16), jv0 = 16 * (item % (Dv / 16));
-        if (r >= n) continue;
-        const size_t off = ((tok0 + r) * H + h) * Dv + jv0;
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(v + off);
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(v + off + 8);
-        float4 w4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) w4[u] = *reinterpret_cast<const float4 *>(wg + off + 4 * u);
-        const uint32_t vw_[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        const float wv[16] = {w4[0].x, w4[0].y, w4[0].z, w4[0].w, w4[1].x, w4[1].y, w4[1].z, w4[1].w,
-                              w4[2].x, w4[2].y, w4[2].z, w4[2].w, w4[3].x, w4[3].y, w4[3].z, w4[3].w};
-        uint32_t out[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vw_[e]));
-            out[e] = tc::pack_bf16(f.x * wv[2 * e], f.y * wv[2 * e + 1]);
-        }
-        uint4 *dst = reinterpret_cast<uint4 *>(vw + off);
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    }
     TCW(9);
 }
 
