@@ -496,7 +496,10 @@ struct L {
     // [1] gamma_last, [2] [4] the final scans' warp totals, [8 + w] warp w's part of <dS', S>
     static constexpr int SM_SCAL = SM_MISC + NF * 64 * 4;
     static constexpr int SM_BAR = SM_SCAL + 64;
-    static constexpr int SMEM_BYTES = SM_BAR + 5 * 8 + 16 + 1024;
+    // [0] TMA  [1] phase A  [2] phase B  [3] phase C: dP, dA'  [4] phase D
+    // [5] K K^T  [6] phase C: dQ, dK
+    static constexpr int NBAR = 7;
+    static constexpr int SMEM_BYTES = SM_BAR + NBAR * 8 + 16 + 1024;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     static_assert(VB >= PANEL && SM_SD % 1024 == 0 && SM_MISC % 1024 == 0, "layout");
 };
@@ -527,9 +530,9 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
     cx.base = base;
-    cx.bar = reinterpret_cast<uint64_t *>(base + Ly::SM_BAR);  // [0] TMA [1] A [2] B [3] C [4] D
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly::SM_BAR + 40);
-    cx.abort = reinterpret_cast<volatile uint32_t *>(base + Ly::SM_BAR + 44);
+    cx.bar = reinterpret_cast<uint64_t *>(base + Ly::SM_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly::SM_BAR + Ly::NBAR * 8);
+    cx.abort = reinterpret_cast<volatile uint32_t *>(base + Ly::SM_BAR + Ly::NBAR * 8 + 4);
     cx.err = &g_bwd_error;
     float *fv = reinterpret_cast<float *>(base + Ly::SM_MISC);
     float *g2s = fv + Ly::F_G2 * 64, *bes = fv + Ly::F_BE * 64, *gams = fv + Ly::F_GAM * 64,
@@ -547,7 +550,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     TG(0);
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(cx.bar + i, 1);
+        for (int i = 0; i < Ly::NBAR; ++i) mbar_init(cx.bar + i, 1);
         *cx.abort = 0u;
         fence_mbar_init();
     }
@@ -677,11 +680,15 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int j = 0; j < C / 16; ++j)
                 mma_bf16(tmem + 2 * DV, desc_sw128(sP + j * 2048, PANEL, 1024),
                          desc_sw128(sDO + j * 2048, PANEL, 1024), idesc_bf16(64, DV, true, true), j > 0);
+        }
+        mma_commit(cx.bar + 1);
+        // K K^T is read by epilogue C only
+        if (landed) {
 #pragma unroll
             for (int j = 0; j < DK / 16; ++j)
                 mma_bf16(tmem + TM_KK, kdesc(sK, j), kdesc(sK, j), idesc_bf16(64, 64, false, false), j > 0);
         }
-        mma_commit(cx.bar + 1);
+        mma_commit(cx.bar + 5);
     }
     bool ok = tc::warp_wait(cx, 1, 0);
     tc_fence_after();
@@ -820,12 +827,19 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     //                  dK = (D o U') dS' + (-beta gamma o Z) S
     if (tid == 0) {
         tc_fence_after();
+        const uint32_t id64 = idesc_bf16(64, 64, false, false), idk = idesc_bf16(64, DK, false, true);
         if (ok) {
-            const uint32_t id64 = idesc_bf16(64, 64, false, false), idk = idesc_bf16(64, DK, false, true);
 #pragma unroll
             for (int j = 0; j < DV / 16; ++j) {
                 mma_bf16(tmem + TM_DP, kdesc(sDO, j), kdesc(sUT, j), id64, j > 0);
                 mma_bf16(tmem + TM_DA, kdesc(sZT, j), kdesc(sUT, j), id64, j > 0);
+            }
+        }
+        mma_commit(cx.bar + 3);
+        // the wider dQ and dK products run while epilogue C reads dP and dA'
+        if (ok) {
+#pragma unroll
+            for (int j = 0; j < DV / 16; ++j) {
                 mma_bf16(tmem + TM_Q2, kdesc(sOG, j), desc_sw128(sSD + j * 2048, Ly::SD_PANEL, 1024), idk,
                          j > 0);
                 mma_bf16(tmem + TM_K2, kdesc(sUD, j),
@@ -836,9 +850,10 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mma_bf16(tmem + TM_K2, kdesc(sZB, j), desc_sw128(sSD + j * 2048, Ly::SD_PANEL, 1024),
                          idk, 1u);
         }
-        mma_commit(cx.bar + 3);
+        mma_commit(cx.bar + 6);
     }
     ok = tc::warp_wait(cx, 3, 0) && ok;
+    ok = tc::warp_wait(cx, 5, 0) && ok;
     tc_fence_after();
     TG(8);
     // epilogue C (row r, columns i0 = 32 hf + 16 sub .. + 15 of the 64 x 64 matrices):
@@ -849,17 +864,6 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // E^T (row-major scratch): entry (i, r) holds E_ri
         __nv_bfloat16 *est = reinterpret_cast<__nv_bfloat16 *>(base + Ly::SM_ES);
         float xr = 0.f, dgr = 0.f, qs = 0.f;
-        // keys 64 hf + 16 pc (lanes 0-15), + 32 (lanes 16-31)
-#pragma unroll 1
-        for (int pc = 0; pc < 2; ++pc) {
-            float x[16], qv[16];
-            tmem_ld16x2<32>(la_ + TM_Q2 + 64 * hf + 16 * pc, x);
-            tmem_wait_ld();
-            load16_bf16(base + Ly::SM_Q + hf * PANEL, r, pc + 2 * sub, qv);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) qs = fmaf(x[j], qv[j], qs);
-        }
-        TG(13);
         const int i0 = 32 * hf + 16 * sub;
         float ev[16];
         {
@@ -887,8 +891,6 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 dp[e] = dpg;
             }
             tc::store16_bf16(base + Ly::SM_DP, r, i0 >> 4, dp);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) est[(i0 + e) * C + r] = __float2bfloat16_rn(ev[e]);
             // column sums over the 16 rows of each half-warp
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -903,6 +905,23 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
                 for (int e = 0; e < 16; ++e) cs_x[64 * q + i0 + e] = col[e];
             }
+        }
+        TG(13);
+        // once the dQ and dK products have completed: E^T over their operand
+        // -beta gamma o Z, and gamma_r (dO S)_r . q_r (keys 64 hf + 16 pc in lanes
+        // 0-15, + 32 in lanes 16-31)
+        ok = tc::warp_wait(cx, 6, 0) && ok;
+        tc_fence_after();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) est[(i0 + e) * C + r] = __float2bfloat16_rn(ev[e]);
+#pragma unroll 1
+        for (int pc = 0; pc < 2; ++pc) {
+            float x[16], qv[16];
+            tmem_ld16x2<32>(la_ + TM_Q2 + 64 * hf + 16 * pc, x);
+            tmem_wait_ld();
+            load16_bf16(base + Ly::SM_Q + hf * PANEL, r, pc + 2 * sub, qv);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) qs = fmaf(x[j], qv[j], qs);
         }
         xr += __shfl_xor_sync(0xffffffffu, xr, 16);
         dgr += __shfl_xor_sync(0xffffffffu, dgr, 16);
