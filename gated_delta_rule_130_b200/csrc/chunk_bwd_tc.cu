@@ -1075,22 +1075,21 @@ bool make_map_wt(CUtensorMap *m, const void *ptr, long long n_tiles) {
 }
 
 struct Ws {
-    __nv_bfloat16 *pt, *wt, *tr, *S_hist, *dS_hist, *o_scratch;
+    __nv_bfloat16 *pt, *wt, *tr, *S_hist, *dS_hist;
     size_t bytes;
 };
 
 inline size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace: [P; T''] tiles | W tiles | T tiles | S_hist | dS_hist (both bf16) |
-// the recompute's scratch output.
+// Workspace: [P; T''] tiles | W tiles | T tiles | S_hist | dS_hist (both bf16).
 Ws carve(void *base, int B, int T, int H, int Dv) {
     const size_t NT = ((size_t)T + C - 1) / C, tiles = (size_t)B * NT * H;
     const size_t states = (size_t)B * H * NT * Dv * DK;
-    const size_t sz[6] = {tiles * 2 * C * C * 2, tiles * C * DK * 2, tiles * C * C * 2, states * 2,
-                          states * 2, (size_t)B * T * H * Dv * 2};
+    const size_t sz[5] = {tiles * 2 * C * C * 2, tiles * C * DK * 2, tiles * C * C * 2, states * 2,
+                          states * 2};
     uint8_t *p = static_cast<uint8_t *>(base);
-    size_t off[6], o = 0;
-    for (int i = 0; i < 6; ++i) {
+    size_t off[5], o = 0;
+    for (int i = 0; i < 5; ++i) {
         off[i] = o;
         o += up256(sz[i]);
     }
@@ -1100,7 +1099,6 @@ Ws carve(void *base, int B, int T, int H, int Dv) {
     w.tr = reinterpret_cast<__nv_bfloat16 *>(p + off[2]);
     w.S_hist = reinterpret_cast<__nv_bfloat16 *>(p + off[3]);
     w.dS_hist = reinterpret_cast<__nv_bfloat16 *>(p + off[4]);
-    w.o_scratch = reinterpret_cast<__nv_bfloat16 *>(p + off[5]);
     w.bytes = o;
     return w;
 }
@@ -1157,7 +1155,7 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
     Ws w = carve(workspace, B, T, H, Dv);
     // recompute: the chunk tiles, then the state entering every chunk
     cudaError_t e = launch_recompute_bwd(q, k, v, la, beta, S0, B, T, H, Dv, w.pt, w.wt, w.tr,
-                                         w.S_hist, w.o_scratch, st);
+                                         w.S_hist, st);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mdo, mw, mp, mpt, mt;
     if (!tc::make_map(&mq, q, B, T, H, DK) || !tc::make_map(&mk, k, B, T, H, DK) ||

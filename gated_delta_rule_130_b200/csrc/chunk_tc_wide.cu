@@ -738,12 +738,15 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                                  desc_sw128(up + kk * 2048, 16, 1024), idesc_s, 1u);
                 mma_commit(cx.bar + B_ST_FULL);
                 mma_commit(cx.bar + B_K_EMPTY + sq);
-                // Y += [P; T''] U'  (Y holds gamma Q S^T; rows 64-127 unused)
+                // Y += [P; T''] U'  (Y holds gamma Q S^T; rows 64-127 unused); a call
+                // without an output (the states alone) skips it
+                if (p.o) {
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    mma_bf16(tmem + TM_Y, desc_sw128(vp + BLK + kk * 32, 16, 1024),
-                             desc_sw128(un + kk * 2048, 16, 1024), idesc_x, 1u);
-                mma_commit(cx.bar + B_Y_FULL);
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tmem + TM_Y, desc_sw128(vp + BLK + kk * 32, 16, 1024),
+                                 desc_sw128(un + kk * 2048, 16, 1024), idesc_x, 1u);
+                    mma_commit(cx.bar + B_Y_FULL);
+                }
                 mma_commit(cx.bar + B_VP_EMPTY + s);
             }
             __syncwarp();
@@ -829,20 +832,23 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::warp_arrive(cx, B_U_READY);
                 if (warp == W_STATE0 + 2) TW(c, 9);
             } else {
-                // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y
-                const float gr = gv[GV_GAM + lrow];
-                float x0[16], x1[16];
-                tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
-                tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
-                tmem_wait_ld();
+                // inter-chunk part of the output, gamma_r (Q S^T)_r, into Y (when there
+                // is an output)
+                if (p.o) {
+                    const float gr = gv[GV_GAM + lrow];
+                    float x0[16], x1[16];
+                    tmem_ld16(lane_addr + TM_X + 32 * hf, x0);
+                    tmem_ld16(lane_addr + TM_X + 32 * hf + 16, x1);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    x0[j] *= gr;
-                    x1[j] *= gr;
+                    for (int j = 0; j < 16; ++j) {
+                        x0[j] *= gr;
+                        x1[j] *= gr;
+                    }
+                    tmem_st16(lane_addr + TM_Y + 32 * hf, x0);
+                    tmem_st16(lane_addr + TM_Y + 32 * hf + 16, x1);
+                    tmem_wait_st();
                 }
-                tmem_st16(lane_addr + TM_Y + 32 * hf, x0);
-                tmem_st16(lane_addr + TM_Y + 32 * hf + 16, x1);
-                tmem_wait_st();
                 tc_fence_before();
                 tc::warp_arrive(cx, B_U_READY);
                 if (warp == W_STATE0) TW(c, 13);
@@ -896,14 +902,14 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (!last && !have) break;
             }
             // chunk output rows (TMEM lanes 0-63)
-            if (q < 2) {
+            if (q < 2 && p.o) {
                 if (!tc::warp_wait(cx, B_Y_FULL, c & 1)) break;
                 tc_fence_after();
                 float y0[16], y1[16];
                 tmem_ld16(lane_addr + TM_Y + 32 * hf, y0);
                 tmem_ld16(lane_addr + TM_Y + 32 * hf + 16, y1);
                 tmem_wait_ld();
-                if (p.o && t0 + lrow < T) {
+                if (t0 + lrow < T) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
                         p.o + ((size_t)(sp.off + t0 + lrow) * H + h) * p.Dv + v0 + 32 * hf);
 #pragma unroll
@@ -1281,12 +1287,12 @@ cudaError_t launch_chunk_tcw_seq_cw(const void *qe, const void *kd, const void *
 // The backward's recompute (Dk = 128, gates as given, B sequences of T tokens):
 // the parallel kernel writes per chunk and head the [P; T''] tile, the W tile and
 // T itself (tile index (b NT + c) H + h); the sequential kernel, fed those tiles,
-// records the state entering every chunk in bf16 ([B*H][NT][Dv][128]) and writes
-// its output to o_scratch.
+// records the state entering every chunk in bf16 ([B*H][NT][Dv][128]) and forms
+// no output.
 cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  int B, int T, int H, int Dv, void *pt, void *wt, void *tr,
-                                 void *S_hist, void *o_scratch, cudaStream_t st) {
+                                 void *S_hist, cudaStream_t st) {
     constexpr int DK = 128;
     const long long NT = ((long long)T + tc::C - 1) / tc::C;
     if (B < 1 || NT < 1) return cudaSuccess;
@@ -1311,7 +1317,7 @@ cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
     tcw::Params p;
     p.log_alpha = log_alpha;
     p.S0 = S0;
-    p.o = static_cast<__nv_bfloat16 *>(o_scratch);
+    p.o = nullptr;
     p.S_T = nullptr;
     p.rqk = nullptr;
     p.glk = nullptr;

@@ -68,7 +68,7 @@ cudaError_t launch_chunk_bwd_tc(const void *q, const void *k, const void *v, con
 cudaError_t launch_recompute_bwd(const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta, const float *S0,
                                  int B, int T, int H, int Dv, void *pt, void *wt, void *tr,
-                                 void *S_hist, void *o_scratch, cudaStream_t st);
+                                 void *S_hist, cudaStream_t st);
 
 // Channel-wise gates (decay per key channel, erase gate b on the key side,
 // write gate w on the value side; CUDA cores, Dk <= 128): chunk_cw.cu.

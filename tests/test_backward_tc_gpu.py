@@ -118,13 +118,11 @@ def test_bwd_tc_degenerate_gates(gdn, gate):
 
 def test_bwd_tc_workspace_size(gdn):
     # [P; T''], W and T tiles per chunk and head, the chunk states and the state
-    # gradients (both bf16) and the recompute's scratch output, each region
-    # rounded up to 256 bytes
+    # gradients (both bf16), each region rounded up to 256 bytes
     B, T, H, Dv = 2, 130, 3, 128
     NT = 3
     tiles = B * NT * H
     up = lambda n: (n + 255) // 256 * 256
     want = (up(tiles * 2 * 64 * 64 * 2) + up(tiles * 64 * 128 * 2) + up(tiles * 64 * 64 * 2)
-            + up(B * H * NT * Dv * 128 * 2) + up(B * H * NT * Dv * 128 * 2)
-            + up(B * T * H * Dv * 2))
+            + up(B * H * NT * Dv * 128 * 2) + up(B * H * NT * Dv * 128 * 2))
     assert gdn.chunk_bwd_workspace_size(B, T, H, 128, Dv, 64, torch.bfloat16) == want
