@@ -391,14 +391,6 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tmem_wait_ld();
             tc::store16_bf16(base + SM_SB, lrow, 2 * hf, x0);
             tc::store16_bf16(base + SM_SB, lrow, 2 * hf + 1, x1);
-            {   // dS' of chunk c for the gradient kernel, [Dv][Dk] bf16
-                __nv_bfloat16 *dst = p.dS_hist + ((head * NT + c) * p.Dv + v0 + 32 * hf) * DK + lrow;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    dst[j * DK] = __float2bfloat16_rn(x0[j]);
-                    dst[(16 + j) * DK] = __float2bfloat16_rn(x1[j]);
-                }
-            }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 x0[j] *= gl;
@@ -410,6 +402,20 @@ gdn_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             fence_async_smem();
             tc_fence_before();
             tc::warp_arrive(cx, B_S_READY);
+            {   // dS' of chunk c for the gradient kernel, [Dv][Dk] bf16, from this
+                // thread's own row of the bf16 copy (beside the K dS'^T product)
+                auto *dst = reinterpret_cast<unsigned short *>(p.dS_hist) +
+                            ((head * NT + c) * p.Dv + v0 + 32 * hf) * DK + lrow;
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(
+                        base + SM_SB + sw128_offset(lrow, (4 * hf + k8) * 16));
+                    const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[(size_t)(8 * k8 + e) * DK] = (unsigned short)(e & 1 ? wd[e >> 1] >> 16 : wd[e >> 1] & 0xffffu);
+                }
+            }
             // -dU' rows = -(P^T dO + D o (K dS'^T))
             if (!tc::warp_wait(cx, B_PD_FULL + s, (k >> 1) & 1) || !tc::warp_wait(cx, B_R_FULL, k & 1)) {
                 ok = false;

@@ -873,13 +873,6 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (!last) {
 #pragma unroll
                     for (int pc = 0; pc < NPC; ++pc) tc::store16_bf16(sbuf, key, col0 / 16 + pc, sv[pc]);
-                    if (p.S_hist)  // the state entering chunk c + 1
-#pragma unroll
-                        for (int pc = 0; pc < NPC; ++pc)
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                p.S_hist[(((size_t)head * NT + c + 1) * p.Dv + v0 + col0 + 16 * pc + j) * DK +
-                                         key] = __float2bfloat16_rn(sv[pc][j]);
 #pragma unroll
                     for (int pc = 0; pc < NPC; ++pc)
 #pragma unroll
@@ -899,6 +892,24 @@ gdn_chunk_tcw_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc_fence_before();
                 tc::warp_arrive(cx, B_S_READY);
                 if (warp == W_STATE0) TW(c, 11);
+                if (!last && p.S_hist) {
+                    // the state entering chunk c + 1, from this thread's own bf16 row
+                    // of the copy (after the hand-off, beside the next X product)
+                    auto *dst = reinterpret_cast<unsigned short *>(p.S_hist) +
+                                (((size_t)head * NT + c + 1) * p.Dv + v0 + col0) * DK + key;
+#pragma unroll
+                    for (int pc = 0; pc < NPC; ++pc)
+#pragma unroll
+                        for (int k8 = 0; k8 < 2; ++k8) {
+                            const uint4 u = *reinterpret_cast<const uint4 *>(
+                                sbuf + sw128_offset(key, (2 * (col0 / 16 + pc) + k8) * 16));
+                            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[(size_t)(16 * pc + 8 * k8 + e) * DK] =
+                                    (unsigned short)(e & 1 ? wd[e >> 1] >> 16 : wd[e >> 1] & 0xffffu);
+                        }
+                }
                 if (!last && !have) break;
             }
             // chunk output rows (TMEM lanes 0-63)
