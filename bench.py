@@ -44,9 +44,10 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def measured_traffic(path: str):
+def measured_traffic(path: str, w):
     """DRAM bytes of one call (both tcgen05-path kernels) from the committed ncu
-    summary, or None if the kernel sources changed since the capture."""
+    summary, or None if the call is not the captured workload or the kernel sources
+    changed since the capture."""
     import hashlib
     f = os.path.join(ROOT, "profiles", "traffic_gdn_chunk_fwd_tc.txt")
     if path != "tcgen05" or not os.path.exists(f):
@@ -54,7 +55,10 @@ def measured_traffic(path: str):
     value, ok = None, True
     for line in open(f):
         line = line.strip()
-        if line.startswith("dram_bytes_per_call:"):
+        if line.startswith("workload:"):
+            name = line.split(":", 1)[1].strip()
+            ok = ok and name in I.WORKLOADS and I.workload(name) == w
+        elif line.startswith("dram_bytes_per_call:"):
             value = float(line.split(":", 1)[1])
         elif line.startswith("sha256 "):
             rel, digest = line[len("sha256 "):].split(":", 1)
@@ -285,7 +289,11 @@ def run_ours(args):
     inp_cpu = I.chunk_inputs(w, seed=w.seed + rank)
     inp = {n: (t.to(device) if t is not None else None) for n, t in inp_cpu.items()}
     path = G.chunk_fwd_path(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
-    launches_per_step = {"tcgen05": 2, "simt": 2}[path]
+    # the parallel tile (UT) kernel and the sequential kernel; a split sequence adds
+    # the map initialisation, the two first-pass walks and the scan
+    variant = (G.chunk_fwd_variant(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
+               if path == "tcgen05" else None)
+    launches_per_step = 6 if variant == "split" else 2
     o = torch.empty((w.B, w.T, w.H, w.Dv), dtype=w.torch_dtype, device=device)
     S_T = torch.empty((w.B, w.H, w.Dv, w.Dk), dtype=torch.float32, device=device)
     ws_bytes = G.chunk_fwd_workspace_size(w.B, w.T, w.H, w.Dk, w.Dv, w.chunk, w.torch_dtype)
@@ -330,7 +338,7 @@ def run_ours(args):
     hbm_peak = pk["hbm_gbs"]
     tc_peak = pk["bf16_tflops"]
     roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": gbs / hbm_peak, "traffic": measured_traffic(path),
+                "frac": gbs / hbm_peak, "traffic": measured_traffic(path, w),
                 "kernel": f"gdn_chunk_fwd ({path}, {launches_per_step} launches/step, timed together)",
                 "algorithmic_bytes": Bytes, "peak_source": f"{pk_kind} hbm_gbs",
                 "tc": {"achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s",
@@ -629,7 +637,7 @@ def run_ours(args):
                        "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
                        "l2": "inputs larger than L2 (q,k,v,o = %.0f MB per rank)" %
                              (4 * o.numel() * o.element_size() / 1e6),
-                       "path": path},
+                       "path": path, "variant": variant},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": steps * launches_per_step, "clocks": clocks, "decode": decode,
             "prologue": prologue, "varlen": varlen, "backward": backward,
