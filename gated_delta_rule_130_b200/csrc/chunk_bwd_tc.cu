@@ -570,7 +570,21 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     TG(1);
 
-    // warp 1 issues the copies and warp 2 the prefetches while warp 0 loads the gates
+    const uint32_t sK = smem_u32(base + Ly::SM_K), sQ = smem_u32(base + Ly::SM_Q),
+                   sDO = smem_u32(base + Ly::SM_DO), sSD = smem_u32(base + Ly::SM_SD),
+                   sP = smem_u32(base + Ly::SM_P), sT = smem_u32(base + Ly::SM_T),
+                   sN = smem_u32(base + Ly::SM_N), sDU = smem_u32(base + Ly::SM_DU),
+                   sUD = smem_u32(base + Ly::SM_UD), sZB = smem_u32(base + Ly::SM_ZB),
+                   sZT = smem_u32(base + Ly::SM_ZT), sDP = smem_u32(base + Ly::SM_DP),
+                   sEE = smem_u32(base + Ly::SM_EE), sUT = smem_u32(base + Ly::SM_UT),
+                   sOG = smem_u32(base + Ly::SM_OG);
+    const auto kdesc = [](uint32_t t, int j) {  // K-major operand, step j of 16 along K
+        return desc_sw128(t + (j >> 2) * PANEL + (j & 3) * 32, 16, 1024);
+    };
+
+    // warp 1 issues the copies and then, once they have landed, the products of
+    // phase A (they do not need the gates), and warp 2 the prefetches, while warp 0
+    // loads the gates
     if (tid == 32) {
         uint64_t *fb = cx.bar + 0;
         mbar_arrive_expect_tx(fb, 4 * PANEL + 2 * Ly::VB + 3 * PANEL + 4 * DV * 128);
@@ -592,15 +606,48 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL, &tm_sh, fb, kb * 64, 0, hist);
             tma_load_3d(base + Ly::SM_SD + kb * Ly::SD_PANEL + DV * 128, &tm_dsh, fb, kb * 64, 0, hist);
         }
+        // ---------------- phase A: [K S^T | K dS'^T], P^T dO, K K^T
+        const bool landed = tc::wait_bar(cx, 0, 0);
+        tc_fence_after();
+        if (landed) {
+#pragma unroll
+            for (int j = 0; j < DK / 16; ++j)
+                mma_bf16(tmem, kdesc(sK, j),
+                         desc_sw128(sSD + (j >> 2) * Ly::SD_PANEL + (j & 3) * 32, 16, 1024),
+                         idesc_bf16(64, 2 * DV, false, false), j > 0);
+#pragma unroll
+            for (int j = 0; j < C / 16; ++j)
+                mma_bf16(tmem + 2 * DV, desc_sw128(sP + j * 2048, PANEL, 1024),
+                         desc_sw128(sDO + j * 2048, PANEL, 1024), idesc_bf16(64, DV, true, true), j > 0);
+        }
+        mma_commit(cx.bar + 1);
+        // K K^T is read by epilogue C only
+        if (landed) {
+#pragma unroll
+            for (int j = 0; j < DK / 16; ++j)
+                mma_bf16(tmem + TM_KK, kdesc(sK, j), kdesc(sK, j), idesc_bf16(64, 64, false, false), j > 0);
+        }
+        mma_commit(cx.bar + 5);
     }
-    if (tid == 64) {
+    if (warp == 2) {
         // one CTA per SM: the CTA one wave later (linear index + SM count) finds its
-        // inputs in L2, their DRAM reads overlapping this CTA's products
+        // inputs in L2, their DRAM reads overlapping this CTA's products (the tiles by
+        // lane 0, the gates of its rows by every lane)
         const long long lin = blockIdx.x + (long long)NT * (blockIdx.y + (long long)H * blockIdx.z);
         const long long nxt = lin + p.pf_stride;
         if (p.pf_stride > 0 && nxt < (long long)NT * H * gridDim.z) {
             const int c2 = (int)(nxt % NT), h2 = (int)((nxt / NT) % H), b2 = (int)(nxt / ((long long)NT * H));
             const int t2 = c2 * C, tile2 = (b2 * NT + c2) * H + h2, hist2 = (b2 * H + h2) * NT + c2;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int rr = lane + 32 * hh;
+                if (t2 + rr < T) {
+                    const size_t gi = ((size_t)b2 * T + t2 + rr) * H + h2;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.log_alpha + gi));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.beta + gi));
+                }
+            }
+            if (lane == 0) {
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb) {
                 tma_prefetch_l2_4d(&tm_k, kb * 64, h2, t2, b2);
@@ -615,6 +662,7 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             tma_prefetch_l2_3d(&tm_pt, 0, 0, tile2);
             tma_prefetch_l2_3d(&tm_t, 0, 0, tile2);
+            }
         }
     }
     if (warp == 0) {
@@ -659,43 +707,8 @@ gdn_bwd_grads_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int q = warp & 3, hf = warp >> 2, sub = lane >> 4;
     const int r = 16 * q + (lane & 15);
     const uint32_t la_ = tmem + ((uint32_t)(32 * q) << 16);
-    const uint32_t sK = smem_u32(base + Ly::SM_K), sQ = smem_u32(base + Ly::SM_Q),
-                   sDO = smem_u32(base + Ly::SM_DO), sSD = smem_u32(base + Ly::SM_SD),
-                   sP = smem_u32(base + Ly::SM_P), sT = smem_u32(base + Ly::SM_T),
-                   sN = smem_u32(base + Ly::SM_N), sDU = smem_u32(base + Ly::SM_DU),
-                   sUD = smem_u32(base + Ly::SM_UD), sZB = smem_u32(base + Ly::SM_ZB),
-                   sZT = smem_u32(base + Ly::SM_ZT), sDP = smem_u32(base + Ly::SM_DP),
-                   sEE = smem_u32(base + Ly::SM_EE), sUT = smem_u32(base + Ly::SM_UT),
-                   sOG = smem_u32(base + Ly::SM_OG);
-    const auto kdesc = [](uint32_t t, int j) {  // K-major operand, step j of 16 along K
-        return desc_sw128(t + (j >> 2) * PANEL + (j & 3) * 32, 16, 1024);
-    };
 
-    // ---------------- phase A: [K S^T | K dS'^T], P^T dO, K K^T
-    if (tid == 0) {
-        const bool landed = tc::wait_bar(cx, 0, 0);
-        tc_fence_after();
-        TG(3);
-        if (landed) {
-#pragma unroll
-            for (int j = 0; j < DK / 16; ++j)
-                mma_bf16(tmem, kdesc(sK, j),
-                         desc_sw128(sSD + (j >> 2) * Ly::SD_PANEL + (j & 3) * 32, 16, 1024),
-                         idesc_bf16(64, 2 * DV, false, false), j > 0);
-#pragma unroll
-            for (int j = 0; j < C / 16; ++j)
-                mma_bf16(tmem + 2 * DV, desc_sw128(sP + j * 2048, PANEL, 1024),
-                         desc_sw128(sDO + j * 2048, PANEL, 1024), idesc_bf16(64, DV, true, true), j > 0);
-        }
-        mma_commit(cx.bar + 1);
-        // K K^T is read by epilogue C only
-        if (landed) {
-#pragma unroll
-            for (int j = 0; j < DK / 16; ++j)
-                mma_bf16(tmem + TM_KK, kdesc(sK, j), kdesc(sK, j), idesc_bf16(64, 64, false, false), j > 0);
-        }
-        mma_commit(cx.bar + 5);
-    }
+    TG(3);
     bool ok = tc::warp_wait(cx, 1, 0);
     tc_fence_after();
     TG(4);
