@@ -202,26 +202,46 @@ gdn_ut_cw_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         const int i0 = 16 * I + 8 * sb;
         const int rA = i0 + rp, rB = i0 + 7 - rp;
         float aA[4] = {}, pA[4] = {}, aB[8] = {}, pB[8] = {};
+        // The decay from row i to row r (i <= r) of the sub-block is the product of the
+        // decays between consecutive rows, d_m = 2^(Lam_{m+1} - Lam_m) <= 1 for
+        // m = i .. r - 1: seven exp2 per channel, no overflow for any decay, and the
+        // factors multiply in float32 (a running product down the columns).
+        const int b = 7 - rp;  // rB and rA within the sub-block: b and rp
 #pragma unroll 2
         for (int jb = 0; jb < 4; ++jb) {
             const int j = 32 * ch + 8 * jb + 2 * cs;
-            const float2 lA = ld2(LM, rA, j), lB = ld2(LM, rB, j);
             const float2 bA = ld2(BK, rA, j), bB = ld2(BK, rB, j);
             const float2 qA = ld2(QF, rA, j), qB = ld2(QF, rB, j);
+            float2 l[8], kI[8];
 #pragma unroll
             for (int ii = 0; ii < 8; ++ii) {
-                const float2 lI = ld2(LM, i0 + ii, j), kI = ld2(KF, i0 + ii, j);
-                // exponents are <= 0 where kept (Lam is non-increasing down the rows;
-                // the pairs left out are selected away, whatever their exponent)
-                const bool kB = ii <= 7 - rp;
-                const float eB0 = kB ? tc::ex2(lB.x - lI.x) * kI.x : 0.f;
-                const float eB1 = kB ? tc::ex2(lB.y - lI.y) * kI.y : 0.f;
+                l[ii] = ld2(LM, i0 + ii, j);
+                kI[ii] = ld2(KF, i0 + ii, j);
+            }
+            float2 d[7];
+#pragma unroll
+            for (int m = 0; m < 7; ++m)
+                d[m] = make_float2(tc::ex2(l[m + 1].x - l[m].x), tc::ex2(l[m + 1].y - l[m].y));
+            // row rB: columns ii = b down to 0 (eB = 1 at ii = b, then times d[ii])
+            float2 eB = make_float2(1.f, 1.f), eA = make_float2(1.f, 1.f);
+#pragma unroll
+            for (int ii = 7; ii >= 0; --ii) {
+                if (ii < 7 && ii < b) {
+                    eB.x *= d[ii].x;
+                    eB.y *= d[ii].y;
+                }
+                const bool kB = ii <= b;
+                const float eB0 = kB ? eB.x * kI[ii].x : 0.f, eB1 = kB ? eB.y * kI[ii].y : 0.f;
                 aB[ii] = fmaf(bB.y, eB1, fmaf(bB.x, eB0, aB[ii]));
                 pB[ii] = fmaf(qB.y, eB1, fmaf(qB.x, eB0, pB[ii]));
                 if (ii < 4) {
+                    // row rA: columns ii = rp down to 0
+                    if (ii < 3 && ii < rp) {
+                        eA.x *= d[ii].x;
+                        eA.y *= d[ii].y;
+                    }
                     const bool kA = ii <= rp;
-                    const float eA0 = kA ? tc::ex2(lA.x - lI.x) * kI.x : 0.f;
-                    const float eA1 = kA ? tc::ex2(lA.y - lI.y) * kI.y : 0.f;
+                    const float eA0 = kA ? eA.x * kI[ii].x : 0.f, eA1 = kA ? eA.y * kI[ii].y : 0.f;
                     aA[ii] = fmaf(bA.y, eA1, fmaf(bA.x, eA0, aA[ii]));
                     pA[ii] = fmaf(qA.y, eA1, fmaf(qA.x, eA0, pA[ii]));
                 }
