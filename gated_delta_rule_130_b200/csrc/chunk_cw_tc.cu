@@ -29,8 +29,9 @@
 //         a tcgen05 product);
 //       - inside a diagonal block, rows 8-15 against rows 0-7 factor the same
 //         way through the block's row 7 (mma.sync); the two 8 x 8 diagonal
-//         sub-blocks are summed directly over the channels in float32 (exp2 of
-//         the exact differences), four warps per block;
+//         sub-blocks are summed directly over the channels in float32, the
+//         decay from row i to row r as the product of the consecutive-row
+//         decays 2^(Lam_{m+1} - Lam_m) <= 1, four warps per block;
 //     then the blocked UT solve, W = T (b o K o 2^Lam) (mma.sync), and the
 //     operands of the sequential kernel: [P; T''] (T'' = T with the columns of
 //     rows past the end zeroed), W, Q o 2^Lam, K o 2^(Lam_last - Lam), w o V
